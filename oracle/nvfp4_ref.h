@@ -1,0 +1,102 @@
+/*
+ * nvfp4_ref.h -- CPU oracle for NVFP4 block quantization with ScaleSearch.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This is the plain, slow, single-threaded definition that the CUDA
+ * library is checked against.  Only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg may load it.  It shares no code, header, table or constant generator with the CUDA path.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [NVFP4]  "NVIDIAのFP4推論が50倍の効率を実現" (introl.com), section "超低精度推論を支えるアーキテクチャ":
+ *           E2M1 values (1 sign, 2 exponent, 1 mantissa bit) in 16-value micro-blocks, one E4M3 FP8
+ *           scale per micro-block and one FP32 scale per tensor.
+ *  [E2M1]   "RTX 50 FP4" article (aitroublesolution.com), section "FP4（4ビット浮動小数点）の仕組みと利点":
+ *           the 1/2/1 sign/exponent/mantissa split.
+ *  [SS]     "Search your block floating-point scales!" (gist.science summary of arXiv 2605.12464),
+ *           Method > ScaleSearch (mechanism, search strategy, rationale), ScaleSearchAttention
+ *           (incoherence processing, attention-sink mixed-precision caching).
+ *  [BEV]    "BEVFormer on B200: FP8/FP4 CUDA kernel tuning" (qiita.com), section 7 (scale applied
+ *           back by one multiply; FP8 max 448; two FP4 values per uint8) and its normalised error.
+ *
+ * Arithmetic: IEEE binary32, round-to-nearest-even, no FMA contraction (built with
+ * -ffp-contract=off, no fast-math), subnormals kept.  Converters are integer bit manipulation.
+ *
+ * Parity status: every function below is pinned by the not-gpu tests (library converters,
+ * brute-force search, closed forms, invariants); the exact f* histogram shape on Gaussian data is
+ * qualitative on the pages (bimodal) and is "parity unpinned" beyond that shape.
+ */
+#ifndef NVFP4_REF_H
+#define NVFP4_REF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types (same numbering as the library's dtype codes, by convention only) */
+enum { REF_F32 = 0, REF_BF16 = 1, REF_F16 = 2 };
+
+/* ---- scalar converters ---- */
+/* E2M1 encode: round-to-nearest-even onto {0,.5,1,1.5,2,3,4,6}, |y|>6 saturates to 6,
+ * sign bit kept (negative values that round to zero give code 0x8).  y must be finite. */
+uint8_t ref_e2m1_encode(float y);
+/* E2M1 decode of the low 4 bits of code. */
+float ref_e2m1_decode(uint8_t code);
+/* E4M3 (fn variant: bias 7, no infinities, 0x7F/0xFF = NaN) encode, RNE, saturating at 448. */
+uint8_t ref_e4m3_encode(float v);
+float ref_e4m3_decode(uint8_t code);
+/* dtype helpers: exact widening; RNE narrowing (overflow -> inf, NaN -> quiet NaN). */
+float ref_bf16_to_f32(uint16_t h);
+float ref_f16_to_f32(uint16_t h);
+uint16_t ref_f32_to_bf16(float f);
+uint16_t ref_f32_to_f16(float f);
+
+/* array forms (plain loops over the scalar converters) */
+void ref_e2m1_encode_n(const float* y, int64_t n, uint8_t* out);
+void ref_e4m3_encode_n(const float* v, int64_t n, uint8_t* out);
+void ref_f32_to_bf16_n(const float* v, int64_t n, uint16_t* out);
+void ref_f32_to_f16_n(const float* v, int64_t n, uint16_t* out);
+void ref_f16_to_f32_n(const uint16_t* h, int64_t n, float* out);
+
+/* ---- tensor-level steps ---- */
+/* max |x_i| as the unsigned maximum of the magnitude bits: NaN/Inf propagate.  n may be 0 (-> 0). */
+float ref_tensor_amax(const void* x, int64_t n, int dtype);
+/* per-tensor FP32 scale g = fl(amax / (6*448)) */
+float ref_global_scale(float amax);
+
+/* One 16-element block of ScaleSearch.  x: 16 floats, g: tensor scale, offsets f in [f_lo, f_hi].
+ * Outputs 8 packed code bytes (element 2k low nibble, 2k+1 high nibble), the scale byte, the chosen
+ * offset (-128 when the block has no valid candidate, is all zero or is poisoned) and its SSE. */
+void ref_search_block(const float* x, float g, int f_lo, int f_hi,
+                      uint8_t* codes8, uint8_t* scale, int8_t* fstar, float* sse);
+
+/* Max-scaling written on its own (no candidate loop): scale = E4M3(amax_b/6/g). */
+void ref_maxscale_block(const float* x, float g, uint8_t* codes8, uint8_t* scale, float* sse);
+
+/* Whole-tensor ScaleSearch quantize.  gscale_in: NULL -> computed from the tensor amax.
+ * block_f / block_sse may be NULL.  Returns 0, or -2 if n % 16 != 0. */
+int ref_quantize(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const float* gscale_in,
+                 uint8_t* codes, uint8_t* scales, float* gscale_out, int8_t* block_f, float* block_sse);
+
+/* Same, over a range of blocks [b0, b1) with a given g (used for sampled full-size checks). */
+void ref_quantize_blocks(const void* x, int dtype, int64_t b0, int64_t b1, float g, int f_lo, int f_hi,
+                         uint8_t* codes, uint8_t* scales, int8_t* block_f, float* block_sse);
+
+/* Dequantize: out_i = fl(dec(q_i) * fl(dec(scale_b) * g)), narrowed to out_dtype by RNE. */
+int ref_dequantize(const uint8_t* codes, const uint8_t* scales, float g, int64_t n, int out_dtype, void* out);
+
+/* 16-point fast Walsh-Hadamard transform on each contiguous group of 16, times 1/4. */
+int ref_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype);
+void ref_fwht16_f32(float* a);
+
+/* Mixed-precision KV layout for K[B,H,T,D] (BF16): tokens [0,sink) and [T-recent,T) copied verbatim,
+ * the rest optionally rotated (FWHT-16 along D) and ScaleSearch-quantized along D with one tensor
+ * scale over the (rotated) middle tokens.  codes: [B,H,T_mid,D/2], scales: [B,H,T_mid,D/16]. */
+int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, int sink, int recent,
+                 int rotate, int f_lo, int f_hi, uint16_t* sink_out, uint16_t* recent_out,
+                 uint8_t* codes, uint8_t* scales, float* gscale_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

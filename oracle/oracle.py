@@ -1,0 +1,226 @@
+"""ctypes wrapper around the C oracle (``nvfp4_ref.c``).
+
+TEST INFRASTRUCTURE ONLY.  This is the plain CPU definition of NVFP4 block quantization with
+ScaleSearch that the CUDA library is checked against.  Only ``tests/``, ``__graft_entry__.smoke()``
+and ``bench.py``'s CPU-baseline leg may import it; the library never does.
+
+All array arguments are numpy arrays (contiguous); results come back as new numpy arrays.
+Element types use the codes 0 = float32, 1 = bfloat16 (stored as uint16), 2 = float16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_ref.c")
+_SO = os.path.join(_HERE, "libnvfp4_ref.so")
+CFLAGS = ["-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-Wall"]
+
+F32, BF16, F16 = 0, 1, 2
+_NP_OF = {F32: np.float32, BF16: np.uint16, F16: np.uint16}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libnvfp4_ref.so`` with gcc (strict IEEE flags)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < max(
+        os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "nvfp4_ref.h"))
+    ):
+        subprocess.run(["gcc", *CFLAGS, "-o", _SO, _SRC, "-lm"], check=True)
+    return _SO
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        sig = {
+            "ref_e2m1_encode": (ctypes.c_uint8, [F]),
+            "ref_e2m1_decode": (F, [ctypes.c_uint8]),
+            "ref_e4m3_encode": (ctypes.c_uint8, [F]),
+            "ref_e4m3_decode": (F, [ctypes.c_uint8]),
+            "ref_e2m1_encode_n": (None, [P, I64, P]),
+            "ref_e4m3_encode_n": (None, [P, I64, P]),
+            "ref_f32_to_bf16_n": (None, [P, I64, P]),
+            "ref_f32_to_f16_n": (None, [P, I64, P]),
+            "ref_f16_to_f32_n": (None, [P, I64, P]),
+            "ref_tensor_amax": (F, [P, I64, I]),
+            "ref_global_scale": (F, [F]),
+            "ref_search_block": (None, [P, F, I, I, P, P, P, P]),
+            "ref_maxscale_block": (None, [P, F, P, P, P]),
+            "ref_quantize": (I, [P, I64, I, I, I, P, P, P, P, P, P]),
+            "ref_quantize_blocks": (None, [P, I, I64, I64, F, I, I, P, P, P, P]),
+            "ref_dequantize": (I, [P, P, F, I64, I, P]),
+            "ref_hadamard16": (I, [P, I64, I, P, I]),
+            "ref_fwht16_f32": (None, [P]),
+            "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_of(x: np.ndarray) -> int:
+    if x.dtype == np.float32:
+        return F32
+    raise TypeError("pass float32 arrays, or uint16 arrays with an explicit dtype code")
+
+
+# ---- scalar / array converters ----
+def e2m1_encode(y: np.ndarray) -> np.ndarray:
+    y = np.ascontiguousarray(y, np.float32)
+    out = np.empty(y.shape, np.uint8)
+    lib().ref_e2m1_encode_n(_p(y), y.size, _p(out))
+    return out
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().ref_e4m3_encode_n(_p(v), v.size, _p(out))
+    return out
+
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().ref_e2m1_decode(code))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().ref_e4m3_decode(code))
+
+
+def f32_to_bf16(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().ref_f32_to_bf16_n(_p(v), v.size, _p(out))
+    return out
+
+
+def f32_to_f16(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().ref_f32_to_f16_n(_p(v), v.size, _p(out))
+    return out
+
+
+def f16_to_f32(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, np.uint16)
+    out = np.empty(h.shape, np.float32)
+    lib().ref_f16_to_f32_n(_p(h), h.size, _p(out))
+    return out
+
+
+# ---- tensor steps ----
+def tensor_amax(x: np.ndarray, dtype: int | None = None) -> np.float32:
+    x = np.ascontiguousarray(x)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    return np.float32(lib().ref_tensor_amax(_p(x), x.size, dtype))
+
+
+def global_scale(amax) -> np.float32:
+    return np.float32(lib().ref_global_scale(float(amax)))
+
+
+def search_block(x16: np.ndarray, g, f_lo: int, f_hi: int):
+    x16 = np.ascontiguousarray(x16, np.float32)
+    assert x16.size == 16
+    codes = np.zeros(8, np.uint8)
+    sc = np.zeros(1, np.uint8)
+    fs = np.zeros(1, np.int8)
+    sse = np.zeros(1, np.float32)
+    lib().ref_search_block(_p(x16), float(g), f_lo, f_hi, _p(codes), _p(sc), _p(fs), _p(sse))
+    return codes, int(sc[0]), int(fs[0]), sse[0]
+
+
+def maxscale_block(x16: np.ndarray, g):
+    x16 = np.ascontiguousarray(x16, np.float32)
+    codes = np.zeros(8, np.uint8)
+    sc = np.zeros(1, np.uint8)
+    sse = np.zeros(1, np.float32)
+    lib().ref_maxscale_block(_p(x16), float(g), _p(codes), _p(sc), _p(sse))
+    return codes, int(sc[0]), sse[0]
+
+
+def quantize(x: np.ndarray, f_lo: int = -2, f_hi: int = 6, dtype: int | None = None, gscale_in=None):
+    """Returns (codes[n/2], scales[n/16], g, block_f[n/16], block_sse[n/16])."""
+    x = np.ascontiguousarray(x)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    n = x.size
+    nb = n // 16
+    codes = np.empty(n // 2, np.uint8)
+    scales = np.empty(nb, np.uint8)
+    bf = np.empty(nb, np.int8)
+    bs = np.empty(nb, np.float32)
+    g = np.zeros(1, np.float32)
+    gin = None if gscale_in is None else np.array([gscale_in], np.float32)
+    rc = lib().ref_quantize(_p(x), n, dtype, f_lo, f_hi, _p(gin), _p(codes), _p(scales), _p(g), _p(bf), _p(bs))
+    if rc != 0:
+        raise ValueError(f"ref_quantize returned {rc}")
+    return codes, scales, g[0], bf, bs
+
+
+def quantize_blocks(x: np.ndarray, b0: int, b1: int, g, f_lo: int = -2, f_hi: int = 6, dtype: int | None = None):
+    x = np.ascontiguousarray(x)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    nb = b1 - b0
+    codes = np.empty(nb * 8, np.uint8)
+    scales = np.empty(nb, np.uint8)
+    bf = np.empty(nb, np.int8)
+    bs = np.empty(nb, np.float32)
+    lib().ref_quantize_blocks(_p(x), dtype, b0, b1, float(g), f_lo, f_hi, _p(codes), _p(scales), _p(bf), _p(bs))
+    return codes, scales, bf, bs
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, g, out_dtype: int = F32) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    n = scales.size * 16
+    out = np.empty(n, _NP_OF[out_dtype])
+    rc = lib().ref_dequantize(_p(codes), _p(scales), float(g), n, out_dtype, _p(out))
+    if rc != 0:
+        raise ValueError(f"ref_dequantize returned {rc}")
+    return out
+
+
+def hadamard16(x: np.ndarray, dtype: int | None = None, out_dtype: int = F32) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    out = np.empty(x.size, _NP_OF[out_dtype])
+    rc = lib().ref_hadamard16(_p(x), x.size, dtype, _p(out), out_dtype)
+    if rc != 0:
+        raise ValueError(f"ref_hadamard16 returned {rc}")
+    return out
+
+
+def kv_mixed(k_bf16: np.ndarray, sink: int = 16, recent: int = 16, rotate: int = 1, f_lo: int = -2, f_hi: int = 6):
+    """k_bf16: uint16 array [B,H,T,D].  Returns (sink[B,H,sink,D], recent[B,H,recent,D],
+    codes[B,H,Tm,D/2], scales[B,H,Tm,D/16], g)."""
+    k = np.ascontiguousarray(k_bf16, np.uint16)
+    B, H, T, D = k.shape
+    Tm = T - sink - recent
+    so = np.empty((B, H, sink, D), np.uint16)
+    ro = np.empty((B, H, recent, D), np.uint16)
+    codes = np.empty((B, H, Tm, D // 2), np.uint8)
+    scales = np.empty((B, H, Tm, D // 16), np.uint8)
+    g = np.zeros(1, np.float32)
+    rc = lib().ref_kv_mixed(_p(k), B, H, T, D, sink, recent, rotate, f_lo, f_hi, _p(so), _p(ro), _p(codes), _p(scales), _p(g))
+    if rc != 0:
+        raise ValueError(f"ref_kv_mixed returned {rc}")
+    return so, ro, codes, scales, g[0]

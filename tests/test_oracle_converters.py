@@ -1,0 +1,114 @@
+"""Pins of the oracle's number-format converters against the ml_dtypes / numpy library casts and
+the format definitions (E2M1: 1 sign, 2 exponent, 1 mantissa bit; E4M3 with 448 as largest value)."""
+import ml_dtypes as md
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+GOLDEN = __import__("os").path.join(__import__("os").path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    vals = []
+    with open(f"{GOLDEN}/{name}") as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                vals.append(line.split())
+    return vals
+
+
+def _binade_sweep(e_lo, e_hi):
+    """All float32 bit patterns with biased exponent in [e_lo, e_hi) (every mantissa), per binade."""
+    m = np.arange(1 << 23, dtype=np.uint32)
+    for e in range(e_lo, e_hi):
+        yield ((np.uint32(e) << np.uint32(23)) | m).view(np.float32)
+
+
+def test_e2m1_decode_matches_format_definition():
+    rows = _read_golden("e2m1_values.txt")
+    for code_s, val_s in rows:
+        code = int(code_s, 0)
+        assert O.e2m1_decode(code) == float(val_s)
+        # the same code with the sign bit set decodes to the negated value (including -0)
+        neg = O.e2m1_decode(code | 8)
+        assert neg == -float(val_s) and np.signbit(neg)
+    # and agrees with the library decode of every 4-bit pattern
+    lib = np.arange(16, dtype=np.uint8).view(md.float4_e2m1fn).astype(np.float32)
+    for c in range(16):
+        assert np.float32(O.e2m1_decode(c)).tobytes() == lib[c].tobytes()
+
+
+def test_e4m3_decode_all_codes_vs_library():
+    lib = np.arange(256, dtype=np.uint8).view(md.float8_e4m3fn).astype(np.float32)
+    for c in range(256):
+        v = np.float32(O.e4m3_decode(c))
+        if np.isnan(lib[c]):
+            assert np.isnan(v) and c & 0x7F == 0x7F
+        else:
+            assert v.tobytes() == lib[c].tobytes(), c
+    rows = dict((k, float(v)) for k, v in _read_golden("e4m3_extremes.txt"))
+    assert O.e4m3_decode(0x7E) == rows["max_finite"] == 448.0
+    assert O.e4m3_decode(0x01) == rows["min_subnormal"]
+    assert O.e4m3_decode(0x08) == rows["min_normal"]
+
+
+def test_e2m1_encode_exhaustive_binades_vs_library():
+    # every float32 in [2^-8, 2^5): all E2M1 decision points (0.25 .. 5, saturation at 6) fall inside
+    for y in _binade_sweep(119, 132):
+        ref = np.clip(y, -6, 6).astype(md.float4_e2m1fn).view(np.uint8) & 0xF
+        got = O.e2m1_encode(y)
+        assert np.array_equal(got, ref)
+        got_neg = O.e2m1_encode(-y)
+        assert np.array_equal(got_neg, ref | 8)
+
+
+def test_e2m1_encode_specials():
+    y = np.array([0.0, -0.0, 1e-45, -1e-45, 1e-30, 5.0, 5.000001, 6.0, 6.5, 7.0, 1e30, 3.4e38], np.float32)
+    got = O.e2m1_encode(y)
+    ref = np.clip(y, -6, 6).astype(md.float4_e2m1fn).view(np.uint8)
+    assert np.array_equal(got, ref)
+    assert got[1] == 0x8 and got[3] == 0x8  # negative values rounding to zero keep the sign
+    # random sample over the whole finite range
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 0xFF800000, size=2_000_000, dtype=np.uint64).astype(np.uint32)
+    v = bits.view(np.float32)
+    v = v[np.isfinite(v)]
+    assert np.array_equal(O.e2m1_encode(v), np.clip(v, -6, 6).astype(md.float4_e2m1fn).view(np.uint8))
+
+
+def test_e4m3_encode_exhaustive_binades_vs_library():
+    # every float32 in [2^-17, 2^9) (all E4M3 subnormal/normal decision points up to 448)
+    for v in _binade_sweep(110, 136):
+        ref = v.astype(md.float8_e4m3fn).view(np.uint8)
+        got = O.e4m3_encode(v)
+        lib_range = v <= 464.0
+        assert np.array_equal(got[lib_range], ref[lib_range])
+        assert np.all(got[~lib_range] == 0x7E)
+    # from 2^9 = 512 up, and 448 <= v < 512: the oracle saturates to 448 (0x7E); the library agrees
+    # up to the midpoint 464 and returns NaN beyond it.
+    v = np.linspace(448, 464, 100001, dtype=np.float32)
+    assert np.array_equal(O.e4m3_encode(v), v.astype(md.float8_e4m3fn).view(np.uint8))
+    big = np.array([464.0001, 465, 480, 1e6, 3.4e38, np.inf], np.float32)
+    assert np.all(O.e4m3_encode(big) == 0x7E)
+    assert O.e4m3_encode(np.array([np.nan], np.float32))[0] == 0x7F
+    assert O.e4m3_encode(np.array([-1.0], np.float32))[0] == 0xB8
+    tiny = np.array([0.0, 2.0**-10, 1.5 * 2.0**-10, 2.0**-30, 1e-45], np.float32)
+    assert np.array_equal(O.e4m3_encode(tiny), tiny.astype(md.float8_e4m3fn).view(np.uint8))
+
+
+def test_narrowing_conversions_vs_library():
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0, 1 << 32, size=4_000_000, dtype=np.uint64).astype(np.uint32)
+    v = bits.view(np.float32)
+    fin = v[~np.isnan(v)]
+    assert np.array_equal(O.f32_to_bf16(fin), fin.astype(md.bfloat16).view(np.uint16))
+    assert np.array_equal(O.f32_to_f16(fin), fin.astype(np.float16).view(np.uint16))
+    # midpoints and overflow edges
+    edge = np.array([65504, 65519.99, 65520, 65536, 2.0**-24, 2.0**-25, 1.5 * 2.0**-25, 3.4e38], np.float32)
+    assert np.array_equal(O.f32_to_f16(edge), edge.astype(np.float16).view(np.uint16))
+    assert np.all(np.isnan(O.f16_to_f32(np.array([0x7E00, 0xFC01], np.uint16))))
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ok = (h & 0x7C00) != 0x7C00
+    assert np.array_equal(O.f16_to_f32(h)[ok].view(np.uint32), h.view(np.float16)[ok].astype(np.float32).view(np.uint32))
