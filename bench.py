@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 ScaleSearch hot path on B200.
+
+One step = one pass of the whole path over one synthetic batch resident in HBM:
+  tensor amax -> [all-reduce(max) across ranks] -> tensor scale g -> ScaleSearch quantize (f in [-2,6])
+  -> dequantize to FP32.
+Default workload: the 4 GiB FP32 stream (2^30 elements, mixture 0.9 N(0,1) + 0.1 N(0,16), seed 3), the
+configuration the throughput target is stated on.  Every step's input (4 GiB) is larger than the
+126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Prints ONE JSON line on rank 0.  Times are CUDA events on the launching stream, max over ranks.
+`--impl reference` times the CPU oracle (the plain C definition) on a bounded sample of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 ScaleSearch quantize GB/s (input) and fraction of 8 TB/s HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+SOURCE_NOTE = "synthetic (seeded generators; stand-in for LLM activations / KV keys / BEV value maps)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="stream_f32")
+    ap.add_argument("--f-lo", type=int, default=-2)
+    ap.add_argument("--f-hi", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampler unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) < 4:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                    bits = int(parts[3], 16)
+                except ValueError:
+                    continue
+                for b, name in REASON_BITS.items():
+                    if bits & b and name != "gpu_idle":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle arm
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(name: str, elems: int):
+    """A bounded CPU sample of the workload's recipe (same generator recipe, CPU stream)."""
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    if name == "stream_f32":
+        x = W.stream_f32("cpu", elems / float(1 << 30))
+    else:
+        w = W.make(name, "cpu")
+        x = w.x.reshape(-1)[:elems].contiguous()
+    import numpy as np
+    import torch
+    if x.dtype == torch.float32:
+        return x.numpy().reshape(-1), 0, x.numel()
+    code = 1 if x.dtype == torch.bfloat16 else 2
+    return x.view(torch.int16).numpy().view(np.uint16).reshape(-1), code, x.numel()
+
+
+def oracle_step(xs, code, f_lo, f_hi):
+    from oracle import oracle as O
+    c, s, g, _, _ = O.quantize(xs, f_lo, f_hi, dtype=code)
+    O.dequantize(c, s, g, 0)
+
+
+def time_oracle(name, f_lo, f_hi, budget_s, max_elems=1 << 25):
+    """Pick a sample size whose oracle step takes about budget_s, then time one step."""
+    probe = 1 << 16
+    xs, code, n = oracle_sample(name, probe)
+    t = time.perf_counter()
+    oracle_step(xs, code, f_lo, f_hi)
+    dt = time.perf_counter() - t
+    elems = int(min(max_elems, max(probe, probe * budget_s / max(dt, 1e-6))))
+    elems -= elems % 16
+    xs, code, n = oracle_sample(name, elems)
+    return xs, code, n
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    xs, code, n = time_oracle(args.workload, args.f_lo, args.f_hi, budget)
+    for _ in range(args.warmup):
+        oracle_step(xs, code, args.f_lo, args.f_hi)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(xs, code, args.f_lo, args.f_hi)
+    el = time.perf_counter() - t
+    bytes_in = n * xs.dtype.itemsize
+    val = bytes_in * args.steps / el / 1e9
+    sample = f"first {n} elements of the {args.workload} recipe per step (CPU generator), oracle quantize + dequantize"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
+        "config": workload_config(args),
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args):
+    return {
+        "workload": f"{args.workload}" + (" (FP32 2^30 = 4 GiB, 0.9 N(0,1) + 0.1 N(0,16), seed 3)"
+                                            if args.workload == "stream_f32" else ""),
+        "window": [args.f_lo, args.f_hi],
+        "step": "amax + [allreduce max] + g + ScaleSearch quantize + dequantize FP32",
+        "l2": "inputs larger than L2 (4 GiB per step per GPU), no flush",
+        "block": 16,
+    }
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = W.make(args.workload, dev, 1.0, shard=rank)
+    if w.kind != "quantize":
+        raise SystemExit("bench.py times quantize workloads; kv_bf16 is covered by the parity tests")
+    x = w.x.reshape(-1).contiguous()
+    n = x.numel()
+    esz = x.element_size()
+    torch.cuda.synchronize()
+
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(n // 16, dtype=torch.uint8, device=dev)
+    deq = torch.empty(n, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        nv.tensor_amax(x, out=amax)
+        if world > 1:
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+        nv.global_scale(amax, out=g)
+        if evs:
+            evs[1].record(stream)
+        nv.quantize_ex(x, args.f_lo, args.f_hi, gscale_in=g, want_f=False, want_sse=False, codes=codes,
+                       scales=scales, gscale=None)
+        if evs:
+            evs[2].record(stream)
+        nv.dequantize(codes, scales, g, torch.float32, out=deq)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    amax_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    q_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    dq_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+
+    bytes_in = n * esz
+    value = world * bytes_in * args.steps / (elapsed_ms * 1e-3) / 1e9
+    peak, peak_src = peaks()
+    q_bytes = n * esz + n // 2 + n // 16          # search pass: read x, write codes + scales
+    two_pass_bytes = 2 * n * esz + n // 2 + n // 16
+    dq_bytes = n // 2 + n // 16 + 4 * n
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
+        "config": workload_config(args),
+        "roofline": {"bound": "hbm", "kernel": "quantize (ScaleSearch search + encode pass)",
+                     "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
+                     "traffic": None, "peak_source": peak_src,
+                     "bytes_per_launch": q_bytes},
+        "breakdown_ms": {"amax_and_g": amax_ms, "quantize": q_ms, "dequantize": dq_ms},
+        "quantize_two_pass": {"gbs_input": bytes_in / ((amax_ms + q_ms) * 1e-3) / 1e9,
+                              "gbs_moved": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 1e9,
+                              "frac_of_8TBs": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 8e12},
+        "dequantize": {"gbs_moved": dq_bytes / (dq_ms * 1e-3) / 1e9},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+
+    # end to end through the public API with host buffers: pinned H2D of the input, the step, and a
+    # D2H read of the quantized result (codes, scales, g) every step.
+    if not args.no_e2e and args.e2e_steps > 0:
+        hx = torch.empty(n, dtype=x.dtype, pin_memory=True)
+        hx.copy_(x)
+        hc = torch.empty(n // 2, dtype=torch.uint8, pin_memory=True)
+        hs = torch.empty(n // 16, dtype=torch.uint8, pin_memory=True)
+        hg = torch.empty(1, dtype=torch.float32, pin_memory=True)
+        xin = torch.empty_like(x)
+
+        def e2e_step():
+            xin.copy_(hx, non_blocking=True)
+            nv.tensor_amax(xin, out=amax)
+            if world > 1:
+                dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+            nv.global_scale(amax, out=g)
+            nv.quantize_ex(xin, args.f_lo, args.f_hi, gscale_in=g, want_f=False, want_sse=False, codes=codes,
+                           scales=scales, gscale=None)
+            nv.dequantize(codes, scales, g, torch.float32, out=deq)
+            hc.copy_(codes, non_blocking=True)
+            hs.copy_(scales, non_blocking=True)
+            hg.copy_(g, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * bytes_in * args.e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                       "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": n // 2 + n // 16 + 4}
+        del hx, hc, hs, hg, xin
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xs, code, ns = time_oracle(args.workload, args.f_lo, args.f_hi, args.cpu_seconds)
+        t = time.perf_counter()
+        oracle_step(xs, code, args.f_lo, args.f_hi)
+        el = time.perf_counter() - t
+        line["cpu_baseline"] = {
+            "value": ns * xs.dtype.itemsize / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{ns} elements of the {args.workload} recipe (CPU generator), one quantize + dequantize, "
+                      f"{el:.1f} s single-threaded C",
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

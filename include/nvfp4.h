@@ -1,0 +1,114 @@
+/*
+ * nvfp4.h -- libnvfp4: NVFP4 block quantization with ScaleSearch on NVIDIA B200 (sm_100a).
+ *
+ * NVFP4 ("NVIDIAのFP4推論が50倍の効率を実現", introl.com, section 超低精度推論を支えるアーキテクチャ):
+ * 4-bit E2M1 values (1 sign, 2 exponent, 1 mantissa bit; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6) in
+ * micro-blocks of 16 consecutive elements, one E4M3 (FP8) scale per micro-block and one FP32 scale per
+ * tensor.  ScaleSearch ("Search your block floating-point scales!", gist.science summary of arXiv
+ * 2605.12464, Method > ScaleSearch) replaces the max-scaling block scale s = round(amax_b / 6) by the
+ * best of its integer neighbours: the E4M3 bit pattern of s is read as an integer, an offset f in
+ * [f_lo, f_hi] is added, and the offset whose block squared error is smallest wins.
+ *
+ * Exact semantics (the library is bit-exact with this definition):
+ *   g      = fl(amax / 2688)            amax = max |x_i| over the tensor (NaN / Inf propagate)
+ *   c0     = E4M3_RNE_SAT(fl(fl(amax_b / 6) / g))          amax_b = max |x_i| over the block
+ *   for f in [f_lo, f_hi], visiting 0, -1, +1, -2, +2, ...:
+ *     c = c0 + f must be a positive finite E4M3 code (1..126); d = fl(E4M3(c) * g) != 0; r = fl(1/d) finite
+ *     sse(f) = sum over i = 0..15, in order, in FP32, of fl(e_i * e_i), where
+ *              y = fl(x_i * r), q = E2M1_RNE_SAT(y), e_i = fl(x_i - fl(E2M1(q) * d))
+ *   f* = argmin sse (ties: smaller |f|, then smaller f); scale byte = c0 + f*;
+ *   code_i = E2M1_RNE_SAT(fl(x_i * r*)), element 2k in the low nibble of byte k of its block.
+ * Special blocks: all-zero -> scale 0x00, sign-only codes, f* = -128; no usable candidate -> the same
+ * with sse = sum of x_i^2; a non-finite element, or g NaN / Inf / negative -> scale 0x7F (E4M3 NaN),
+ * codes 0, f* = -128, sse NaN.
+ *
+ * Memory: every pointer argument is device memory owned by the caller unless stated otherwise; the
+ * library allocates nothing and keeps no state between calls except cached device properties.
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls enqueue
+ * work and return without synchronising; outputs are valid once the stream reaches that point.
+ * Overlapping calls on different streams that write the same outputs race, as with any kernel.
+ * Errors: argument errors are reported synchronously as a negative status and nothing is enqueued.
+ * A CUDA launch error is returned as NVFP4_ERR_CUDA.  With the environment variable NVFP4_CHECKED=1
+ * the quantize / kv calls synchronise the stream and return NVFP4_ERR_NONFINITE when the tensor held a
+ * NaN or Inf (the outputs are then poisoned in-band as described above).
+ * Alignment: element buffers must be 16-byte aligned (32-byte aligned inputs use 256-bit loads);
+ * code buffers 8-byte aligned.  Sizes are element counts and must be multiples of 16 (one block).
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { NVFP4_F32 = 0, NVFP4_BF16 = 1, NVFP4_F16 = 2 } nvfp4_dtype;
+
+enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_ARG = -1,       /* null pointer, bad dtype, bad offset window, block != 16 */
+  NVFP4_ERR_SIZE = -2,      /* n < 0, n % 16 != 0, or a shape that does not split into blocks */
+  NVFP4_ERR_ALIGN = -3,     /* a buffer is not aligned as required */
+  NVFP4_ERR_CUDA = -4,      /* a CUDA call failed (launch error) */
+  NVFP4_ERR_NONFINITE = -5  /* checked mode only: the input held NaN / Inf */
+};
+
+/* Human-readable name of a status code (static string). */
+const char* nvfp4_status_str(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int nvfp4_version(void);
+
+/* Tensor amax (the FP32 per-tensor scale's input; NVFP4 page, second-level FP32 scale).
+ * x: n elements of `dtype`.  d_amax: one device float, overwritten with max |x_i| (NaN if any x_i is
+ * NaN, else Inf if any is infinite; 0 for n == 0).  n need not be a multiple of 16. */
+int nvfp4_tensor_amax(const void* x, int64_t n, int dtype, float* d_amax, void* stream);
+
+/* Per-tensor scale from an amax: *d_gscale = fl(*d_amax / 2688).  Both are one device float (they may
+ * alias).  Used by sharded callers after reducing their shard amaxes with a max. */
+int nvfp4_global_scale(const float* d_amax, float* d_gscale, void* stream);
+
+/* ScaleSearch quantize ("Search your block floating-point scales!", Method > ScaleSearch).
+ * x: n elements of `dtype` (n % 16 == 0), blocks of 16 along the contiguous order.
+ * block: must be 16.  f_lo <= f_hi, both in [-126, 126]; {0, 0} is plain max-scaling.
+ * codes: n/2 bytes; scales: n/16 bytes; gscale: one device float receiving g.
+ * Work: one read pass for amax, one read pass for the search and encode. */
+int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi,
+                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
+
+/* Extended quantize.  gscale_in: NULL -> as nvfp4_quantize; else a device float holding g, and the
+ * amax pass is skipped (sharded tensors, calibrated scales); gscale may then be NULL.
+ * block_f: NULL or n/16 int8 receiving f* (-128 for blocks without a scale);
+ * block_sse: NULL or n/16 floats receiving the winning block SSE (the block MSE times 16). */
+int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi,
+                      const float* gscale_in, uint8_t* codes, uint8_t* scales, float* gscale,
+                      int8_t* block_f, float* block_sse, void* stream);
+
+/* Dequantize: out_i = fl(E2M1(code_i) * fl(E4M3(scale_b) * g)), rounded to out_dtype (RNE).
+ * The block scale is applied back by one multiply (BEVFormer-on-B200 page, section 7).
+ * codes: n/2 bytes, scales: n/16 bytes, gscale: one device float, out: n elements. */
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n,
+                     int out_dtype, void* out, void* stream);
+
+/* Hadamard-16 rotation ("Search your block floating-point scales!", ScaleSearchAttention >
+ * incoherence processing): each contiguous group of 16 elements is multiplied by the Sylvester
+ * Hadamard matrix H16 / 4, computed as butterflies with strides 1, 2, 4, 8 in FP32.
+ * x and out: n elements (n % 16 == 0); out may alias x only when dtype == out_dtype. */
+int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype, void* stream);
+
+/* Attention-sink mixed-precision KV layout ("Search your block floating-point scales!",
+ * ScaleSearchAttention > attention-sink-aware mixed-precision caching).
+ * k_bf16: K[B,H,T,D] BF16, contiguous.  D % 16 == 0, T >= sink_tokens + recent_tokens.
+ * sink_bf16: [B,H,sink_tokens,D] and recent_bf16: [B,H,recent_tokens,D] receive the first and last
+ * tokens verbatim.  The T_mid = T - sink - recent middle tokens are rotated along D by FWHT-16 when
+ * rotate != 0 (kept in FP32) and quantized along D with one tensor scale over the rotated middle:
+ * codes [B,H,T_mid,D/2], scales [B,H,T_mid,D/16], gscale one device float. */
+int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                   int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

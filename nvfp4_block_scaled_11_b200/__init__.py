@@ -1,0 +1,195 @@
+"""nvfp4_block_scaled_11_b200 -- Python binding of libnvfp4 (NVFP4 ScaleSearch quantization, sm_100a).
+
+Argument marshalling only: every function checks that its tensors are contiguous CUDA tensors,
+allocates outputs with torch when the caller did not pass them, and calls the C ABI declared in
+``include/nvfp4.h`` with raw device pointers and the current CUDA stream.  All computation happens
+in the library's CUDA kernels; there is no CPU path.  A missing ``libnvfp4.so`` raises.
+
+Element types: torch.float32, torch.bfloat16, torch.float16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
+    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE",
+]
+
+_SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
+_lib = None
+
+DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+DTYPE_OF = {v: k for k, v in DTYPE_CODE.items()}
+
+# C-ABI entry points and their argument types (include/nvfp4.h)
+_P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+_SIGS = {
+    "nvfp4_status_str": (ctypes.c_char_p, [_I]),
+    "nvfp4_version": (_I, []),
+    "nvfp4_tensor_amax": (_I, [_P, _I64, _I, _P, _P]),
+    "nvfp4_global_scale": (_I, [_P, _P, _P]),
+    "nvfp4_quantize": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "nvfp4_quantize_ex": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
+    "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
+    "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int):
+        super().__init__(status_str(status))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libnvfp4 (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_SO):
+            raise RuntimeError(
+                f"libnvfp4.so is not built ({_SO}); run `python -m nvfp4_block_scaled_11_b200.build`"
+            )
+        L = ctypes.CDLL(_SO)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().nvfp4_status_str(status).decode()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise NVFP4Error(rc)
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    try:
+        return DTYPE_CODE[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def tensor_amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """max |x| as a 1-element float32 device tensor (NaN / Inf propagate)."""
+    _cuda(x, "x")
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().nvfp4_tensor_amax(_ptr(x), x.numel(), _dt(x), _ptr(out), _stream(x)))
+    return out
+
+
+def global_scale(amax: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """g = amax / 2688 on the device."""
+    _cuda(amax, "amax")
+    out = torch.empty(1, dtype=torch.float32, device=amax.device) if out is None else out
+    _check(lib().nvfp4_global_scale(_ptr(amax), _ptr(out), _stream(amax)))
+    return out
+
+
+def _alloc_q(x, codes, scales, gscale):
+    n = x.numel()
+    dev = x.device
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev) if codes is None else codes
+    scales = torch.empty(n // 16, dtype=torch.uint8, device=dev) if scales is None else scales
+    gscale = torch.empty(1, dtype=torch.float32, device=dev) if gscale is None else gscale
+    return codes, scales, gscale
+
+
+def quantize(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, block: int = 16, codes=None, scales=None, gscale=None):
+    """ScaleSearch quantize of x (blocks of 16 along the contiguous order).
+
+    Returns (codes uint8[n/2], scales uint8[n/16], gscale float32[1])."""
+    _cuda(x, "x")
+    codes, scales, gscale = _alloc_q(x, codes, scales, gscale)
+    _check(lib().nvfp4_quantize(_ptr(x), x.numel(), _dt(x), block, f_lo, f_hi, _ptr(codes), _ptr(scales),
+                                _ptr(gscale), _stream(x)))
+    return codes, scales, gscale
+
+
+def quantize_ex(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None,
+                want_f: bool = True, want_sse: bool = True, block: int = 16, codes=None, scales=None, gscale=None,
+                block_f=None, block_sse=None):
+    """Quantize with optional external tensor scale and per-block outputs.
+
+    Returns (codes, scales, gscale, block_f int8[n/16] or None, block_sse float32[n/16] or None)."""
+    _cuda(x, "x")
+    n = x.numel()
+    if gscale_in is not None:
+        _cuda(gscale_in, "gscale_in")
+        keep = gscale
+    codes, scales, gscale = _alloc_q(x, codes, scales, gscale)
+    if gscale_in is not None and keep is None:
+        gscale = None  # g comes from gscale_in; no copy requested
+    if want_f and block_f is None:
+        block_f = torch.empty(n // 16, dtype=torch.int8, device=x.device)
+    if want_sse and block_sse is None:
+        block_sse = torch.empty(n // 16, dtype=torch.float32, device=x.device)
+    _check(lib().nvfp4_quantize_ex(_ptr(x), n, _dt(x), block, f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
+                                   _ptr(scales), _ptr(gscale), _ptr(block_f), _ptr(block_sse), _stream(x)))
+    return codes, scales, gscale, block_f, block_sse
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    """Dequantize n = 16 * scales.numel() elements to out_dtype."""
+    _cuda(codes, "codes"), _cuda(scales, "scales"), _cuda(gscale, "gscale")
+    n = scales.numel() * 16
+    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
+    _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), _ptr(gscale), n, DTYPE_CODE[out.dtype], _ptr(out),
+                                  _stream(codes)))
+    return out
+
+
+def hadamard16(x: torch.Tensor, out_dtype=None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """FWHT-16 / 4 on every contiguous group of 16 elements."""
+    _cuda(x, "x")
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    out = torch.empty(x.shape, dtype=out_dtype, device=x.device) if out is None else out
+    _check(lib().nvfp4_hadamard16(_ptr(x), x.numel(), _dt(x), _ptr(out), DTYPE_CODE[out.dtype], _stream(x)))
+    return out
+
+
+def kv_mixed(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = True, f_lo: int = -2, f_hi: int = 6):
+    """Mixed-precision KV layout of K[B,H,T,D] (BF16).
+
+    Returns (sink bf16[B,H,sink,D], recent bf16[B,H,recent,D], codes uint8[B,H,Tm,D/2],
+    scales uint8[B,H,Tm,D/16], gscale float32[1])."""
+    _cuda(k, "k")
+    if k.dtype != torch.bfloat16 or k.dim() != 4:
+        raise TypeError("k must be a 4-D bfloat16 tensor [B,H,T,D]")
+    B, H, T, D = k.shape
+    Tm = T - sink - recent
+    dev = k.device
+    so = torch.empty((B, H, sink, D), dtype=torch.bfloat16, device=dev)
+    ro = torch.empty((B, H, recent, D), dtype=torch.bfloat16, device=dev)
+    codes = torch.empty((B, H, max(Tm, 0), D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((B, H, max(Tm, 0), D // 16), dtype=torch.uint8, device=dev)
+    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(lib().nvfp4_kv_mixed(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), f_lo, f_hi, _ptr(so),
+                                _ptr(ro), _ptr(codes), _ptr(scales), _ptr(gscale), _stream(k)))
+    return so, ro, codes, scales, gscale

@@ -1,0 +1,408 @@
+// kernels.cuh -- libnvfp4 kernels for sm_100a: tensor amax, ScaleSearch quantize, dequantize,
+// Hadamard-16 and the pieces of the mixed-precision KV layout.
+//
+// Sources (web pages, by title and section):
+//   "NVIDIAのFP4推論が50倍の効率を実現" (introl.com), 超低精度推論を支えるアーキテクチャ: the NVFP4 format.
+//   "Search your block floating-point scales!" (gist.science summary of arXiv 2605.12464),
+//     Method > ScaleSearch: the scale search; ScaleSearchAttention: Hadamard rotation, sink/recent KV.
+//   "BEVFormer on B200: FP8/FP4 CUDA kernel tuning" (qiita.com), section 7: scale applied back by one
+//     multiply; two FP4 codes per byte.
+#pragma once
+
+#include <float.h>
+
+#include "device.cuh"
+
+namespace nvfp4 {
+
+constexpr float kTensorDiv = 2688.0f;  // 6 (largest E2M1) * 448 (largest E4M3)
+
+// =================================================================================================
+// Tensor amax: unsigned max of the magnitude bits (NaN > Inf > finite, so both propagate), reduced
+// per CTA and merged with one atomicMax into a caller word that was zeroed beforehand.
+// =================================================================================================
+template <int DT>
+__device__ __forceinline__ uint32_t mag_max_words(const uint32_t* w, int nw, uint32_t m) {
+#pragma unroll
+  for (int k = 0; k < nw; ++k) {
+    if (DT == DT_F32) m = max(m, w[k] & 0x7FFFFFFFu);
+    else m = __vmaxu2(m, w[k] & 0x7FFF7FFFu);  // two 16-bit magnitudes per word
+  }
+  return m;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t mag_to_f32bits(uint32_t m) {
+  if (DT == DT_F32) return m;
+  uint32_t h = max(m & 0xFFFFu, m >> 16);
+  if (DT == DT_BF16) return h << 16;
+  return __float_as_uint(__half2float(__ushort_as_half((unsigned short)h)));
+}
+
+template <int DT>
+__global__ void __launch_bounds__(512) amax_kernel(const char* __restrict__ x, int64_t n, int v8,
+                                                   uint32_t* __restrict__ out) {
+  constexpr int ES = DT == DT_F32 ? 4 : 2;
+  constexpr int EPV = 32 / ES;  // elements per 32-byte vector
+  const int64_t nvec = n / EPV;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m = 0;
+  if (v8) {
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+      uint32_t a[8], b[8], c[8], d[8];
+      ld_v8(x + 32 * i, a);
+      ld_v8(x + 32 * (i + stride), b);
+      ld_v8(x + 32 * (i + 2 * stride), c);
+      ld_v8(x + 32 * (i + 3 * stride), d);
+      m = mag_max_words<DT>(a, 8, m);
+      m = mag_max_words<DT>(b, 8, m);
+      m = mag_max_words<DT>(c, 8, m);
+      m = mag_max_words<DT>(d, 8, m);
+    }
+    for (; i < nvec; i += stride) {
+      uint32_t a[8];
+      ld_v8(x + 32 * i, a);
+      m = mag_max_words<DT>(a, 8, m);
+    }
+  } else {
+    for (; i < nvec; i += stride) {
+      uint32_t a[4], b[4];
+      ld_v4(x + 32 * i, a);
+      ld_v4(x + 32 * i + 16, b);
+      m = mag_max_words<DT>(a, 4, m);
+      m = mag_max_words<DT>(b, 4, m);
+    }
+  }
+  m = mag_to_f32bits<DT>(m);
+  // ragged tail (n % EPV elements), one element per thread of the first CTA
+  if (blockIdx.x == 0) {
+    const int64_t t = nvec * EPV + threadIdx.x;
+    if (t < n) {
+      uint32_t b;
+      if (DT == DT_F32) b = reinterpret_cast<const uint32_t*>(x)[t] & 0x7FFFFFFFu;
+      else {
+        uint32_t h = reinterpret_cast<const uint16_t*>(x)[t] & 0x7FFFu;
+        b = mag_to_f32bits<DT>(h);
+      }
+      m = max(m, b);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ uint32_t s[32];
+  if ((threadIdx.x & 31) == 0) s[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? s[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (threadIdx.x == 0 && m) atomicMax(out, m);
+  }
+}
+
+// g = fl(amax / 2688), in place or into another word.
+__global__ void global_scale_kernel(const float* amax, float* g) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *g = __fdiv_rn(*amax, kTensorDiv);
+}
+
+// =================================================================================================
+// ScaleSearch quantize.
+// =================================================================================================
+struct QuantParams {
+  const char* x;       // input base (bytes)
+  int64_t nblocks;
+  int f_lo, f_hi;
+  const float* g_src;  // device word: g itself, or the tensor amax when g_is_amax
+  int g_is_amax;
+  uint8_t* codes;
+  uint8_t* scales;
+  int8_t* block_f;     // optional
+  float* block_sse;    // optional
+  int v8;              // input base is 32-byte aligned
+  // mixed KV layout: blocks run over the middle tokens of K[BH, T, D]
+  int64_t T, Tm, sink, D, bpr;  // bpr = D / 16
+};
+
+// Candidate table for one launch: d[c] = fl(E4M3(c) * g), r[c] = fl(1 / d[c]); r = 0 marks a code that
+// cannot be a scale (c outside 1..126, d == 0 or 1/d not finite).
+struct CandTable {
+  float d[128];
+  float r[128];
+};
+
+__device__ __forceinline__ void build_cand_table(CandTable& t, float g) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    float d = __fmul_rn(e4m3_value((uint32_t)c), g);
+    float r = __frcp_rn(d);
+    bool ok = c >= 1 && c <= 126 && d != 0.0f && fabsf(r) <= FLT_MAX;
+    t.d[c] = d;
+    t.r[c] = ok ? r : 0.0f;
+  }
+}
+
+// Block squared error of candidate (d, r), summed in FP32 in element order (the definition).
+__device__ __forceinline__ float block_sse_exact(const float (&a)[16], float d, float r) {
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    float y0 = __fmul_rn(a[i], r), y1 = __fmul_rn(a[i + 1], r);
+    uint32_t h2 = e2m1x2_to_f16x2(e2m1x2(y1, y0));
+    float e0 = __fsub_rn(a[i], __fmul_rn(f16lo(h2), d));
+    float e1 = __fsub_rn(a[i + 1], __fmul_rn(f16hi(h2), d));
+    s = __fadd_rn(s, __fmul_rn(e0, e0));
+    s = __fadd_rn(s, __fmul_rn(e1, e1));
+  }
+  return s;
+}
+
+template <int DT, bool KV, bool ROT>
+__global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
+  __shared__ CandTable tab;
+  float g = *p.g_src;
+  if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
+  const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);  // NaN, Inf or negative
+  build_cand_table(tab, g);
+  __syncthreads();
+
+  constexpr int ES = DT == DT_F32 ? 4 : 2;
+  const int span = max(abs(p.f_lo), abs(p.f_hi));
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < p.nblocks; b += stride) {
+    int64_t elem;
+    if (KV) {
+      const int64_t per_bh = p.Tm * p.bpr;
+      const int64_t bh = b / per_bh;
+      const int64_t rem = b - bh * per_bh;
+      const int64_t t = rem / p.bpr;
+      const int64_t j = rem - t * p.bpr;
+      elem = (bh * p.T + p.sink + t) * p.D + 16 * j;
+    } else {
+      elem = 16 * b;
+    }
+    float x[16];
+    load_block<DT>(p.x + elem * ES, p.v8 != 0, x);
+    if (ROT) fwht16(x);
+
+    float a[16];
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      a[i] = fabsf(x[i]);
+      m = max(m, __float_as_uint(x[i]) & 0x7FFFFFFFu);
+    }
+
+    uint32_t lo = 0, hi = 0;  // packed codes
+    int scale, fstar = -128;
+    float sse;
+    if (g_bad || m >= 0x7F800000u) {  // poisoned block
+      scale = 0x7F;
+      sse = __uint_as_float(0x7FFFFFFFu);
+    } else {
+      float best = 0.0f;
+      int c0 = 0;
+      if (m != 0) {
+        const float t = __fdiv_rn(__uint_as_float(m), 6.0f);
+        c0 = e4m3_code(__fdiv_rn(t, g));
+        for (int jv = 0; jv <= 2 * span; ++jv) {
+          const int f = (jv == 0) ? 0 : ((jv & 1) ? -((jv + 1) >> 1) : (jv >> 1));
+          if (f < p.f_lo || f > p.f_hi) continue;
+          const int c = c0 + f;
+          if (c < 1 || c > 126) continue;
+          const float r = tab.r[c];
+          if (r == 0.0f) continue;
+          const float s = block_sse_exact(a, tab.d[c], r);
+          if (fstar == -128 || s < best) {
+            best = s;
+            fstar = f;
+          }
+        }
+      }
+      if (fstar != -128) {
+        const int cs = c0 + fstar;
+        const float r = tab.r[cs];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          lo |= (e2m1x2(__fmul_rn(x[2 * k + 1], r), __fmul_rn(x[2 * k], r)) & 0xFFu) << (8 * k);
+          hi |= (e2m1x2(__fmul_rn(x[2 * k + 9], r), __fmul_rn(x[2 * k + 8], r)) & 0xFFu) << (8 * k);
+        }
+        scale = cs;
+        sse = best;
+      } else {
+        // zero block, or no usable candidate: sign-only zero codes, scale 0
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint32_t nib = ((__float_as_uint(x[2 * k]) >> 31) << 3) | ((__float_as_uint(x[2 * k + 1]) >> 31) << 7);
+          if (k < 4) lo |= nib << (8 * k);
+          else hi |= nib << (8 * (k - 4));
+        }
+        scale = 0;
+        float s = 0.0f;
+        if (m != 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s = __fadd_rn(s, __fmul_rn(x[i], x[i]));
+        }
+        sse = s;
+      }
+    }
+    reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(lo, hi);
+    p.scales[b] = (uint8_t)scale;
+    if (p.block_f) p.block_f[b] = (int8_t)fstar;
+    if (p.block_sse) p.block_sse[b] = sse;
+  }
+}
+
+// =================================================================================================
+// Dequantize: one thread per block; the block step d = fl(E4M3(scale) * g) is applied by one multiply.
+// =================================================================================================
+template <int OT>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                         const uint8_t* __restrict__ scales,
+                                                         const float* __restrict__ gsrc, int64_t nblocks,
+                                                         char* __restrict__ out, int v8) {
+  const float g = *gsrc;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    const uint2 cw = reinterpret_cast<const uint2*>(codes)[b];
+    const float d = __fmul_rn(e4m3_value(scales[b]), g);
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xFFu;
+      const uint32_t h2 = e2m1x2_to_f16x2(byte);
+      v[2 * k] = __fmul_rn(f16lo(h2), d);
+      v[2 * k + 1] = __fmul_rn(f16hi(h2), d);
+    }
+    if (OT == DT_F32) {
+      char* o = out + 64 * b;
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(v[i]);
+      if (v8) {
+        uint32_t a[8], c[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { a[i] = w[i]; c[i] = w[8 + i]; }
+        st_v8(o, a);
+        st_v8(o + 32, c);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
+      }
+    } else {
+      char* o = out + 32 * b;
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (OT == DT_BF16) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&h);
+        } else {
+          __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+      }
+      if (v8) st_v8(o, w);
+      else {
+        st_v4(o, w);
+        st_v4(o + 16, w + 4);
+      }
+    }
+  }
+}
+
+// =================================================================================================
+// Hadamard-16: one thread per group of 16.
+// =================================================================================================
+template <int DT, int OT>
+__global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict__ x, int64_t ngroups,
+                                                         char* __restrict__ out, int v8_in, int v8_out) {
+  constexpr int ES = DT == DT_F32 ? 4 : 2;
+  constexpr int OS = OT == DT_F32 ? 4 : 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < ngroups; b += stride) {
+    float a[16];
+    load_block<DT>(x + 16 * ES * b, v8_in != 0, a);
+    fwht16(a);
+    char* o = out + 16 * OS * b;
+    if (OT == DT_F32) {
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(a[i]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
+    } else {
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (OT == DT_BF16) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * k], a[2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&h);
+        } else {
+          __half2 h = __floats2half2_rn(a[2 * k], a[2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+      }
+      st_v4(o, w);
+      st_v4(o + 16, w + 4);
+    }
+  }
+}
+
+// =================================================================================================
+// Mixed-precision KV layout helpers.
+// =================================================================================================
+// Copy the first `sink` and last `recent` token rows of every (batch, head) verbatim (16-byte units).
+__global__ void __launch_bounds__(256) kv_copy_kernel(const char* __restrict__ k, int64_t BH, int64_t T,
+                                                      int64_t row_bytes, int64_t sink, int64_t recent,
+                                                      char* __restrict__ sink_out, char* __restrict__ recent_out) {
+  const int64_t units_per_row = row_bytes / 16;
+  const int64_t per_bh = (sink + recent) * units_per_row;
+  const int64_t total = BH * per_bh;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += stride) {
+    const int64_t bh = u / per_bh;
+    const int64_t r = u - bh * per_bh;
+    const int64_t tok = r / units_per_row;
+    const int64_t w = r - tok * units_per_row;
+    const char* src;
+    char* dst;
+    if (tok < sink) {
+      src = k + ((bh * T + tok) * row_bytes) + 16 * w;
+      dst = sink_out + ((bh * sink + tok) * row_bytes) + 16 * w;
+    } else {
+      const int64_t tr = tok - sink;
+      src = k + ((bh * T + (T - recent) + tr) * row_bytes) + 16 * w;
+      dst = recent_out + ((bh * recent + tr) * row_bytes) + 16 * w;
+    }
+    uint32_t v[4];
+    ld_v4(src, v);
+    st_v4(dst, v);
+  }
+}
+
+// amax over the (optionally rotated) middle tokens; one thread per 16-group.
+template <bool ROT>
+__global__ void __launch_bounds__(256) kv_amax_kernel(const char* __restrict__ k, int64_t ngroups, int64_t T,
+                                                      int64_t Tm, int64_t sink, int64_t D, int64_t bpr, int v8,
+                                                      uint32_t* __restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  uint32_t m = 0;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < ngroups; b += stride) {
+    const int64_t per_bh = Tm * bpr;
+    const int64_t bh = b / per_bh;
+    const int64_t rem = b - bh * per_bh;
+    const int64_t t = rem / bpr;
+    const int64_t j = rem - t * bpr;
+    const int64_t elem = (bh * T + sink + t) * D + 16 * j;
+    float x[16];
+    load_block<DT_BF16>(k + 2 * elem, v8 != 0, x);
+    if (ROT) fwht16(x);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(x[i]) & 0x7FFFFFFFu);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(out, m);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,292 @@
+// nvfp4_api.cu -- the libnvfp4 C ABI (include/nvfp4.h): argument validation and kernel launches.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "kernels.cuh"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    int s = 0;
+    cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev);
+    g_dev[dev].sms = s > 0 ? s : 148;
+  }
+  return g_dev[dev].sms;
+}
+
+// Persistent-style grid: enough CTAs for `items` at `per_cta` items each, capped at `ctas_per_sm` per SM.
+int grid_for(int64_t items, int per_cta, int ctas_per_sm) {
+  int64_t need = (items + per_cta - 1) / per_cta;
+  int64_t cap = (int64_t)sm_count() * ctas_per_sm;
+  if (need < 1) need = 1;
+  return (int)(need < cap ? need : cap);
+}
+
+bool checked_mode() {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* e = getenv("NVFP4_CHECKED");
+    mode = (e && e[0] == '1') ? 1 : 0;
+  }
+  return mode == 1;
+}
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline bool dtype_ok(int dt) { return dt == DT_F32 || dt == DT_BF16 || dt == DT_F16; }
+inline int esize(int dt) { return dt == DT_F32 ? 4 : 2; }
+
+int last_error() { return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+int check_finite_sync(const float* g_dev, cudaStream_t s) {
+  if (!checked_mode() || g_dev == nullptr) return NVFP4_OK;
+  float g = 0.0f;
+  if (cudaMemcpyAsync(&g, g_dev, sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  return (g == g && g <= 3.402823466e38f) ? NVFP4_OK : NVFP4_ERR_NONFINITE;
+}
+
+int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_t s) {
+  const int64_t vecs = n * esize(dtype) / 32;
+  const int grid = grid_for(vecs > 0 ? vecs : 1, 512 * 4, 2);
+  const int v8 = aligned(x, 32) ? 1 : 0;
+  const char* xp = static_cast<const char*>(x);
+  switch (dtype) {
+    case DT_F32: amax_kernel<DT_F32><<<grid, 512, 0, s>>>(xp, n, v8, word); break;
+    case DT_BF16: amax_kernel<DT_BF16><<<grid, 512, 0, s>>>(xp, n, v8, word); break;
+    default: amax_kernel<DT_F16><<<grid, 512, 0, s>>>(xp, n, v8, word); break;
+  }
+  return last_error();
+}
+
+template <bool KV, bool ROT>
+int launch_quantize_t(int dtype, const QuantParams& p, cudaStream_t s) {
+  const int grid = grid_for(p.nblocks, 256, 4);
+  switch (dtype) {
+    case DT_F32: quantize_kernel<DT_F32, KV, ROT><<<grid, 256, 0, s>>>(p); break;
+    case DT_BF16: quantize_kernel<DT_BF16, KV, ROT><<<grid, 256, 0, s>>>(p); break;
+    default: quantize_kernel<DT_F16, KV, ROT><<<grid, 256, 0, s>>>(p); break;
+  }
+  return last_error();
+}
+
+int window_ok(int f_lo, int f_hi) { return f_lo <= f_hi && f_lo >= -126 && f_hi <= 126; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_str(int status) {
+  switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_ARG: return "NVFP4_ERR_ARG: invalid argument";
+    case NVFP4_ERR_SIZE: return "NVFP4_ERR_SIZE: size is not a whole number of 16-element blocks";
+    case NVFP4_ERR_ALIGN: return "NVFP4_ERR_ALIGN: buffer misaligned";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA: CUDA error";
+    case NVFP4_ERR_NONFINITE: return "NVFP4_ERR_NONFINITE: input held NaN or Inf";
+    default: return "NVFP4: unknown status";
+  }
+}
+
+int nvfp4_version(void) { return 100; }
+
+int nvfp4_tensor_amax(const void* x, int64_t n, int dtype, float* d_amax, void* stream) {
+  if (!dtype_ok(dtype) || d_amax == nullptr || (n > 0 && x == nullptr)) return NVFP4_ERR_ARG;
+  if (n < 0) return NVFP4_ERR_SIZE;
+  if ((n > 0 && !aligned(x, 16)) || !aligned(d_amax, 4)) return NVFP4_ERR_ALIGN;
+  cudaStream_t s = S(stream);
+  if (cudaMemsetAsync(d_amax, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (n == 0) return NVFP4_OK;
+  return launch_amax(x, n, dtype, reinterpret_cast<uint32_t*>(d_amax), s);
+}
+
+int nvfp4_global_scale(const float* d_amax, float* d_gscale, void* stream) {
+  if (d_amax == nullptr || d_gscale == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(d_amax, 4) || !aligned(d_gscale, 4)) return NVFP4_ERR_ALIGN;
+  global_scale_kernel<<<1, 32, 0, S(stream)>>>(d_amax, d_gscale);
+  return last_error();
+}
+
+int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi, const float* gscale_in,
+                      uint8_t* codes, uint8_t* scales, float* gscale, int8_t* block_f, float* block_sse,
+                      void* stream) {
+  if (!dtype_ok(dtype) || block != 16 || !window_ok(f_lo, f_hi)) return NVFP4_ERR_ARG;
+  if (gscale_in == nullptr && gscale == nullptr) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
+  if ((n > 0 && !aligned(x, 16)) || (n > 0 && !aligned(codes, 8)) || (gscale && !aligned(gscale, 4)) ||
+      (gscale_in && !aligned(gscale_in, 4)) || (block_sse && !aligned(block_sse, 4)))
+    return NVFP4_ERR_ALIGN;
+  cudaStream_t s = S(stream);
+  QuantParams p{};
+  p.x = static_cast<const char*>(x);
+  p.nblocks = n / 16;
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.codes = codes;
+  p.scales = scales;
+  p.block_f = block_f;
+  p.block_sse = block_sse;
+  p.v8 = aligned(x, 32) ? 1 : 0;
+  if (gscale_in == nullptr) {
+    // gscale doubles as the amax accumulator: zero, reduce, quantize (reads it as amax), then g.
+    if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (n > 0) {
+      int rc = launch_amax(x, n, dtype, reinterpret_cast<uint32_t*>(gscale), s);
+      if (rc) return rc;
+      p.g_src = gscale;
+      p.g_is_amax = 1;
+      rc = launch_quantize_t<false, false>(dtype, p, s);
+      if (rc) return rc;
+    }
+    global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
+    if (int rc = last_error()) return rc;
+    return check_finite_sync(gscale, s);
+  }
+  p.g_src = gscale_in;
+  p.g_is_amax = 0;
+  if (n > 0) {
+    if (int rc = launch_quantize_t<false, false>(dtype, p, s)) return rc;
+  }
+  if (gscale && gscale != gscale_in) {
+    if (cudaMemcpyAsync(gscale, gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+  }
+  return check_finite_sync(gscale_in, s);
+}
+
+int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi, uint8_t* codes,
+                   uint8_t* scales, float* gscale, void* stream) {
+  if (gscale == nullptr) return NVFP4_ERR_ARG;
+  return nvfp4_quantize_ex(x, n, dtype, block, f_lo, f_hi, nullptr, codes, scales, gscale, nullptr, nullptr,
+                           stream);
+}
+
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,
+                     void* out, void* stream) {
+  if (!dtype_ok(out_dtype) || gscale == nullptr) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n == 0) return NVFP4_OK;
+  if (codes == nullptr || scales == nullptr || out == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
+  const int64_t nb = n / 16;
+  const int grid = grid_for(nb, 256, 8);
+  const int v8 = aligned(out, 32) ? 1 : 0;
+  char* o = static_cast<char*>(out);
+  cudaStream_t s = S(stream);
+  switch (out_dtype) {
+    case DT_F32: dequantize_kernel<DT_F32><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+    case DT_BF16: dequantize_kernel<DT_BF16><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+    default: dequantize_kernel<DT_F16><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+  }
+  return last_error();
+}
+
+int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype, void* stream) {
+  if (!dtype_ok(dtype) || !dtype_ok(out_dtype)) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n == 0) return NVFP4_OK;
+  if (x == nullptr || out == nullptr) return NVFP4_ERR_ARG;
+  if (x == out && dtype != out_dtype) return NVFP4_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16)) return NVFP4_ERR_ALIGN;
+  const int64_t ng = n / 16;
+  const int grid = grid_for(ng, 256, 8);
+  const int v8i = aligned(x, 32) ? 1 : 0, v8o = aligned(out, 32) ? 1 : 0;
+  const char* xp = static_cast<const char*>(x);
+  char* o = static_cast<char*>(out);
+  cudaStream_t s = S(stream);
+#define NVFP4_H16(DI, DO) hadamard16_kernel<DI, DO><<<grid, 256, 0, s>>>(xp, ng, o, v8i, v8o)
+  if (dtype == DT_F32) {
+    if (out_dtype == DT_F32) NVFP4_H16(DT_F32, DT_F32);
+    else if (out_dtype == DT_BF16) NVFP4_H16(DT_F32, DT_BF16);
+    else NVFP4_H16(DT_F32, DT_F16);
+  } else if (dtype == DT_BF16) {
+    if (out_dtype == DT_F32) NVFP4_H16(DT_BF16, DT_F32);
+    else if (out_dtype == DT_BF16) NVFP4_H16(DT_BF16, DT_BF16);
+    else NVFP4_H16(DT_BF16, DT_F16);
+  } else {
+    if (out_dtype == DT_F32) NVFP4_H16(DT_F16, DT_F32);
+    else if (out_dtype == DT_BF16) NVFP4_H16(DT_F16, DT_BF16);
+    else NVFP4_H16(DT_F16, DT_F16);
+  }
+#undef NVFP4_H16
+  return last_error();
+}
+
+int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                   int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
+  if (!window_ok(f_lo, f_hi) || gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
+    return NVFP4_ERR_SIZE;
+  const int64_t BH = B * H;
+  const int64_t Tm = T - sink_tokens - recent_tokens;
+  const int64_t ngroups = BH * Tm * (D / 16);
+  if (BH > 0 && k_bf16 == nullptr) return NVFP4_ERR_ARG;
+  if (BH > 0 && sink_tokens > 0 && sink_bf16 == nullptr) return NVFP4_ERR_ARG;
+  if (BH > 0 && recent_tokens > 0 && recent_bf16 == nullptr) return NVFP4_ERR_ARG;
+  if (ngroups > 0 && (codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
+  if ((BH > 0 && !aligned(k_bf16, 16)) || (sink_bf16 && !aligned(sink_bf16, 16)) ||
+      (recent_bf16 && !aligned(recent_bf16, 16)) || (codes && !aligned(codes, 8)) || !aligned(gscale, 4))
+    return NVFP4_ERR_ALIGN;
+  cudaStream_t s = S(stream);
+  const char* k = static_cast<const char*>(k_bf16);
+  if (BH > 0 && sink_tokens + recent_tokens > 0) {
+    const int64_t units = BH * (sink_tokens + recent_tokens) * (D * 2 / 16);
+    kv_copy_kernel<<<grid_for(units, 256, 8), 256, 0, s>>>(k, BH, T, D * 2, sink_tokens, recent_tokens,
+                                                           static_cast<char*>(sink_bf16),
+                                                           static_cast<char*>(recent_bf16));
+    if (int rc = last_error()) return rc;
+  }
+  if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (ngroups > 0) {
+    const int v8 = aligned(k_bf16, 32) ? 1 : 0;
+    const int grid = grid_for(ngroups, 256, 8);
+    uint32_t* word = reinterpret_cast<uint32_t*>(gscale);
+    if (rotate) kv_amax_kernel<true><<<grid, 256, 0, s>>>(k, ngroups, T, Tm, sink_tokens, D, D / 16, v8, word);
+    else kv_amax_kernel<false><<<grid, 256, 0, s>>>(k, ngroups, T, Tm, sink_tokens, D, D / 16, v8, word);
+    if (int rc = last_error()) return rc;
+    QuantParams p{};
+    p.x = k;
+    p.nblocks = ngroups;
+    p.f_lo = f_lo;
+    p.f_hi = f_hi;
+    p.g_src = gscale;
+    p.g_is_amax = 1;
+    p.codes = codes;
+    p.scales = scales;
+    p.v8 = v8;
+    p.T = T;
+    p.Tm = Tm;
+    p.sink = sink_tokens;
+    p.D = D;
+    p.bpr = D / 16;
+    int rc = rotate ? launch_quantize_t<true, true>(DT_BF16, p, s) : launch_quantize_t<true, false>(DT_BF16, p, s);
+    if (rc) return rc;
+  }
+  global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
+  if (int rc = last_error()) return rc;
+  return check_finite_sync(gscale, s);
+}
+
+}  // extern "C"

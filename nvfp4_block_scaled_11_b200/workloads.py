@@ -38,9 +38,10 @@ class Workload:
     note: str
 
 
-def _gen(seed: int, device) -> torch.Generator:
+def _gen(seed: int, device, shard: int = 0) -> torch.Generator:
+    """Generator for one workload; shard k > 0 (another rank's slice) gets its own stream."""
     g = torch.Generator(device=device)
-    g.manual_seed(seed)
+    g.manual_seed(seed + 7919 * shard)
     return g
 
 
@@ -80,10 +81,10 @@ def kv_bf16(device="cpu", scale: float = 1.0, heads: int = 8, head_dim: int = 12
     return k.to(torch.bfloat16)
 
 
-def stream_f32(device="cpu", scale: float = 1.0) -> torch.Tensor:
+def stream_f32(device="cpu", scale: float = 1.0, shard: int = 0) -> torch.Tensor:
     n = max(1 << 14, int((1 << 30) * scale))
     n -= n % 16
-    g = _gen(3, device)
+    g = _gen(3, device, shard)
     a = torch.randn((n,), generator=g, device=device, dtype=torch.float32)
     b = torch.randn((n,), generator=g, device=device, dtype=torch.float32)
     pick = torch.rand((n,), generator=g, device=device) < 0.1
@@ -103,7 +104,7 @@ def bev_f16(device="cpu", scale: float = 1.0) -> torch.Tensor:
     return v.to(torch.float16)
 
 
-def make(name: str, device="cpu", scale: float = 1.0) -> Workload:
+def make(name: str, device="cpu", scale: float = 1.0, shard: int = 0) -> Workload:
     if name == "act_f32":
         return Workload(name, act_f32(device, scale), -2, 6, "quantize", "FP32 [1024,4096] N(0,1), seed 0")
     if name == "act_bf16":
@@ -113,7 +114,7 @@ def make(name: str, device="cpu", scale: float = 1.0) -> Workload:
         return Workload(name, kv_bf16(device, scale), -2, 6, "kv",
                         "BF16 K [1,8,32768,128] N(0,1) + N(0,2) bias on 4 channels, seed 2")
     if name == "stream_f32":
-        return Workload(name, stream_f32(device, scale), -2, 6, "quantize",
+        return Workload(name, stream_f32(device, scale, shard), -2, 6, "quantize",
                         "FP32 2^30 mixture 0.9 N(0,1) + 0.1 N(0,16), seed 3")
     if name == "bev_f16":
         return Workload(name, bev_f16(device, scale), -2, 6, "quantize",

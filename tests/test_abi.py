@@ -1,0 +1,84 @@
+"""The C-ABI library loads and exports every symbol include/nvfp4.h declares; argument validation
+rejects bad calls synchronously (these calls return before any CUDA work, so no GPU is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_11_b200 as nv
+from nvfp4_block_scaled_11_b200 import build as nvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+def _declared():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nvbuild.build()
+    return nv.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 9
+    for name in names:
+        assert hasattr(L, name), name
+        assert name in nv._SIGS, f"binding lacks {name}"
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert nv.status_str(code).startswith("NVFP4")
+    assert L.nvfp4_version() >= 100
+
+
+V = ctypes.c_void_p
+
+
+def test_quantize_argument_errors(L):
+    fake = V(0x10000)  # 16-byte aligned, never dereferenced: validation fails first
+    codes, scales, g = V(0x20000), V(0x30000), V(0x40000)
+    # n not a multiple of 16
+    assert L.nvfp4_quantize(fake, 17, 0, 16, -2, 6, codes, scales, g, None) == -2
+    assert L.nvfp4_quantize(fake, -16, 0, 16, -2, 6, codes, scales, g, None) == -2
+    # block != 16, bad dtype, bad window, missing gscale
+    assert L.nvfp4_quantize(fake, 32, 0, 32, -2, 6, codes, scales, g, None) == -1
+    assert L.nvfp4_quantize(fake, 32, 7, 16, -2, 6, codes, scales, g, None) == -1
+    assert L.nvfp4_quantize(fake, 32, 0, 16, 3, 2, codes, scales, g, None) == -1
+    assert L.nvfp4_quantize(fake, 32, 0, 16, -200, 6, codes, scales, g, None) == -1
+    assert L.nvfp4_quantize(fake, 32, 0, 16, -2, 6, codes, scales, None, None) == -1
+    assert L.nvfp4_quantize(None, 32, 0, 16, -2, 6, codes, scales, g, None) == -1
+    # misaligned input / codes
+    assert L.nvfp4_quantize(V(0x10008), 32, 0, 16, -2, 6, codes, scales, g, None) == -3
+    assert L.nvfp4_quantize(fake, 32, 0, 16, -2, 6, V(0x20004), scales, g, None) == -3
+
+
+def test_other_entry_point_errors(L):
+    fake = V(0x10000)
+    assert L.nvfp4_dequantize(fake, fake, fake, 24, 0, fake, None) == -2
+    assert L.nvfp4_dequantize(fake, fake, None, 32, 0, fake, None) == -1
+    assert L.nvfp4_dequantize(fake, fake, fake, 32, 9, fake, None) == -1
+    assert L.nvfp4_dequantize(fake, fake, fake, 32, 0, V(0x10004), None) == -3
+    assert L.nvfp4_hadamard16(fake, 20, 0, fake, 0, None) == -2
+    assert L.nvfp4_hadamard16(fake, 32, 0, fake, 1, None) == -1  # in place across dtypes
+    assert L.nvfp4_tensor_amax(fake, 10, 5, fake, None) == -1
+    assert L.nvfp4_tensor_amax(V(0x10002), 10, 0, fake, None) == -3
+    assert L.nvfp4_global_scale(None, fake, None) == -1
+    # kv: T smaller than sink + recent, D not a multiple of 16
+    assert L.nvfp4_kv_mixed(fake, 1, 1, 20, 128, 16, 16, 1, -2, 6, fake, fake, fake, fake, fake, None) == -2
+    assert L.nvfp4_kv_mixed(fake, 1, 1, 64, 120, 16, 16, 1, -2, 6, fake, fake, fake, fake, fake, None) == -2
+    assert L.nvfp4_kv_mixed(fake, 1, 1, 64, 128, 16, 16, 1, 5, 4, fake, fake, fake, fake, fake, None) == -1
+    assert L.nvfp4_quantize_ex(fake, 32, 0, 16, -2, 6, None, fake, fake, None, None, None, None) == -1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        nv.quantize(torch.zeros(32))
