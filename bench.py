@@ -40,6 +40,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="stream_f32")
+    ap.add_argument("--scale", type=float, default=1.0, help="fraction of the workload size (profiling runs)")
     ap.add_argument("--f-lo", type=int, default=-2)
     ap.add_argument("--f-hi", type=int, default=6)
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -181,9 +182,10 @@ def run_reference(args, rank, world):
 
 
 def workload_config(args):
+    full = args.workload == "stream_f32" and args.scale == 1.0
     return {
-        "workload": f"{args.workload}" + (" (FP32 2^30 = 4 GiB, 0.9 N(0,1) + 0.1 N(0,16), seed 3)"
-                                            if args.workload == "stream_f32" else ""),
+        "workload": f"{args.workload}" + (" (FP32 2^30 = 4 GiB, 0.9 N(0,1) + 0.1 N(0,16), seed 3)" if full
+                                            else f" scaled by {args.scale}"),
         "window": [args.f_lo, args.f_hi],
         "step": "amax + [allreduce max] + g + ScaleSearch quantize + dequantize FP32",
         "l2": "inputs larger than L2 (4 GiB per step per GPU), no flush",
@@ -216,7 +218,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    w = W.make(args.workload, dev, 1.0, shard=rank)
+    w = W.make(args.workload, dev, args.scale, shard=rank)
     if w.kind != "quantize":
         raise SystemExit("bench.py times quantize workloads; kv_bf16 is covered by the parity tests")
     x = w.x.reshape(-1).contiguous()

@@ -7,7 +7,7 @@
 #include <mutex>
 
 #include "../../include/nvfp4.h"
-#include "kernels.cuh"
+#include "search.cuh"
 
 using namespace nvfp4;
 
@@ -79,13 +79,33 @@ int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_
   return last_error();
 }
 
+template <int DT, bool KV, bool ROT, int NC>
+void launch_search(const QuantParams& p, cudaStream_t s) {
+  const int grid = grid_for(p.nblocks, 256, 3);
+  if (p.block_sse) quantize_search_kernel<DT, KV, ROT, NC, true><<<grid, 256, 0, s>>>(p);
+  else quantize_search_kernel<DT, KV, ROT, NC, false><<<grid, 256, 0, s>>>(p);
+}
+
+template <int DT, bool KV, bool ROT>
+void launch_quantize_dt(const QuantParams& p, cudaStream_t s) {
+  switch (p.f_hi - p.f_lo + 1) {
+    case 1: launch_search<DT, KV, ROT, 1>(p, s); break;
+    case 9: launch_search<DT, KV, ROT, 9>(p, s); break;
+    case 17: launch_search<DT, KV, ROT, 17>(p, s); break;
+    default: quantize_kernel<DT, KV, ROT><<<grid_for(p.nblocks, 256, 4), 256, 0, s>>>(p); break;
+  }
+}
+
 template <bool KV, bool ROT>
 int launch_quantize_t(int dtype, const QuantParams& p, cudaStream_t s) {
-  const int grid = grid_for(p.nblocks, 256, 4);
-  switch (dtype) {
-    case DT_F32: quantize_kernel<DT_F32, KV, ROT><<<grid, 256, 0, s>>>(p); break;
-    case DT_BF16: quantize_kernel<DT_BF16, KV, ROT><<<grid, 256, 0, s>>>(p); break;
-    default: quantize_kernel<DT_F16, KV, ROT><<<grid, 256, 0, s>>>(p); break;
+  if (KV) {
+    launch_quantize_dt<DT_BF16, KV, ROT>(p, s);
+  } else {
+    switch (dtype) {
+      case DT_F32: launch_quantize_dt<DT_F32, KV, ROT>(p, s); break;
+      case DT_BF16: launch_quantize_dt<DT_BF16, KV, ROT>(p, s); break;
+      default: launch_quantize_dt<DT_F16, KV, ROT>(p, s); break;
+    }
   }
   return last_error();
 }

@@ -1,0 +1,410 @@
+// search.cuh -- ScaleSearch quantize for sm_100a with a certified fast score.
+//
+// "Search your block floating-point scales!" (gist.science summary of arXiv 2605.12464), Method >
+// ScaleSearch: every offset f of the default E4M3 scale code is scored by the block's squared error and
+// the best one wins.  The definition scores candidate d (r = fl(1/d)) by the in-order FP32 fold
+//     F = sum_i fl(e_i^2),  e_i = fl(x_i - fl(E2M1(fl(x_i r)) d)).
+// Scoring all candidates that way costs about seven FP32 operations per candidate and element.  This
+// kernel scores them instead in the scaled domain,
+//     P = fl(d^2) * sum_i (v_i - y_i)^2,  y_i = fl(x_i r),  v_i = E2M1(y_i),
+// with the E2M1 rounding and its decode done by the hardware converters (the code never leaves an 8-bit
+// register), v_i - y_i formed with one rounding by a mixed-precision subtract, and the squares
+// accumulated with packed FP32 FMAs: three FP32 pipe slots per candidate and element.
+//
+// P differs from F only by rounding.  For blocks whose magnitudes keep every intermediate normal
+// (2^-40 <= amax_b <= 2^40, every candidate d >= 2^-40, every y <= 1024) the difference is bounded by
+//     |F - P| <= 2^-15 * P + 2^-15 * amax_b * Dmax + 2^-36 * amax_b^2 + 2^-140,
+//     Dmax = max(d_hi, amax_b - 6 d_lo)   (d_lo / d_hi: smallest / largest candidate scale):
+// both F and P are perturbations of the real sum of (x_i - v_i d)^2 by the roundings of r, y, the
+// products and the sums, and |x_i - v_i d| <= d * max(1, y_max - 6) bounds the cross terms.  When the
+// runner-up's score exceeds the best score by more than twice that bound, the best candidate of the
+// score is the best candidate of the definition and no exact work is needed.  Otherwise every
+// candidate that is not so separated is re-scored with the definition, and the definition's tie rule
+// decides.  Blocks outside the covered range, or whose window leaves the codes 1..126, are scored with
+// the definition throughout.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace nvfp4 {
+
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 pk2(float lo, float hi) {
+  u64 r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(u64 v, float& lo, float& hi) {
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// Exact E2M1 roundings of (lo, hi), returned as the f16 halves of one register (RNE, saturating).
+__device__ __forceinline__ uint32_t e2m1_round2(float lo, float hi) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %2, %1; cvt.rn.f16x2.e2m1x2 %0, t; }"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
+// (v_lo - y_lo, v_hi - y_hi) with v the f16 halves of h2 (exact values): one rounding each.
+__device__ __forceinline__ u64 vsub2(uint32_t h2, float ylo, float yhi) {
+  float lo, hi;
+  asm("{ .reg .b16 l, h; mov.b32 {l,h}, %2; sub.rn.f32.f16 %0, l, %3; sub.rn.f32.f16 %1, h, %4; }"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2), "f"(ylo), "f"(yhi));
+  return pk2(lo, hi);
+}
+// E2M1 codes of 8 values packed into a word, value 2k in the low nibble of byte k.
+__device__ __forceinline__ uint32_t e2m1_pack8(u64 p0, u64 p1, u64 p2, u64 p3) {
+  float a0, a1, b0, b1, c0, c1, d0, d1;
+  upk2(p0, a0, a1);
+  upk2(p1, b0, b1);
+  upk2(p2, c0, c1);
+  upk2(p3, d0, d1);
+  uint32_t r;
+  asm("{ .reg .b8 t0, t1, t2, t3;\n"
+      "  cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n"
+      "  cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n"
+      "  cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n"
+      "  cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n"
+      "  mov.b32 %0, {t0, t1, t2, t3}; }"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1), "f"(d0), "f"(d1));
+  return r;
+}
+// max(m, |a|, |b|) with NaN propagation.
+__device__ __forceinline__ float absmax3_nan(float m, float a, float b) {
+  float d;
+  asm("{ .reg .f32 u, v; abs.f32 u, %2; abs.f32 v, %3; max.NaN.f32 %0, %1, u, v; }"
+      : "=f"(d)
+      : "f"(m), "f"(a), "f"(b));
+  return d;
+}
+
+// Candidate table for one launch, one 16-byte entry per code: d = fl(E4M3(c) * g), r = fl(1 / d),
+// dd = fl(d * d); r = 0 marks a code that cannot be a scale (outside 1..126, d == 0 or 1/d not finite).
+struct CandEntry {
+  float d, r, dd, pad;
+};
+
+__device__ __forceinline__ void build_cand_entries(CandEntry* t, float g) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float d = __fmul_rn(e4m3_value((uint32_t)c), g);
+    const float r = __frcp_rn(d);
+    const bool ok = c >= 1 && c <= 126 && d != 0.0f && fabsf(r) <= FLT_MAX;
+    t[c] = CandEntry{d, ok ? r : 0.0f, __fmul_rn(d, d), 0.0f};
+  }
+}
+
+// Default code c0(a) = E4M3(fl(fl(a / 6) / g)) of a block with amax a > 0.  c0 is non-decreasing in a,
+// so it is fixed by the thresholds T[k] = min{a : c0(a) >= k}: c0(a) = max{k : T[k] <= a}.  Each
+// threshold is found once per CTA by bisection over the bit patterns of non-negative floats (their
+// integer order is their numeric order), evaluating c0 exactly as defined; T[0] = 0, T[127] = +Inf.
+__device__ __forceinline__ int c0_exact(float a, float g) {
+  return a == 0.0f ? 0 : e4m3_code(__fdiv_rn(__fdiv_rn(a, 6.0f), g));
+}
+
+__device__ __forceinline__ void build_c0_thresholds(float* T, float g) {
+  for (int k = threadIdx.x; k < 128; k += blockDim.x) {
+    float t;
+    if (k == 0) {
+      t = 0.0f;
+    } else if (k == 127) {
+      t = __uint_as_float(0x7F800000u);
+    } else {
+      uint32_t lo = 0u, hi = 0x7F800000u;  // c0(lo) < k <= c0(hi)
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (c0_exact(__uint_as_float(mid), g) >= k) hi = mid;
+        else lo = mid;
+      }
+      t = __uint_as_float(hi);
+    }
+    T[k] = t;
+  }
+}
+
+// c0 of a finite a > 0 from the thresholds: a close first guess from one multiply, then exact steps.
+__device__ __forceinline__ int c0_from_thresholds(const float* T, float a, float inv6g) {
+  int c = e4m3_code(__fmul_rn(a, inv6g));
+  while (T[c + 1] <= a) ++c;
+  while (T[c] > a) --c;
+  return c;
+}
+
+// The definition: in-order FP32 fold of the squared errors of candidate (d, r).
+__device__ __forceinline__ float block_sse_def(const float (&x)[16], float d, float r) {
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float y0 = __fmul_rn(x[i], r), y1 = __fmul_rn(x[i + 1], r);
+    const uint32_t h2 = e2m1_round2(y0, y1);
+    const float e0 = __fsub_rn(x[i], __fmul_rn(f16lo(h2), d));
+    const float e1 = __fsub_rn(x[i + 1], __fmul_rn(f16hi(h2), d));
+    s = __fadd_rn(s, __fmul_rn(e0, e0));
+    s = __fadd_rn(s, __fmul_rn(e1, e1));
+  }
+  return s;
+}
+
+// One element pair of the scaled-domain score: acc += (v - y)^2 for y = x * r, v = E2M1(y), both lanes.
+__device__ __forceinline__ u64 score_pair(u64 acc, u64 x2, u64 rr) {
+  asm("{ .reg .b64 y2, e2; .reg .f32 ylo, yhi, elo, ehi; .reg .b8 q; .reg .b32 h2; .reg .b16 hl, hh;\n"
+      "  mul.rn.f32x2 y2, %1, %2;\n"
+      "  mov.b64 {ylo, yhi}, y2;\n"
+      "  cvt.rn.satfinite.e2m1x2.f32 q, yhi, ylo;\n"
+      "  cvt.rn.f16x2.e2m1x2 h2, q;\n"
+      "  mov.b32 {hl, hh}, h2;\n"
+      "  sub.rn.f32.f16 elo, hl, ylo;\n"
+      "  sub.rn.f32.f16 ehi, hh, yhi;\n"
+      "  mov.b64 e2, {elo, ehi};\n"
+      "  fma.rn.f32x2 %0, e2, e2, %0; }"
+      : "+l"(acc)
+      : "l"(x2), "l"(rr));
+  return acc;
+}
+
+// Scaled-domain score of one candidate: sum over the block of (v - y)^2 (any order), times d^2.
+__device__ __forceinline__ float score_scaled(const u64 (&x2)[8], float r, float dd) {
+  const u64 rr = pk2(r, r);
+  u64 acc = 0ull;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc = score_pair(acc, x2[k], rr);
+  float lo, hi;
+  upk2(acc, lo, hi);
+  return __fmul_rn(__fadd_rn(lo, hi), dd);
+}
+
+__device__ __forceinline__ bool better(float s, int f, float bs, int bf) {
+  // definition order: smaller sse, then smaller |f|, then smaller f
+  if (s != bs) return s < bs;
+  if (abs(f) != abs(bf)) return abs(f) < abs(bf);
+  return f < bf;
+}
+
+// Score every usable candidate of the window with the definition; visit 0, -1, +1, ... and keep the
+// first strictly smaller SSE (the definition's tie rule).
+__device__ __forceinline__ void search_def(const float (&x)[16], int c0, int f_lo, int f_hi, const CandEntry* tab,
+                                           int& fstar, float& best) {
+  const int span = max(abs(f_lo), abs(f_hi));
+  fstar = -128;
+  best = 0.0f;
+  for (int jv = 0; jv <= 2 * span; ++jv) {
+    const int f = (jv == 0) ? 0 : ((jv & 1) ? -((jv + 1) >> 1) : (jv >> 1));
+    if (f < f_lo || f > f_hi) continue;
+    const int c = c0 + f;
+    if (c < 1 || c > 126) continue;
+    const CandEntry e = tab[c];
+    if (e.r == 0.0f) continue;
+    const float s = block_sse_def(x, e.d, e.r);
+    if (fstar == -128 || s < best) {
+      best = s;
+      fstar = f;
+    }
+  }
+}
+
+struct Block16 {
+  float v[16];
+};
+
+// Near tie (rare): every candidate whose score is within thr is re-scored with the definition and the
+// definition's tie rule picks among them.  Out of line to keep the hot loop small.
+__device__ __noinline__ void resolve_near_tie(Block16 blk, int clo, int nc, int f_lo, float thr, const CandEntry* tab,
+                                              int* fstar_out, float* best_out) {
+  u64 x2[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x2[k] = pk2(blk.v[2 * k], blk.v[2 * k + 1]);
+  int fstar = -128;
+  float best = 0.0f;
+#pragma unroll 1
+  for (int j = 0; j < nc; ++j) {
+    const CandEntry e = tab[clo + j];
+    if (score_scaled(x2, e.r, e.dd) <= thr) {
+      const float s = block_sse_def(blk.v, e.d, e.r);
+      const int f = f_lo + j;
+      if (fstar == -128 || better(s, f, best, fstar)) {
+        best = s;
+        fstar = f;
+      }
+    }
+  }
+  *fstar_out = fstar;
+  *best_out = best;
+}
+
+// The definition over the whole window (blocks the fast score does not cover).  Out of line.
+__device__ __noinline__ void search_def_block(Block16 blk, int c0, int f_lo, int f_hi, const CandEntry* tab,
+                                              int* fstar_out, float* best_out) {
+  int fstar;
+  float best;
+  search_def(blk.v, c0, f_lo, f_hi, tab, fstar, best);
+  *fstar_out = fstar;
+  *best_out = best;
+}
+
+// Certified fast search over the NC offsets f_lo .. f_lo + NC - 1 of the default code c0.  Returns
+// false (outputs untouched) when the block is outside what the error bound covers.
+template <int NC, bool WANT_SSE>
+__device__ __forceinline__ bool search_fast(const float (&x)[16], float amax_b, int c0, int f_lo,
+                                            const CandEntry* tab, int& fstar, float& best) {
+  const int clo = c0 + f_lo, chi = c0 + f_lo + NC - 1;
+  if (clo < 1 || chi > 126 || !(amax_b >= 0x1p-40f && amax_b <= 0x1p40f)) return false;
+  const CandEntry elo = tab[clo];
+  if (elo.r == 0.0f || !(elo.d >= 0x1p-40f) || !(__fmul_rn(amax_b, elo.r) <= 1024.0f)) return false;
+  const float dhi = tab[chi].d;
+
+  u64 x2[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x2[k] = pk2(x[2 * k], x[2 * k + 1]);
+  // keys: score bits with the candidate index in the low 5 bits (unsigned order = score order);
+  // m1 / m2 track the smallest and the second smallest key
+  uint32_t m1 = 0xFFFFFFFFu, m2 = 0xFFFFFFFFu;
+#pragma unroll
+  for (int j = 0; j < NC; ++j) {
+    const CandEntry e = tab[clo + j];
+    const float s = score_scaled(x2, e.r, e.dd);
+    const uint32_t key = (__float_as_uint(s) & ~31u) | (uint32_t)j;
+    m2 = min(m2, max(m1, key));
+    m1 = min(m1, key);
+  }
+  const float pbest = __uint_as_float(m1 & ~31u);
+  const float p2 = __uint_as_float(m2 & ~31u);
+  const float dmax = fmaxf(dhi, __fsub_rn(__fmul_rn(amax_b, 1.000001f), __fmul_rn(6.0f, elo.d)));
+  const float beta = __fadd_rn(__fmul_rn(__fmul_rn(amax_b, dmax), 0x1p-15f),
+                               __fadd_rn(__fmul_rn(__fmul_rn(amax_b, amax_b), 0x1p-36f), 0x1p-140f));
+  // a candidate whose score is above thr is certainly worse than the best under the definition
+  const float thr = __fmul_rn(__fadd_rn(__fmul_rn(pbest, 1.0f + 0x1p-13f), __fmul_rn(beta, 2.5f)), 1.0f + 0x1p-13f);
+  if (p2 > thr) {
+    fstar = f_lo + (int)(m1 & 31u);
+    best = 0.0f;
+    if (WANT_SSE) {
+      const CandEntry e = tab[c0 + fstar];
+      best = block_sse_def(x, e.d, e.r);
+    }
+    return true;
+  }
+  Block16 blk;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) blk.v[i] = x[i];
+  resolve_near_tie(blk, clo, NC, f_lo, thr, tab, &fstar, &best);
+  return true;
+}
+
+template <int DT, bool KV, bool ROT, int NC, bool WANT_SSE>
+__device__ __forceinline__ void quantize_one_block(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                                   float inv6g, bool g_bad, int64_t b, float (&x)[16]) {
+  if (ROT) fwht16(x);
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) amax_b = absmax3_nan(amax_b, x[i], x[i + 1]);
+
+  uint32_t lo = 0u, hi = 0u;
+  int scale = 0, fstar = -128, c0 = 0;
+  float sse = 0.0f;
+  if (g_bad || !(amax_b <= FLT_MAX)) {  // NaN / Inf element, or unusable g: poisoned block
+    scale = 0x7F;
+    sse = __uint_as_float(0x7FFFFFFFu);
+  } else {
+    if (amax_b != 0.0f) {
+      c0 = c0_from_thresholds(thr, amax_b, inv6g);
+      if (NC == 1) {
+        const int c = c0 + p.f_lo;
+        if (c >= 1 && c <= 126 && tab[c].r != 0.0f) {
+          fstar = p.f_lo;
+          if (WANT_SSE) sse = block_sse_def(x, tab[c].d, tab[c].r);
+        }
+      } else if (!search_fast<NC, WANT_SSE>(x, amax_b, c0, p.f_lo, tab, fstar, sse)) {
+        Block16 blk;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) blk.v[i] = x[i];
+        search_def_block(blk, c0, p.f_lo, p.f_lo + NC - 1, tab, &fstar, &sse);
+      }
+    }
+    if (fstar != -128) {
+      scale = c0 + fstar;
+      const float r = tab[scale].r;
+      const u64 rr = pk2(r, r);
+      lo = e2m1_pack8(mul2(pk2(x[0], x[1]), rr), mul2(pk2(x[2], x[3]), rr), mul2(pk2(x[4], x[5]), rr),
+                      mul2(pk2(x[6], x[7]), rr));
+      hi = e2m1_pack8(mul2(pk2(x[8], x[9]), rr), mul2(pk2(x[10], x[11]), rr), mul2(pk2(x[12], x[13]), rr),
+                      mul2(pk2(x[14], x[15]), rr));
+    } else {
+      // all-zero block or no usable candidate: sign-only zero codes, scale 0, sse = sum of x^2
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t nib =
+            ((__float_as_uint(x[2 * k]) >> 31) << 3) | ((__float_as_uint(x[2 * k + 1]) >> 31) << 7);
+        if (k < 4) lo |= nib << (8 * k);
+        else hi |= nib << (8 * (k - 4));
+      }
+      if (WANT_SSE && amax_b != 0.0f) {
+        float s = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s = __fadd_rn(s, __fmul_rn(x[i], x[i]));
+        sse = s;
+      }
+    }
+  }
+  reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(lo, hi);
+  p.scales[b] = (uint8_t)scale;
+  if (p.block_f) p.block_f[b] = (int8_t)fstar;
+  if (WANT_SSE) p.block_sse[b] = sse;
+}
+
+template <int DT, bool KV>
+__device__ __forceinline__ const char* block_src(const QuantParams& p, int64_t b) {
+  constexpr int ES = DT == DT_F32 ? 4 : 2;
+  int64_t elem;
+  if (KV) {
+    const int64_t per_bh = p.Tm * p.bpr;
+    const int64_t bh = b / per_bh;
+    const int64_t rem = b - bh * per_bh;
+    const int64_t t = rem / p.bpr;
+    const int64_t j = rem - t * p.bpr;
+    elem = (bh * p.T + p.sink + t) * p.D + 16 * j;
+  } else {
+    elem = 16 * b;
+  }
+  return p.x + elem * ES;
+}
+
+// One thread per 16-element block, grid-stride, with the next block's loads in flight while the
+// current block is searched.
+template <int DT, bool KV, bool ROT, int NC, bool WANT_SSE>
+__global__ void __launch_bounds__(256, 3) quantize_search_kernel(QuantParams p) {
+  __shared__ CandEntry tab[128];
+  __shared__ float thr[128];
+  float g = *p.g_src;
+  if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
+  const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
+  build_cand_entries(tab, g);
+  if (!g_bad) build_c0_thresholds(thr, g);
+  __syncthreads();
+  const float inv6g = __frcp_rn(__fmul_rn(6.0f, g));
+
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const bool v8 = p.v8 != 0;
+  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  float xn[16];
+  if (b < p.nblocks) load_block<DT>(block_src<DT, KV>(p, b), v8, xn);
+  for (; b < p.nblocks; b += stride) {
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = xn[i];
+    if (b + stride < p.nblocks) load_block<DT>(block_src<DT, KV>(p, b + stride), v8, xn);
+    quantize_one_block<DT, KV, ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x);
+  }
+}
+
+}  // namespace nvfp4

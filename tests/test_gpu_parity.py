@@ -296,3 +296,23 @@ def test_full_size_sampled(name):
     out = nv.dequantize(codes, scales, g, torch.float32)
     rd = O.dequantize(codes.view(-1, 8)[ti].cpu().numpy().reshape(-1), rs, rg)
     assert same_f32(out.view(-1, 16)[ti].cpu().numpy(), rd)
+
+
+def test_many_blocks_with_natural_near_ties():
+    """2^20 blocks: about 0.1% of them have a runner-up within 2e-4 of the best score, which exercises
+    the fast score's certification and its fall back to the definition."""
+    x = W.stream_f32("cpu", 2 ** -6)
+    check_quantize(x, -2, 6)
+    check_quantize(x, -8, 8)
+
+
+def test_exact_ties_on_dyadic_blocks():
+    """Dyadic values with a power-of-two tensor scale make many candidates' SSEs exactly equal; the
+    definition's tie rule (smaller |f|, then smaller f) must decide."""
+    rng = np.random.default_rng(21)
+    vals = rng.integers(-24, 25, size=(1 << 16, 16)) / 8.0
+    vals[:, 0] = np.where(rng.random(1 << 16) < 0.5, 3.0, -3.0)
+    x = torch.from_numpy(vals.astype(np.float32).reshape(-1))
+    for gin in (2.0 ** -6, 2.0 ** -8, 3.0 * 2.0 ** -9):
+        check_quantize(x, -2, 6, gscale_in=gin)
+        check_quantize(x, -8, 8, gscale_in=gin)
