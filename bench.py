@@ -60,6 +60,25 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def captured_traffic(kernel_key: str, elements: int):
+    """DRAM bytes per launch from the committed ncu record, scaled to `elements`; None when the kernel
+    sources changed since the capture (the counters then no longer describe this build)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+            rec = json.load(fh)[kernel_key]
+        h = hashlib.sha256()
+        for f in rec["source_files"]:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != rec["source_sha256"]:
+            return None
+        per = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["captured_elements"]
+        return per * elements
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------------------------------------
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------------
@@ -296,7 +315,9 @@ def main():
         "config": workload_config(args),
         "roofline": {"bound": "hbm", "kernel": "quantize (ScaleSearch search + encode pass)",
                      "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
-                     "traffic": None, "peak_source": peak_src,
+                     "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0>", n)
+                     if (x.dtype == torch.float32 and (args.f_lo, args.f_hi) == (-2, 6)) else None,
+                     "peak_source": peak_src,
                      "bytes_per_launch": q_bytes},
         "breakdown_ms": {"amax_and_g": amax_ms, "quantize": q_ms, "dequantize": dq_ms},
         "quantize_two_pass": {"gbs_input": bytes_in / ((amax_ms + q_ms) * 1e-3) / 1e9,

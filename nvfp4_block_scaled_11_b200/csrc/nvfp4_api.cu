@@ -81,7 +81,7 @@ int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_
 
 template <int DT, bool KV, bool ROT, int NC>
 void launch_search(const QuantParams& p, cudaStream_t s) {
-  const int grid = grid_for(p.nblocks, 256, 3);
+  const int grid = grid_for(p.nblocks, 256, NVFP4_SEARCH_CTAS_PER_SM);
   if (p.block_sse) quantize_search_kernel<DT, KV, ROT, NC, true><<<grid, 256, 0, s>>>(p);
   else quantize_search_kernel<DT, KV, ROT, NC, false><<<grid, 256, 0, s>>>(p);
 }
@@ -98,7 +98,7 @@ void launch_quantize_dt(const QuantParams& p, cudaStream_t s) {
 
 template <bool KV, bool ROT>
 int launch_quantize_t(int dtype, const QuantParams& p, cudaStream_t s) {
-  if (KV) {
+  if constexpr (KV) {
     launch_quantize_dt<DT_BF16, KV, ROT>(p, s);
   } else {
     switch (dtype) {

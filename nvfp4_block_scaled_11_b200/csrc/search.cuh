@@ -91,10 +91,38 @@ __device__ __forceinline__ float absmax3_nan(float m, float a, float b) {
   return d;
 }
 
-// Candidate table for one launch, one 16-byte entry per code: d = fl(E4M3(c) * g), r = fl(1 / d),
-// dd = fl(d * d); r = 0 marks a code that cannot be a scale (outside 1..126, d == 0 or 1/d not finite).
-struct CandEntry {
-  float d, r, dd, pad;
+__device__ __forceinline__ void ld_v4_b64(const void* p, u64& a, u64& b, u64& c, u64& d) {
+  asm("ld.global.nc.L1::no_allocate.v4.b64 {%0,%1,%2,%3}, [%4];" : "=l"(a), "=l"(b), "=l"(c), "=l"(d) : "l"(p));
+}
+__device__ __forceinline__ void ld_v2_b64(const void* p, u64& a, u64& b) {
+  asm("ld.global.nc.L1::no_allocate.v2.b64 {%0,%1}, [%2];" : "=l"(a), "=l"(b) : "l"(p));
+}
+
+// One 16-element block as 8 packed FP32 pairs (element 2k low, 2k+1 high).  32-byte aligned sources
+// use 256-bit loads, 16-byte aligned ones 128-bit loads; 16-bit inputs are widened exactly.
+template <int DT>
+__device__ __forceinline__ void load_pairs(const char* src, bool v8, u64 (&x2)[8]) {
+  if (DT == DT_F32) {
+    if (v8) {
+      ld_v4_b64(src, x2[0], x2[1], x2[2], x2[3]);
+      ld_v4_b64(src + 32, x2[4], x2[5], x2[6], x2[7]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ld_v2_b64(src + 16 * k, x2[2 * k], x2[2 * k + 1]);
+    }
+  } else {
+    float x[16];
+    load_block<DT>(src, v8, x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x2[k] = pk2(x[2 * k], x[2 * k + 1]);
+  }
+}
+
+// Candidate table for one launch, one 16-byte entry per code: d = fl(E4M3(c) * g), r = fl(1 / d) (stored
+// twice so that (r, r) loads as one aligned register pair), dd = fl(d * d); r = 0 marks a code that
+// cannot be a scale (outside 1..126, d == 0 or 1/d not finite).
+struct __align__(16) CandEntry {
+  float r, r2, dd, d;
 };
 
 __device__ __forceinline__ void build_cand_entries(CandEntry* t, float g) {
@@ -102,7 +130,8 @@ __device__ __forceinline__ void build_cand_entries(CandEntry* t, float g) {
     const float d = __fmul_rn(e4m3_value((uint32_t)c), g);
     const float r = __frcp_rn(d);
     const bool ok = c >= 1 && c <= 126 && d != 0.0f && fabsf(r) <= FLT_MAX;
-    t[c] = CandEntry{d, ok ? r : 0.0f, __fmul_rn(d, d), 0.0f};
+    const float rs = ok ? r : 0.0f;
+    t[c] = CandEntry{rs, rs, __fmul_rn(d, d), d};
   }
 }
 
@@ -157,33 +186,57 @@ __device__ __forceinline__ float block_sse_def(const float (&x)[16], float d, fl
   return s;
 }
 
+__device__ __forceinline__ float block_sse_def_pairs(const u64 (&x2)[8], float d, float r) {
+  float x[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
+  return block_sse_def(x, d, r);
+}
+
 // One element pair of the scaled-domain score: acc += (v - y)^2 for y = x * r, v = E2M1(y), both lanes.
+// FIRST: acc is not read (the first pair of a candidate starts the sum with a product).
+template <bool FIRST>
 __device__ __forceinline__ u64 score_pair(u64 acc, u64 x2, u64 rr) {
-  asm("{ .reg .b64 y2, e2; .reg .f32 ylo, yhi, elo, ehi; .reg .b8 q; .reg .b32 h2; .reg .b16 hl, hh;\n"
-      "  mul.rn.f32x2 y2, %1, %2;\n"
-      "  mov.b64 {ylo, yhi}, y2;\n"
-      "  cvt.rn.satfinite.e2m1x2.f32 q, yhi, ylo;\n"
-      "  cvt.rn.f16x2.e2m1x2 h2, q;\n"
-      "  mov.b32 {hl, hh}, h2;\n"
-      "  sub.rn.f32.f16 elo, hl, ylo;\n"
-      "  sub.rn.f32.f16 ehi, hh, yhi;\n"
-      "  mov.b64 e2, {elo, ehi};\n"
-      "  fma.rn.f32x2 %0, e2, e2, %0; }"
-      : "+l"(acc)
-      : "l"(x2), "l"(rr));
+  if (FIRST) {
+    asm("{ .reg .b64 y2, e2; .reg .f32 ylo, yhi, elo, ehi; .reg .b8 q; .reg .b32 h2; .reg .b16 hl, hh;\n"
+        "  mul.rn.f32x2 y2, %1, %2;\n"
+        "  mov.b64 {ylo, yhi}, y2;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 q, yhi, ylo;\n"
+        "  cvt.rn.f16x2.e2m1x2 h2, q;\n"
+        "  mov.b32 {hl, hh}, h2;\n"
+        "  sub.rn.f32.f16 elo, hl, ylo;\n"
+        "  sub.rn.f32.f16 ehi, hh, yhi;\n"
+        "  mov.b64 e2, {elo, ehi};\n"
+        "  mul.rn.f32x2 %0, e2, e2; }"
+        : "=l"(acc)
+        : "l"(x2), "l"(rr));
+  } else {
+    asm("{ .reg .b64 y2, e2; .reg .f32 ylo, yhi, elo, ehi; .reg .b8 q; .reg .b32 h2; .reg .b16 hl, hh;\n"
+        "  mul.rn.f32x2 y2, %1, %2;\n"
+        "  mov.b64 {ylo, yhi}, y2;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 q, yhi, ylo;\n"
+        "  cvt.rn.f16x2.e2m1x2 h2, q;\n"
+        "  mov.b32 {hl, hh}, h2;\n"
+        "  sub.rn.f32.f16 elo, hl, ylo;\n"
+        "  sub.rn.f32.f16 ehi, hh, yhi;\n"
+        "  mov.b64 e2, {elo, ehi};\n"
+        "  fma.rn.f32x2 %0, e2, e2, %0; }"
+        : "+l"(acc)
+        : "l"(x2), "l"(rr));
+  }
   return acc;
 }
 
 // Scaled-domain score of one candidate: sum over the block of (v - y)^2 (any order), times d^2.
-__device__ __forceinline__ float score_scaled(const u64 (&x2)[8], float r, float dd) {
-  const u64 rr = pk2(r, r);
-  u64 acc = 0ull;
+__device__ __forceinline__ float score_scaled(const u64 (&x2)[8], u64 rr, float dd) {
+  u64 acc = score_pair<true>(0ull, x2[0], rr);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc = score_pair(acc, x2[k], rr);
+  for (int k = 1; k < 8; ++k) acc = score_pair<false>(acc, x2[k], rr);
   float lo, hi;
   upk2(acc, lo, hi);
   return __fmul_rn(__fadd_rn(lo, hi), dd);
 }
+
 
 __device__ __forceinline__ bool better(float s, int f, float bs, int bf) {
   // definition order: smaller sse, then smaller |f|, then smaller f
@@ -214,49 +267,12 @@ __device__ __forceinline__ void search_def(const float (&x)[16], int c0, int f_l
   }
 }
 
-struct Block16 {
-  float v[16];
-};
-
-// Near tie (rare): every candidate whose score is within thr is re-scored with the definition and the
-// definition's tie rule picks among them.  Out of line to keep the hot loop small.
-__device__ __noinline__ void resolve_near_tie(Block16 blk, int clo, int nc, int f_lo, float thr, const CandEntry* tab,
-                                              int* fstar_out, float* best_out) {
-  u64 x2[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) x2[k] = pk2(blk.v[2 * k], blk.v[2 * k + 1]);
-  int fstar = -128;
-  float best = 0.0f;
-#pragma unroll 1
-  for (int j = 0; j < nc; ++j) {
-    const CandEntry e = tab[clo + j];
-    if (score_scaled(x2, e.r, e.dd) <= thr) {
-      const float s = block_sse_def(blk.v, e.d, e.r);
-      const int f = f_lo + j;
-      if (fstar == -128 || better(s, f, best, fstar)) {
-        best = s;
-        fstar = f;
-      }
-    }
-  }
-  *fstar_out = fstar;
-  *best_out = best;
-}
-
-// The definition over the whole window (blocks the fast score does not cover).  Out of line.
-__device__ __noinline__ void search_def_block(Block16 blk, int c0, int f_lo, int f_hi, const CandEntry* tab,
-                                              int* fstar_out, float* best_out) {
-  int fstar;
-  float best;
-  search_def(blk.v, c0, f_lo, f_hi, tab, fstar, best);
-  *fstar_out = fstar;
-  *best_out = best;
-}
-
 // Certified fast search over the NC offsets f_lo .. f_lo + NC - 1 of the default code c0.  Returns
-// false (outputs untouched) when the block is outside what the error bound covers.
+// true with fstar / best set when the fast score decides the block; false when the block must be scored
+// with the definition (outside the range the error bound covers, window leaving the codes 1..126, or a
+// runner-up too close to the best).
 template <int NC, bool WANT_SSE>
-__device__ __forceinline__ bool search_fast(const float (&x)[16], float amax_b, int c0, int f_lo,
+__device__ __forceinline__ bool search_fast(const u64 (&x2)[8], float amax_b, int c0, int f_lo,
                                             const CandEntry* tab, int& fstar, float& best) {
   const int clo = c0 + f_lo, chi = c0 + f_lo + NC - 1;
   if (clo < 1 || chi > 126 || !(amax_b >= 0x1p-40f && amax_b <= 0x1p40f)) return false;
@@ -264,102 +280,141 @@ __device__ __forceinline__ bool search_fast(const float (&x)[16], float amax_b, 
   if (elo.r == 0.0f || !(elo.d >= 0x1p-40f) || !(__fmul_rn(amax_b, elo.r) <= 1024.0f)) return false;
   const float dhi = tab[chi].d;
 
-  u64 x2[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) x2[k] = pk2(x[2 * k], x[2 * k + 1]);
   // keys: score bits with the candidate index in the low 5 bits (unsigned order = score order);
   // m1 / m2 track the smallest and the second smallest key
   uint32_t m1 = 0xFFFFFFFFu, m2 = 0xFFFFFFFFu;
 #pragma unroll
   for (int j = 0; j < NC; ++j) {
-    const CandEntry e = tab[clo + j];
-    const float s = score_scaled(x2, e.r, e.dd);
+    const float4 e = reinterpret_cast<const float4*>(tab)[clo + j];  // r, r, dd, d
+    const float s = score_scaled(x2, pk2(e.x, e.y), e.z);
     const uint32_t key = (__float_as_uint(s) & ~31u) | (uint32_t)j;
     m2 = min(m2, max(m1, key));
     m1 = min(m1, key);
   }
   const float pbest = __uint_as_float(m1 & ~31u);
   const float p2 = __uint_as_float(m2 & ~31u);
-  const float dmax = fmaxf(dhi, __fsub_rn(__fmul_rn(amax_b, 1.000001f), __fmul_rn(6.0f, elo.d)));
-  const float beta = __fadd_rn(__fmul_rn(__fmul_rn(amax_b, dmax), 0x1p-15f),
-                               __fadd_rn(__fmul_rn(__fmul_rn(amax_b, amax_b), 0x1p-36f), 0x1p-140f));
-  // a candidate whose score is above thr is certainly worse than the best under the definition
-  const float thr = __fmul_rn(__fadd_rn(__fmul_rn(pbest, 1.0f + 0x1p-13f), __fmul_rn(beta, 2.5f)), 1.0f + 0x1p-13f);
-  if (p2 > thr) {
-    fstar = f_lo + (int)(m1 & 31u);
-    best = 0.0f;
-    if (WANT_SSE) {
-      const CandEntry e = tab[c0 + fstar];
-      best = block_sse_def(x, e.d, e.r);
-    }
-    return true;
+  // bound terms (see the header): the arithmetic only has to stay an upper bound, so it uses FMAs
+  const float dmax = fmaxf(dhi, __fmaf_rn(amax_b, 1.000001f, -6.0f * elo.d));
+  const float beta = __fmaf_rn(amax_b, __fmaf_rn(amax_b, 0x1p-36f, dmax * 0x1p-15f), 0x1p-140f);
+  const float thr = __fmaf_rn(pbest, 1.0f + 0x1p-12f, beta * 2.51f);
+  if (!(p2 > thr)) return false;  // near tie: the definition decides
+  fstar = f_lo + (int)(m1 & 31u);
+  best = 0.0f;
+  if (WANT_SSE) {
+    const CandEntry e = tab[c0 + fstar];
+    best = block_sse_def_pairs(x2, e.d, e.r);
   }
-  Block16 blk;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) blk.v[i] = x[i];
-  resolve_near_tie(blk, clo, NC, f_lo, thr, tab, &fstar, &best);
   return true;
 }
 
-template <int DT, bool KV, bool ROT, int NC, bool WANT_SSE>
-__device__ __forceinline__ void quantize_one_block(const QuantParams& p, const CandEntry* tab, const float* thr,
-                                                   float inv6g, bool g_bad, int64_t b, float (&x)[16]) {
-  if (ROT) fwht16(x);
+__device__ __forceinline__ void encode_pairs(const u64 (&x2)[8], float r, uint32_t& wlo, uint32_t& whi) {
+  const u64 rr = pk2(r, r);
+  wlo = e2m1_pack8(mul2(x2[0], rr), mul2(x2[1], rr), mul2(x2[2], rr), mul2(x2[3], rr));
+  whi = e2m1_pack8(mul2(x2[4], rr), mul2(x2[5], rr), mul2(x2[6], rr), mul2(x2[7], rr));
+}
+
+__device__ __forceinline__ float block_amax_nan(const u64 (&x2)[8]) {
   float amax_b = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) amax_b = absmax3_nan(amax_b, x[i], x[i + 1]);
+  for (int k = 0; k < 8; ++k) {
+    float lo, hi;
+    upk2(x2[k], lo, hi);
+    amax_b = absmax3_nan(amax_b, lo, hi);
+  }
+  return amax_b;
+}
 
-  uint32_t lo = 0u, hi = 0u;
-  int scale = 0, fstar = -128, c0 = 0;
-  float sse = 0.0f;
-  if (g_bad || !(amax_b <= FLT_MAX)) {  // NaN / Inf element, or unusable g: poisoned block
+template <bool ROT>
+__device__ __forceinline__ void maybe_rotate(u64 (&x2)[8]) {
+  if (ROT) {
+    float t[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) upk2(x2[k], t[2 * k], t[2 * k + 1]);
+    fwht16(t);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x2[k] = pk2(t[2 * k], t[2 * k + 1]);
+  }
+}
+
+template <bool WANT_SSE>
+__device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, const u64 (&x2)[8], const CandEntry* tab,
+                                            int c0, int fstar, float sse, bool poisoned, float amax_b) {
+  uint32_t wlo = 0u, whi = 0u;
+  int scale;
+  if (poisoned) {
     scale = 0x7F;
     sse = __uint_as_float(0x7FFFFFFFu);
+  } else if (fstar != -128) {
+    scale = c0 + fstar;
+    encode_pairs(x2, tab[scale].r, wlo, whi);
   } else {
-    if (amax_b != 0.0f) {
-      c0 = c0_from_thresholds(thr, amax_b, inv6g);
-      if (NC == 1) {
-        const int c = c0 + p.f_lo;
-        if (c >= 1 && c <= 126 && tab[c].r != 0.0f) {
-          fstar = p.f_lo;
-          if (WANT_SSE) sse = block_sse_def(x, tab[c].d, tab[c].r);
-        }
-      } else if (!search_fast<NC, WANT_SSE>(x, amax_b, c0, p.f_lo, tab, fstar, sse)) {
-        Block16 blk;
+    // all-zero block or no usable candidate: sign-only zero codes, scale 0, sse = sum of x^2
+    scale = 0;
+    float s = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) blk.v[i] = x[i];
-        search_def_block(blk, c0, p.f_lo, p.f_lo + NC - 1, tab, &fstar, &sse);
+    for (int k = 0; k < 8; ++k) {
+      float lo, hi;
+      upk2(x2[k], lo, hi);
+      const uint32_t nib = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
+      if (k < 4) wlo |= nib << (8 * k);
+      else whi |= nib << (8 * (k - 4));
+      if (WANT_SSE) {
+        s = __fadd_rn(s, __fmul_rn(lo, lo));
+        s = __fadd_rn(s, __fmul_rn(hi, hi));
       }
     }
-    if (fstar != -128) {
-      scale = c0 + fstar;
-      const float r = tab[scale].r;
-      const u64 rr = pk2(r, r);
-      lo = e2m1_pack8(mul2(pk2(x[0], x[1]), rr), mul2(pk2(x[2], x[3]), rr), mul2(pk2(x[4], x[5]), rr),
-                      mul2(pk2(x[6], x[7]), rr));
-      hi = e2m1_pack8(mul2(pk2(x[8], x[9]), rr), mul2(pk2(x[10], x[11]), rr), mul2(pk2(x[12], x[13]), rr),
-                      mul2(pk2(x[14], x[15]), rr));
-    } else {
-      // all-zero block or no usable candidate: sign-only zero codes, scale 0, sse = sum of x^2
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t nib =
-            ((__float_as_uint(x[2 * k]) >> 31) << 3) | ((__float_as_uint(x[2 * k + 1]) >> 31) << 7);
-        if (k < 4) lo |= nib << (8 * k);
-        else hi |= nib << (8 * (k - 4));
-      }
-      if (WANT_SSE && amax_b != 0.0f) {
-        float s = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) s = __fadd_rn(s, __fmul_rn(x[i], x[i]));
-        sse = s;
-      }
-    }
+    sse = (WANT_SSE && amax_b != 0.0f) ? s : 0.0f;
   }
-  reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(lo, hi);
+  reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(wlo, whi);
   p.scales[b] = (uint8_t)scale;
   if (p.block_f) p.block_f[b] = (int8_t)fstar;
   if (WANT_SSE) p.block_sse[b] = sse;
+}
+
+// Fast path for one block.  Returns true when the block needs the definition (outputs not written).
+template <bool ROT, int NC, bool WANT_SSE>
+__device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                                    float inv6g, bool g_bad, int64_t b, u64 (&x2)[8]) {
+  maybe_rotate<ROT>(x2);
+  const float amax_b = block_amax_nan(x2);
+  const bool poisoned = g_bad || !(amax_b <= FLT_MAX);  // NaN / Inf element, or unusable g
+  int c0 = 0, fstar = -128;
+  float sse = 0.0f;
+  if (!poisoned && amax_b != 0.0f) {
+    c0 = c0_from_thresholds(thr, amax_b, inv6g);
+    if (NC == 1) {
+      const int c = c0 + p.f_lo;
+      if (c >= 1 && c <= 126 && tab[c].r != 0.0f) {
+        fstar = p.f_lo;
+        if (WANT_SSE) sse = block_sse_def_pairs(x2, tab[c].d, tab[c].r);
+      }
+    } else if (!search_fast<NC, WANT_SSE>(x2, amax_b, c0, p.f_lo, tab, fstar, sse)) {
+      return true;
+    }
+  }
+  write_block<WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  return false;
+}
+
+// The definition for one block (deferred blocks): same outputs, every candidate scored in order.
+template <int DT, bool KV, bool ROT, bool WANT_SSE>
+__device__ __forceinline__ void quantize_block_def(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                                   float inv6g, bool g_bad, int64_t b, const char* src, bool v8) {
+  u64 x2[8];
+  load_pairs<DT>(src, v8, x2);
+  maybe_rotate<ROT>(x2);
+  const float amax_b = block_amax_nan(x2);
+  const bool poisoned = g_bad || !(amax_b <= FLT_MAX);
+  int c0 = 0, fstar = -128;
+  float sse = 0.0f;
+  if (!poisoned && amax_b != 0.0f) {
+    c0 = c0_from_thresholds(thr, amax_b, inv6g);
+    float x[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
+    search_def(x, c0, p.f_lo, p.f_hi, tab, fstar, sse);
+  }
+  write_block<WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
 }
 
 template <int DT, bool KV>
@@ -379,12 +434,19 @@ __device__ __forceinline__ const char* block_src(const QuantParams& p, int64_t b
   return p.x + elem * ES;
 }
 
-// One thread per 16-element block, grid-stride, with the next block's loads in flight while the
-// current block is searched.
+// One thread per 16-element block, grid-stride in warp-uniform rounds, the next block's loads in flight
+// while the current one is searched.  Blocks the fast score cannot decide are queued per warp (ballot)
+// and scored with the definition 32 at a time, one per lane, so a rare block does not stall its warp.
+constexpr int kDeferCap = 64;
+#ifndef NVFP4_SEARCH_CTAS_PER_SM
+#define NVFP4_SEARCH_CTAS_PER_SM 2
+#endif
+
 template <int DT, bool KV, bool ROT, int NC, bool WANT_SSE>
-__global__ void __launch_bounds__(256, 3) quantize_search_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search_kernel(QuantParams p) {
   __shared__ CandEntry tab[128];
   __shared__ float thr[128];
+  __shared__ int64_t defer[8][kDeferCap];
   float g = *p.g_src;
   if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
   const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
@@ -393,17 +455,44 @@ __global__ void __launch_bounds__(256, 3) quantize_search_kernel(QuantParams p) 
   __syncthreads();
   const float inv6g = __frcp_rn(__fmul_rn(6.0f, g));
 
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lanes_below = (1u << lane) - 1u;
+  int64_t* dlist = defer[warp];
+  int dcount = 0;  // warp-uniform
+  auto flush = [&]() {
+    __syncwarp();
+    for (int e = lane; e < dcount; e += 32) {
+      const int64_t bd = dlist[e];
+      quantize_block_def<DT, KV, ROT, WANT_SSE>(p, tab, thr, inv6g, g_bad, bd, block_src<DT, KV>(p, bd), p.v8 != 0);
+    }
+    __syncwarp();
+    dcount = 0;
+  };
+
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const bool v8 = p.v8 != 0;
   int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  float xn[16];
-  if (b < p.nblocks) load_block<DT>(block_src<DT, KV>(p, b), v8, xn);
-  for (; b < p.nblocks; b += stride) {
-    float x[16];
+  const int64_t warp0 = b - lane;
+  u64 xn[8];
+  if (b < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b), v8, xn);
+  for (int64_t wb = warp0; wb < p.nblocks; wb += stride, b += stride) {
+    const bool active = b < p.nblocks;
+    u64 x2[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = xn[i];
-    if (b + stride < p.nblocks) load_block<DT>(block_src<DT, KV>(p, b + stride), v8, xn);
-    quantize_one_block<DT, KV, ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x);
+    for (int k = 0; k < 8; ++k) x2[k] = xn[k];
+    if (b + stride < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b + stride), v8, xn);
+    const bool deferred = active && quantize_block_fast<ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
+    if constexpr (NC > 1) {  // a single-offset window never needs the definition pass
+      const unsigned m = __ballot_sync(0xFFFFFFFFu, deferred);
+      if (m) {
+        if (deferred) dlist[dcount + __popc(m & lanes_below)] = b;
+        dcount += __popc(m);
+        if (dcount > kDeferCap - 32) flush();
+      }
+    }
+  }
+  if constexpr (NC > 1) {
+    if (dcount) flush();
   }
 }
 
