@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time the eager step only (no CUDA graph replay)")
     return ap.parse_args()
 
 
@@ -145,6 +146,12 @@ def oracle_sample(name: str, elems: int):
     from nvfp4_block_scaled_11_b200 import workloads as W
     if name == "stream_f32":
         x = W.stream_f32("cpu", elems / float(1 << 30))
+    elif name == "kv_bf16":
+        import numpy as np
+        import torch
+        T = max(64, elems // 128)
+        k = W.kv_bf16("cpu", scale=T / 32768, heads=1)
+        return k.view(torch.int16).numpy().view(np.uint16), "kv", k.numel()
     else:
         w = W.make(name, "cpu")
         x = w.x.reshape(-1)[:elems].contiguous()
@@ -158,6 +165,10 @@ def oracle_sample(name: str, elems: int):
 
 def oracle_step(xs, code, f_lo, f_hi):
     from oracle import oracle as O
+    if code == "kv":
+        _, _, c, s, g = O.kv_mixed(xs, 16, 16, 1, f_lo, f_hi)
+        O.dequantize(c.reshape(-1), s.reshape(-1), g, 1)
+        return
     c, s, g, _, _ = O.quantize(xs, f_lo, f_hi, dtype=code)
     O.dequantize(c, s, g, 0)
 
@@ -201,13 +212,26 @@ def run_reference(args, rank, world):
 
 
 def workload_config(args):
-    full = args.workload == "stream_f32" and args.scale == 1.0
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    notes = {
+        "stream_f32": "FP32 2^30 = 4 GiB, 0.9 N(0,1) + 0.1 N(0,16), seed 3",
+        "act_f32": "FP32 [1024,4096] N(0,1), seed 0",
+        "act_bf16": "BF16 [8192,8192] 0.5*t(3), 1% outlier columns x20, seed 1",
+        "kv_bf16": "BF16 K [1,8,32768,128], N(0,1) + N(0,2) bias on 4 channels, seed 2",
+        "bev_f16": "FP16 [6,30825,8,32] N(0,1) x level gain 1,2,4,8, seed 5",
+    }
+    big = args.workload == "stream_f32"
+    name = f"{args.workload} ({notes.get(args.workload, '')})"
+    if args.scale != 1.0:
+        name += f" scaled by {args.scale}"
     return {
-        "workload": f"{args.workload}" + (" (FP32 2^30 = 4 GiB, 0.9 N(0,1) + 0.1 N(0,16), seed 3)" if full
-                                            else f" scaled by {args.scale}"),
+        "workload": name,
         "window": [args.f_lo, args.f_hi],
-        "step": "amax + [allreduce max] + g + ScaleSearch quantize + dequantize FP32",
-        "l2": "inputs larger than L2 (4 GiB per step per GPU), no flush",
+        "step": ("kv_mixed (sink/recent copy + FWHT-16 + amax + ScaleSearch) + dequantize BF16"
+                 if args.workload == "kv_bf16" else
+                 "amax + [allreduce max] + g + ScaleSearch quantize + dequantize"),
+        "l2": ("inputs larger than L2 (4 GiB per step per GPU), no flush" if big and args.scale == 1.0 else
+               "L2 flushed between steps by a 256 MiB write (not timed)"),
         "block": 16,
     }
 
@@ -238,34 +262,49 @@ def main():
                                 device_id=dev)
 
     w = W.make(args.workload, dev, args.scale, shard=rank)
-    if w.kind != "quantize":
-        raise SystemExit("bench.py times quantize workloads; kv_bf16 is covered by the parity tests")
-    x = w.x.reshape(-1).contiguous()
+    x = w.x.contiguous()
     n = x.numel()
     esz = x.element_size()
+    kv = w.kind == "kv"
     torch.cuda.synchronize()
 
     amax = torch.empty(1, dtype=torch.float32, device=dev)
     g = torch.empty(1, dtype=torch.float32, device=dev)
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
-    scales = torch.empty(n // 16, dtype=torch.uint8, device=dev)
-    deq = torch.empty(n, dtype=torch.float32, device=dev)
+    if kv:
+        B, H, T, D = x.shape
+        n_q = B * H * (T - 32) * D          # quantized middle tokens
+        deq = torch.empty(n_q, dtype=torch.bfloat16, device=dev)
+    else:
+        x = x.reshape(-1)
+        n_q = n
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(n // 16, dtype=torch.uint8, device=dev)
+        deq = torch.empty(n, dtype=x.dtype, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # inputs that fit in L2 are evicted between timed steps by writing a 256 MiB buffer (not timed)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if n * esz < (512 << 20) else None
 
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        nv.tensor_amax(x, out=amax)
-        if world > 1:
-            dist.all_reduce(amax, op=dist.ReduceOp.MAX)
-        nv.global_scale(amax, out=g)
-        if evs:
-            evs[1].record(stream)
-        nv.quantize_ex(x, args.f_lo, args.f_hi, gscale_in=g, want_f=False, want_sse=False, codes=codes,
-                       scales=scales, gscale=None)
-        if evs:
-            evs[2].record(stream)
-        nv.dequantize(codes, scales, g, torch.float32, out=deq)
+        if kv:
+            _, _, kc, ks, kg = nv.kv_mixed(x, 16, 16, True, args.f_lo, args.f_hi)
+            if evs:
+                evs[1].record(stream)
+                evs[2].record(stream)
+            nv.dequantize(kc.reshape(-1), ks.reshape(-1), kg, torch.bfloat16, out=deq)
+        else:
+            nv.tensor_amax(x, out=amax)
+            if world > 1:
+                dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+            nv.global_scale(amax, out=g)
+            if evs:
+                evs[1].record(stream)
+            nv.quantize_ex(x, args.f_lo, args.f_hi, gscale_in=g, want_f=False, want_sse=False, codes=codes,
+                           scales=scales, gscale=None)
+            if evs:
+                evs[2].record(stream)
+            nv.dequantize(codes, scales, g, deq.dtype, out=deq)
         if evs:
             evs[3].record(stream)
 
@@ -285,13 +324,51 @@ def main():
         dist.barrier()
     t0.record(stream)
     for k in range(args.steps):
+        if flush is not None:
+            flush.fill_(float(k))
         step(evs[k])
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    elapsed_ms = t0.elapsed_time(t1)
+    if flush is None:
+        elapsed_ms = t0.elapsed_time(t1)
+    else:  # the flushes are not part of the step
+        elapsed_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    eager_ms = elapsed_ms
+    graph_used = False
+    if world == 1 and not args.no_graph:
+        # the same step captured once as a CUDA graph and replayed: removes the host launch latency
+        # that dominates the small configurations (the per-stage breakdown stays the eager one)
+        cg = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()  # warm the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(cg, stream=side):
+            step()
+        for _ in range(max(1, args.warmup)):
+            cg.replay()
+        torch.cuda.synchronize()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        ga = torch.cuda.Event(enable_timing=True)
+        gb = torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for k in range(args.steps):
+            if flush is not None:
+                flush.fill_(float(-k))
+            gev[k][0].record(stream)
+            cg.replay()
+            gev[k][1].record(stream)
+        gb.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ga.elapsed_time(gb) if flush is None else sum(a.elapsed_time(b) for a, b in gev)
+        del cg
+        if graph_ms < elapsed_ms:
+            elapsed_ms = graph_ms
+            graph_used = True
     amax_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     q_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     dq_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -303,31 +380,39 @@ def main():
     bytes_in = n * esz
     value = world * bytes_in * args.steps / (elapsed_ms * 1e-3) / 1e9
     peak, peak_src = peaks()
-    q_bytes = n * esz + n // 2 + n // 16          # search pass: read x, write codes + scales
-    two_pass_bytes = 2 * n * esz + n // 2 + n // 16
-    dq_bytes = n // 2 + n // 16 + 4 * n
-    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    q_bytes = n_q * esz + n_q // 2 + n_q // 16          # search pass: read x, write codes + scales
+    two_pass_bytes = 2 * n_q * esz + n_q // 2 + n_q // 16
+    dq_bytes = n_q // 2 + n_q // 16 + deq.element_size() * n_q
+    if kv:
+        # one fused call: copies + rotated amax + rotated search; report the call against its bytes
+        q_ms = amax_ms + q_ms
+        amax_ms = 0.0
+    q_gbs = (two_pass_bytes if kv else q_bytes) / (q_ms * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
         "config": workload_config(args),
-        "roofline": {"bound": "hbm", "kernel": "quantize (ScaleSearch search + encode pass)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "kv_mixed (amax + search passes)" if kv else
+                     "quantize (ScaleSearch search + encode pass)",
                      "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
                      "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0>", n)
-                     if (x.dtype == torch.float32 and (args.f_lo, args.f_hi) == (-2, 6)) else None,
+                     if (not kv and x.dtype == torch.float32 and (args.f_lo, args.f_hi) == (-2, 6)) else None,
                      "peak_source": peak_src,
-                     "bytes_per_launch": q_bytes},
+                     "bytes_per_launch": two_pass_bytes if kv else q_bytes},
         "breakdown_ms": {"amax_and_g": amax_ms, "quantize": q_ms, "dequantize": dq_ms},
-        "quantize_two_pass": {"gbs_input": bytes_in / ((amax_ms + q_ms) * 1e-3) / 1e9,
+        "quantize_two_pass": {"gbs_input": n_q * esz / ((amax_ms + q_ms) * 1e-3) / 1e9,
                               "gbs_moved": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 1e9,
                               "frac_of_8TBs": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 8e12},
         "dequantize": {"gbs_moved": dq_bytes / (dq_ms * 1e-3) / 1e9},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (5 if kv else 4) * args.steps,
         "clocks": clocks,
+        "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / args.steps},
     }
-
+    if kv:
+        args.no_e2e = True
     # end to end through the public API with host buffers: pinned H2D of the input, the step, and a
     # D2H read of the quantized result (codes, scales, g) every step.
     if not args.no_e2e and args.e2e_steps > 0:
