@@ -328,8 +328,13 @@ __global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict_
       uint32_t w[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(a[i]);
+      if (v8_out) {
+        st_v8(o, static_cast<const uint32_t*>(w));
+        st_v8(o + 32, w + 8);
+      } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
+        for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
+      }
     } else {
       uint32_t w[8];
 #pragma unroll
@@ -342,8 +347,12 @@ __global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict_
           w[k] = *reinterpret_cast<uint32_t*>(&h);
         }
       }
-      st_v4(o, w);
-      st_v4(o + 16, w + 4);
+      if (v8_out) {
+        st_v8(o, w);
+      } else {
+        st_v4(o, w);
+        st_v4(o + 16, w + 4);
+      }
     }
   }
 }
