@@ -136,31 +136,43 @@ __device__ __forceinline__ void build_cand_entries(CandEntry* t, float g) {
 }
 
 // Default code c0(a) = E4M3(fl(fl(a / 6) / g)) of a block with amax a > 0.  c0 is non-decreasing in a,
-// so it is fixed by the thresholds T[k] = min{a : c0(a) >= k}: c0(a) = max{k : T[k] <= a}.  Each
-// threshold is found once per CTA by bisection over the bit patterns of non-negative floats (their
-// integer order is their numeric order), evaluating c0 exactly as defined; T[0] = 0, T[127] = +Inf.
+// so it is fixed by the thresholds T[k] = min{a : c0(a) >= k}: c0(a) = max{k : T[k] <= a}; T[0] = 0,
+// T[127] = +Inf.  The E4M3 rounding boundary below code k is the midpoint m_k of the values of codes k-1
+// and k, so T[k] lies within a few ulps of fl(fl(m_k g) 6): a short walk over neighbouring floats,
+// evaluating c0 exactly as defined, stops at the float a with c0(a) >= k > c0(a - 1ulp), which is T[k]
+// (the bit patterns of non-negative floats are ordered like their values).  When the estimate is not
+// a positive finite float, or the walk needs more than a few steps (extreme g), bisection over the
+// whole float range finds the same threshold.
 __device__ __forceinline__ int c0_exact(float a, float g) {
   return a == 0.0f ? 0 : e4m3_code(__fdiv_rn(__fdiv_rn(a, 6.0f), g));
 }
 
-__device__ __forceinline__ void build_c0_thresholds(float* T, float g) {
-  for (int k = threadIdx.x; k < 128; k += blockDim.x) {
-    float t;
-    if (k == 0) {
-      t = 0.0f;
-    } else if (k == 127) {
-      t = __uint_as_float(0x7F800000u);
-    } else {
-      uint32_t lo = 0u, hi = 0x7F800000u;  // c0(lo) < k <= c0(hi)
-      while (hi - lo > 1u) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (c0_exact(__uint_as_float(mid), g) >= k) hi = mid;
-        else lo = mid;
+__device__ __forceinline__ float c0_threshold(int k, float g) {
+  const float m = __fmul_rn(0.5f, __fadd_rn(e4m3_value((uint32_t)(k - 1)), e4m3_value((uint32_t)k)));
+  const float a0 = __fmul_rn(__fmul_rn(m, g), 6.0f);
+  if (a0 > 0.0f && a0 <= FLT_MAX) {
+    uint32_t u = __float_as_uint(a0);
+    for (int it = 0; it < 8; ++it) {
+      if (c0_exact(__uint_as_float(u), g) >= k) {
+        if (u == 0u || c0_exact(__uint_as_float(u - 1u), g) < k) return __uint_as_float(u);
+        --u;
+      } else {
+        ++u;
       }
-      t = __uint_as_float(hi);
     }
-    T[k] = t;
   }
+  uint32_t lo = 0u, hi = 0x7F800000u;  // c0(lo) < k <= c0(hi)
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    if (c0_exact(__uint_as_float(mid), g) >= k) hi = mid;
+    else lo = mid;
+  }
+  return __uint_as_float(hi);
+}
+
+__device__ __forceinline__ void build_c0_thresholds(float* T, float g) {
+  for (int k = threadIdx.x; k < 128; k += blockDim.x)
+    T[k] = k == 0 ? 0.0f : (k == 127 ? __uint_as_float(0x7F800000u) : c0_threshold(k, g));
 }
 
 // c0 of a finite a > 0 from the thresholds: a close first guess from one multiply, then exact steps.
