@@ -431,3 +431,24 @@ void ref_f32_to_f16_n(const float* v, int64_t n, uint16_t* out) {
 void ref_f16_to_f32_n(const uint16_t* h, int64_t n, float* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = ref_f16_to_f32(h[i]);
 }
+
+/* ---- tensor-core consumer layout of the block scales (see the header) ---- */
+int64_t ref_sf_mma_bytes(int64_t rows, int64_t bpr) {
+  const int64_t row_tiles = (rows + 127) / 128, col_tiles = (bpr + 3) / 4;
+  return row_tiles * col_tiles * 512;
+}
+
+int64_t ref_sf_mma_offset(int64_t r, int64_t c, int64_t bpr) {
+  const int64_t col_tiles = (bpr + 3) / 4;
+  const int64_t tile = (r / 128) * col_tiles + c / 4;   /* column tiles of a row tile are consecutive */
+  const int64_t rr = r % 128, cc = c % 4;
+  return tile * 512 + 16 * (rr % 32) + 4 * (rr / 32) + cc;
+}
+
+void ref_scales_to_mma(const uint8_t* lin, int64_t batch, int64_t rows, int64_t bpr, uint8_t* out) {
+  const int64_t per = ref_sf_mma_bytes(rows, bpr);
+  for (int64_t i = 0; i < batch * per; ++i) out[i] = 0;
+  for (int64_t l = 0; l < batch; ++l)
+    for (int64_t r = 0; r < rows; ++r)
+      for (int64_t c = 0; c < bpr; ++c) out[l * per + ref_sf_mma_offset(r, c, bpr)] = lin[(l * rows + r) * bpr + c];
+}

@@ -22,7 +22,9 @@
  *
  * Parity status: every function below is pinned by the not-gpu tests (library converters,
  * brute-force search, closed forms, invariants); the exact f* histogram shape on Gaussian data is
- * qualitative on the pages (bimodal) and is "parity unpinned" beyond that shape.
+ * qualitative on the pages (bimodal) and is "parity unpinned" beyond that shape.  The block-scale tile
+ * layout is pinned by an independent reshape construction of the documented tile array, hand-checked
+ * offsets, padding and bijectivity; the NVFP4 product (oracle.py) by exact rational arithmetic.
  */
 #ifndef NVFP4_REF_H
 #define NVFP4_REF_H
@@ -95,6 +97,20 @@ void ref_fwht16_f32(float* a);
 int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, int sink, int recent,
                  int rotate, int f_lo, int f_hi, uint16_t* sink_out, uint16_t* recent_out,
                  uint8_t* codes, uint8_t* scales, float* gscale_out);
+
+/* ---- tensor-core consumer layout of the block scales ----
+ * [SS] ScaleSearchAttention runs QK^T and PV as NVFP4 products on the tensor cores with FP32
+ * accumulation.  The pages do not describe how the tensor cores read the block scales; this follows
+ * NVIDIA's public description of the block-scaled MMA operands (PTX ISA, tcgen05 block scaling; cuBLAS
+ * "1D block scaling factors layout"): a scale matrix of `rows` rows and `bpr` 16-element blocks per row
+ * is cut into tiles of 128 rows x 4 block columns (512 bytes; rows padded to 128, columns to 4).
+ * Tiles are stored row tile by row tile, the column tiles of one row tile consecutively.  Inside a
+ * tile, the scale of row r and column c is byte 16 * (r mod 32) + 4 * (r div 32) + c.
+ * Padding bytes are zero.  A batch of matrices stores its tiles matrix after matrix. */
+int64_t ref_sf_mma_bytes(int64_t rows, int64_t bpr);                  /* one matrix, padded */
+int64_t ref_sf_mma_offset(int64_t r, int64_t c, int64_t bpr);        /* byte of (row r, block c) */
+/* scales in row-major [batch, rows, bpr] order -> the tile layout (out: batch * ref_sf_mma_bytes) */
+void ref_scales_to_mma(const uint8_t* lin, int64_t batch, int64_t rows, int64_t bpr, uint8_t* out);
 
 #ifdef __cplusplus
 }

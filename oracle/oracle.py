@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
             "ref_hadamard16": (I, [P, I64, I, P, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+            "ref_sf_mma_bytes": (I64, [I64, I64]),
+            "ref_sf_mma_offset": (I64, [I64, I64, I64]),
+            "ref_scales_to_mma": (None, [P, I64, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -224,3 +227,75 @@ def kv_mixed(k_bf16: np.ndarray, sink: int = 16, recent: int = 16, rotate: int =
     if rc != 0:
         raise ValueError(f"ref_kv_mixed returned {rc}")
     return so, ro, codes, scales, g[0]
+
+
+# ---- tensor-core consumer: block-scale tile layout and the NVFP4 product ----
+def sf_mma_bytes(rows: int, bpr: int) -> int:
+    """Bytes of one [rows, bpr] scale matrix in the 128x4 tile layout (padded)."""
+    return int(lib().ref_sf_mma_bytes(rows, bpr))
+
+
+def sf_mma_offset(r: int, c: int, bpr: int) -> int:
+    return int(lib().ref_sf_mma_offset(r, c, bpr))
+
+
+def scales_to_mma(scales: np.ndarray, batch: int, rows: int, bpr: int) -> np.ndarray:
+    """Row-major [batch, rows, bpr] scale bytes -> the tile layout (padding zero)."""
+    lin = np.ascontiguousarray(scales, np.uint8).reshape(-1)
+    if lin.size != batch * rows * bpr:
+        raise ValueError("scales size does not match batch * rows * bpr")
+    out = np.empty(batch * sf_mma_bytes(rows, bpr), np.uint8)
+    lib().ref_scales_to_mma(_p(lin), batch, rows, bpr, _p(out))
+    return out
+
+
+def quantize_mma(x: np.ndarray, f_lo: int = -2, f_hi: int = 6, dtype: int | None = None, gscale_in=None):
+    """Quantize x [batch, rows, cols] (or [rows, cols]) along cols; scales in the tile layout.
+
+    Returns (codes [batch*rows*cols/2], sf_mma, g)."""
+    if x.ndim == 2:
+        x = x[None]
+    batch, rows, cols = x.shape
+    codes, scales, g, _, _ = quantize(x.reshape(-1), f_lo, f_hi, dtype, gscale_in)
+    return codes, scales_to_mma(scales, batch, rows, cols // 16), g
+
+
+_E2M1_TAB = None
+_E4M3_TAB = None
+
+
+def _tables():
+    global _E2M1_TAB, _E4M3_TAB
+    if _E2M1_TAB is None:
+        _E2M1_TAB = np.array([e2m1_decode(c) for c in range(16)], np.float64)
+        _E4M3_TAB = np.array([e4m3_decode(c) for c in range(256)], np.float64)
+    return _E2M1_TAB, _E4M3_TAB
+
+
+def block_values(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Exact real values E2M1(q) * E4M3(s) (without the tensor scale) of a [rows, cols] matrix, fp64."""
+    t2, t4 = _tables()
+    c = np.ascontiguousarray(codes, np.uint8).reshape(rows, cols // 2)
+    q = np.empty((rows, cols), np.uint8)
+    q[:, 0::2] = c & 15      # element 2k: low nibble
+    q[:, 1::2] = c >> 4      # element 2k+1: high nibble
+    sv = t4[np.ascontiguousarray(scales, np.uint8).reshape(rows, cols // 16)]
+    return t2[q] * np.repeat(sv, 16, axis=1)
+
+
+def gemm_nt(a_codes, a_scales, g_a, b_codes, b_scales, g_b, M: int, N: int, K: int, alpha: float = 1.0,
+            batch: int = 1) -> np.ndarray:
+    """D[l] = alpha * g_a * g_b * A[l] B[l]^T in fp64 from row-major codes and row-major (linear) scales.
+
+    Each product of two E2M1 values and two E4M3 scales is exact in fp64; the sums are a library matmul."""
+    A = np.ascontiguousarray(a_codes).reshape(batch, -1)
+    As = np.ascontiguousarray(a_scales).reshape(batch, -1)
+    B = np.ascontiguousarray(b_codes).reshape(batch, -1)
+    Bs = np.ascontiguousarray(b_scales).reshape(batch, -1)
+    out = np.empty((batch, M, N), np.float64)
+    scale = float(alpha) * float(g_a) * float(g_b)
+    for l in range(batch):
+        av = block_values(A[l], As[l], M, K)
+        bv = block_values(B[l], Bs[l], N, K)
+        out[l] = (av @ bv.T) * scale
+    return out
