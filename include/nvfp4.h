@@ -108,6 +108,55 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
+/* ---- Tensor-core consumer ("Search your block floating-point scales!", ScaleSearchAttention: QK^T and
+ * PV run as NVFP4 products on the tensor cores with FP32 accumulation) ----
+ *
+ * Scale tile layout.  The block-scaled tensor-core MMA reads block scales in NVIDIA's documented tile
+ * format (PTX ISA, tcgen05 block scaling; not described on the pages): a matrix of `rows` rows with
+ * `cols` / 16 blocks per row is cut into 512-byte tiles of 128 rows x 4 block columns (rows padded to a
+ * multiple of 128, block columns to a multiple of 4, padding bytes zero).  Tiles are stored row tile
+ * by row tile, the column tiles of one row tile consecutively; inside a tile the scale of row r and
+ * block column c is byte 16 * (r mod 32) + 4 * (r div 32) + c.  A batch stores its matrices one after
+ * another.  The codes keep the row-major packed layout of nvfp4_quantize. */
+
+/* Bytes of the tile-layout scales of `batch` matrices of [rows, cols] (cols % 16 == 0); negative status
+ * on invalid sizes. */
+int64_t nvfp4_sf_mma_bytes(int64_t rows, int64_t cols, int64_t batch);
+
+/* nvfp4_quantize_ex for x [batch, rows, cols] (contiguous, blocks along cols, cols % 16 == 0) with the
+ * scales written in the tile layout: sf receives nvfp4_sf_mma_bytes(rows, cols, batch) bytes.
+ * gscale_in / gscale as in nvfp4_quantize_ex (one tensor scale for the whole batch).
+ * The whole tensor must hold fewer than 2^32 blocks (NVFP4_ERR_SIZE otherwise). */
+int nvfp4_quantize_mma(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
+                       const float* gscale_in, uint8_t* codes, uint8_t* sf, float* gscale, void* stream);
+
+/* nvfp4_kv_mixed with the middle-token scales in the tile layout: each (batch, head) is one
+ * [T_mid, D] matrix, so sf receives nvfp4_sf_mma_bytes(T_mid, D, B * H) bytes; it feeds
+ * nvfp4_gemm_nt as the K operand of Q K^T directly. */
+int nvfp4_kv_mixed_mma(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                       int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                       uint8_t* codes, uint8_t* sf, float* gscale, void* stream);
+
+/* Batched NVFP4 product on the tensor cores:
+ *   D[l][m][n] = alpha * g_a * g_b * sum_k A[l][m][k] * B[l][n][k]     (FP32 accumulation)
+ * where A[l][m][k] = E2M1(a code) * E4M3(a scale) is operand A before its tensor scale (likewise B).
+ * a_codes: [batch, M, K/2] packed codes (nvfp4_quantize_mma of a [batch, M, K] tensor), a_sf its tile
+ * layout scales, a_gscale its device tensor scale; b_* likewise for [batch, N, K].
+ * d: [batch, M, N] row-major, d_dtype NVFP4_F32 or NVFP4_BF16 (RNE from FP32).
+ * alpha_work: one device float owned by the caller; it receives fl(fl(alpha * g_a) * g_b), which the
+ * epilogue multiplies in, so it must not be shared with a concurrent call on another stream.
+ * Requirements: K % 32 == 0 (NVFP4_ERR_SIZE); codes, scales and d 16-byte aligned and N * sizeof(d
+ * element) a multiple of 16 (NVFP4_ERR_ALIGN); all sizes below 2^31.  K == 0 writes zeros.
+ * A scale byte 0x7F (a poisoned block) makes the outputs that use it NaN. */
+int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gscale, const uint8_t* b_codes,
+                  const uint8_t* b_sf, const float* b_gscale, int64_t batch, int64_t M, int64_t N, int64_t K,
+                  float alpha, void* d, int d_dtype, float* alpha_work, void* stream);
+
+/* Host only, for verification: the byte offsets at which nvfp4_gemm_nt reads the scale of (matrix l,
+ * row r, block column c), for l < batch, r < rows, c < K/16 in that (row-major) order, into out
+ * (batch * rows * K/16 entries).  No device work. */
+int nvfp4_gemm_sf_offsets(int64_t rows, int64_t K, int64_t batch, int64_t* out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,7 +16,8 @@ import torch
 
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
-    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE",
+    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "kv_mixed_mma",
+    "gemm_nt", "gemm_sf_offsets",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -37,6 +38,11 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_sf_mma_bytes": (_I64, [_I64, _I64, _I64]),
+    "nvfp4_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "nvfp4_kv_mixed_mma": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_gemm_nt": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P, _P]),
+    "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),
 }
 
 
@@ -193,3 +199,88 @@ def kv_mixed(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = T
     _check(lib().nvfp4_kv_mixed(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), f_lo, f_hi, _ptr(so),
                                 _ptr(ro), _ptr(codes), _ptr(scales), _ptr(gscale), _stream(k)))
     return so, ro, codes, scales, gscale
+
+
+# ---- tensor-core consumer: scales in the MMA tile layout, NVFP4 x NVFP4 product ----
+def sf_mma_bytes(rows: int, cols: int, batch: int = 1) -> int:
+    """Bytes of the tile-layout scales of `batch` [rows, cols] matrices (padded to 128 rows x 4 blocks)."""
+    nb = lib().nvfp4_sf_mma_bytes(rows, cols, batch)
+    if nb < 0:
+        raise NVFP4Error(int(nb))
+    return int(nb)
+
+
+def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None):
+    """Quantize x [rows, cols] or [batch, rows, cols] along cols with the scales in the tensor-core tile
+    layout.  Returns (codes uint8[..., rows, cols/2] (x's rank), sf uint8[sf_mma_bytes], gscale float32[1])."""
+    _cuda(x, "x")
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be [rows, cols] or [batch, rows, cols]")
+    batch, rows, cols = (1, *x.shape) if x.dim() == 2 else x.shape
+    dev = x.device
+    codes = torch.empty((*x.shape[:-1], cols // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(sf_mma_bytes(rows, cols, batch), dtype=torch.uint8, device=dev)
+    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    if gscale_in is not None:
+        _cuda(gscale_in, "gscale_in")
+    _check(lib().nvfp4_quantize_mma(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
+                                    _ptr(sf), _ptr(gscale), _stream(x)))
+    return codes, sf, gscale
+
+
+def kv_mixed_mma(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = True, f_lo: int = -2,
+                 f_hi: int = 6):
+    """kv_mixed with the middle-token scales of every (batch, head) in the tensor-core tile layout.
+
+    Returns (sink, recent, codes uint8[B,H,Tm,D/2], sf uint8[sf_mma_bytes(Tm, D, B*H)], gscale)."""
+    _cuda(k, "k")
+    if k.dtype != torch.bfloat16 or k.dim() != 4:
+        raise TypeError("k must be a 4-D bfloat16 tensor [B,H,T,D]")
+    B, H, T, D = k.shape
+    Tm = max(T - sink - recent, 0)
+    dev = k.device
+    so = torch.empty((B, H, sink, D), dtype=torch.bfloat16, device=dev)
+    ro = torch.empty((B, H, recent, D), dtype=torch.bfloat16, device=dev)
+    codes = torch.empty((B, H, Tm, D // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(max(sf_mma_bytes(Tm, D, B * H), 1), dtype=torch.uint8, device=dev)
+    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(lib().nvfp4_kv_mixed_mma(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), f_lo, f_hi, _ptr(so),
+                                    _ptr(ro), _ptr(codes), _ptr(sf), _ptr(gscale), _stream(k)))
+    return so, ro, codes, sf, gscale
+
+
+def gemm_nt(a_codes: torch.Tensor, a_sf: torch.Tensor, a_gscale: torch.Tensor, b_codes: torch.Tensor,
+            b_sf: torch.Tensor, b_gscale: torch.Tensor, alpha: float = 1.0, out_dtype=torch.float32,
+            out: torch.Tensor | None = None, alpha_work: torch.Tensor | None = None) -> torch.Tensor:
+    """D[l] = alpha * g_a * g_b * A[l] B[l]^T on the tensor cores (FP32 accumulation).
+
+    a_codes: uint8 [M, K/2] or [batch, M, K/2] (quantize_mma output), b_codes: [.., N, K/2] likewise;
+    returns D [M, N] or [batch, M, N] in out_dtype (float32 or bfloat16)."""
+    for t, nm in ((a_codes, "a_codes"), (a_sf, "a_sf"), (a_gscale, "a_gscale"), (b_codes, "b_codes"),
+                  (b_sf, "b_sf"), (b_gscale, "b_gscale")):
+        _cuda(t, nm)
+    squeeze = a_codes.dim() == 2
+    a3 = a_codes if a_codes.dim() == 3 else a_codes.unsqueeze(0)
+    b3 = b_codes if b_codes.dim() == 3 else b_codes.unsqueeze(0)
+    batch, M, K2 = a3.shape
+    if b3.shape[0] != batch or b3.shape[2] != K2:
+        raise ValueError("a_codes and b_codes disagree on batch or K")
+    N, K = b3.shape[1], 2 * K2
+    dev = a_codes.device
+    if out is None:
+        out = torch.empty((batch, M, N), dtype=out_dtype, device=dev)
+    _cuda(out, "out")
+    if alpha_work is None:
+        alpha_work = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(lib().nvfp4_gemm_nt(_ptr(a_codes), _ptr(a_sf), _ptr(a_gscale), _ptr(b_codes), _ptr(b_sf), _ptr(b_gscale),
+                               batch, M, N, K, float(alpha), _ptr(out), DTYPE_CODE[out.dtype], _ptr(alpha_work),
+                               _stream(a_codes)))
+    return out[0] if squeeze and out.dim() == 3 else out
+
+
+def gemm_sf_offsets(rows: int, K: int, batch: int = 1):
+    """Host-side: byte offsets at which gemm_nt reads scale (l, r, c), as a numpy int64 array."""
+    import numpy as np
+    out = np.empty(batch * rows * (K // 16), np.int64)
+    _check(lib().nvfp4_gemm_sf_offsets(rows, K, batch, out.ctypes.data))
+    return out

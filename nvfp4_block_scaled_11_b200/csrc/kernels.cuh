@@ -122,7 +122,23 @@ struct QuantParams {
   int v8;              // input base is 32-byte aligned
   // mixed KV layout: blocks run over the middle tokens of K[BH, T, D]
   int64_t T, Tm, sink, D, bpr;  // bpr = D / 16
+  // scales in the tensor-core tile layout when sf_bpr > 0: the blocks form matrices of sf_rows rows and
+  // sf_bpr blocks per row (fewer than 2^32 blocks in all); each matrix's scales take sf_mat_bytes bytes
+  uint32_t sf_bpr, sf_rows, sf_ctiles;  // sf_ctiles = ceil(sf_bpr / 4)
+  int64_t sf_mat_bytes;
 };
+
+// Byte of block b's scale.  Linear: b.  Tile layout (block-scaled tensor-core MMA operand): 512-byte
+// tiles of 128 rows x 4 block columns, the column tiles of a row tile consecutive, and inside a tile
+// row r, column c at 16 * (r mod 32) + 4 * (r div 32) + c.
+__device__ __forceinline__ int64_t scale_index(const QuantParams& p, int64_t b) {
+  if (p.sf_bpr == 0u) return b;
+  const uint32_t ub = (uint32_t)b, per = p.sf_rows * p.sf_bpr;
+  const uint32_t mat = ub / per, rem = ub - mat * per;
+  const uint32_t r = rem / p.sf_bpr, c = rem - r * p.sf_bpr;
+  const uint32_t in_mat = ((r >> 7) * p.sf_ctiles + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u);
+  return (int64_t)mat * p.sf_mat_bytes + in_mat;
+}
 
 // Candidate table for one launch: d[c] = fl(E4M3(c) * g), r[c] = fl(1 / d[c]); r = 0 marks a code that
 // cannot be a scale (c outside 1..126, d == 0 or 1/d not finite).
@@ -246,7 +262,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
       }
     }
     reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(lo, hi);
-    p.scales[b] = (uint8_t)scale;
+    p.scales[scale_index(p, b)] = (uint8_t)scale;
     if (p.block_f) p.block_f[b] = (int8_t)fstar;
     if (p.block_sse) p.block_sse[b] = sse;
   }

@@ -112,6 +112,58 @@ int launch_quantize_t(int dtype, const QuantParams& p, cudaStream_t s) {
 
 int window_ok(int f_lo, int f_hi) { return f_lo <= f_hi && f_lo >= -126 && f_hi <= 126; }
 
+// Shared body of the quantize entry points; `sf` carries the tile-layout fields (sf.sf_bpr == 0: linear).
+int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const float* gscale_in, uint8_t* codes,
+                  uint8_t* scales, float* gscale, int8_t* block_f, float* block_sse, const QuantParams& sf,
+                  cudaStream_t s) {
+  if (!dtype_ok(dtype) || !window_ok(f_lo, f_hi)) return NVFP4_ERR_ARG;
+  if (gscale_in == nullptr && gscale == nullptr) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
+  if ((n > 0 && !aligned(x, 16)) || (n > 0 && !aligned(codes, 8)) || (gscale && !aligned(gscale, 4)) ||
+      (gscale_in && !aligned(gscale_in, 4)) || (block_sse && !aligned(block_sse, 4)))
+    return NVFP4_ERR_ALIGN;
+  QuantParams p{};
+  p.x = static_cast<const char*>(x);
+  p.nblocks = n / 16;
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.codes = codes;
+  p.scales = scales;
+  p.block_f = block_f;
+  p.block_sse = block_sse;
+  p.v8 = aligned(x, 32) ? 1 : 0;
+  p.sf_bpr = sf.sf_bpr;
+  p.sf_rows = sf.sf_rows;
+  p.sf_ctiles = sf.sf_ctiles;
+  p.sf_mat_bytes = sf.sf_mat_bytes;
+  if (gscale_in == nullptr) {
+    // gscale doubles as the amax accumulator: zero, reduce, quantize (reads it as amax), then g.
+    if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (n > 0) {
+      int rc = launch_amax(x, n, dtype, reinterpret_cast<uint32_t*>(gscale), s);
+      if (rc) return rc;
+      p.g_src = gscale;
+      p.g_is_amax = 1;
+      rc = launch_quantize_t<false, false>(dtype, p, s);
+      if (rc) return rc;
+    }
+    global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
+    if (int rc = last_error()) return rc;
+    return check_finite_sync(gscale, s);
+  }
+  p.g_src = gscale_in;
+  p.g_is_amax = 0;
+  if (n > 0) {
+    if (int rc = launch_quantize_t<false, false>(dtype, p, s)) return rc;
+  }
+  if (gscale && gscale != gscale_in) {
+    if (cudaMemcpyAsync(gscale, gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+  }
+  return check_finite_sync(gscale_in, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -150,49 +202,38 @@ int nvfp4_global_scale(const float* d_amax, float* d_gscale, void* stream) {
 int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi, const float* gscale_in,
                       uint8_t* codes, uint8_t* scales, float* gscale, int8_t* block_f, float* block_sse,
                       void* stream) {
-  if (!dtype_ok(dtype) || block != 16 || !window_ok(f_lo, f_hi)) return NVFP4_ERR_ARG;
-  if (gscale_in == nullptr && gscale == nullptr) return NVFP4_ERR_ARG;
-  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
-  if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
-  if ((n > 0 && !aligned(x, 16)) || (n > 0 && !aligned(codes, 8)) || (gscale && !aligned(gscale, 4)) ||
-      (gscale_in && !aligned(gscale_in, 4)) || (block_sse && !aligned(block_sse, 4)))
-    return NVFP4_ERR_ALIGN;
+  if (block != 16) return NVFP4_ERR_ARG;
+  return quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes, scales, gscale, block_f, block_sse, QuantParams{},
+                       S(stream));
+}
+
+int64_t nvfp4_sf_mma_bytes(int64_t rows, int64_t cols, int64_t batch) {
+  if (rows < 0 || cols < 0 || batch < 0) return NVFP4_ERR_ARG;
+  if (cols % 16 != 0) return NVFP4_ERR_SIZE;
+  return batch * ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
+}
+
+int nvfp4_quantize_mma(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
+                       const float* gscale_in, uint8_t* codes, uint8_t* sf, float* gscale, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_ARG;
+  if (cols % 16 != 0) return NVFP4_ERR_SIZE;
+  const int64_t n = batch * rows * cols;
+  if (n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (n > 0 && sf == nullptr) return NVFP4_ERR_ARG;
   cudaStream_t s = S(stream);
-  QuantParams p{};
-  p.x = static_cast<const char*>(x);
-  p.nblocks = n / 16;
-  p.f_lo = f_lo;
-  p.f_hi = f_hi;
-  p.codes = codes;
-  p.scales = scales;
-  p.block_f = block_f;
-  p.block_sse = block_sse;
-  p.v8 = aligned(x, 32) ? 1 : 0;
-  if (gscale_in == nullptr) {
-    // gscale doubles as the amax accumulator: zero, reduce, quantize (reads it as amax), then g.
-    if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (n > 0) {
-      int rc = launch_amax(x, n, dtype, reinterpret_cast<uint32_t*>(gscale), s);
-      if (rc) return rc;
-      p.g_src = gscale;
-      p.g_is_amax = 1;
-      rc = launch_quantize_t<false, false>(dtype, p, s);
-      if (rc) return rc;
-    }
-    global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
-    if (int rc = last_error()) return rc;
-    return check_finite_sync(gscale, s);
-  }
-  p.g_src = gscale_in;
-  p.g_is_amax = 0;
+  QuantParams lay{};
   if (n > 0) {
-    if (int rc = launch_quantize_t<false, false>(dtype, p, s)) return rc;
-  }
-  if (gscale && gscale != gscale_in) {
-    if (cudaMemcpyAsync(gscale, gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    const int64_t bpr = cols / 16;
+    lay.sf_bpr = (uint32_t)bpr;
+    lay.sf_rows = (uint32_t)rows;
+    lay.sf_ctiles = (uint32_t)((bpr + 3) / 4);
+    lay.sf_mat_bytes = ((rows + 127) / 128) * 128 * (int64_t)lay.sf_ctiles * 4;
+    // padding bytes (rows up to a multiple of 128, block columns up to a multiple of 4) must read as 0
+    if ((rows % 128 != 0 || bpr % 4 != 0) &&
+        cudaMemsetAsync(sf, 0, (size_t)(batch * lay.sf_mat_bytes), s) != cudaSuccess)
       return NVFP4_ERR_CUDA;
   }
-  return check_finite_sync(gscale_in, s);
+  return quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes, sf, gscale, nullptr, nullptr, lay, s);
 }
 
 int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi, uint8_t* codes,
@@ -253,9 +294,9 @@ int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dty
   return last_error();
 }
 
-int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
-                   int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
-                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
+static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                         int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                         uint8_t* codes, uint8_t* scales, float* gscale, bool mma, void* stream) {
   if (!window_ok(f_lo, f_hi) || gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
     return NVFP4_ERR_SIZE;
@@ -266,6 +307,7 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
   if (BH > 0 && sink_tokens > 0 && sink_bf16 == nullptr) return NVFP4_ERR_ARG;
   if (BH > 0 && recent_tokens > 0 && recent_bf16 == nullptr) return NVFP4_ERR_ARG;
   if (ngroups > 0 && (codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
+  if (mma && ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
   if ((BH > 0 && !aligned(k_bf16, 16)) || (sink_bf16 && !aligned(sink_bf16, 16)) ||
       (recent_bf16 && !aligned(recent_bf16, 16)) || (codes && !aligned(codes, 8)) || !aligned(gscale, 4))
     return NVFP4_ERR_ALIGN;
@@ -301,12 +343,36 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
     p.sink = sink_tokens;
     p.D = D;
     p.bpr = D / 16;
+    if (mma) {
+      // the scales of each (batch, head) form a [Tm, D/16] matrix in the tensor-core tile layout
+      p.sf_bpr = (uint32_t)(D / 16);
+      p.sf_rows = (uint32_t)Tm;
+      p.sf_ctiles = (uint32_t)((D / 16 + 3) / 4);
+      p.sf_mat_bytes = ((Tm + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
+      if ((Tm % 128 != 0 || (D / 16) % 4 != 0) &&
+          cudaMemsetAsync(scales, 0, (size_t)(BH * p.sf_mat_bytes), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    }
     int rc = rotate ? launch_quantize_t<true, true>(DT_BF16, p, s) : launch_quantize_t<true, false>(DT_BF16, p, s);
     if (rc) return rc;
   }
   global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
   if (int rc = last_error()) return rc;
   return check_finite_sync(gscale, s);
+}
+
+int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                   int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                   uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
+  return kv_mixed_impl(k_bf16, B, H, T, D, sink_tokens, recent_tokens, rotate, f_lo, f_hi, sink_bf16, recent_bf16,
+                       codes, scales, gscale, false, stream);
+}
+
+int nvfp4_kv_mixed_mma(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                       int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                       uint8_t* codes, uint8_t* sf, float* gscale, void* stream) {
+  return kv_mixed_impl(k_bf16, B, H, T, D, sink_tokens, recent_tokens, rotate, f_lo, f_hi, sink_bf16, recent_bf16,
+                       codes, sf, gscale, true, stream);
 }
 
 }  // extern "C"

@@ -378,7 +378,7 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
     sse = (WANT_SSE && amax_b != 0.0f) ? s : 0.0f;
   }
   reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(wlo, whi);
-  p.scales[b] = (uint8_t)scale;
+  p.scales[scale_index(p, b)] = (uint8_t)scale;
   if (p.block_f) p.block_f[b] = (int8_t)fstar;
   if (WANT_SSE) p.block_sse[b] = sse;
 }
