@@ -10,6 +10,10 @@ configuration the throughput target is stated on.  Every step's input (4 GiB) is
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
+Workloads: stream_f32 (default), act_f32, act_bf16, kv_bf16, bev_f16, and gemm_nvfp4 -- the tensor-core
+consumer: ScaleSearch-quantized BF16 activations [8192, 8192] times NVFP4 weights [8192, 8192] on the
+tensor cores, reported in TFLOP/s against the FP4 tensor roofline.
+
 Prints ONE JSON line on rank 0.  Times are CUDA events on the launching stream, max over ranks.
 `--impl reference` times the CPU oracle (the plain C definition) on a bounded sample of the same
 workload on the host cores.
@@ -237,6 +241,232 @@ def workload_config(args):
 
 
 # ------------------------------------------------------------------------------------------------
+# Tensor-core consumer workload: an NVFP4 linear layer
+# ------------------------------------------------------------------------------------------------
+GEMM_METRIC = "NVFP4 linear layer TFLOP/s (ScaleSearch-quantized activations x NVFP4 weights, tensor cores)"
+FP4_PER_BF16 = 4.0   # nominal dense FP4 / BF16 tensor throughput ratio of B200 (9 / 2.25 PFLOP/s)
+
+
+def gemm_shape(args):
+    return max(128, int(8192 * args.scale)), 8192, 8192     # M (tokens), N (outputs), K (inputs)
+
+
+def gemm_config(args):
+    M, N, K = gemm_shape(args)
+    return {
+        "workload": f"gemm_nvfp4 (activations BF16 [{M},{K}] 0.5*t(3) with 1% outlier columns x20, seed 1; "
+                    f"weights BF16 [{N},{K}] N(0,1/{K}), seed 11)",
+        "window": [args.f_lo, args.f_hi],
+        "step": "activations: amax + g + ScaleSearch quantize with tile-layout scales; "
+                "then D = g_a g_w A W^T on the tensor cores (NVFP4 x NVFP4, FP32 accumulate) -> BF16",
+        "weights": "quantized once before timing (ScaleSearch [-2,6], tile-layout scales)",
+        "l2": "L2 flushed between steps by a 256 MiB write (not timed)",
+        "M": M, "N": N, "K": K, "block": 16,
+    }
+
+
+def oracle_gemm_sample(args, rows=64, w_rows=1024):
+    """Oracle work for the CPU baseline: quantize `rows` activation rows and multiply them (fp64, exact
+    products) by `w_rows` weight rows quantized beforehand.  Returns (step function, flops per step)."""
+    import numpy as np
+    import torch
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    from oracle import oracle as O
+    K = gemm_shape(args)[2]
+    xa = W.act_bf16("cpu", rows / 8192.0)[:rows].contiguous()
+    xw = W.weight_bf16("cpu", w_rows, K)
+    a16 = xa.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    w16 = xw.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    wc, ws, wg, _, _ = O.quantize(w16, args.f_lo, args.f_hi, dtype=O.BF16)
+
+    def step():
+        ac, as_, ag, _, _ = O.quantize(a16, args.f_lo, args.f_hi, dtype=O.BF16)
+        O.gemm_nt(ac, as_, ag, wc, ws, wg, rows, w_rows, K)
+
+    return step, 2.0 * rows * w_rows * K, f"{rows} activation rows x {w_rows} weight rows, K = {K}"
+
+
+def run_gemm_reference(args, rank, world):
+    if rank != 0:
+        return
+    step, flops, desc = oracle_gemm_sample(args)
+    for _ in range(min(args.warmup, 3)):
+        step()
+    steps = max(1, min(args.steps, 20))
+    t = time.perf_counter()
+    for _ in range(steps):
+        step()
+    el = time.perf_counter() - t
+    val = flops * steps / el / 1e12
+    line = {
+        "impl": "reference", "metric": GEMM_METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": min(args.warmup, 3), "ms_per_step": el / steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4 x fp4 -> f64 (oracle)", "data": SOURCE_NOTE,
+        "config": gemm_config(args),
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": torch_threads(), "kind": "oracle",
+                         "sample": desc + ": oracle quantize (C, 1 thread) + fp64 numpy product"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def torch_threads():
+    try:
+        import numpy as np  # noqa: F401
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_gemm(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    M, N, K = gemm_shape(args)
+    x = W.act_bf16(dev, M / 8192.0)[:M].contiguous()
+    w = W.weight_bf16(dev, N, K)
+    wc, wsf, wg = nv.quantize_mma(w, args.f_lo, args.f_hi)
+    del w
+    ac = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    asf = torch.empty(nv.sf_mma_bytes(M, K), dtype=torch.uint8, device=dev)
+    ag = torch.empty(1, dtype=torch.float32, device=dev)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    aw = torch.empty(1, dtype=torch.float32, device=dev)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        nv.quantize_mma(x, args.f_lo, args.f_hi, codes=ac, sf=asf, gscale=ag)
+        if evs:
+            evs[1].record(stream)
+        nv.gemm_nt(ac, asf, ag, wc, wsf, wg, out=d, alpha_work=aw)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        step(evs[k])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    eager_ms = elapsed_ms
+    graph_used = False
+    if world == 1 and not args.no_graph:
+        cg = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(cg, stream=side):
+            step()
+        for _ in range(max(1, args.warmup)):
+            cg.replay()
+        torch.cuda.synchronize()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.fill_(float(-k))
+            gev[k][0].record(stream)
+            cg.replay()
+            gev[k][1].record(stream)
+        torch.cuda.synchronize()
+        graph_ms = sum(a.elapsed_time(b) for a, b in gev)
+        del cg
+        if graph_ms < elapsed_ms:
+            elapsed_ms, graph_used = graph_ms, True
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    g_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    flops = 2.0 * M * N * K
+    bf16_peak, src = tensor_peak()
+    fp4_peak = bf16_peak * FP4_PER_BF16
+    achieved = flops / (g_ms * 1e-3) / 1e12
+    line = {
+        "metric": GEMM_METRIC, "value": world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4 (e2m1 x e2m1, e4m3 block scales)",
+        "data": SOURCE_NOTE, "config": gemm_config(args),
+        "roofline": {"bound": "tensor", "kernel": "NVFP4 block-scaled GEMM (tcgen05, 128x128x256 tile)",
+                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "traffic": None, "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g} (nominal fp4/bf16 ratio)",
+                     "flops_per_launch": flops},
+        "breakdown_ms": {"quantize_activations": q_ms, "gemm": g_ms},
+        "quantize_activations": {"gbs_input": M * K * 2 / (q_ms * 1e-3) / 1e9},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+        "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / args.steps},
+    }
+    if not args.no_e2e and args.e2e_steps > 0:
+        hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        hx.copy_(x)
+        hd = torch.empty(d.shape, dtype=d.dtype, pin_memory=True)
+        xin = torch.empty_like(x)
+
+        def e2e_step():
+            xin.copy_(hx, non_blocking=True)
+            nv.quantize_mma(xin, args.f_lo, args.f_hi, codes=ac, sf=asf, gscale=ag)
+            nv.gemm_nt(ac, asf, ag, wc, wsf, wg, out=d, alpha_work=aw)
+            hd.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": hx.numel() * hx.element_size(),
+                       "d2h_bytes_per_step": hd.numel() * hd.element_size()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_o, fl, desc = oracle_gemm_sample(args)
+        step_o()
+        t = time.perf_counter()
+        step_o()
+        el = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "cores": torch_threads(), "kind": "oracle",
+                                "sample": desc + f": oracle quantize (C, 1 thread) + fp64 numpy product, {el:.2f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 def main():
@@ -245,7 +475,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        if args.workload == "gemm_nvfp4":
+            run_gemm_reference(args, rank, world)
+        else:
+            run_reference(args, rank, world)
         return
 
     import torch
@@ -261,6 +494,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
+    if args.workload == "gemm_nvfp4":
+        run_gemm(args, rank, world, dev)
+        return
     w = W.make(args.workload, dev, args.scale, shard=rank)
     x = w.x.contiguous()
     n = x.numel()

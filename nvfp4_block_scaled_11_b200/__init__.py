@@ -210,7 +210,9 @@ def sf_mma_bytes(rows: int, cols: int, batch: int = 1) -> int:
     return int(nb)
 
 
-def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None):
+def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None,
+                 codes: torch.Tensor | None = None, sf: torch.Tensor | None = None,
+                 gscale: torch.Tensor | None = None):
     """Quantize x [rows, cols] or [batch, rows, cols] along cols with the scales in the tensor-core tile
     layout.  Returns (codes uint8[..., rows, cols/2] (x's rank), sf uint8[sf_mma_bytes], gscale float32[1])."""
     _cuda(x, "x")
@@ -218,9 +220,14 @@ def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torc
         raise ValueError("x must be [rows, cols] or [batch, rows, cols]")
     batch, rows, cols = (1, *x.shape) if x.dim() == 2 else x.shape
     dev = x.device
-    codes = torch.empty((*x.shape[:-1], cols // 2), dtype=torch.uint8, device=dev)
-    sf = torch.empty(sf_mma_bytes(rows, cols, batch), dtype=torch.uint8, device=dev)
-    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    if codes is None:
+        codes = torch.empty((*x.shape[:-1], cols // 2), dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(sf_mma_bytes(rows, cols, batch), dtype=torch.uint8, device=dev)
+    if gscale is None:
+        gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    if codes.numel() * 2 != x.numel() or sf.numel() < sf_mma_bytes(rows, cols, batch):
+        raise ValueError("codes / sf buffers are too small")
     if gscale_in is not None:
         _cuda(gscale_in, "gscale_in")
     _check(lib().nvfp4_quantize_mma(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),

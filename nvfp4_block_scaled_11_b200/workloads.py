@@ -104,6 +104,13 @@ def bev_f16(device="cpu", scale: float = 1.0) -> torch.Tensor:
     return v.to(torch.float16)
 
 
+def weight_bf16(device="cpu", n_out: int = 8192, n_in: int = 8192) -> torch.Tensor:
+    """Linear-layer weights [n_out, n_in]: N(0, 1/n_in) (variance-preserving init), BF16, seed 11."""
+    g = _gen(11, device)
+    w = torch.randn((n_out, n_in), generator=g, device=device, dtype=torch.float32)
+    return (w * n_in ** -0.5).to(torch.bfloat16)
+
+
 def make(name: str, device="cpu", scale: float = 1.0, shard: int = 0) -> Workload:
     if name == "act_f32":
         return Workload(name, act_f32(device, scale), -2, 6, "quantize", "FP32 [1024,4096] N(0,1), seed 0")
