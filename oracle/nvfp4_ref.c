@@ -415,6 +415,20 @@ int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, 
   return 0;
 }
 
+int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, int64_t n, int64_t D, int rotate,
+                  float g, int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0) {
+  if (BH < 0 || n < 0 || D <= 0 || D % 16 != 0 || t0 < 0 || t0 + n > cap || first < 0) return -2;
+  float blk[16];
+  for (int64_t bh = 0; bh < BH; ++bh)
+    for (int64_t t = 0; t < n; ++t)
+      for (int64_t j = 0; j < D / 16; ++j) {
+        const int64_t out = (bh * cap + t0 + t) * (D / 16) + j;
+        load_row_group(k, bh * ld_bh + (first + t) * D + 16 * j, rotate, blk);
+        ref_search_block(blk, g, f_lo, f_hi, codes + 8 * out, scales + out, 0, 0);
+      }
+  return 0;
+}
+
 /* ---- array forms of the scalar converters (plain loops; used by the converter sweeps) ---- */
 void ref_e2m1_encode_n(const float* y, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = ref_e2m1_encode(y[i]);

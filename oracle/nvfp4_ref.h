@@ -98,6 +98,15 @@ int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, 
                  int rotate, int f_lo, int f_hi, uint16_t* sink_out, uint16_t* recent_out,
                  uint8_t* codes, uint8_t* scales, float* gscale_out);
 
+/* Incremental KV append for decode ([SS] attention-sink mixed-precision caching, with the cache
+ * growing one token group at a time): tokens [first, first+n) of every (batch, head) row block of the
+ * BF16 buffer k (row block bh starts at element bh * ld_bh; token t at + t * D) are optionally
+ * rotated (FWHT-16 along D) and quantized along D with the given tensor scale g (the prefill's),
+ * into rows [t0, t0+n) of a cache of `cap` rows per (batch, head):
+ * codes [BH, cap, D/2], scales [BH, cap, D/16] (row-major).  Other rows are left untouched.  */
+int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, int64_t n, int64_t D, int rotate,
+                  float g, int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0);
+
 /* ---- tensor-core consumer layout of the block scales ----
  * [SS] ScaleSearchAttention runs QK^T and PV as NVFP4 products on the tensor cores with FP32
  * accumulation.  The pages do not describe how the tensor cores read the block scales; this follows

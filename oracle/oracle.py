@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "ref_hadamard16": (I, [P, I64, I, P, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+            "ref_kv_append": (I, [P, I64, I64, I64, I64, I64, I, F, I, I, P, P, I64, I64]),
             "ref_sf_mma_bytes": (I64, [I64, I64]),
             "ref_sf_mma_offset": (I64, [I64, I64, I64]),
             "ref_scales_to_mma": (None, [P, I64, I64, I64, P]),
@@ -299,3 +300,17 @@ def gemm_nt(a_codes, a_scales, g_a, b_codes, b_scales, g_b, M: int, N: int, K: i
         bv = block_values(B[l], Bs[l], N, K)
         out[l] = (av @ bv.T) * scale
     return out
+
+
+def kv_append(k_rows: np.ndarray, first: int, n: int, g, codes: np.ndarray, scales: np.ndarray, t0: int,
+              rotate: int = 1, f_lo: int = -2, f_hi: int = 6) -> None:
+    """Quantize tokens [first, first+n) of every (batch, head) of k_rows (uint16 BF16 [BH, T, D]) with the
+    tensor scale g into rows [t0, t0+n) of codes [BH, cap, D/2] / scales [BH, cap, D/16], in place."""
+    k = np.ascontiguousarray(k_rows, np.uint16)
+    BH, T, D = k.shape
+    cap = codes.shape[1]
+    assert codes.flags.c_contiguous and scales.flags.c_contiguous
+    rc = lib().ref_kv_append(_p(k), BH, T * D, first, n, D, rotate, float(g), f_lo, f_hi, _p(codes), _p(scales),
+                             cap, t0)
+    if rc != 0:
+        raise ValueError(f"ref_kv_append returned {rc}")
