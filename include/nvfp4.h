@@ -108,6 +108,26 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
+/* ---- Incremental KV cache for decode ("Search your block floating-point scales!", ScaleSearchAttention >
+ * attention-sink mixed-precision caching, applied while the sequence grows) ----
+ * The tensor scale is fixed at prefill; later tokens are quantized with it as they leave the BF16
+ * window of recent tokens (values beyond 448 * 6 * g saturate). */
+
+/* Tensor scale of a prefill: g = fl(amax / 2688) over the (rotated when rotate != 0) middle tokens
+ * [sink_tokens, T - recent_tokens) of K[B,H,T,D] (BF16), exactly as nvfp4_kv_mixed computes it. */
+int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens, int recent_tokens,
+                    int rotate, float* gscale, void* stream);
+
+/* Quantize tokens [first, first + n) of every (batch, head) of the BF16 buffer k_bf16 [BH, T, D]
+ * (optionally rotated by FWHT-16 along D) with the tensor scale *gscale into rows [t0, t0 + n) of an
+ * NVFP4 cache with `cap` rows per (batch, head): codes [BH, cap, D/2]; scales [BH, cap, D/16] when
+ * scale_layout == 0, or the tensor-core tile layout of BH matrices [cap, D] when scale_layout == 1
+ * (nvfp4_sf_mma_bytes(cap, D, BH) bytes; padding bytes are not written).  Other rows are untouched.
+ * Requires first + n <= T and t0 + n <= cap (NVFP4_ERR_SIZE). */
+int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, int64_t n, int64_t D, int rotate,
+                    int f_lo, int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
+                    int scale_layout, void* stream);
+
 /* ---- Tensor-core consumer ("Search your block floating-point scales!", ScaleSearchAttention: QK^T and
  * PV run as NVFP4 products on the tensor cores with FP32 accumulation) ----
  *

@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "kv_mixed_mma",
-    "gemm_nt", "gemm_sf_offsets",
+    "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -38,6 +38,8 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_kv_gscale": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
+    "nvfp4_kv_append": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _P]),
     "nvfp4_sf_mma_bytes": (_I64, [_I64, _I64, _I64]),
     "nvfp4_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "nvfp4_kv_mixed_mma": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
@@ -291,3 +293,33 @@ def gemm_sf_offsets(rows: int, K: int, batch: int = 1):
     out = np.empty(batch * rows * (K // 16), np.int64)
     _check(lib().nvfp4_gemm_sf_offsets(rows, K, batch, out.ctypes.data))
     return out
+
+
+# ---- incremental KV cache (decode) ----
+def kv_gscale(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = True,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """Tensor scale over the (rotated) middle tokens of K[B,H,T,D] (BF16), as kv_mixed computes it."""
+    _cuda(k, "k")
+    if k.dtype != torch.bfloat16 or k.dim() != 4:
+        raise TypeError("k must be a 4-D bfloat16 tensor [B,H,T,D]")
+    B, H, T, D = k.shape
+    out = torch.empty(1, dtype=torch.float32, device=k.device) if out is None else out
+    _check(lib().nvfp4_kv_gscale(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), _ptr(out), _stream(k)))
+    return out
+
+
+def kv_append(k_rows: torch.Tensor, first: int, n: int, gscale: torch.Tensor, codes: torch.Tensor,
+              scales: torch.Tensor, t0: int, rotate: bool = True, f_lo: int = -2, f_hi: int = 6,
+              tile_layout: bool = False) -> None:
+    """Quantize tokens [first, first+n) of k_rows [..., T, D] (BF16, contiguous; leading dims = batch x
+    heads) with the tensor scale gscale into rows [t0, t0+n) of codes [..., cap, D/2] and scales
+    ([..., cap, D/16], or the tile layout of the per-head [cap, D] matrices when tile_layout)."""
+    for t, nm in ((k_rows, "k_rows"), (gscale, "gscale"), (codes, "codes"), (scales, "scales")):
+        _cuda(t, nm)
+    if k_rows.dtype != torch.bfloat16:
+        raise TypeError("k_rows must be bfloat16")
+    T, D = k_rows.shape[-2], k_rows.shape[-1]
+    BH = k_rows.numel() // max(T * D, 1)
+    cap = codes.shape[-2]
+    _check(lib().nvfp4_kv_append(_ptr(k_rows), BH, T, first, n, D, int(bool(rotate)), f_lo, f_hi, _ptr(gscale),
+                                 _ptr(codes), _ptr(scales), cap, t0, 1 if tile_layout else 0, _stream(k_rows)))

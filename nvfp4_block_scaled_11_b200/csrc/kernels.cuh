@@ -126,7 +126,18 @@ struct QuantParams {
   // sf_bpr blocks per row (fewer than 2^32 blocks in all); each matrix's scales take sf_mat_bytes bytes
   uint32_t sf_bpr, sf_rows, sf_ctiles;  // sf_ctiles = ceil(sf_bpr / 4)
   int64_t sf_mat_bytes;
+  // KV append: when out_cap > 0 the Tm token rows of each (batch, head) handled by this launch are
+  // written to rows out_t0 .. out_t0 + Tm - 1 of a cache with out_cap rows per (batch, head)
+  int64_t out_cap, out_t0;
 };
+
+// Output block index of block b (input order): b itself, or its row in the KV cache being appended to.
+__device__ __forceinline__ int64_t out_block(const QuantParams& p, int64_t b) {
+  if (p.out_cap == 0) return b;
+  const int64_t per = p.Tm * p.bpr;
+  const int64_t bh = b / per, rem = b - bh * per;  // rem = token * bpr + block column
+  return (bh * p.out_cap + p.out_t0) * p.bpr + rem;
+}
 
 // Byte of block b's scale.  Linear: b.  Tile layout (block-scaled tensor-core MMA operand): 512-byte
 // tiles of 128 rows x 4 block columns, the column tiles of a row tile consecutive, and inside a tile
@@ -261,10 +272,11 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
         sse = s;
       }
     }
-    reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(lo, hi);
-    p.scales[scale_index(p, b)] = (uint8_t)scale;
-    if (p.block_f) p.block_f[b] = (int8_t)fstar;
-    if (p.block_sse) p.block_sse[b] = sse;
+    const int64_t ob = out_block(p, b);
+    reinterpret_cast<uint2*>(p.codes)[ob] = make_uint2(lo, hi);
+    p.scales[scale_index(p, ob)] = (uint8_t)scale;
+    if (p.block_f) p.block_f[ob] = (int8_t)fstar;
+    if (p.block_sse) p.block_sse[ob] = sse;
   }
 }
 

@@ -361,6 +361,70 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   return check_finite_sync(gscale, s);
 }
 
+int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens, int recent_tokens,
+                    int rotate, float* gscale, void* stream) {
+  if (gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
+    return NVFP4_ERR_SIZE;
+  const int64_t Tm = T - sink_tokens - recent_tokens;
+  const int64_t ngroups = B * H * Tm * (D / 16);
+  if (ngroups > 0 && k_bf16 == nullptr) return NVFP4_ERR_ARG;
+  if ((ngroups > 0 && !aligned(k_bf16, 16)) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
+  cudaStream_t s = S(stream);
+  if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (ngroups > 0) {
+    const char* k = static_cast<const char*>(k_bf16);
+    const int v8 = aligned(k_bf16, 32) ? 1 : 0;
+    const int grid = grid_for(ngroups, 256, 8);
+    uint32_t* word = reinterpret_cast<uint32_t*>(gscale);
+    if (rotate) kv_amax_kernel<true><<<grid, 256, 0, s>>>(k, ngroups, T, Tm, sink_tokens, D, D / 16, v8, word);
+    else kv_amax_kernel<false><<<grid, 256, 0, s>>>(k, ngroups, T, Tm, sink_tokens, D, D / 16, v8, word);
+    if (int rc = last_error()) return rc;
+  }
+  global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
+  if (int rc = last_error()) return rc;
+  return check_finite_sync(gscale, s);
+}
+
+int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, int64_t n, int64_t D, int rotate,
+                    int f_lo, int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
+                    int scale_layout, void* stream) {
+  if (!window_ok(f_lo, f_hi) || gscale == nullptr || (scale_layout != 0 && scale_layout != 1)) return NVFP4_ERR_ARG;
+  if (BH < 0 || T < 0 || n < 0 || first < 0 || t0 < 0 || cap < 0 || D <= 0 || D % 16 != 0) return NVFP4_ERR_SIZE;
+  if (first + n > T || t0 + n > cap) return NVFP4_ERR_SIZE;
+  if (scale_layout == 1 && BH * cap * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (BH == 0 || n == 0) return NVFP4_OK;
+  if (k_bf16 == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(k_bf16, 16) || !aligned(codes, 8) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
+  QuantParams p{};
+  p.x = static_cast<const char*>(k_bf16);
+  p.nblocks = BH * n * (D / 16);
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.g_src = gscale;
+  p.g_is_amax = 0;
+  p.codes = codes;
+  p.scales = scales;
+  p.v8 = aligned(k_bf16, 32) ? 1 : 0;
+  p.T = T;
+  p.Tm = n;
+  p.sink = first;
+  p.D = D;
+  p.bpr = D / 16;
+  p.out_cap = cap;
+  p.out_t0 = t0;
+  if (scale_layout == 1) {
+    p.sf_bpr = (uint32_t)(D / 16);
+    p.sf_rows = (uint32_t)cap;
+    p.sf_ctiles = (uint32_t)((D / 16 + 3) / 4);
+    p.sf_mat_bytes = ((cap + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
+  }
+  cudaStream_t s = S(stream);
+  const int rc = rotate ? launch_quantize_t<true, true>(DT_BF16, p, s) : launch_quantize_t<true, false>(DT_BF16, p, s);
+  if (rc) return rc;
+  return check_finite_sync(gscale, s);
+}
+
 int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {

@@ -377,10 +377,11 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
     }
     sse = (WANT_SSE && amax_b != 0.0f) ? s : 0.0f;
   }
-  reinterpret_cast<uint2*>(p.codes)[b] = make_uint2(wlo, whi);
-  p.scales[scale_index(p, b)] = (uint8_t)scale;
-  if (p.block_f) p.block_f[b] = (int8_t)fstar;
-  if (WANT_SSE) p.block_sse[b] = sse;
+  const int64_t ob = out_block(p, b);
+  reinterpret_cast<uint2*>(p.codes)[ob] = make_uint2(wlo, whi);
+  p.scales[scale_index(p, ob)] = (uint8_t)scale;
+  if (p.block_f) p.block_f[ob] = (int8_t)fstar;
+  if (WANT_SSE) p.block_sse[ob] = sse;
 }
 
 // Fast path for one block.  Returns true when the block needs the definition (outputs not written).

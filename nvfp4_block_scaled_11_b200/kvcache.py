@@ -1,0 +1,109 @@
+"""Attention-sink mixed-precision K/V cache that grows during decode.
+
+"Search your block floating-point scales!" (gist.science summary of arXiv 2605.12464),
+ScaleSearchAttention > attention-sink-aware mixed-precision caching: the first and the last block of
+the KV cache stay in full precision and the blocks in between are NVFP4.  During decode the last block
+moves: every new token enters a BF16 window of recent tokens, and once the window holds two groups of
+`recent` tokens the older group is quantized (one `nvfp4_kv_append` launch, Hadamard-rotated along
+head_dim when `rotate`) into the NVFP4 middle.  The window therefore always keeps between `recent` and
+2 * recent - 1 of the newest tokens in BF16.
+
+The tensor scale is fixed by the prefill (`nvfp4_kv_gscale` over the rotated middle tokens, as in
+`nvfp4_kv_mixed`); later tokens use it unchanged, so values beyond 448 * 6 * g saturate.
+
+Host-side bookkeeping only: token rows are moved with tensor copies, every quantization runs in the
+library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import kv_append, kv_gscale, sf_mma_bytes
+
+
+class NVFP4KVCache:
+    """K (or V) cache of B x H heads of dimension D with room for `capacity` NVFP4 middle tokens.
+
+    Attributes (device tensors):
+      sink   [B, H, sink, D] bf16      first tokens, verbatim
+      window [B, H, 2*recent, D] bf16  ring of the newest tokens; valid slots head .. head + n_window - 1
+      codes  [B, H, capacity, D/2]     NVFP4 middle, rows 0 .. n_mid - 1 valid
+      scales [B, H, capacity, D/16]    or the tensor-core tile layout of the B*H [capacity, D] matrices
+      gscale [1] float32               tensor scale (fixed at prefill)
+    """
+
+    def __init__(self, B: int, H: int, D: int, capacity: int, sink: int = 16, recent: int = 16, rotate: bool = True,
+                 f_lo: int = -2, f_hi: int = 6, tile_layout: bool = False, device="cuda"):
+        if D % 16 or recent <= 0 or sink < 0 or capacity < 0:
+            raise ValueError("D must be a multiple of 16; recent > 0; sink, capacity >= 0")
+        self.B, self.H, self.D, self.capacity = B, H, D, capacity
+        self.n_sink_max, self.recent, self.rotate, self.f_lo, self.f_hi = sink, recent, rotate, f_lo, f_hi
+        self.tile_layout = tile_layout
+        dev = torch.device(device)
+        self.sink = torch.zeros((B, H, sink, D), dtype=torch.bfloat16, device=dev)
+        self.window = torch.zeros((B, H, 2 * recent, D), dtype=torch.bfloat16, device=dev)
+        self.codes = torch.zeros((B, H, capacity, D // 2), dtype=torch.uint8, device=dev)
+        if tile_layout:
+            self.scales = torch.zeros(max(sf_mma_bytes(capacity, D, B * H), 1), dtype=torch.uint8, device=dev)
+        else:
+            self.scales = torch.zeros((B, H, capacity, D // 16), dtype=torch.uint8, device=dev)
+        self.gscale = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.n_sink = 0
+        self.n_mid = 0
+        self.head = 0        # first valid window slot: 0 or recent
+        self.n_window = 0
+        self.prefilled = False
+
+    @property
+    def length(self) -> int:
+        return self.n_sink + self.n_mid + self.n_window
+
+    def prefill(self, k: torch.Tensor) -> None:
+        """Start the cache from K[B, H, T, D] (BF16), T >= sink + recent: the tensor scale over the rotated
+        middle, the middle quantized into rows 0 .. T - sink - recent - 1, sink and window verbatim."""
+        B, H, T, D = k.shape
+        if (B, H, D) != (self.B, self.H, self.D) or k.dtype != torch.bfloat16:
+            raise ValueError("k must be bfloat16 [B, H, T, D] matching the cache")
+        s, r = self.n_sink_max, self.recent
+        if T < s + r:
+            raise ValueError("prefill needs at least sink + recent tokens")
+        k = k.contiguous()
+        n_mid = T - s - r
+        if n_mid > self.capacity:
+            raise ValueError("prefill middle exceeds the cache capacity")
+        kv_gscale(k, s, r, self.rotate, out=self.gscale)
+        if n_mid:
+            kv_append(k, s, n_mid, self.gscale, self.codes, self.scales, 0, self.rotate, self.f_lo, self.f_hi,
+                      self.tile_layout)
+        self.sink.copy_(k[:, :, :s])
+        self.window[:, :, :r].copy_(k[:, :, T - r:])
+        self.n_sink, self.n_mid, self.head, self.n_window = s, n_mid, 0, r
+        self.prefilled = True
+
+    def append(self, k_new: torch.Tensor) -> None:
+        """Append tokens K_new[B, H, n, D] (BF16) in order."""
+        if not self.prefilled:
+            raise RuntimeError("prefill first")
+        r = self.recent
+        for i in range(k_new.shape[2]):
+            if self.n_window == 2 * r:
+                self._flush_group()
+            slot = (self.head + self.n_window) % (2 * r)
+            self.window[:, :, slot].copy_(k_new[:, :, i])
+            self.n_window += 1
+
+    def _flush_group(self) -> None:
+        r = self.recent
+        if self.n_mid + r > self.capacity:
+            raise RuntimeError("NVFP4 cache capacity exceeded")
+        # the oldest `recent` window tokens are the contiguous slots head .. head + recent - 1
+        kv_append(self.window, self.head, r, self.gscale, self.codes, self.scales, self.n_mid, self.rotate,
+                  self.f_lo, self.f_hi, self.tile_layout)
+        self.n_mid += r
+        self.head = (self.head + r) % (2 * r)
+        self.n_window -= r
+
+    def recent_tokens(self) -> torch.Tensor:
+        """The BF16 window in token order, [B, H, n_window, D]."""
+        idx = [(self.head + i) % (2 * self.recent) for i in range(self.n_window)]
+        return self.window[:, :, idx]

@@ -1,0 +1,105 @@
+"""Incremental KV cache (decode) through the C ABI against the oracle: bit-exact codes and scales."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_11_b200 as nv
+from nvfp4_block_scaled_11_b200 import workloads as W
+from nvfp4_block_scaled_11_b200.kvcache import NVFP4KVCache
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _u16(t):
+    return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _k(T, heads=2, D=128):
+    k = W.kv_bf16("cpu", scale=T / 32768, heads=heads, head_dim=D)
+    return k
+
+
+@pytest.mark.parametrize("rotate", [True, False])
+@pytest.mark.parametrize("tile", [False, True])
+def test_kv_append_matches_oracle(rotate, tile):
+    k = _k(64, heads=3)[0]                      # [BH=3, T, D]
+    BH, T, D = k.shape
+    first, n, cap, t0 = 7, 20, 300, 131         # rows 131..150 cross a 128-row tile boundary
+    g = torch.tensor([0.0023], dtype=torch.float32)
+    codes = torch.full((BH, cap, D // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    if tile:
+        scales = torch.full((nv.sf_mma_bytes(cap, D, BH),), 0xAA, dtype=torch.uint8, device="cuda")
+    else:
+        scales = torch.full((BH, cap, D // 16), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.kv_append(k.cuda(), first, n, g.cuda(), codes, scales, t0, rotate=rotate, tile_layout=tile)
+    rc = np.full((BH, cap, D // 2), 0xAA, np.uint8)
+    rs = np.full((BH, cap, D // 16), 0xAA, np.uint8)
+    O.kv_append(_u16(k), first, n, g.item(), rc, rs, t0, rotate=int(rotate))
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    if not tile:
+        assert np.array_equal(scales.cpu().numpy(), rs)
+    else:
+        want = np.full(nv.sf_mma_bytes(cap, D, BH), 0xAA, np.uint8)
+        per = O.sf_mma_bytes(cap, D // 16)
+        for l in range(BH):
+            for r in range(t0, t0 + n):
+                for c in range(D // 16):
+                    want[l * per + O.sf_mma_offset(r, c, D // 16)] = rs[l, r, c]
+        assert np.array_equal(scales.cpu().numpy(), want)
+
+
+def test_kv_gscale_matches_kv_mixed():
+    k = _k(200)
+    g = nv.kv_gscale(k.cuda())
+    *_, rg = O.kv_mixed(_u16(k))
+    assert g.item() == rg
+    g0 = nv.kv_gscale(k.cuda(), rotate=False)
+    *_, rg0 = O.kv_mixed(_u16(k), rotate=0)
+    assert g0.item() == rg0
+
+
+def test_kv_append_errors():
+    k = torch.zeros((2, 32, 64), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(1, device="cuda")
+    codes = torch.zeros((2, 8, 32), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((2, 8, 4), dtype=torch.uint8, device="cuda")
+    with pytest.raises(nv.NVFP4Error) as e:
+        nv.kv_append(k, 0, 5, g, codes, scales, 4)        # rows 4..8 exceed the 8-row cache
+    assert e.value.status == -2
+    with pytest.raises(nv.NVFP4Error) as e:
+        nv.kv_append(k, 30, 4, g, codes, scales, 0)       # tokens 30..33 exceed T = 32
+    assert e.value.status == -2
+    nv.kv_append(k, 0, 0, g, codes, scales, 8)             # nothing to do
+
+
+@pytest.mark.parametrize("tile", [False, True])
+def test_decode_cache_matches_oracle_sequence(tile):
+    B, H, D, T0 = 1, 2, 128, 90
+    full = _k(T0 + 60, heads=H)                  # the whole sequence: prefill + decoded tokens
+    Tfull = full.shape[2]
+    pre = full[:, :, :T0].contiguous()
+    cache = NVFP4KVCache(B, H, D, capacity=256, tile_layout=tile)
+    cache.prefill(pre.cuda())
+    t = T0
+    for _ in range(37):                          # one token per step
+        cache.append(full[:, :, t:t + 1].cuda())
+        t += 1
+    cache.append(full[:, :, t:Tfull].cuda())     # then a chunk
+    torch.cuda.synchronize()
+    assert cache.length == Tfull
+    # oracle: g from the prefill, the middle = tokens [16, 16 + n_mid) of the whole sequence
+    *_, g = O.kv_mixed(_u16(pre))
+    assert cache.gscale.item() == g
+    n_mid = cache.n_mid
+    assert n_mid == Tfull - 16 - cache.n_window and cache.recent <= cache.n_window < 2 * cache.recent
+    rc = np.zeros((B * H, 256, D // 2), np.uint8)
+    rs = np.zeros((B * H, 256, D // 16), np.uint8)
+    O.kv_append(_u16(full).reshape(B * H, Tfull, D), 16, n_mid, g, rc, rs, 0)
+    assert np.array_equal(cache.codes.cpu().numpy().reshape(B * H, 256, D // 2)[:, :n_mid], rc[:, :n_mid])
+    if tile:
+        assert np.array_equal(cache.scales.cpu().numpy(), O.scales_to_mma(rs, B * H, 256, D // 16))
+    else:
+        assert np.array_equal(cache.scales.cpu().numpy().reshape(B * H, 256, D // 16)[:, :n_mid], rs[:, :n_mid])
+    assert torch.equal(cache.sink.cpu(), full[:, :, :16])
+    assert torch.equal(cache.recent_tokens().cpu(), full[:, :, Tfull - cache.n_window:])
