@@ -429,6 +429,64 @@ int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, i
   return 0;
 }
 
+/* ---- MXFP4 (see the header) ---- */
+/* floor(log2(a)) of a finite a > 0, from its bit pattern */
+static int ilog2_floor(float a) {
+  const uint32_t b = f2u(a) & 0x7FFFFFFFu;
+  const int e = (int)(b >> 23);
+  if (e > 0) return e - 127;
+  int msb = 22;                              /* subnormal: a = m * 2^-149 with m = b */
+  while (!((b >> msb) & 1u)) --msb;
+  return msb - 149;
+}
+
+/* 2^k exactly, k in [-149, 127] */
+static float pow2f(int k) {
+  return k >= -126 ? u2f((uint32_t)(k + 127) << 23) : u2f(1u << (k + 149));
+}
+
+int ref_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales) {
+  if (n < 0 || n % 32 != 0) return -2;
+  for (int64_t b = 0; b < n / 32; ++b) {
+    float v[32], amax = 0.0f;
+    int bad = 0;
+    for (int i = 0; i < 32; ++i) {
+      v[i] = load_elem(x, dtype, 32 * b + i);
+      const float a = fabsf(v[i]);
+      if (!(a <= FLT_MAX)) bad = 1;
+      else if (a > amax) amax = a;
+    }
+    uint8_t* c = codes + 16 * b;
+    if (bad) {
+      scales[b] = 0xFF;
+      for (int i = 0; i < 16; ++i) c[i] = 0;
+      continue;
+    }
+    int e = amax == 0.0f ? -127 : ilog2_floor(amax) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    scales[b] = (uint8_t)(e + 127);
+    const float inv = pow2f(-e);             /* x / 2^e as an exact multiply (RNE if subnormal) */
+    for (int i = 0; i < 16; ++i) {
+      const uint8_t lo = ref_e2m1_encode(v[2 * i] * inv), hi = ref_e2m1_encode(v[2 * i + 1] * inv);
+      c[i] = (uint8_t)(lo | (hi << 4));
+    }
+  }
+  return 0;
+}
+
+int ref_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n, int out_dtype, void* out) {
+  if (n < 0 || n % 32 != 0) return -2;
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const float X = scales[b] == 0xFF ? qnan() : pow2f((int)scales[b] - 127);
+    for (int i = 0; i < 32; ++i) {
+      const uint8_t q = (uint8_t)((codes[16 * b + i / 2] >> (4 * (i & 1))) & 15u);
+      store_elem(out, out_dtype, 32 * b + i, ref_e2m1_decode(q) * X);
+    }
+  }
+  return 0;
+}
+
 /* ---- array forms of the scalar converters (plain loops; used by the converter sweeps) ---- */
 void ref_e2m1_encode_n(const float* y, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = ref_e2m1_encode(y[i]);

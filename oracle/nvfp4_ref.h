@@ -107,6 +107,17 @@ int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, 
 int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, int64_t n, int64_t D, int rotate,
                   float g, int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0);
 
+/* ---- MXFP4, the power-of-two-scaled comparison format ----
+ * [NV] compares NVFP4 with "simple power-of-two scaling like MXFP4".  MXFP4 as the OCP Microscaling
+ * (MX) v1.0 specification defines it: blocks of 32 elements, one E8M0 scale X = 2^e with
+ * e = floor(log2(amax_b)) - 2 (2 = the exponent of E2M1's largest value 6), clamped to [-127, 127];
+ * elements E2M1_RNE_SAT(x / X).  Scale byte = e + 127.  All-zero block: e = -127 (byte 0).  A block
+ * with a NaN or Inf element: scale byte 0xFF (E8M0 NaN), codes 0.  Nibble order as for NVFP4.
+ * codes: n/2 bytes, scales: n/32 bytes, n % 32 == 0. */
+int ref_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales);
+/* x_i = E2M1(q_i) * 2^(s - 127) (exact in FP32), rounded to out_dtype; scale byte 0xFF gives NaN. */
+int ref_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n, int out_dtype, void* out);
+
 /* ---- tensor-core consumer layout of the block scales ----
  * [SS] ScaleSearchAttention runs QK^T and PV as NVFP4 products on the tensor cores with FP32
  * accumulation.  The pages do not describe how the tensor cores read the block scales; this follows

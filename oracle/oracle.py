@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
             "ref_hadamard16": (I, [P, I64, I, P, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+            "ref_mxfp4_quantize": (I, [P, I64, I, P, P]),
+            "ref_mxfp4_dequantize": (I, [P, P, I64, I, P]),
             "ref_kv_append": (I, [P, I64, I64, I64, I64, I64, I, F, I, I, P, P, I64, I64]),
             "ref_sf_mma_bytes": (I64, [I64, I64]),
             "ref_sf_mma_offset": (I64, [I64, I64, I64]),
@@ -314,3 +316,27 @@ def kv_append(k_rows: np.ndarray, first: int, n: int, g, codes: np.ndarray, scal
                              cap, t0)
     if rc != 0:
         raise ValueError(f"ref_kv_append returned {rc}")
+
+
+# ---- MXFP4 (comparison format) ----
+def mxfp4_quantize(x: np.ndarray, dtype: int | None = None):
+    """(codes n/2, E8M0 scales n/32) of x (n % 32 == 0)."""
+    x = np.ascontiguousarray(x).reshape(-1)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    codes = np.empty(x.size // 2, np.uint8)
+    scales = np.empty(x.size // 32, np.uint8)
+    rc = lib().ref_mxfp4_quantize(_p(x), x.size, dtype, _p(codes), _p(scales))
+    if rc != 0:
+        raise ValueError(f"ref_mxfp4_quantize returned {rc}")
+    return codes, scales
+
+
+def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray, out_dtype: int = F32) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    n = scales.size * 32
+    out = np.empty(n, _NP_OF[out_dtype])
+    rc = lib().ref_mxfp4_dequantize(_p(codes), _p(scales), n, out_dtype, _p(out))
+    if rc != 0:
+        raise ValueError(f"ref_mxfp4_dequantize returned {rc}")
+    return out
