@@ -108,6 +108,18 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
+/* ---- MXFP4, the comparison format ("NVIDIAのFP4推論が50倍の効率を実現", 超低精度推論を支えるアーキテクチャ:
+ * NVFP4 against simple power-of-two scaling such as MXFP4) ----
+ * MXFP4 as the OCP Microscaling (MX) v1.0 specification defines it (not on the pages): blocks of 32
+ * elements, one E8M0 scale X = 2^e, e = floor(log2(amax_b)) - 2 clamped to [-127, 127] (scale byte
+ * e + 127; all-zero block: byte 0), elements E2M1_RNE_SAT(x / X) packed two per byte (element 2k in
+ * the low nibble); a block holding NaN or Inf gets scale byte 0xFF and codes 0.
+ * codes: n/2 bytes (16-byte aligned), scales: n/32 bytes, n % 32 == 0. */
+int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales, void* stream);
+/* out_i = E2M1(code_i) * 2^(scale - 127) (exact in FP32), RNE to out_dtype; scale byte 0xFF gives NaN. */
+int nvfp4_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n, int out_dtype, void* out,
+                           void* stream);
+
 /* ---- Incremental KV cache for decode ("Search your block floating-point scales!", ScaleSearchAttention >
  * attention-sink mixed-precision caching, applied while the sequence grows) ----
  * The tensor scale is fixed at prefill; later tokens are quantized with it as they leave the BF16

@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "kv_mixed_mma",
-    "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append",
+    "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -38,6 +38,8 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_mxfp4_quantize": (_I, [_P, _I64, _I, _P, _P, _P]),
+    "nvfp4_mxfp4_dequantize": (_I, [_P, _P, _I64, _I, _P, _P]),
     "nvfp4_kv_gscale": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
     "nvfp4_kv_append": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _P]),
     "nvfp4_sf_mma_bytes": (_I64, [_I64, _I64, _I64]),
@@ -323,3 +325,24 @@ def kv_append(k_rows: torch.Tensor, first: int, n: int, gscale: torch.Tensor, co
     cap = codes.shape[-2]
     _check(lib().nvfp4_kv_append(_ptr(k_rows), BH, T, first, n, D, int(bool(rotate)), f_lo, f_hi, _ptr(gscale),
                                  _ptr(codes), _ptr(scales), cap, t0, 1 if tile_layout else 0, _stream(k_rows)))
+
+
+# ---- MXFP4 (comparison format) ----
+def mxfp4_quantize(x: torch.Tensor, codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """MXFP4 (32-element blocks, E8M0 power-of-two scales).  Returns (codes uint8[n/2], scales uint8[n/32])."""
+    _cuda(x, "x")
+    n = x.numel()
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=x.device) if codes is None else codes
+    scales = torch.empty(n // 32, dtype=torch.uint8, device=x.device) if scales is None else scales
+    _check(lib().nvfp4_mxfp4_quantize(_ptr(x), n, _dt(x), _ptr(codes), _ptr(scales), _stream(x)))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out_dtype=torch.float32,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    _cuda(codes, "codes"), _cuda(scales, "scales")
+    n = scales.numel() * 32
+    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
+    _check(lib().nvfp4_mxfp4_dequantize(_ptr(codes), _ptr(scales), n, DTYPE_CODE[out.dtype], _ptr(out),
+                                        _stream(codes)))
+    return out

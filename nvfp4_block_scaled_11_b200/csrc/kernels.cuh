@@ -386,6 +386,106 @@ __global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict_
 }
 
 // =================================================================================================
+// MXFP4 (the power-of-two-scaled format NVFP4 is compared against): OCP Microscaling v1.0 -- blocks of
+// 32, one E8M0 scale 2^e with e = floor(log2 amax_b) - 2 (clamped to [-127, 127]), elements
+// E2M1_RNE_SAT(x * 2^-e); all-zero block e = -127; a NaN / Inf element -> scale 0xFF, codes 0.
+// =================================================================================================
+// 2^k as an exact float for k in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2_exact(int k) {
+  return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << (k + 149));
+}
+
+template <int DT>
+__global__ void __launch_bounds__(256) mxfp4_quantize_kernel(const char* __restrict__ x, int64_t nblocks, int v8,
+                                                             uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int ES = DT == DT_F32 ? 4 : 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    float v0[16], v1[16];
+    load_block<DT>(x + 32 * ES * b, v8 != 0, v0);
+    load_block<DT>(x + 32 * ES * b + 16 * ES, v8 != 0, v1);
+    uint32_t mb = 0u;  // largest magnitude bit pattern: integer order = numeric order; NaN / Inf >= 0x7F800000
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mb = max(mb, max(__float_as_uint(v0[i]) & 0x7FFFFFFFu, __float_as_uint(v1[i]) & 0x7FFFFFFFu));
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    int sbyte = 0xFF;
+    if (mb < 0x7F800000u) {
+      const int ex = (int)(mb >> 23);
+      int e = mb == 0u ? -127 : (ex > 0 ? ex - 127 : (31 - __clz((int)mb)) - 149) - 2;
+      e = max(e, -127);
+      sbyte = e + 127;
+      const float inv = pow2_exact(-e);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float lo = k < 8 ? v0[2 * k] : v1[2 * k - 16], hi = k < 8 ? v0[2 * k + 1] : v1[2 * k - 15];
+        w[k >> 2] |= (e2m1x2(__fmul_rn(hi, inv), __fmul_rn(lo, inv)) & 0xFFu) << (8 * (k & 3));
+      }
+    }
+    reinterpret_cast<uint4*>(codes)[b] = make_uint4(w[0], w[1], w[2], w[3]);
+    scales[b] = (uint8_t)sbyte;
+  }
+}
+
+template <int OT>
+__device__ __forceinline__ void store16(char* o, const float (&v)[16], bool v8) {
+  if (OT == DT_F32) {
+    uint32_t a[8], c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { a[i] = __float_as_uint(v[i]); c[i] = __float_as_uint(v[8 + i]); }
+    if (v8) {
+      st_v8(o, a);
+      st_v8(o + 32, c);
+    } else {
+      st_v4(o, a); st_v4(o + 16, a + 4); st_v4(o + 32, c); st_v4(o + 48, c + 4);
+    }
+  } else {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (OT == DT_BF16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&h);
+      } else {
+        __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&h);
+      }
+    }
+    if (v8) {
+      st_v8(o, w);
+    } else {
+      st_v4(o, w);
+      st_v4(o + 16, w + 4);
+    }
+  }
+}
+
+template <int OT>
+__global__ void __launch_bounds__(256) mxfp4_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                               const uint8_t* __restrict__ scales, int64_t nblocks,
+                                                               char* __restrict__ out, int v8) {
+  constexpr int OS = OT == DT_F32 ? 4 : 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    const uint4 cw = reinterpret_cast<const uint4*>(codes)[b];
+    const uint32_t s = scales[b];
+    const float X = s == 0xFFu ? __uint_as_float(0x7FC00000u) : pow2_exact((int)s - 127);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t byte = (words[2 * half + (k >> 2)] >> (8 * (k & 3))) & 0xFFu;
+        const uint32_t h2 = e2m1x2_to_f16x2(byte);
+        v[2 * k] = __fmul_rn(f16lo(h2), X);
+        v[2 * k + 1] = __fmul_rn(f16hi(h2), X);
+      }
+      store16<OT>(out + (32 * b + 16 * half) * OS, v, v8 != 0);
+    }
+  }
+}
+
+// =================================================================================================
 // Mixed-precision KV layout helpers.
 // =================================================================================================
 // Copy the first `sink` and last `recent` token rows of every (batch, head) verbatim (16-byte units).

@@ -361,6 +361,45 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   return check_finite_sync(gscale, s);
 }
 
+int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales, void* stream) {
+  if (!dtype_ok(dtype)) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 32 != 0) return NVFP4_ERR_SIZE;
+  if (n == 0) return NVFP4_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16)) return NVFP4_ERR_ALIGN;
+  const int64_t nb = n / 32;
+  const int grid = grid_for(nb, 256, 8);
+  const int v8 = aligned(x, 32) ? 1 : 0;
+  const char* xp = static_cast<const char*>(x);
+  cudaStream_t s = S(stream);
+  switch (dtype) {
+    case DT_F32: mxfp4_quantize_kernel<DT_F32><<<grid, 256, 0, s>>>(xp, nb, v8, codes, scales); break;
+    case DT_BF16: mxfp4_quantize_kernel<DT_BF16><<<grid, 256, 0, s>>>(xp, nb, v8, codes, scales); break;
+    default: mxfp4_quantize_kernel<DT_F16><<<grid, 256, 0, s>>>(xp, nb, v8, codes, scales); break;
+  }
+  return last_error();
+}
+
+int nvfp4_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n, int out_dtype, void* out,
+                           void* stream) {
+  if (!dtype_ok(out_dtype)) return NVFP4_ERR_ARG;
+  if (n < 0 || n % 32 != 0) return NVFP4_ERR_SIZE;
+  if (n == 0) return NVFP4_OK;
+  if (codes == nullptr || scales == nullptr || out == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(out, 16)) return NVFP4_ERR_ALIGN;
+  const int64_t nb = n / 32;
+  const int grid = grid_for(nb, 256, 8);
+  const int v8 = aligned(out, 32) ? 1 : 0;
+  char* o = static_cast<char*>(out);
+  cudaStream_t s = S(stream);
+  switch (out_dtype) {
+    case DT_F32: mxfp4_dequantize_kernel<DT_F32><<<grid, 256, 0, s>>>(codes, scales, nb, o, v8); break;
+    case DT_BF16: mxfp4_dequantize_kernel<DT_BF16><<<grid, 256, 0, s>>>(codes, scales, nb, o, v8); break;
+    default: mxfp4_dequantize_kernel<DT_F16><<<grid, 256, 0, s>>>(codes, scales, nb, o, v8); break;
+  }
+  return last_error();
+}
+
 int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens, int recent_tokens,
                     int rotate, float* gscale, void* stream) {
   if (gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
