@@ -429,6 +429,41 @@ int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, i
   return 0;
 }
 
+/* ---- multi-scale deformable attention forward (see the header) ---- */
+static double msda_corner(const float* value, int64_t b, int64_t key0, int64_t H, int64_t W, int64_t yy, int64_t xx,
+                          int64_t nkeys, int64_t heads, int64_t ch, int64_t h, int64_t c) {
+  if (yy < 0 || xx < 0 || yy >= H || xx >= W) return 0.0;
+  const int64_t key = key0 + yy * W + xx;
+  return (double)value[((b * nkeys + key) * heads + h) * ch + c];
+}
+
+int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* start, const float* loc, const float* w,
+                     int64_t bs, int64_t nkeys, int64_t heads, int64_t ch, int64_t L, int64_t P, int64_t nq, double* out) {
+  for (int64_t b = 0; b < bs; ++b)
+    for (int64_t q = 0; q < nq; ++q)
+      for (int64_t h = 0; h < heads; ++h)
+        for (int64_t c = 0; c < ch; ++c) {
+          double acc = 0.0;
+          for (int64_t l = 0; l < L; ++l) {
+            const int64_t H = shapes[2 * l], W = shapes[2 * l + 1];
+            for (int64_t p = 0; p < P; ++p) {
+              const int64_t i = (((b * nq + q) * heads + h) * L + l) * P + p;
+              const double x = (double)loc[2 * i] * (double)W - 0.5, y = (double)loc[2 * i + 1] * (double)H - 0.5;
+              if (!(x > -1.0 && y > -1.0 && x < (double)W && y < (double)H)) continue;
+              const int64_t x0 = (int64_t)floor(x), y0 = (int64_t)floor(y);
+              const double fx = x - (double)x0, fy = y - (double)y0;
+              const double v = (1 - fy) * (1 - fx) * msda_corner(value, b, start[l], H, W, y0, x0, nkeys, heads, ch, h, c) +
+                               (1 - fy) * fx * msda_corner(value, b, start[l], H, W, y0, x0 + 1, nkeys, heads, ch, h, c) +
+                               fy * (1 - fx) * msda_corner(value, b, start[l], H, W, y0 + 1, x0, nkeys, heads, ch, h, c) +
+                               fy * fx * msda_corner(value, b, start[l], H, W, y0 + 1, x0 + 1, nkeys, heads, ch, h, c);
+              acc += (double)w[i] * v;
+            }
+          }
+          out[((b * nq + q) * heads + h) * ch + c] = acc;
+        }
+  return 0;
+}
+
 /* ---- MXFP4 (see the header) ---- */
 /* floor(log2(a)) of a finite a > 0, from its bit pattern */
 static int ilog2_floor(float a) {

@@ -107,6 +107,18 @@ int ref_kv_mixed(const uint16_t* k, int64_t B, int64_t H, int64_t T, int64_t D, 
 int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, int64_t n, int64_t D, int rotate,
                   float g, int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0);
 
+/* ---- Multi-scale deformable attention forward on quantized values ----
+ * [BEV] section 5-7: only the value tensor is stored in low precision; sampling locations, attention
+ * weights, the bilinear interpolation and the accumulation stay in full precision.  For every batch
+ * b, query q and head h:
+ *   out[b,q,h,c] = sum_l sum_p w[b,q,h,l,p] * bilinear_l(value[b, start_l + .., h, c], x * W_l - 0.5, y * H_l - 0.5)
+ * with (x, y) = loc[b,q,h,l,p], level l a H_l x W_l map starting at key start_l, bilinear weights from
+ * the fractional parts and corners outside the map contributing zero.  value: [bs, nkeys, heads, ch]
+ * (FP32, e.g. the dequantized NVFP4 values); loc: [bs, nq, heads, L, P, 2]; w: [bs, nq, heads, L, P];
+ * shapes: L pairs (H_l, W_l), start: L key offsets; out: [bs, nq, heads, ch] in double. */
+int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* start, const float* loc, const float* w,
+                     int64_t bs, int64_t nkeys, int64_t heads, int64_t ch, int64_t L, int64_t P, int64_t nq, double* out);
+
 /* ---- MXFP4, the power-of-two-scaled comparison format ----
  * [NV] compares NVFP4 with "simple power-of-two scaling like MXFP4".  MXFP4 as the OCP Microscaling
  * (MX) v1.0 specification defines it: blocks of 32 elements, one E8M0 scale X = 2^e with

@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "ref_hadamard16": (I, [P, I64, I, P, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+            "ref_msda_forward": (I, [P, P, P, P, P, I64, I64, I64, I64, I64, I64, I64, P]),
             "ref_mxfp4_quantize": (I, [P, I64, I, P, P]),
             "ref_mxfp4_dequantize": (I, [P, P, I64, I, P]),
             "ref_kv_append": (I, [P, I64, I64, I64, I64, I64, I, F, I, I, P, P, I64, I64]),
@@ -339,4 +340,21 @@ def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray, out_dtype: int = F32
     rc = lib().ref_mxfp4_dequantize(_p(codes), _p(scales), n, out_dtype, _p(out))
     if rc != 0:
         raise ValueError(f"ref_mxfp4_dequantize returned {rc}")
+    return out
+
+
+# ---- multi-scale deformable attention forward ----
+def msda_forward(value: np.ndarray, shapes, loc: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """value float32 [bs, nkeys, heads, ch]; shapes [(H_l, W_l)]; loc float32 [bs, nq, heads, L, P, 2];
+    w float32 [bs, nq, heads, L, P].  Returns float64 [bs, nq, heads, ch]."""
+    value = np.ascontiguousarray(value, np.float32)
+    loc = np.ascontiguousarray(loc, np.float32)
+    w = np.ascontiguousarray(w, np.float32)
+    bs, nkeys, heads, ch = value.shape
+    _, nq, _, L, P, _ = loc.shape
+    sh = np.ascontiguousarray(np.asarray(shapes, np.int64).reshape(L, 2))
+    start = np.ascontiguousarray(np.concatenate([[0], np.cumsum(sh[:, 0] * sh[:, 1])[:-1]]).astype(np.int64))
+    assert int((sh[:, 0] * sh[:, 1]).sum()) == nkeys
+    out = np.empty((bs, nq, heads, ch), np.float64)
+    lib().ref_msda_forward(_p(value), _p(sh), _p(start), _p(loc), _p(w), bs, nkeys, heads, ch, L, P, nq, _p(out))
     return out
