@@ -108,6 +108,28 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
+/* ---- Multi-scale deformable attention forward on NVFP4 values ("自動運転モデル BEVFormer の NVIDIA Blackwell
+ * B200 FP8/FP4 CUDAカーネル・チューニング", sections 5-7: only the value tensor is low precision; locations,
+ * weights, interpolation and accumulation stay FP32) ----
+ *   out[b,q,h,c] = sum_l sum_p w[b,q,h,l,p] * bilinear(value level l, head h, channel c; x * W_l - 0.5, y * H_l - 0.5)
+ * (x, y) = loc[b,q,h,l,p]; corners outside the H_l x W_l map contribute zero; level l occupies keys
+ * start_l = sum_{k<l} H_k W_k .. of the value tensor.
+ * shapes: HOST array of L (H_l, W_l) pairs, 1 <= L <= 8, sum H_l W_l == nkeys (NVFP4_ERR_SIZE).
+ * loc: [bs, nq, heads, L, P, 2] FP32, w: [bs, nq, heads, L, P] FP32, out: [bs, nq, heads, ch] FP32
+ * (32-byte aligned).  ch (channels per head) must be 16, 32 or 64. */
+
+/* Values as NVFP4 quantized along the channels: codes [bs, nkeys, heads, ch/2] (16-byte aligned),
+ * scales [bs, nkeys, heads, ch/16] (E4M3 block scales), gscale the device tensor scale; the value
+ * used is E2M1(code) * E4M3(scale) * g (the g multiply is applied once to each output). */
+int nvfp4_msda_forward_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t bs,
+                             int64_t nkeys, int64_t heads, int64_t ch, const int64_t* shapes, int L, int P, int64_t nq,
+                             const float* loc, const float* w, float* out, void* stream);
+
+/* The full-precision twin: value [bs, nkeys, heads, ch] in dtype (FP32 / BF16 / F16, 16-byte aligned). */
+int nvfp4_msda_forward(const void* value, int dtype, int64_t bs, int64_t nkeys, int64_t heads, int64_t ch,
+                       const int64_t* shapes, int L, int P, int64_t nq, const float* loc, const float* w, float* out,
+                       void* stream);
+
 /* ---- MXFP4, the comparison format ("NVIDIAのFP4推論が50倍の効率を実現", 超低精度推論を支えるアーキテクチャ:
  * NVFP4 against simple power-of-two scaling such as MXFP4) ----
  * MXFP4 as the OCP Microscaling (MX) v1.0 specification defines it (not on the pages): blocks of 32

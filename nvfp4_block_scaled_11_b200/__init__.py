@@ -18,6 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
+    "msda_forward",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -38,6 +39,8 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_msda_forward_nvfp4": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
+    "nvfp4_msda_forward": (_I, [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
     "nvfp4_mxfp4_quantize": (_I, [_P, _I64, _I, _P, _P, _P]),
     "nvfp4_mxfp4_dequantize": (_I, [_P, _P, _I64, _I, _P, _P]),
     "nvfp4_kv_gscale": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
@@ -345,4 +348,36 @@ def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out_dtype=torch.
     out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
     _check(lib().nvfp4_mxfp4_dequantize(_ptr(codes), _ptr(scales), n, DTYPE_CODE[out.dtype], _ptr(out),
                                         _stream(codes)))
+    return out
+
+
+# ---- multi-scale deformable attention forward on NVFP4 (or full-precision) values ----
+def msda_forward(value, shapes, loc: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """value: a tensor [bs, nkeys, heads, ch] (float32 / bfloat16 / float16), or the NVFP4 triple
+    (codes uint8 [bs, nkeys, heads, ch/2], scales uint8 [bs, nkeys, heads, ch/16], gscale float32[1]);
+    shapes: sequence of (H_l, W_l); loc [bs, nq, heads, L, P, 2] and w [bs, nq, heads, L, P] float32.
+    Returns out [bs, nq, heads, ch] float32."""
+    import numpy as np
+    _cuda(loc, "loc"), _cuda(w, "w")
+    sh = np.ascontiguousarray(np.asarray(shapes, np.int64).reshape(-1, 2))
+    bs, nq, heads, L, P, _ = loc.shape
+    if isinstance(value, (tuple, list)):
+        codes, scales, gscale = value
+        for t, nm in ((codes, "codes"), (scales, "scales"), (gscale, "gscale")):
+            _cuda(t, nm)
+        _, nkeys, _, ch2 = codes.shape
+        ch = 2 * ch2
+    else:
+        _cuda(value, "value")
+        _, nkeys, _, ch = value.shape
+    if out is None:
+        out = torch.empty((bs, nq, heads, ch), dtype=torch.float32, device=loc.device)
+    _cuda(out, "out")
+    shp = sh.ctypes.data
+    if isinstance(value, (tuple, list)):
+        _check(lib().nvfp4_msda_forward_nvfp4(_ptr(codes), _ptr(scales), _ptr(gscale), bs, nkeys, heads, ch, shp,
+                                              L, P, nq, _ptr(loc), _ptr(w), _ptr(out), _stream(loc)))
+    else:
+        _check(lib().nvfp4_msda_forward(_ptr(value), _dt(value), bs, nkeys, heads, ch, shp, L, P, nq, _ptr(loc),
+                                        _ptr(w), _ptr(out), _stream(loc)))
     return out

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/nvfp4.h"
+#include "msda.cuh"
 #include "search.cuh"
 
 using namespace nvfp4;
@@ -162,6 +163,45 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
       return NVFP4_ERR_CUDA;
   }
   return check_finite_sync(gscale_in, s);
+}
+
+// Validation shared by the two deformable-attention entry points; fills the level fields of p.
+int msda_setup(MsdaParams& p, int64_t bs, int64_t nkeys, int64_t heads, int64_t ch, const int64_t* shapes, int L, int P,
+               int64_t nq, const float* loc, const float* w, float* out) {
+  if (L < 1 || L > kMsdaMaxLevels || P < 1 || shapes == nullptr) return NVFP4_ERR_ARG;
+  if (bs < 0 || nkeys < 0 || heads < 0 || nq < 0 || (ch != 16 && ch != 32 && ch != 64)) return NVFP4_ERR_SIZE;
+  int64_t keys = 0;
+  for (int l = 0; l < L; ++l) {
+    const int64_t H = shapes[2 * l], W = shapes[2 * l + 1];
+    if (H < 1 || W < 1 || H >= (1 << 24) || W >= (1 << 24)) return NVFP4_ERR_SIZE;
+    p.H[l] = (int)H;
+    p.W[l] = (int)W;
+    p.start[l] = keys;
+    keys += H * W;
+  }
+  if (keys != nkeys) return NVFP4_ERR_SIZE;
+  p.nkeys = nkeys;
+  p.heads = heads;
+  p.nq = nq;
+  p.total = bs * nq * heads;
+  p.L = L;
+  p.P = P;
+  p.loc = loc;
+  p.w = w;
+  p.out = out;
+  if (p.total == 0) return NVFP4_OK;
+  if (loc == nullptr || w == nullptr || out == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(loc, 4) || !aligned(w, 4) || !aligned(out, 32)) return NVFP4_ERR_ALIGN;
+  return NVFP4_OK;
+}
+
+template <int VT>
+int msda_launch(const MsdaParams& p, int64_t ch, cudaStream_t s) {
+  const int grid = grid_for(p.total, 128, 16);
+  if (ch == 16) msda_forward_kernel<VT, 16><<<grid, 128, 0, s>>>(p);
+  else if (ch == 32) msda_forward_kernel<VT, 32><<<grid, 128, 0, s>>>(p);
+  else msda_forward_kernel<VT, 64><<<grid, 128, 0, s>>>(p);
+  return last_error();
 }
 
 }  // namespace
@@ -359,6 +399,36 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
   if (int rc = last_error()) return rc;
   return check_finite_sync(gscale, s);
+}
+
+int nvfp4_msda_forward_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t bs,
+                             int64_t nkeys, int64_t heads, int64_t ch, const int64_t* shapes, int L, int P, int64_t nq,
+                             const float* loc, const float* w, float* out, void* stream) {
+  MsdaParams p{};
+  if (int rc = msda_setup(p, bs, nkeys, heads, ch, shapes, L, P, nq, loc, w, out)) return rc;
+  if (p.total == 0) return NVFP4_OK;
+  if (codes == nullptr || scales == nullptr || gscale == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
+  p.codes = codes;
+  p.scales = scales;
+  p.gsrc = gscale;
+  return msda_launch<MSDA_NVFP4>(p, ch, S(stream));
+}
+
+int nvfp4_msda_forward(const void* value, int dtype, int64_t bs, int64_t nkeys, int64_t heads, int64_t ch,
+                       const int64_t* shapes, int L, int P, int64_t nq, const float* loc, const float* w, float* out,
+                       void* stream) {
+  if (!dtype_ok(dtype)) return NVFP4_ERR_ARG;
+  MsdaParams p{};
+  if (int rc = msda_setup(p, bs, nkeys, heads, ch, shapes, L, P, nq, loc, w, out)) return rc;
+  if (p.total == 0) return NVFP4_OK;
+  if (value == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(value, 16)) return NVFP4_ERR_ALIGN;
+  p.value = static_cast<const char*>(value);
+  cudaStream_t s = S(stream);
+  if (dtype == DT_F32) return msda_launch<MSDA_F32>(p, ch, s);
+  if (dtype == DT_F16) return msda_launch<MSDA_F16>(p, ch, s);
+  return msda_launch<MSDA_BF16>(p, ch, s);
 }
 
 int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales, void* stream) {

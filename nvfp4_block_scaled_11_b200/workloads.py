@@ -111,6 +111,19 @@ def weight_bf16(device="cpu", n_out: int = 8192, n_in: int = 8192) -> torch.Tens
     return (w * n_in ** -0.5).to(torch.bfloat16)
 
 
+def msda_inputs(device="cpu", nq: int = 10000, bs: int = 6, heads: int = 8, points: int = 4, scale: float = 1.0):
+    """Sampling locations and attention weights for deformable attention over the `bev_f16` value maps
+    (levels LEVELS): loc [bs, nq, heads, L, P, 2] ~ U(-0.05, 1.05) (some points fall off the map),
+    w [bs, nq, heads, L, P] = softmax over the L*P points of N(0, 1) logits; seed 13."""
+    nq = max(1, int(nq * scale))
+    g = _gen(13, device)
+    L = len(LEVELS)
+    loc = torch.rand((bs, nq, heads, L, points, 2), generator=g, device=device) * 1.1 - 0.05
+    logits = torch.randn((bs, nq, heads, L * points), generator=g, device=device)
+    w = torch.softmax(logits, dim=-1).reshape(bs, nq, heads, L, points)
+    return loc.contiguous(), w.contiguous()
+
+
 def make(name: str, device="cpu", scale: float = 1.0, shard: int = 0) -> Workload:
     if name == "act_f32":
         return Workload(name, act_f32(device, scale), -2, 6, "quantize", "FP32 [1024,4096] N(0,1), seed 0")
