@@ -12,7 +12,8 @@ configuration the throughput target is stated on.  Every step's input (4 GiB) is
 
 Workloads: stream_f32 (default), act_f32, act_bf16, kv_bf16, bev_f16, and gemm_nvfp4 -- the tensor-core
 consumer: ScaleSearch-quantized BF16 activations [8192, 8192] times NVFP4 weights [8192, 8192] on the
-tensor cores, reported in TFLOP/s against the FP4 tensor roofline.
+tensor cores, reported in TFLOP/s against the FP4 tensor roofline; and msda_nvfp4 -- deformable attention
+over the BEVFormer value maps with ScaleSearch NVFP4 values, reported in queries/s.
 
 Prints ONE JSON line on rank 0.  Times are CUDA events on the launching stream, max over ranks.
 `--impl reference` times the CPU oracle (the plain C definition) on a bounded sample of the same
@@ -458,6 +459,204 @@ def run_gemm(args, rank, world, dev):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------------------------
+# Deformable attention on NVFP4 values (BEVFormer value maps)
+# ------------------------------------------------------------------------------------------------
+MSDA_METRIC = "deformable attention forward queries/s (ScaleSearch NVFP4 values, BEVFormer value maps)"
+
+
+def msda_config(args):
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    bs, nq, heads, L, P = 6, max(1, int(10000 * args.scale)), 8, len(W.LEVELS), 4   # as W.msda_inputs draws them
+    return {
+        "workload": f"msda_nvfp4 (value FP16 [6,30825,8,32] = bev_f16, levels {list(W.LEVELS)}; {nq} queries per "
+                    f"camera, {L} levels x {P} points, loc ~ U(-0.05,1.05), softmax weights; seeds 5, 13)",
+        "window": [args.f_lo, args.f_hi],
+        "step": "value: amax + g + ScaleSearch quantize (blocks of 16 channels); deformable attention forward "
+                "gathering NVFP4 values, FP32 interpolation and accumulation",
+        "l2": "L2 flushed between steps by a 256 MiB write (not timed)",
+        "bs": bs, "nq": nq, "heads": heads, "levels": L, "points": P, "channels": 32,
+    }
+
+
+def oracle_msda_sample(args, per_camera=10000):
+    import numpy as np
+    import torch
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    from oracle import oracle as O
+    value = W.bev_f16("cpu")
+    bs, nk, heads, ch = value.shape
+    loc, w = W.msda_inputs("cpu", scale=args.scale)
+    vh = value.contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    c, sc, g, _, _ = O.quantize(vh, args.f_lo, args.f_hi, dtype=O.F16)
+    vq = O.dequantize(c, sc, g).reshape(bs, nk, heads, ch)
+    per_camera = min(per_camera, loc.shape[1])
+    ls, ws = loc[:, :per_camera].contiguous().numpy(), w[:, :per_camera].contiguous().numpy()
+
+    def step():
+        O.msda_forward(vq, W.LEVELS, ls, ws)
+
+    return step, bs * per_camera, f"{per_camera} queries per camera x {bs} cameras, fp64 oracle forward on " \
+                                  f"oracle-quantized values (value quantization not timed)"
+
+
+def run_msda(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    value = W.bev_f16(dev)
+    bs, nk, heads, ch = value.shape
+    loc, w = W.msda_inputs(dev, scale=args.scale)
+    nq, L, P = loc.shape[1], loc.shape[3], loc.shape[4]
+    n = value.numel()
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(n // 16, dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    out = torch.empty((bs, nq, heads, ch), dtype=torch.float32, device=dev)
+    trip = (codes.view(bs, nk, heads, ch // 2), scales.view(bs, nk, heads, ch // 16), g)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        nv.quantize(value.reshape(-1), args.f_lo, args.f_hi, codes=codes, scales=scales, gscale=g)
+        if evs:
+            evs[1].record(stream)
+        nv.msda_forward(trip, W.LEVELS, loc, w, out=out)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        step(evs[k])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    m_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    def twin_ms(v):
+        ts = []
+        for k in range(max(3, args.steps // 10) + 3):
+            flush.fill_(float(k))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            nv.msda_forward(v, W.LEVELS, loc, w, out=out)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.mean(ts[3:])
+
+    f16_ms = twin_ms(value)
+    v32 = value.float()
+    f32_ms = twin_ms(v32)
+    # accuracy of the NVFP4 path against the FP32-value forward (normalised absolute error)
+    o4 = nv.msda_forward(trip, W.LEVELS, loc, w).double()
+    o32 = nv.msda_forward(v32, W.LEVELS, loc, w).double()
+    nae = float((o4 - o32).abs().mean() / o32.abs().mean())
+    del v32, o4, o32
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    peak, src = peaks()
+    msda_bytes = n // 2 + n // 16 + loc.numel() * 4 + w.numel() * 4 + out.numel() * 4
+    achieved = msda_bytes / (m_ms * 1e-3) / 1e9
+    line = {
+        "metric": MSDA_METRIC, "value": world * bs * nq * args.steps / (elapsed_ms * 1e-3), "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 values, f32 math",
+        "data": SOURCE_NOTE, "config": msda_config(args),
+        "roofline": {"bound": "hbm", "kernel": "msda_forward_kernel<NVFP4, 32> (gather-latency bound; value map "
+                     "resident in L2)", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": src, "bytes_per_launch": msda_bytes},
+        "breakdown_ms": {"quantize_value": q_ms, "msda_nvfp4": m_ms, "msda_f16_twin": f16_ms, "msda_f32_twin": f32_ms},
+        "value_bytes": {"nvfp4": n // 2 + n // 16, "f16": n * 2, "f32": n * 4},
+        "normalised_abs_error_vs_f32_values": nae,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_e2e and args.e2e_steps > 0:
+        hv = torch.empty(value.shape, dtype=value.dtype, pin_memory=True)
+        hv.copy_(value)
+        hl = torch.empty(loc.shape, dtype=loc.dtype, pin_memory=True)
+        hl.copy_(loc)
+        hw = torch.empty(w.shape, dtype=w.dtype, pin_memory=True)
+        hw.copy_(w)
+        ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dv, dl, dw = torch.empty_like(value), torch.empty_like(loc), torch.empty_like(w)
+
+        def e2e_step():
+            dv.copy_(hv, non_blocking=True)
+            dl.copy_(hl, non_blocking=True)
+            dw.copy_(hw, non_blocking=True)
+            nv.quantize(dv.reshape(-1), args.f_lo, args.f_hi, codes=codes, scales=scales, gscale=g)
+            nv.msda_forward(trip, W.LEVELS, dl, dw, out=out)
+            ho.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * bs * nq * args.e2e_steps / (e2e_ms * 1e-3), "unit": "queries/s",
+                       "h2d_bytes_per_step": (hv.numel() * 2 + hl.numel() * 4 + hw.numel() * 4),
+                       "d2h_bytes_per_step": ho.numel() * 4}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_o, nqs, desc = oracle_msda_sample(args)
+        t = time.perf_counter()
+        step_o()
+        el = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": nqs / el, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                "sample": desc + f", {el:.2f} s single-threaded C"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_msda_reference(args, rank, world):
+    if rank != 0:
+        return
+    step, nqs, desc = oracle_msda_sample(args)
+    steps = max(1, min(args.steps, 5))
+    step()
+    t = time.perf_counter()
+    for _ in range(steps):
+        step()
+    el = time.perf_counter() - t
+    val = nqs * steps / el
+    print(json.dumps({
+        "impl": "reference", "metric": MSDA_METRIC, "value": val, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": 1, "ms_per_step": el / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 oracle", "data": SOURCE_NOTE, "config": msda_config(args),
+        "cpu_baseline": {"value": val, "unit": "queries/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -477,6 +676,8 @@ def main():
     if args.impl == "reference":
         if args.workload == "gemm_nvfp4":
             run_gemm_reference(args, rank, world)
+        elif args.workload == "msda_nvfp4":
+            run_msda_reference(args, rank, world)
         else:
             run_reference(args, rank, world)
         return
@@ -496,6 +697,9 @@ def main():
 
     if args.workload == "gemm_nvfp4":
         run_gemm(args, rank, world, dev)
+        return
+    if args.workload == "msda_nvfp4":
+        run_msda(args, rank, world, dev)
         return
     w = W.make(args.workload, dev, args.scale, shard=rank)
     x = w.x.contiguous()
