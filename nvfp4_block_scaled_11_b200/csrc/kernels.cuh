@@ -131,12 +131,30 @@ struct QuantParams {
   int64_t out_cap, out_t0;
 };
 
+// KV launches cover fewer than 2^32 blocks (checked by the host), so block indices split with 32-bit
+// arithmetic: block b is (bh, t, j) = (head row, middle token, block column).
+__device__ __forceinline__ void kv_split(int64_t b, int64_t Tm, int64_t bpr, uint32_t& bh, uint32_t& t, uint32_t& j) {
+  const uint32_t ub = (uint32_t)b, per = (uint32_t)(Tm * bpr), ubpr = (uint32_t)bpr;
+  bh = ub / per;
+  const uint32_t rem = ub - bh * per;
+  t = rem / ubpr;
+  j = rem - t * ubpr;
+}
+
+// Element offset of KV block b in K[BH, T, D]: middle token t of head row bh, block column j.
+__device__ __forceinline__ int64_t kv_block_elem(int64_t b, int64_t Tm, int64_t bpr, int64_t T, int64_t sink,
+                                                 int64_t D) {
+  uint32_t bh, t, j;
+  kv_split(b, Tm, bpr, bh, t, j);
+  return ((int64_t)bh * T + sink + t) * D + 16 * (int64_t)j;
+}
+
 // Output block index of block b (input order): b itself, or its row in the KV cache being appended to.
 __device__ __forceinline__ int64_t out_block(const QuantParams& p, int64_t b) {
   if (p.out_cap == 0) return b;
-  const int64_t per = p.Tm * p.bpr;
-  const int64_t bh = b / per, rem = b - bh * per;  // rem = token * bpr + block column
-  return (bh * p.out_cap + p.out_t0) * p.bpr + rem;
+  uint32_t bh, t, j;
+  kv_split(b, p.Tm, p.bpr, bh, t, j);
+  return ((int64_t)bh * p.out_cap + p.out_t0 + t) * p.bpr + j;
 }
 
 // Byte of block b's scale.  Linear: b.  Tile layout (block-scaled tensor-core MMA operand): 512-byte
@@ -198,12 +216,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < p.nblocks; b += stride) {
     int64_t elem;
     if (KV) {
-      const int64_t per_bh = p.Tm * p.bpr;
-      const int64_t bh = b / per_bh;
-      const int64_t rem = b - bh * per_bh;
-      const int64_t t = rem / p.bpr;
-      const int64_t j = rem - t * p.bpr;
-      elem = (bh * p.T + p.sink + t) * p.D + 16 * j;
+      elem = kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D);
     } else {
       elem = 16 * b;
     }
@@ -525,12 +538,7 @@ __global__ void __launch_bounds__(256) kv_amax_kernel(const char* __restrict__ k
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t m = 0;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < ngroups; b += stride) {
-    const int64_t per_bh = Tm * bpr;
-    const int64_t bh = b / per_bh;
-    const int64_t rem = b - bh * per_bh;
-    const int64_t t = rem / bpr;
-    const int64_t j = rem - t * bpr;
-    const int64_t elem = (bh * T + sink + t) * D + 16 * j;
+    const int64_t elem = kv_block_elem(b, Tm, bpr, T, sink, D);
     float x[16];
     load_block<DT_BF16>(k + 2 * elem, v8 != 0, x);
     if (ROT) fwht16(x);

@@ -347,7 +347,7 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   if (BH > 0 && sink_tokens > 0 && sink_bf16 == nullptr) return NVFP4_ERR_ARG;
   if (BH > 0 && recent_tokens > 0 && recent_bf16 == nullptr) return NVFP4_ERR_ARG;
   if (ngroups > 0 && (codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
-  if (mma && ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if ((BH > 0 && !aligned(k_bf16, 16)) || (sink_bf16 && !aligned(sink_bf16, 16)) ||
       (recent_bf16 && !aligned(recent_bf16, 16)) || (codes && !aligned(codes, 8)) || !aligned(gscale, 4))
     return NVFP4_ERR_ALIGN;
@@ -477,6 +477,7 @@ int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t
     return NVFP4_ERR_SIZE;
   const int64_t Tm = T - sink_tokens - recent_tokens;
   const int64_t ngroups = B * H * Tm * (D / 16);
+  if (ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if (ngroups > 0 && k_bf16 == nullptr) return NVFP4_ERR_ARG;
   if ((ngroups > 0 && !aligned(k_bf16, 16)) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
   cudaStream_t s = S(stream);
@@ -502,6 +503,7 @@ int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, in
   if (BH < 0 || T < 0 || n < 0 || first < 0 || t0 < 0 || cap < 0 || D <= 0 || D % 16 != 0) return NVFP4_ERR_SIZE;
   if (first + n > T || t0 + n > cap) return NVFP4_ERR_SIZE;
   if (scale_layout == 1 && BH * cap * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (BH * n * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if (BH == 0 || n == 0) return NVFP4_OK;
   if (k_bf16 == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(k_bf16, 16) || !aligned(codes, 8) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;

@@ -435,12 +435,7 @@ __device__ __forceinline__ const char* block_src(const QuantParams& p, int64_t b
   constexpr int ES = DT == DT_F32 ? 4 : 2;
   int64_t elem;
   if (KV) {
-    const int64_t per_bh = p.Tm * p.bpr;
-    const int64_t bh = b / per_bh;
-    const int64_t rem = b - bh * per_bh;
-    const int64_t t = rem / p.bpr;
-    const int64_t j = rem - t * p.bpr;
-    elem = (bh * p.T + p.sink + t) * p.D + 16 * j;
+    elem = kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D);
   } else {
     elem = 16 * b;
   }
@@ -460,6 +455,11 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   __shared__ CandEntry tab[128];
   __shared__ float thr[128];
   __shared__ int64_t defer[8][kDeferCap];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const bool v8 = p.v8 != 0;
+  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  u64 xn[8];
+  if (b < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b), v8, xn);  // in flight while the tables are built
   float g = *p.g_src;
   if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
   const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
@@ -482,12 +482,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
     dcount = 0;
   };
 
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const bool v8 = p.v8 != 0;
-  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t warp0 = b - lane;
-  u64 xn[8];
-  if (b < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b), v8, xn);
   for (int64_t wb = warp0; wb < p.nblocks; wb += stride, b += stride) {
     const bool active = b < p.nblocks;
     u64 x2[8];
