@@ -103,7 +103,8 @@ int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dty
  * sink_bf16: [B,H,sink_tokens,D] and recent_bf16: [B,H,recent_tokens,D] receive the first and last
  * tokens verbatim.  The T_mid = T - sink - recent middle tokens are rotated along D by FWHT-16 when
  * rotate != 0 (kept in FP32) and quantized along D with one tensor scale over the rotated middle:
- * codes [B,H,T_mid,D/2], scales [B,H,T_mid,D/16], gscale one device float. */
+ * codes [B,H,T_mid,D/2], scales [B,H,T_mid,D/16], gscale one device float.
+ * B * H * T_mid * D / 16 must be below 2^32 (NVFP4_ERR_SIZE). */
 int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
@@ -157,7 +158,7 @@ int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t
  * NVFP4 cache with `cap` rows per (batch, head): codes [BH, cap, D/2]; scales [BH, cap, D/16] when
  * scale_layout == 0, or the tensor-core tile layout of BH matrices [cap, D] when scale_layout == 1
  * (nvfp4_sf_mma_bytes(cap, D, BH) bytes; padding bytes are not written).  Other rows are untouched.
- * Requires first + n <= T and t0 + n <= cap (NVFP4_ERR_SIZE). */
+ * Requires first + n <= T, t0 + n <= cap and BH * n * D / 16 < 2^32 (NVFP4_ERR_SIZE). */
 int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, int64_t n, int64_t D, int rotate,
                     int f_lo, int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
                     int scale_layout, void* stream);
