@@ -8,10 +8,10 @@
 //   out[b,q,h,c] = g * sum_l sum_p w * sum_corners bilinear_weight * E2M1(code) * E4M3(block scale)
 // with corners outside the level's map contributing zero (sampling at loc * size - 0.5).
 //
-// One thread per (batch, query, head) keeps the head's CH channels in registers: the location,
-// bounds test and bilinear weights of a sampling point are computed once for all channels, each
-// corner is one gather of CH/2 code bytes plus CH/16 scale bytes, the block scale is folded into the
-// corner weight and the channel updates are packed FP32x2 FMAs.  The full-precision twin (FP32 / F16
+// A thread owns a slice of whole 16-channel blocks of one (batch, query, head) in registers: the
+// location, bounds test and bilinear weights of a sampling point are computed once per slice, each
+// corner is one gather of the slice's code bytes plus its scale bytes, the block scale is folded into
+// the corner weight and the channel updates are packed FP32x2 FMAs.  The full-precision twin (FP32 / F16
 // / BF16 values) runs the same loop on plain values, for the footprint / speed comparison.
 #pragma once
 
@@ -36,70 +36,95 @@ struct MsdaParams {
   int64_t start[kMsdaMaxLevels];
 };
 
-// acc[k] += cw * (value pair k) for the CH/2 channel pairs of one corner.
-template <int VT, int CH>
-__device__ __forceinline__ void msda_corner(const MsdaParams& p, int64_t kh, float cw, u64 (&acc)[CH / 2]) {
+// Raw bytes of one corner's channel slice [coff, coff + CHT) (kh = key * heads + head): loaded for all
+// four corners of a sampling point before any of them is used, so the gathers overlap.
+template <int VT, int CHT>
+struct CornerData {
+  static constexpr int kWords = VT == MSDA_NVFP4 ? CHT / 8 : (VT == MSDA_F32 ? CHT : CHT / 2);
+  uint32_t w[kWords];
+  uint32_t sc;  // NVFP4: the CHT/16 scale bytes (little-endian)
+};
+
+template <int VT, int CH, int CHT>
+__device__ __forceinline__ void msda_load(const MsdaParams& p, int64_t kh, int coff, CornerData<VT, CHT>& d) {
   if constexpr (VT == MSDA_NVFP4) {
-    const uint8_t* cp = p.codes + kh * (CH / 2);
-    uint32_t cw32[CH / 8];
-    if constexpr (CH == 16) {
+    const uint8_t* cp = p.codes + kh * (CH / 2) + coff / 2;
+    if constexpr (CHT == 16) {
       const uint2 v = *reinterpret_cast<const uint2*>(cp);
-      cw32[0] = v.x; cw32[1] = v.y;
+      d.w[0] = v.x; d.w[1] = v.y;
     } else {
 #pragma unroll
-      for (int k = 0; k < CH / 32; ++k) {
+      for (int k = 0; k < CHT / 32; ++k) {
         const uint4 v = *reinterpret_cast<const uint4*>(cp + 16 * k);
-        cw32[4 * k] = v.x; cw32[4 * k + 1] = v.y; cw32[4 * k + 2] = v.z; cw32[4 * k + 3] = v.w;
+        d.w[4 * k] = v.x; d.w[4 * k + 1] = v.y; d.w[4 * k + 2] = v.z; d.w[4 * k + 3] = v.w;
       }
     }
-    const uint8_t* sp = p.scales + kh * (CH / 16);
+    const uint8_t* sp = p.scales + kh * (CH / 16) + coff / 16;
+    d.sc = 0u;
 #pragma unroll
-    for (int blk = 0; blk < CH / 16; ++blk) {
-      const float s = __fmul_rn(cw, e4m3_value(sp[blk]));   // corner weight x block scale
-      const u64 ss = pk2(s, s);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {                            // byte k of the block: channels 2k, 2k+1
-        const uint32_t byte = (cw32[2 * blk + (k >> 2)] >> (8 * (k & 3))) & 0xFFu;
-        const uint32_t h2 = e2m1x2_to_f16x2(byte);
-        acc[8 * blk + k] = fma2(pk2(f16lo(h2), f16hi(h2)), ss, acc[8 * blk + k]);
-      }
-    }
-  } else if constexpr (VT == MSDA_F32) {
-    const float4* vp = reinterpret_cast<const float4*>(p.value + kh * CH * 4);
-    const u64 cc = pk2(cw, cw);
-#pragma unroll
-    for (int k = 0; k < CH / 4; ++k) {
-      const float4 v = vp[k];
-      acc[2 * k] = fma2(pk2(v.x, v.y), cc, acc[2 * k]);
-      acc[2 * k + 1] = fma2(pk2(v.z, v.w), cc, acc[2 * k + 1]);
-    }
+    for (int blk = 0; blk < CHT / 16; ++blk) d.sc |= (uint32_t)sp[blk] << (8 * blk);
   } else {
-    const uint4* vp = reinterpret_cast<const uint4*>(p.value + kh * CH * 2);
-    const u64 cc = pk2(cw, cw);
+    constexpr int ES = VT == MSDA_F32 ? 4 : 2;
+    const uint4* vp = reinterpret_cast<const uint4*>(p.value + (kh * CH + coff) * ES);
 #pragma unroll
-    for (int k = 0; k < CH / 8; ++k) {
+    for (int k = 0; k < CornerData<VT, CHT>::kWords / 4; ++k) {
       const uint4 v = vp[k];
-      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float lo = VT == MSDA_F16 ? f16lo(wd[j]) : bf16lo(wd[j]);
-        const float hi = VT == MSDA_F16 ? f16hi(wd[j]) : bf16hi(wd[j]);
-        acc[4 * k + j] = fma2(pk2(lo, hi), cc, acc[4 * k + j]);
-      }
+      d.w[4 * k] = v.x; d.w[4 * k + 1] = v.y; d.w[4 * k + 2] = v.z; d.w[4 * k + 3] = v.w;
     }
   }
 }
 
-template <int VT, int CH>
+// acc[k] += cw * (value pair k) for the CHT/2 channel pairs of one loaded corner.
+template <int VT, int CHT>
+__device__ __forceinline__ void msda_accumulate(const CornerData<VT, CHT>& d, float cw, u64 (&acc)[CHT / 2]) {
+  if constexpr (VT == MSDA_NVFP4) {
+#pragma unroll
+    for (int blk = 0; blk < CHT / 16; ++blk) {
+      const float s = __fmul_rn(cw, e4m3_value((d.sc >> (8 * blk)) & 0xFFu));   // corner weight x block scale
+      const u64 ss = pk2(s, s);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {                                             // channels 2k, 2k+1 of the block
+        const uint32_t byte = (d.w[2 * blk + (k >> 2)] >> (8 * (k & 3))) & 0xFFu;
+        const uint32_t h2 = e2m1x2_to_f16x2(byte);
+        acc[8 * blk + k] = fma2(pk2(f16lo(h2), f16hi(h2)), ss, acc[8 * blk + k]);
+      }
+    }
+  } else {
+    const u64 cc = pk2(cw, cw);
+#pragma unroll
+    for (int k = 0; k < CHT / 2; ++k) {
+      float lo, hi;
+      if (VT == MSDA_F32) {
+        lo = __uint_as_float(d.w[2 * k]);
+        hi = __uint_as_float(d.w[2 * k + 1]);
+      } else if (VT == MSDA_F16) {
+        lo = f16lo(d.w[k]);
+        hi = f16hi(d.w[k]);
+      } else {
+        lo = bf16lo(d.w[k]);
+        hi = bf16hi(d.w[k]);
+      }
+      acc[k] = fma2(pk2(lo, hi), cc, acc[k]);
+    }
+  }
+}
+
+// SPLIT threads share one (batch, query, head), each owning CH / SPLIT consecutive channels (whole
+// 16-channel blocks).
+template <int VT, int CH, int SPLIT>
 __global__ void __launch_bounds__(128) msda_forward_kernel(MsdaParams p) {
+  constexpr int CHT = CH / SPLIT;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const float g = VT == MSDA_NVFP4 ? *p.gsrc : 1.0f;
-  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < p.total; t += stride) {
+  const int64_t nthreads = p.total * SPLIT;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < nthreads; u += stride) {
+    const int64_t t = u / SPLIT;
+    const int coff = (int)(u - t * SPLIT) * CHT;
     const int64_t h = t % p.heads;
     const int64_t b = t / (p.heads * p.nq);
-    u64 acc[CH / 2];
+    u64 acc[CHT / 2];
 #pragma unroll
-    for (int k = 0; k < CH / 2; ++k) acc[k] = 0ull;
+    for (int k = 0; k < CHT / 2; ++k) acc[k] = 0ull;
     const float* lp = p.loc + t * p.L * p.P * 2;
     const float* wp = p.w + t * p.L * p.P;
     for (int l = 0; l < p.L; ++l) {
@@ -115,25 +140,27 @@ __global__ void __launch_bounds__(128) msda_forward_kernel(MsdaParams p) {
         const int x0 = (int)xf, y0 = (int)yf;
         const float fx = __fsub_rn(x, xf), fy = __fsub_rn(y, yf);
         const float gx = __fsub_rn(1.0f, fx), gy = __fsub_rn(1.0f, fy);
+        // the four corners: off-map ones read an on-map address and are skipped when accumulating
+        CornerData<VT, CHT> d[4];
+        bool ok[4];
+        float cw[4];
 #pragma unroll
-        for (int cy = 0; cy < 2; ++cy) {
-          const int yy = y0 + cy;
-          if (yy < 0 || yy >= H) continue;
-          const float wy = __fmul_rn(wt, cy ? fy : gy);
-#pragma unroll
-          for (int cx = 0; cx < 2; ++cx) {
-            const int xx = x0 + cx;
-            if (xx < 0 || xx >= W) continue;
-            const float cw = __fmul_rn(wy, cx ? fx : gx);
-            msda_corner<VT, CH>(p, (key0 + (int64_t)yy * W + xx) * p.heads + h, cw, acc);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int yy = y0 + (c >> 1), xx = x0 + (c & 1);
+          ok[c] = yy >= 0 && yy < H && xx >= 0 && xx < W;
+          const int ys = min(max(yy, 0), H - 1), xs = min(max(xx, 0), W - 1);
+          cw[c] = __fmul_rn(__fmul_rn(wt, (c >> 1) ? fy : gy), (c & 1) ? fx : gx);
+          msda_load<VT, CH, CHT>(p, (key0 + (int64_t)ys * W + xs) * p.heads + h, coff, d[c]);
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (ok[c]) msda_accumulate<VT, CHT>(d[c], cw[c], acc);
       }
     }
-    // write the head's channels (scaled by g for NVFP4): CH * 4 bytes, 32-byte aligned
-    float* o = p.out + t * CH;
+    // write this thread's channels (scaled by g for NVFP4): CHT * 4 bytes, 32-byte aligned
+    float* o = p.out + t * CH + coff;
 #pragma unroll
-    for (int k = 0; k < CH / 8; ++k) {
+    for (int k = 0; k < CHT / 8; ++k) {
       uint32_t v[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {

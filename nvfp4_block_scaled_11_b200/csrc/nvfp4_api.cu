@@ -195,12 +195,20 @@ int msda_setup(MsdaParams& p, int64_t bs, int64_t nkeys, int64_t heads, int64_t 
   return NVFP4_OK;
 }
 
+// Channels per thread: NVFP4 values keep a whole head per thread (its gathers are 8-16 bytes, so the
+// per-point location work dominates); full-precision twins split a head into 16-channel slices (their
+// gathers are 32-64 bytes per slice, and more threads in flight hide them better).  Both measured.
+template <int VT, int CH>
+void msda_launch_ch(const MsdaParams& p, cudaStream_t s) {
+  constexpr int SPLIT = VT == MSDA_NVFP4 ? 1 : CH / 16;
+  msda_forward_kernel<VT, CH, SPLIT><<<grid_for(p.total * SPLIT, 128, 16), 128, 0, s>>>(p);
+}
+
 template <int VT>
 int msda_launch(const MsdaParams& p, int64_t ch, cudaStream_t s) {
-  const int grid = grid_for(p.total, 128, 16);
-  if (ch == 16) msda_forward_kernel<VT, 16><<<grid, 128, 0, s>>>(p);
-  else if (ch == 32) msda_forward_kernel<VT, 32><<<grid, 128, 0, s>>>(p);
-  else msda_forward_kernel<VT, 64><<<grid, 128, 0, s>>>(p);
+  if (ch == 16) msda_launch_ch<VT, 16>(p, s);
+  else if (ch == 32) msda_launch_ch<VT, 32>(p, s);
+  else msda_launch_ch<VT, 64>(p, s);
   return last_error();
 }
 
