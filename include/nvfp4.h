@@ -185,6 +185,14 @@ int64_t nvfp4_sf_mma_bytes(int64_t rows, int64_t cols, int64_t batch);
 int nvfp4_quantize_mma(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
                        const float* gscale_in, uint8_t* codes, uint8_t* sf, float* gscale, void* stream);
 
+/* The transposed operand: x [batch, rows, cols] (contiguous) quantized in blocks of 16 consecutive
+ * ROWS of each column (rows % 16 == 0), written as the [batch, cols, rows] matrices: codes_t
+ * [batch, cols, rows/2] and sf_t the tile layout of cols-row matrices (nvfp4_sf_mma_bytes(cols, rows,
+ * batch) bytes).  The same as nvfp4_quantize_mma of the transposed tensor; used for V in P V^T, where
+ * the product contracts over tokens.  One tensor scale for the whole tensor. */
+int nvfp4_quantize_mma_t(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
+                         const float* gscale_in, uint8_t* codes_t, uint8_t* sf_t, float* gscale, void* stream);
+
 /* nvfp4_kv_mixed with the middle-token scales in the tile layout: each (batch, head) is one
  * [T_mid, D] matrix, so sf receives nvfp4_sf_mma_bytes(T_mid, D, B * H) bytes; it feeds
  * nvfp4_gemm_nt as the K operand of Q K^T directly. */

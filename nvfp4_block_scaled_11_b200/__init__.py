@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
-    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "kv_mixed_mma",
+    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
     "msda_forward",
 ]
@@ -47,6 +47,7 @@ _SIGS = {
     "nvfp4_kv_append": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _P]),
     "nvfp4_sf_mma_bytes": (_I64, [_I64, _I64, _I64]),
     "nvfp4_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "nvfp4_quantize_mma_t": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "nvfp4_kv_mixed_mma": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_gemm_nt": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P, _P]),
     "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),
@@ -239,6 +240,29 @@ def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torc
         _cuda(gscale_in, "gscale_in")
     _check(lib().nvfp4_quantize_mma(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
                                     _ptr(sf), _ptr(gscale), _stream(x)))
+    return codes, sf, gscale
+
+
+def quantize_mma_t(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None,
+                   codes: torch.Tensor | None = None, sf: torch.Tensor | None = None,
+                   gscale: torch.Tensor | None = None):
+    """Quantize x [rows, cols] or [batch, rows, cols] in blocks of 16 rows per column, written transposed:
+    codes uint8[..., cols, rows/2], sf (tile layout of the [cols, rows] matrices), gscale float32[1]."""
+    _cuda(x, "x")
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be [rows, cols] or [batch, rows, cols]")
+    batch, rows, cols = (1, *x.shape) if x.dim() == 2 else x.shape
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((*x.shape[:-2], cols, rows // 2), dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.empty(sf_mma_bytes(cols, rows, batch), dtype=torch.uint8, device=dev)
+    if gscale is None:
+        gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    if gscale_in is not None:
+        _cuda(gscale_in, "gscale_in")
+    _check(lib().nvfp4_quantize_mma_t(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
+                                      _ptr(sf), _ptr(gscale), _stream(x)))
     return codes, sf, gscale
 
 

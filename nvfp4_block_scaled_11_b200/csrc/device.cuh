@@ -117,6 +117,21 @@ __device__ __forceinline__ void load_block(const char* p, bool v8, float (&x)[16
   }
 }
 
+// 16 elements of one column: element i at p + i * stride_bytes (a warp reads consecutive columns).
+template <int DT>
+__device__ __forceinline__ void load_column(const char* p, int64_t stride_bytes, float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const char* q = p + i * stride_bytes;
+    if (DT == DT_F32) {
+      x[i] = __ldg(reinterpret_cast<const float*>(q));
+    } else {
+      const uint32_t h = __ldg(reinterpret_cast<const unsigned short*>(q));
+      x[i] = DT == DT_BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
+    }
+  }
+}
+
 // 16-point Walsh-Hadamard butterflies (strides 1, 2, 4, 8), then times 1/4; FP32, no contraction.
 __device__ __forceinline__ void fwht16(float (&a)[16]) {
 #pragma unroll

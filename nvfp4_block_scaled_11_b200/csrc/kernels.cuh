@@ -129,7 +129,23 @@ struct QuantParams {
   // KV append: when out_cap > 0 the Tm token rows of each (batch, head) handled by this launch are
   // written to rows out_t0 .. out_t0 + Tm - 1 of a cache with out_cap rows per (batch, head)
   int64_t out_cap, out_t0;
+  // column blocks (source mode SRC_COLS): x is [batch, rows, tr_cols] and a block is 16 consecutive
+  // rows of one column; tr_rb = rows / 16.  Blocks run column-fastest, so a warp reads rows of
+  // consecutive columns; outputs are the transposed [batch, tr_cols, rows] layout.
+  int64_t tr_cols, tr_rb;
 };
+
+// Where the 16 elements of a block come from.
+enum { SRC_LINEAR = 0, SRC_KV = 1, SRC_COLS = 2 };
+
+// Column-mode block b -> (batch l, column c, row block rb); fewer than 2^32 blocks (host-checked).
+__device__ __forceinline__ void cols_split(const QuantParams& p, int64_t b, uint32_t& l, uint32_t& c, uint32_t& rb) {
+  const uint32_t ub = (uint32_t)b, C = (uint32_t)p.tr_cols, RB = (uint32_t)p.tr_rb;
+  const uint32_t rest = ub / C;
+  c = ub - rest * C;
+  l = rest / RB;
+  rb = rest - l * RB;
+}
 
 // KV launches cover fewer than 2^32 blocks (checked by the host), so block indices split with 32-bit
 // arithmetic: block b is (bh, t, j) = (head row, middle token, block column).
@@ -149,12 +165,23 @@ __device__ __forceinline__ int64_t kv_block_elem(int64_t b, int64_t Tm, int64_t 
   return ((int64_t)bh * T + sink + t) * D + 16 * (int64_t)j;
 }
 
-// Output block index of block b (input order): b itself, or its row in the KV cache being appended to.
+// Output block index of block b (input order), fixed by the source mode at compile time: linear blocks
+// land where they are read; KV blocks land in rows out_t0.. of a cap-row cache when appending
+// (out_cap > 0); column blocks land in the transposed layout (row c of matrix l, block rb).
+template <int MODE>
 __device__ __forceinline__ int64_t out_block(const QuantParams& p, int64_t b) {
-  if (p.out_cap == 0) return b;
-  uint32_t bh, t, j;
-  kv_split(b, p.Tm, p.bpr, bh, t, j);
-  return ((int64_t)bh * p.out_cap + p.out_t0 + t) * p.bpr + j;
+  if constexpr (MODE == SRC_COLS) {
+    uint32_t l, c, rb;
+    cols_split(p, b, l, c, rb);
+    return ((int64_t)l * p.tr_cols + c) * p.tr_rb + rb;
+  } else if constexpr (MODE == SRC_KV) {
+    if (p.out_cap == 0) return b;
+    uint32_t bh, t, j;
+    kv_split(b, p.Tm, p.bpr, bh, t, j);
+    return ((int64_t)bh * p.out_cap + p.out_t0 + t) * p.bpr + j;
+  } else {
+    return b;
+  }
 }
 
 // Byte of block b's scale.  Linear: b.  Tile layout (block-scaled tensor-core MMA operand): 512-byte
@@ -201,7 +228,7 @@ __device__ __forceinline__ float block_sse_exact(const float (&a)[16], float d, 
   return s;
 }
 
-template <int DT, bool KV, bool ROT>
+template <int DT, int MODE, bool ROT>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
   __shared__ CandTable tab;
   float g = *p.g_src;
@@ -214,14 +241,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
   const int span = max(abs(p.f_lo), abs(p.f_hi));
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < p.nblocks; b += stride) {
-    int64_t elem;
-    if (KV) {
-      elem = kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D);
-    } else {
-      elem = 16 * b;
-    }
     float x[16];
-    load_block<DT>(p.x + elem * ES, p.v8 != 0, x);
+    if (MODE == SRC_COLS) {
+      uint32_t l, c, rb;
+      cols_split(p, b, l, c, rb);
+      load_column<DT>(p.x + (((int64_t)l * p.tr_rb + rb) * 16 * p.tr_cols + c) * ES, p.tr_cols * ES, x);
+    } else {
+      const int64_t elem = MODE == SRC_KV ? kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D) : 16 * b;
+      load_block<DT>(p.x + elem * ES, p.v8 != 0, x);
+    }
     if (ROT) fwht16(x);
 
     float a[16];
@@ -285,7 +313,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
         sse = s;
       }
     }
-    const int64_t ob = out_block(p, b);
+    const int64_t ob = out_block<MODE>(p, b);
     reinterpret_cast<uint2*>(p.codes)[ob] = make_uint2(lo, hi);
     p.scales[scale_index(p, ob)] = (uint8_t)scale;
     if (p.block_f) p.block_f[ob] = (int8_t)fstar;

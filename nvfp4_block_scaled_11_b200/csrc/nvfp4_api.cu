@@ -80,32 +80,33 @@ int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_
   return last_error();
 }
 
-template <int DT, bool KV, bool ROT, int NC>
+template <int DT, int MODE, bool ROT, int NC>
 void launch_search(const QuantParams& p, cudaStream_t s) {
   const int grid = grid_for(p.nblocks, 256, NVFP4_SEARCH_CTAS_PER_SM);
-  if (p.block_sse) quantize_search_kernel<DT, KV, ROT, NC, true><<<grid, 256, 0, s>>>(p);
-  else quantize_search_kernel<DT, KV, ROT, NC, false><<<grid, 256, 0, s>>>(p);
+  if (p.block_sse) quantize_search_kernel<DT, MODE, ROT, NC, true><<<grid, 256, 0, s>>>(p);
+  else quantize_search_kernel<DT, MODE, ROT, NC, false><<<grid, 256, 0, s>>>(p);
 }
 
-template <int DT, bool KV, bool ROT>
+template <int DT, int MODE, bool ROT>
 void launch_quantize_dt(const QuantParams& p, cudaStream_t s) {
   switch (p.f_hi - p.f_lo + 1) {
-    case 1: launch_search<DT, KV, ROT, 1>(p, s); break;
-    case 9: launch_search<DT, KV, ROT, 9>(p, s); break;
-    case 17: launch_search<DT, KV, ROT, 17>(p, s); break;
-    default: quantize_kernel<DT, KV, ROT><<<grid_for(p.nblocks, 256, 4), 256, 0, s>>>(p); break;
+    case 1: launch_search<DT, MODE, ROT, 1>(p, s); break;
+    case 9: launch_search<DT, MODE, ROT, 9>(p, s); break;
+    case 17: launch_search<DT, MODE, ROT, 17>(p, s); break;
+    default: quantize_kernel<DT, MODE, ROT><<<grid_for(p.nblocks, 256, 4), 256, 0, s>>>(p); break;
   }
 }
 
-template <bool KV, bool ROT>
+// MODE: SRC_LINEAR (any dtype), SRC_KV (BF16 keys), SRC_COLS (any dtype, never rotated).
+template <int MODE, bool ROT>
 int launch_quantize_t(int dtype, const QuantParams& p, cudaStream_t s) {
-  if constexpr (KV) {
-    launch_quantize_dt<DT_BF16, KV, ROT>(p, s);
+  if constexpr (MODE == SRC_KV) {
+    launch_quantize_dt<DT_BF16, MODE, ROT>(p, s);
   } else {
     switch (dtype) {
-      case DT_F32: launch_quantize_dt<DT_F32, KV, ROT>(p, s); break;
-      case DT_BF16: launch_quantize_dt<DT_BF16, KV, ROT>(p, s); break;
-      default: launch_quantize_dt<DT_F16, KV, ROT>(p, s); break;
+      case DT_F32: launch_quantize_dt<DT_F32, MODE, ROT>(p, s); break;
+      case DT_BF16: launch_quantize_dt<DT_BF16, MODE, ROT>(p, s); break;
+      default: launch_quantize_dt<DT_F16, MODE, ROT>(p, s); break;
     }
   }
   return last_error();
@@ -138,6 +139,8 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
   p.sf_rows = sf.sf_rows;
   p.sf_ctiles = sf.sf_ctiles;
   p.sf_mat_bytes = sf.sf_mat_bytes;
+  p.tr_cols = sf.tr_cols;
+  p.tr_rb = sf.tr_rb;
   if (gscale_in == nullptr) {
     // gscale doubles as the amax accumulator: zero, reduce, quantize (reads it as amax), then g.
     if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -146,7 +149,7 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
       if (rc) return rc;
       p.g_src = gscale;
       p.g_is_amax = 1;
-      rc = launch_quantize_t<false, false>(dtype, p, s);
+      rc = p.tr_cols ? launch_quantize_t<SRC_COLS, false>(dtype, p, s) : launch_quantize_t<SRC_LINEAR, false>(dtype, p, s);
       if (rc) return rc;
     }
     global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
@@ -156,7 +159,9 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
   p.g_src = gscale_in;
   p.g_is_amax = 0;
   if (n > 0) {
-    if (int rc = launch_quantize_t<false, false>(dtype, p, s)) return rc;
+    if (int rc = p.tr_cols ? launch_quantize_t<SRC_COLS, false>(dtype, p, s)
+                           : launch_quantize_t<SRC_LINEAR, false>(dtype, p, s))
+      return rc;
   }
   if (gscale && gscale != gscale_in) {
     if (cudaMemcpyAsync(gscale, gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -284,6 +289,30 @@ int nvfp4_quantize_mma(const void* x, int64_t batch, int64_t rows, int64_t cols,
   return quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes, sf, gscale, nullptr, nullptr, lay, s);
 }
 
+int nvfp4_quantize_mma_t(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
+                         const float* gscale_in, uint8_t* codes_t, uint8_t* sf_t, float* gscale, void* stream) {
+  if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_ARG;
+  if (rows % 16 != 0) return NVFP4_ERR_SIZE;
+  const int64_t n = batch * rows * cols;
+  if (n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (n > 0 && sf_t == nullptr) return NVFP4_ERR_ARG;
+  cudaStream_t s = S(stream);
+  QuantParams lay{};
+  if (n > 0) {
+    const int64_t bpr = rows / 16;           // blocks per row of the transposed [cols, rows] matrix
+    lay.sf_bpr = (uint32_t)bpr;
+    lay.sf_rows = (uint32_t)cols;
+    lay.sf_ctiles = (uint32_t)((bpr + 3) / 4);
+    lay.sf_mat_bytes = ((cols + 127) / 128) * 128 * (int64_t)lay.sf_ctiles * 4;
+    lay.tr_cols = cols;
+    lay.tr_rb = bpr;
+    if ((cols % 128 != 0 || bpr % 4 != 0) &&
+        cudaMemsetAsync(sf_t, 0, (size_t)(batch * lay.sf_mat_bytes), s) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+  }
+  return quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes_t, sf_t, gscale, nullptr, nullptr, lay, s);
+}
+
 int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int f_hi, uint8_t* codes,
                    uint8_t* scales, float* gscale, void* stream) {
   if (gscale == nullptr) return NVFP4_ERR_ARG;
@@ -401,7 +430,7 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
           cudaMemsetAsync(scales, 0, (size_t)(BH * p.sf_mat_bytes), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     }
-    int rc = rotate ? launch_quantize_t<true, true>(DT_BF16, p, s) : launch_quantize_t<true, false>(DT_BF16, p, s);
+    int rc = rotate ? launch_quantize_t<SRC_KV, true>(DT_BF16, p, s) : launch_quantize_t<SRC_KV, false>(DT_BF16, p, s);
     if (rc) return rc;
   }
   global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
@@ -539,7 +568,7 @@ int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, in
     p.sf_mat_bytes = ((cap + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
   }
   cudaStream_t s = S(stream);
-  const int rc = rotate ? launch_quantize_t<true, true>(DT_BF16, p, s) : launch_quantize_t<true, false>(DT_BF16, p, s);
+  const int rc = rotate ? launch_quantize_t<SRC_KV, true>(DT_BF16, p, s) : launch_quantize_t<SRC_KV, false>(DT_BF16, p, s);
   if (rc) return rc;
   return check_finite_sync(gscale, s);
 }

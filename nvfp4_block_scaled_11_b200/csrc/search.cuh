@@ -348,7 +348,7 @@ __device__ __forceinline__ void maybe_rotate(u64 (&x2)[8]) {
   }
 }
 
-template <bool WANT_SSE>
+template <int MODE, bool WANT_SSE>
 __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, const u64 (&x2)[8], const CandEntry* tab,
                                             int c0, int fstar, float sse, bool poisoned, float amax_b) {
   uint32_t wlo = 0u, whi = 0u;
@@ -377,7 +377,7 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
     }
     sse = (WANT_SSE && amax_b != 0.0f) ? s : 0.0f;
   }
-  const int64_t ob = out_block(p, b);
+  const int64_t ob = out_block<MODE>(p, b);
   reinterpret_cast<uint2*>(p.codes)[ob] = make_uint2(wlo, whi);
   p.scales[scale_index(p, ob)] = (uint8_t)scale;
   if (p.block_f) p.block_f[ob] = (int8_t)fstar;
@@ -385,7 +385,7 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
 }
 
 // Fast path for one block.  Returns true when the block needs the definition (outputs not written).
-template <bool ROT, int NC, bool WANT_SSE>
+template <int MODE, bool ROT, int NC, bool WANT_SSE>
 __device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const CandEntry* tab, const float* thr,
                                                     float inv6g, bool g_bad, int64_t b, u64 (&x2)[8]) {
   maybe_rotate<ROT>(x2);
@@ -405,17 +405,15 @@ __device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const 
       return true;
     }
   }
-  write_block<WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
   return false;
 }
 
-// The definition for one block (deferred blocks): same outputs, every candidate scored in order.
-template <int DT, bool KV, bool ROT, bool WANT_SSE>
-__device__ __forceinline__ void quantize_block_def(const QuantParams& p, const CandEntry* tab, const float* thr,
-                                                   float inv6g, bool g_bad, int64_t b, const char* src, bool v8) {
-  u64 x2[8];
-  load_pairs<DT>(src, v8, x2);
-  maybe_rotate<ROT>(x2);
+// The definition for one block already in registers (rotated if the path rotates): same outputs as the
+// fast path, every candidate scored in order.
+template <int MODE, bool WANT_SSE>
+__device__ __forceinline__ void quantize_block_def_x2(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                                      float inv6g, bool g_bad, int64_t b, const u64 (&x2)[8]) {
   const float amax_b = block_amax_nan(x2);
   const bool poisoned = g_bad || !(amax_b <= FLT_MAX);
   int c0 = 0, fstar = -128;
@@ -427,19 +425,41 @@ __device__ __forceinline__ void quantize_block_def(const QuantParams& p, const C
     for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
     search_def(x, c0, p.f_lo, p.f_hi, tab, fstar, sse);
   }
-  write_block<WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
 }
 
-template <int DT, bool KV>
+// First element of block b (linear and KV modes: the 16 elements are contiguous).
+template <int DT, int MODE>
 __device__ __forceinline__ const char* block_src(const QuantParams& p, int64_t b) {
   constexpr int ES = DT == DT_F32 ? 4 : 2;
-  int64_t elem;
-  if (KV) {
-    elem = kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D);
-  } else {
-    elem = 16 * b;
-  }
+  const int64_t elem = MODE == SRC_KV ? kv_block_elem(b, p.Tm, p.bpr, p.T, p.sink, p.D) : 16 * b;
   return p.x + elem * ES;
+}
+
+// Block b as 8 packed FP32 pairs, from whichever source mode the launch uses.
+template <int DT, int MODE>
+__device__ __forceinline__ void load_block_pairs(const QuantParams& p, int64_t b, bool v8, u64 (&x2)[8]) {
+  if constexpr (MODE == SRC_COLS) {
+    constexpr int ES = DT == DT_F32 ? 4 : 2;
+    uint32_t l, c, rb;
+    cols_split(p, b, l, c, rb);
+    float x[16];
+    load_column<DT>(p.x + (((int64_t)l * p.tr_rb + rb) * 16 * p.tr_cols + c) * ES, p.tr_cols * ES, x);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x2[k] = pk2(x[2 * k], x[2 * k + 1]);
+  } else {
+    load_pairs<DT>(block_src<DT, MODE>(p, b), v8, x2);
+  }
+}
+
+// The definition for one block (deferred blocks): reload, rotate, score every candidate in order.
+template <int DT, int MODE, bool ROT, bool WANT_SSE>
+__device__ __forceinline__ void quantize_block_def(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                                   float inv6g, bool g_bad, int64_t b, bool v8) {
+  u64 x2[8];
+  load_block_pairs<DT, MODE>(p, b, v8, x2);
+  maybe_rotate<ROT>(x2);
+  quantize_block_def_x2<MODE, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
 }
 
 // One thread per 16-element block, grid-stride in warp-uniform rounds, the next block's loads in flight
@@ -450,7 +470,7 @@ constexpr int kDeferCap = 64;
 #define NVFP4_SEARCH_CTAS_PER_SM 2
 #endif
 
-template <int DT, bool KV, bool ROT, int NC, bool WANT_SSE>
+template <int DT, int MODE, bool ROT, int NC, bool WANT_SSE>
 __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search_kernel(QuantParams p) {
   __shared__ CandEntry tab[128];
   __shared__ float thr[128];
@@ -459,7 +479,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   const bool v8 = p.v8 != 0;
   int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   u64 xn[8];
-  if (b < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b), v8, xn);  // in flight while the tables are built
+  if (b < p.nblocks) load_block_pairs<DT, MODE>(p, b, v8, xn);  // in flight while the tables are built
   float g = *p.g_src;
   if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
   const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
     __syncwarp();
     for (int e = lane; e < dcount; e += 32) {
       const int64_t bd = dlist[e];
-      quantize_block_def<DT, KV, ROT, WANT_SSE>(p, tab, thr, inv6g, g_bad, bd, block_src<DT, KV>(p, bd), p.v8 != 0);
+      quantize_block_def<DT, MODE, ROT, WANT_SSE>(p, tab, thr, inv6g, g_bad, bd, p.v8 != 0);
     }
     __syncwarp();
     dcount = 0;
@@ -488,8 +508,8 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
     u64 x2[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) x2[k] = xn[k];
-    if (b + stride < p.nblocks) load_pairs<DT>(block_src<DT, KV>(p, b + stride), v8, xn);
-    const bool deferred = active && quantize_block_fast<ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
+    if (b + stride < p.nblocks) load_block_pairs<DT, MODE>(p, b + stride, v8, xn);
+    const bool deferred = active && quantize_block_fast<MODE, ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
     if constexpr (NC > 1) {  // a single-offset window never needs the definition pass
       const unsigned m = __ballot_sync(0xFFFFFFFFu, deferred);
       if (m) {

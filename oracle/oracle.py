@@ -358,3 +358,11 @@ def msda_forward(value: np.ndarray, shapes, loc: np.ndarray, w: np.ndarray) -> n
     out = np.empty((bs, nq, heads, ch), np.float64)
     lib().ref_msda_forward(_p(value), _p(sh), _p(start), _p(loc), _p(w), bs, nkeys, heads, ch, L, P, nq, _p(out))
     return out
+
+
+def quantize_mma_t(x: np.ndarray, f_lo: int = -2, f_hi: int = 6, dtype: int | None = None, gscale_in=None):
+    """x [batch, rows, cols] (or [rows, cols]) quantized in blocks of 16 rows per column: the tile-layout
+    quantization of the transposed matrices.  Returns (codes [batch*cols*rows/2], sf_mma, g)."""
+    if x.ndim == 2:
+        x = x[None]
+    return quantize_mma(np.ascontiguousarray(np.swapaxes(x, 1, 2)), f_lo, f_hi, dtype, gscale_in)

@@ -203,3 +203,25 @@ def test_gemm_nt_full_size_sampled():
         ref = O.gemm_nt(rac, ras, rga, rbc, rbs, rgb, 1, len(cols), K)[0, 0]
         bound = _gemm_bound(rac, ras, rbc, rbs, 1, len(cols), K, 1, float(rga) * float(rgb))[0, 0]
         assert (np.abs(dc[r, cols].astype(np.float64) - ref) <= (K + 4) * U * bound + 1e-37).all(), r
+
+
+@pytest.mark.parametrize("shape,dtype", [((1, 128, 64), torch.float32), ((2, 96, 130), torch.bfloat16),
+                                         ((3, 16, 33), torch.float16), ((1, 4096, 128), torch.bfloat16)])
+def test_quantize_mma_t_bit_exact(shape, dtype):
+    x = _x(shape, 200 + shape[2], dtype)
+    codes, sf, g = nv.quantize_mma_t(x.cuda())
+    rc, rsf, rg = O.quantize_mma_t(_np(x).reshape(shape), dtype=_odt(x))
+    assert g.item() == rg
+    assert codes.shape == (shape[0], shape[2], shape[1] // 2)
+    assert np.array_equal(codes.cpu().numpy().reshape(-1), rc)
+    assert np.array_equal(sf.cpu().numpy(), rsf)
+
+
+def test_quantize_mma_t_windows_and_external_scale():
+    x = _x((2, 64, 40), 9)
+    gin = torch.tensor([0.004], dtype=torch.float32)
+    for lo, hi in ((0, 0), (-8, 8), (-1, 3)):
+        codes, sf, _ = nv.quantize_mma_t(x.cuda(), lo, hi, gscale_in=gin.cuda())
+        rc, rsf, _ = O.quantize_mma_t(x.numpy(), lo, hi, gscale_in=0.004)
+        assert np.array_equal(codes.cpu().numpy().reshape(-1), rc), (lo, hi)
+        assert np.array_equal(sf.cpu().numpy(), rsf), (lo, hi)
