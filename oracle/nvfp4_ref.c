@@ -18,6 +18,7 @@ static uint32_t f2u(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
 static float u2f(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
 
 static float qnan(void) { return u2f(0x7FC00000u); }
+static float pow2f(int k);
 
 /* Nearest integer to a non-negative finite w < 2^24, ties to even, from w's bits. */
 static uint32_t rne_int(float w) {
@@ -461,6 +462,55 @@ int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* s
           }
           out[((b * nq + q) * heads + h) * ch + c] = acc;
         }
+  return 0;
+}
+
+/* ---- FP4 attention softmax (see the header) ---- */
+float ref_exp_ss(float x) {
+  if (x != x) return x;
+  if (x < -104.0f) return 0.0f;
+  const float log2e = 0x1.715476p+0f;                  /* fl(1 / ln 2) */
+  const float ln2_hi = 0x1.62e4p-1f;                   /* ln 2 rounded to 16 significant bits */
+  const float ln2_lo = 0x1.7f7d1cp-20f;                /* fl(ln 2 - ln2_hi) */
+  const float n = rintf(x * log2e);
+  const float r = (x - n * ln2_hi) - n * ln2_lo;
+  float p = 0x1.a01a02p-13f;                           /* 1/7! */
+  p = p * r + 0x1.6c16c2p-10f;                         /* 1/6! */
+  p = p * r + 0x1.111112p-7f;                          /* 1/5! */
+  p = p * r + 0x1.555556p-5f;                          /* 1/4! */
+  p = p * r + 0x1.555556p-3f;                          /* 1/3! */
+  p = p * r + 0x1p-1f;                                 /* 1/2! */
+  p = p * r + 1.0f;
+  p = p * r + 1.0f;
+  const int k = (int)n;
+  if (k >= -126) return p * pow2f(k);
+  return (p * pow2f(k + 64)) * pow2f(-64);
+}
+
+int ref_softmax_quantize(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
+                         int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, float* row_max, float* row_sum) {
+  if (batch < 0 || Tq < 0 || Tk < 0 || Tk % 16 != 0) return -2;
+  const float g = ref_global_scale(1.0f);
+  float blk[16];
+  for (int64_t row = 0; row < batch * Tq; ++row) {
+    const int64_t q = row % Tq;
+    const float* sr = s + row * Tk;
+    float m = -INFINITY;
+    for (int64_t k = 0; k < Tk; ++k)
+      if (!causal || k <= q + q_offset) m = sr[k] > m ? sr[k] : m;
+    float l = 0.0f;
+    for (int64_t j = 0; j < Tk / 16; ++j) {
+      for (int i = 0; i < 16; ++i) {
+        const int64_t k = 16 * j + i;
+        blk[i] = (!causal || k <= q + q_offset) ? ref_exp_ss(sr[k] - m) : 0.0f;
+        l = l + blk[i];
+      }
+      const int64_t b = row * (Tk / 16) + j;
+      ref_search_block(blk, g, f_lo, f_hi, codes + 8 * b, scales + b, 0, 0);
+    }
+    row_max[row] = m;
+    row_sum[row] = l;
+  }
   return 0;
 }
 

@@ -119,6 +119,23 @@ int ref_kv_append(const uint16_t* k, int64_t BH, int64_t ld_bh, int64_t first, i
 int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* start, const float* loc, const float* w,
                      int64_t bs, int64_t nkeys, int64_t heads, int64_t ch, int64_t L, int64_t P, int64_t nq, double* out);
 
+/* ---- FP4 attention: softmax numerators quantized for the P V^T product ----
+ * [SS] ScaleSearchAttention runs P V^T in NVFP4 on the tensor cores.  The pages do not say how P is
+ * formed; this takes the flash-attention form: for each row q of the scores S [batch, Tq, Tk],
+ * m = max over the allowed keys, P~ = exp(S - m) (allowed keys) or 0 (masked keys; causal: key k is
+ * allowed for query q iff k <= q + q_offset), l = sum of P~ (FP32, in key order), and P~ quantized with
+ * ScaleSearch along the keys with the tensor scale g = fl(1 / 2688) (the tensor amax of P~ is 1).
+ * exp is ref_exp_ss below, so both implementations produce the same P~ bit for bit. */
+
+/* exp(x) in FP32 by Cody-Waite reduction and a degree-7 Taylor polynomial (published method, fixed
+ * operation order, no FMA): n = rint(x * log2(e)), r = (x - n * ln2_hi) - n * ln2_lo with ln2 split at 16
+ * significant bits (n * ln2_hi exact), p = Horner(1, 1, 1/2!, ..., 1/7!) at r, result p * 2^n (scaled in
+ * two exact steps below 2^-126).  x < -104 gives 0; NaN gives NaN. */
+float ref_exp_ss(float x);
+
+int ref_softmax_quantize(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
+                         int f_lo, int f_hi, uint8_t* codes, uint8_t* scales, float* row_max, float* row_sum);
+
 /* ---- MXFP4, the power-of-two-scaled comparison format ----
  * [NV] compares NVFP4 with "simple power-of-two scaling like MXFP4".  MXFP4 as the OCP Microscaling
  * (MX) v1.0 specification defines it: blocks of 32 elements, one E8M0 scale X = 2^e with

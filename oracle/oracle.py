@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
             "ref_hadamard16": (I, [P, I64, I, P, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
+            "ref_exp_ss": (F, [F]),
+            "ref_softmax_quantize": (I, [P, I64, I64, I64, I, I64, I, I, P, P, P, P]),
             "ref_msda_forward": (I, [P, P, P, P, P, I64, I64, I64, I64, I64, I64, I64, P]),
             "ref_mxfp4_quantize": (I, [P, I64, I, P, P]),
             "ref_mxfp4_dequantize": (I, [P, P, I64, I, P]),
@@ -366,3 +368,24 @@ def quantize_mma_t(x: np.ndarray, f_lo: int = -2, f_hi: int = 6, dtype: int | No
     if x.ndim == 2:
         x = x[None]
     return quantize_mma(np.ascontiguousarray(np.swapaxes(x, 1, 2)), f_lo, f_hi, dtype, gscale_in)
+
+
+# ---- FP4 attention softmax ----
+def exp_ss(x) -> np.float32:
+    return np.float32(lib().ref_exp_ss(float(x)))
+
+
+def softmax_quantize(s: np.ndarray, causal: bool = False, q_offset: int = 0, f_lo: int = -2, f_hi: int = 6):
+    """s float32 [batch, Tq, Tk].  Returns (codes [batch,Tq,Tk/2], scales [batch,Tq,Tk/16] (row-major),
+    row_max [batch,Tq], row_sum [batch,Tq], g) for P~ = exp(S - m) quantized with g = fl(1/2688)."""
+    s = np.ascontiguousarray(s, np.float32)
+    batch, Tq, Tk = s.shape
+    codes = np.empty((batch, Tq, Tk // 2), np.uint8)
+    scales = np.empty((batch, Tq, Tk // 16), np.uint8)
+    m = np.empty((batch, Tq), np.float32)
+    l = np.empty((batch, Tq), np.float32)
+    rc = lib().ref_softmax_quantize(_p(s), batch, Tq, Tk, int(bool(causal)), q_offset, f_lo, f_hi, _p(codes),
+                                    _p(scales), _p(m), _p(l))
+    if rc != 0:
+        raise ValueError(f"ref_softmax_quantize returned {rc}")
+    return codes, scales, m, l, global_scale(1.0)
