@@ -215,6 +215,24 @@ int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs
                   const uint8_t* b_sf, const float* b_gscale, int64_t batch, int64_t M, int64_t N, int64_t K,
                   float alpha, void* d, int d_dtype, float* alpha_work, void* stream);
 
+/* Softmax numerators for the P V^T product of FP4 attention ([SS] ScaleSearchAttention; the pages do
+ * not say how P is formed, this is the flash-attention form).  s: scores [batch, Tq, Tk] FP32 (16-byte
+ * aligned, Tk % 16 == 0).  For each row (b, q): m = max over the allowed keys (causal != 0: key k is
+ * allowed iff k <= q + q_offset), P~_k = exp(S_k - m) for allowed keys and 0 otherwise, l = sum_k P~_k.
+ * exp is a fixed FP32 method: n = rint(x log2 e), r = (x - n ln2_hi) - n ln2_lo (ln 2 split at 16
+ * significant bits), p = degree-7 Taylor polynomial of e^r in Horner form, result p 2^n (0 below -104).
+ * P~ is ScaleSearch-quantized along the keys (window [f_lo, f_hi] of 1, 9 or 17 offsets) with the tensor
+ * scale g = fl(1/2688): codes [batch, Tq, Tk/2], sf the tile layout of the [Tq, Tk] matrices
+ * (nvfp4_sf_mma_bytes(Tq, Tk, batch) bytes), *gscale = g, row_max / row_sum [batch * Tq] (FP32; the
+ * sum's order is unspecified).  Then O = (P~ V) / l: nvfp4_gemm_nt of (codes, sf, gscale) with V from
+ * nvfp4_quantize_mma_t, followed by nvfp4_rows_divide. */
+int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
+                               int f_lo, int f_hi, uint8_t* codes, uint8_t* sf, float* gscale, float* row_max,
+                               float* row_sum, void* stream);
+
+/* x[r, c] = fl(x[r, c] / l[r]) for an FP32 [rows, cols] matrix (cols % 4 == 0, 16-byte aligned). */
+int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream);
+
 /* Host only, for verification: the byte offsets at which nvfp4_gemm_nt reads the scale of (matrix l,
  * row r, block column c), for l < batch, r < rows, c < K/16 in that (row-major) order, into out
  * (batch * rows * K/16 entries).  No device work. */

@@ -18,7 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
-    "msda_forward",
+    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -50,6 +50,8 @@ _SIGS = {
     "nvfp4_quantize_mma_t": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "nvfp4_kv_mixed_mma": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_gemm_nt": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P, _P]),
+    "nvfp4_softmax_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_rows_divide": (_I, [_P, _P, _I64, _I64, _P]),
     "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),
 }
 
@@ -405,3 +407,51 @@ def msda_forward(value, shapes, loc: torch.Tensor, w: torch.Tensor, out: torch.T
         _check(lib().nvfp4_msda_forward(_ptr(value), _dt(value), bs, nkeys, heads, ch, shp, L, P, nq, _ptr(loc),
                                         _ptr(w), _ptr(out), _stream(loc)))
     return out
+
+
+# ---- FP4 attention (ScaleSearchAttention numerics, unfused) ----
+def softmax_quantize_mma(s: torch.Tensor, causal: bool = False, q_offset: int = 0, f_lo: int = -2, f_hi: int = 6):
+    """s float32 [batch, Tq, Tk] (or [Tq, Tk]).  Returns (codes [.., Tq, Tk/2], sf tile layout, gscale[1],
+    row_max [batch*Tq], row_sum [batch*Tq]) for the softmax numerators P~ = exp(S - m)."""
+    _cuda(s, "s")
+    batch, Tq, Tk = (1, *s.shape) if s.dim() == 2 else s.shape
+    dev = s.device
+    codes = torch.empty((*s.shape[:-1], Tk // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(max(sf_mma_bytes(Tq, Tk, batch), 1), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    m = torch.empty(batch * Tq, dtype=torch.float32, device=dev)
+    l = torch.empty(batch * Tq, dtype=torch.float32, device=dev)
+    _check(lib().nvfp4_softmax_quantize_mma(_ptr(s), batch, Tq, Tk, int(bool(causal)), q_offset, f_lo, f_hi,
+                                            _ptr(codes), _ptr(sf), _ptr(g), _ptr(m), _ptr(l), _stream(s)))
+    return codes, sf, g, m, l
+
+
+def rows_divide(x: torch.Tensor, l: torch.Tensor) -> torch.Tensor:
+    """In place: x[r, :] /= l[r] for x float32 [..., cols] viewed as rows."""
+    _cuda(x, "x"), _cuda(l, "l")
+    cols = x.shape[-1]
+    _check(lib().nvfp4_rows_divide(_ptr(x), _ptr(l), x.numel() // max(cols, 1), cols, _stream(x)))
+    return x
+
+
+def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, rotate: bool = True,
+                  scale: float | None = None, f_lo: int = -2, f_hi: int = 6):
+    """Attention with every product in NVFP4 on the tensor cores ("Search your block floating-point
+    scales!", ScaleSearchAttention; unfused): q [H, Tq, D], k and v [H, Tk, D].
+      rotate: Hadamard-16 along D on q and k (Q K^T unchanged, outliers spread);
+      S = scale * Q K^T (NVFP4 x NVFP4, FP32 accumulation);  P~ = exp(S - rowmax) quantized with ScaleSearch;
+      O = (P~ V) / rowsum with V quantized along the tokens.  Causal: query i sees keys <= i + Tk - Tq.
+    Returns O [H, Tq, D] float32."""
+    H, Tq, D = q.shape
+    Tk = k.shape[1]
+    scale = D ** -0.5 if scale is None else scale
+    if rotate:
+        q = hadamard16(q.contiguous(), out_dtype=torch.float32)
+        k = hadamard16(k.contiguous(), out_dtype=torch.float32)
+    qc, qsf, qg = quantize_mma(q.contiguous(), f_lo, f_hi)
+    kc, ksf, kg = quantize_mma(k.contiguous(), f_lo, f_hi)
+    s = gemm_nt(qc, qsf, qg, kc, ksf, kg, alpha=scale)
+    pc, psf, pg, _, l = softmax_quantize_mma(s, causal, Tk - Tq, f_lo, f_hi)
+    vc, vsf, vg = quantize_mma_t(v.contiguous(), f_lo, f_hi)
+    o = gemm_nt(pc, psf, pg, vc, vsf, vg)
+    return rows_divide(o, l)

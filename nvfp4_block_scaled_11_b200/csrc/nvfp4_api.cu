@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/nvfp4.h"
+#include "attention.cuh"
 #include "msda.cuh"
 #include "search.cuh"
 
@@ -466,6 +467,49 @@ int nvfp4_msda_forward(const void* value, int dtype, int64_t bs, int64_t nkeys, 
   if (dtype == DT_F32) return msda_launch<MSDA_F32>(p, ch, s);
   if (dtype == DT_F16) return msda_launch<MSDA_F16>(p, ch, s);
   return msda_launch<MSDA_BF16>(p, ch, s);
+}
+
+int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
+                               int f_lo, int f_hi, uint8_t* codes, uint8_t* sf, float* gscale, float* row_max,
+                               float* row_sum, void* stream) {
+  const int nc = f_hi - f_lo + 1;
+  if (!window_ok(f_lo, f_hi) || (nc != 1 && nc != 9 && nc != 17) || gscale == nullptr) return NVFP4_ERR_ARG;
+  if (batch < 0 || Tq < 0 || Tk < 0 || Tk % 16 != 0) return NVFP4_ERR_SIZE;
+  const int64_t rows = batch * Tq, bpr = Tk / 16;
+  if (rows * bpr >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  cudaStream_t st = S(stream);
+  if (rows == 0 || Tk == 0) return NVFP4_OK;
+  if (s == nullptr || codes == nullptr || sf == nullptr || row_max == nullptr || row_sum == nullptr)
+    return NVFP4_ERR_ARG;
+  if (!aligned(s, 16) || !aligned(codes, 8) || !aligned(gscale, 4) || !aligned(row_max, 4) || !aligned(row_sum, 4))
+    return NVFP4_ERR_ALIGN;
+  QuantParams p{};
+  p.nblocks = rows * bpr;
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.codes = codes;
+  p.scales = sf;
+  p.sf_bpr = (uint32_t)bpr;
+  p.sf_rows = (uint32_t)Tq;
+  p.sf_ctiles = (uint32_t)((bpr + 3) / 4);
+  p.sf_mat_bytes = ((Tq + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
+  if ((Tq % 128 != 0 || bpr % 4 != 0) && cudaMemsetAsync(sf, 0, (size_t)(batch * p.sf_mat_bytes), st) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  SoftmaxParams a{s, rows, Tq, Tk, causal ? 1 : 0, q_offset, aligned(s, 32) ? 1 : 0, row_max, row_sum, gscale};
+  const int grid = grid_for(rows * 32, 256, 4);
+  if (nc == 9) softmax_quantize_kernel<9><<<grid, 256, 0, st>>>(p, a);
+  else if (nc == 1) softmax_quantize_kernel<1><<<grid, 256, 0, st>>>(p, a);
+  else softmax_quantize_kernel<17><<<grid, 256, 0, st>>>(p, a);
+  return last_error();
+}
+
+int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream) {
+  if (rows < 0 || cols < 0 || cols % 4 != 0) return NVFP4_ERR_SIZE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (x == nullptr || l == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(l, 4)) return NVFP4_ERR_ALIGN;
+  rows_divide_kernel<<<grid_for(rows * cols / 4, 256, 8), 256, 0, S(stream)>>>(x, l, rows, cols);
+  return last_error();
 }
 
 int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales, void* stream) {

@@ -1,0 +1,99 @@
+"""FP4 attention (ScaleSearchAttention numerics, unfused) against the oracle.
+
+* softmax_quantize_mma on host-made scores: codes, tile-layout scales, g and row maxima bit-exact
+  (exp is the same published method on both sides); row sums within the FP32 summation bound.
+* The whole pipeline: the GPU's scores come from FP32 tensor-core accumulation, the oracle's from the
+  float64 product rounded once, so a softmax numerator can land on the other side of a rounding
+  boundary now and then.  The test bounds how often P codes differ (< 0.5 %) and the output's
+  deviation (relative Frobenius < 2e-3), far below what a wrong layout, scale or mask produces."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_11_b200 as nv
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+U = 2.0 ** -24
+
+
+def _scores(batch, Tq, Tk, seed, scale=2.5):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((batch, Tq, Tk), generator=g) * scale).float()
+
+
+@pytest.mark.parametrize("batch,Tq,Tk,causal,q_offset,window", [
+    (2, 37, 96, False, 0, (-2, 6)), (1, 130, 2048, True, 1918, (-2, 6)), (3, 8, 64, True, 0, (-2, 6)),
+    (1, 64, 256, False, 0, (0, 0)), (1, 64, 256, True, 192, (-8, 8))])
+def test_softmax_quantize_matches_oracle(batch, Tq, Tk, causal, q_offset, window):
+    s = _scores(batch, Tq, Tk, Tq + Tk)
+    codes, sf, g, m, l = nv.softmax_quantize_mma(s.cuda(), causal, q_offset, *window)
+    torch.cuda.synchronize()
+    rc, rs, rm, rl, rg = O.softmax_quantize(s.numpy(), causal, q_offset, *window)
+    assert g.item() == rg
+    assert np.array_equal(m.cpu().numpy(), rm.reshape(-1))
+    assert np.array_equal(codes.cpu().numpy().reshape(-1), rc.reshape(-1))
+    assert np.array_equal(sf.cpu().numpy(), O.scales_to_mma(rs, batch, Tq, Tk // 16))
+    assert (np.abs(l.cpu().numpy() - rl.reshape(-1)) <= (Tk + 4) * U * rl.reshape(-1)).all()
+
+
+def test_softmax_quantize_poisons_nan_block():
+    s = _scores(1, 4, 64, 3)
+    s[0, 2, 37] = float("nan")
+    codes, sf, g, m, l = nv.softmax_quantize_mma(s.cuda())
+    rc, rs, rm, rl, _ = O.softmax_quantize(s.numpy())
+    assert np.array_equal(codes.cpu().numpy().reshape(-1), rc.reshape(-1))
+    assert np.array_equal(sf.cpu().numpy(), O.scales_to_mma(rs, 1, 4, 4))
+    assert rs[0, 2, 2] == 0x7F
+
+
+def test_rows_divide_exact():
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn((3, 5, 8), generator=g)
+    l = torch.rand(15, generator=g) + 0.5
+    y = nv.rows_divide(x.clone().cuda(), l.cuda()).cpu().numpy()
+    want = (x.numpy().reshape(15, 8) / l.numpy()[:, None]).astype(np.float32)
+    assert np.array_equal(y.reshape(15, 8), want)
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_fp4_pipeline_matches_oracle(causal):
+    H, Tq, Tk, D = 2, 64, 256, 128
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn((H, Tq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
+    o = nv.attention_fp4(q.cuda(), k.cuda(), v.cuda(), causal=causal).cpu().numpy().astype(np.float64)
+    # the oracle's pipeline
+    scale = D ** -0.5
+    qr = O.hadamard16(_u16(q).reshape(-1), dtype=O.BF16, out_dtype=O.F32)
+    kr = O.hadamard16(_u16(k).reshape(-1), dtype=O.BF16, out_dtype=O.F32)
+    qc, qs, qg, _, _ = O.quantize(qr)
+    kc, ks, kg, _, _ = O.quantize(kr)
+    s = O.gemm_nt(qc, qs, qg, kc, ks, kg, Tq, Tk, D, scale, H).astype(np.float32)
+    pc, ps, pm, pl, pg = O.softmax_quantize(s, causal, Tk - Tq)
+    vc, vsf, vg = O.quantize_mma_t(_u16(v).reshape(H, Tk, D), dtype=O.BF16)
+    vcodes, vscales, _, _, _ = O.quantize(np.ascontiguousarray(np.swapaxes(_u16(v).reshape(H, Tk, D), 1, 2)).reshape(-1),
+                                          dtype=O.BF16)
+    ov = O.gemm_nt(pc, ps, pg, vcodes, vscales, vg, Tq, D, Tk, 1.0, H) / pl[..., None]
+    # the GPU's P for the same comparison
+    qc_g, qsf_g, qg_g = nv.quantize_mma(nv.hadamard16(q.cuda(), out_dtype=torch.float32))
+    kc_g, ksf_g, kg_g = nv.quantize_mma(nv.hadamard16(k.cuda(), out_dtype=torch.float32))
+    s_g = nv.gemm_nt(qc_g, qsf_g, qg_g, kc_g, ksf_g, kg_g, alpha=scale)
+    pc_g, _, _, _, _ = nv.softmax_quantize_mma(s_g, causal, Tk - Tq)
+    differ = np.mean(pc_g.cpu().numpy().reshape(-1) != pc.reshape(-1))
+    assert differ < 5e-3, differ
+    rel = np.linalg.norm(o - ov) / np.linalg.norm(ov)
+    assert rel < 2e-3, rel
+    # and against full-precision attention: the quantization error of NVFP4 attention
+    qf, kf, vf = q.double(), k.double(), v.double()
+    sf = torch.einsum("hqd,hkd->hqk", qf, kf) * scale
+    if causal:
+        sf = sf.masked_fill(torch.arange(Tk)[None, :] > torch.arange(Tq)[:, None] + (Tk - Tq), float("-inf"))
+    of = torch.einsum("hqk,hkd->hqd", torch.softmax(sf, -1), vf).numpy()
+    nae = np.abs(o - of).mean() / np.abs(of).mean()
+    assert nae < 0.25, nae
