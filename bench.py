@@ -13,7 +13,8 @@ configuration the throughput target is stated on.  Every step's input (4 GiB) is
 Workloads: stream_f32 (default), act_f32, act_bf16, kv_bf16, bev_f16, and gemm_nvfp4 -- the tensor-core
 consumer: ScaleSearch-quantized BF16 activations [8192, 8192] times NVFP4 weights [8192, 8192] on the
 tensor cores, reported in TFLOP/s against the FP4 tensor roofline; and msda_nvfp4 -- deformable attention
-over the BEVFormer value maps with ScaleSearch NVFP4 values, reported in queries/s.
+over the BEVFormer value maps with ScaleSearch NVFP4 values, reported in queries/s; and attn_nvfp4 --
+causal attention with NVFP4 Q K^T and P V^T on the tensor cores, reported in TFLOP/s.
 
 Prints ONE JSON line on rank 0.  Times are CUDA events on the launching stream, max over ranks.
 `--impl reference` times the CPU oracle (the plain C definition) on a bounded sample of the same
@@ -657,6 +658,192 @@ def run_msda_reference(args, rank, world):
     }), flush=True)
 
 
+# ------------------------------------------------------------------------------------------------
+# FP4 attention (ScaleSearchAttention numerics, unfused)
+# ------------------------------------------------------------------------------------------------
+ATTN_METRIC = "FP4 attention TFLOP/s (4*H*Tq*Tk*D per step; NVFP4 Q K^T and P V^T on the tensor cores)"
+
+
+def attn_config(args, shape):
+    H, Tq, Tk, D = shape
+    return {
+        "workload": f"attn_nvfp4 (q [{H},{Tq},{D}] N(0,1) seed 21; k = KV-cache keys [{H},{Tk},{D}] (N(0,1) + channel "
+                    f"bias, seed 2); v [{H},{Tk},{D}] N(0,1) seed 22; BF16; causal, queries at the end)",
+        "window": [args.f_lo, args.f_hi],
+        "step": "Hadamard-16 on q, k; ScaleSearch NVFP4 quantize of q, k (tile layout) and of v along tokens; "
+                "S = Q K^T (FP4 tensor cores); softmax numerators quantized with ScaleSearch; O = P~ V^T "
+                "(FP4 tensor cores) / rowsum",
+        "l2": "inputs and scores larger than L2 (S is 2.1 GB), no flush",
+        "H": H, "Tq": Tq, "Tk": Tk, "D": D,
+    }
+
+
+def run_attn(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    q, k, v = W.attn_inputs(dev, scale=args.scale)
+    H, Tq, D = q.shape
+    Tk = k.shape[1]
+    stream = torch.cuda.current_stream(dev)
+    scale = D ** -0.5
+    # every intermediate preallocated, so the step launches kernels only (no allocator calls)
+    f32, u8 = torch.float32, torch.uint8
+    E = lambda *shape, dt=f32: torch.empty(shape, dtype=dt, device=dev)
+    qr, kr = E(H, Tq, D), E(H, Tk, D)
+    qc, qsf, qg = E(H, Tq, D // 2, dt=u8), E(nv.sf_mma_bytes(Tq, D, H), dt=u8), E(1)
+    kc, ksf, kg = E(H, Tk, D // 2, dt=u8), E(nv.sf_mma_bytes(Tk, D, H), dt=u8), E(1)
+    vc, vsf, vg = E(H, D, Tk // 2, dt=u8), E(nv.sf_mma_bytes(D, Tk, H), dt=u8), E(1)
+    s_buf = E(H, Tq, Tk)
+    pc, psf, pg = E(H, Tq, Tk // 2, dt=u8), E(nv.sf_mma_bytes(Tq, Tk, H), dt=u8), E(1)
+    m_buf, l_buf, o, aw1, aw2 = E(H * Tq), E(H * Tq), E(H, Tq, D), E(1), E(1)
+
+    def step(evs=None):
+        def mark(i):
+            if evs:
+                evs[i].record(stream)
+        mark(0)
+        nv.hadamard16(q, out=qr)
+        nv.hadamard16(k, out=kr)
+        nv.quantize_mma(qr, args.f_lo, args.f_hi, codes=qc, sf=qsf, gscale=qg)
+        nv.quantize_mma(kr, args.f_lo, args.f_hi, codes=kc, sf=ksf, gscale=kg)
+        nv.quantize_mma_t(v, args.f_lo, args.f_hi, codes=vc, sf=vsf, gscale=vg)
+        mark(1)
+        nv.gemm_nt(qc, qsf, qg, kc, ksf, kg, alpha=scale, out=s_buf, alpha_work=aw1)
+        mark(2)
+        nv.softmax_quantize_mma(s_buf, True, Tk - Tq, args.f_lo, args.f_hi, codes=pc, sf=psf, g=pg, m=m_buf, l=l_buf)
+        mark(3)
+        nv.gemm_nt(pc, psf, pg, vc, vsf, vg, out=o, alpha_work=aw2)
+        mark(4)
+        nv.rows_divide(o, l_buf)
+        mark(5)
+        return o
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    steps = max(1, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    eager_ms = elapsed_ms
+    graph_used = False
+    if world == 1 and not args.no_graph:
+        cg = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(cg, stream=side):
+            step()
+        for _ in range(max(1, args.warmup)):
+            cg.replay()
+        torch.cuda.synchronize()
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(steps):
+            cg.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ga.elapsed_time(gb)
+        del cg
+        if graph_ms < elapsed_ms:
+            elapsed_ms, graph_used = graph_ms, True
+    stage = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(5)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    flops = 4.0 * H * Tq * Tk * D
+    bf16_peak, src = tensor_peak()
+    fp4_peak = bf16_peak * FP4_PER_BF16
+    hbm_peak, hsrc = peaks()
+    sm_bytes = H * Tq * Tk * 4 + H * Tq * Tk // 2 + H * Tq * Tk // 16 + 2 * H * Tq * 4
+    # accuracy against full-precision attention on the last 64 queries of head 0
+    qf, kf, vf = q[0, -64:].double(), k[0].double(), v[0].double()
+    sref = (qf @ kf.T) * scale
+    mask = torch.arange(Tk, device=dev)[None, :] > torch.arange(Tq - 64, Tq, device=dev)[:, None] + (Tk - Tq)
+    oref = torch.softmax(sref.masked_fill(mask, float("-inf")), -1) @ vf
+    nae = float((o[0, -64:].double() - oref).abs().mean() / oref.abs().mean())
+    line = {
+        "metric": ATTN_METRIC, "value": world * flops * steps / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 operands, f32 accumulation", "data": SOURCE_NOTE, "config": attn_config(args, (H, Tq, Tk, D)),
+        "roofline": {"bound": "hbm", "kernel": "softmax_quantize_kernel (reads the FP32 scores, writes NVFP4 P)",
+                     "achieved": sm_bytes / (stage[2] * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": sm_bytes / (stage[2] * 1e-3) / 1e9 / hbm_peak, "traffic": None, "peak_source": hsrc,
+                     "bytes_per_launch": sm_bytes},
+        "products": {"qk_tflops": 2.0 * H * Tq * Tk * D / (stage[1] * 1e-3) / 1e12,
+                     "pv_tflops": 2.0 * H * Tq * Tk * D / (stage[3] * 1e-3) / 1e12,
+                     "fp4_peak": fp4_peak, "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g}"},
+        "breakdown_ms": {"rotate_and_quantize_qkv": stage[0], "qk_product": stage[1], "softmax_quantize": stage[2],
+                         "pv_product": stage[3], "rows_divide": stage[4]},
+        "normalised_abs_error_vs_fp64_attention": nae,
+        "gpu_launches": 20 * steps,
+        "clocks": clocks,
+        "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = attn_oracle_baseline(args)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def attn_oracle_baseline(args, Tq=64, Tk=1024):
+    """The oracle pipeline on one head, Tq x Tk, timed on one host core."""
+    import numpy as np
+    import torch
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    from oracle import oracle as O
+    q, k, v = W.attn_inputs("cpu", scale=Tk / 32768)
+    D = q.shape[2]
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    qh, kh, vh = u16(q[0, -Tq:]), u16(k[0, :Tk]), u16(v[0, :Tk])
+    t = time.perf_counter()
+    qc, qs, qg, _, _ = O.quantize(O.hadamard16(qh.reshape(-1), dtype=O.BF16, out_dtype=O.F32))
+    kc, ks, kg, _, _ = O.quantize(O.hadamard16(kh.reshape(-1), dtype=O.BF16, out_dtype=O.F32))
+    s = O.gemm_nt(qc, qs, qg, kc, ks, kg, Tq, Tk, D, D ** -0.5).astype(np.float32)
+    pc, ps, _, pl, pg = O.softmax_quantize(s, True, Tk - Tq)
+    vc, vs, vg, _, _ = O.quantize(np.ascontiguousarray(vh.T).reshape(-1), dtype=O.BF16)
+    O.gemm_nt(pc, ps, pg, vc, vs, vg, Tq, D, Tk) / pl[..., None]
+    el = time.perf_counter() - t
+    return {"value": 4.0 * Tq * Tk * D / el / 1e12, "unit": "TFLOP/s", "cores": torch_threads(), "kind": "oracle",
+            "sample": f"one head, {Tq} queries x {Tk} keys, D = {D}: the oracle pipeline (C quantize and softmax, "
+                      f"fp64 numpy products), {el:.2f} s"}
+
+
+def run_attn_reference(args, rank, world):
+    if rank != 0:
+        return
+    base = attn_oracle_baseline(args)
+    print(json.dumps({
+        "impl": "reference", "metric": ATTN_METRIC, "value": base["value"], "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": 1, "warmup": 0, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4 operands, f64 oracle", "data": SOURCE_NOTE,
+        "config": attn_config(args, (8, 2048, 32768, 128)), "cpu_baseline": base,
+        "e2e": {"value": base["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -678,6 +865,8 @@ def main():
             run_gemm_reference(args, rank, world)
         elif args.workload == "msda_nvfp4":
             run_msda_reference(args, rank, world)
+        elif args.workload == "attn_nvfp4":
+            run_attn_reference(args, rank, world)
         else:
             run_reference(args, rank, world)
         return
@@ -700,6 +889,9 @@ def main():
         return
     if args.workload == "msda_nvfp4":
         run_msda(args, rank, world, dev)
+        return
+    if args.workload == "attn_nvfp4":
+        run_attn(args, rank, world, dev)
         return
     w = W.make(args.workload, dev, args.scale, shard=rank)
     x = w.x.contiguous()

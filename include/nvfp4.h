@@ -219,8 +219,9 @@ int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs
  * not say how P is formed, this is the flash-attention form).  s: scores [batch, Tq, Tk] FP32 (16-byte
  * aligned, Tk % 16 == 0).  For each row (b, q): m = max over the allowed keys (causal != 0: key k is
  * allowed iff k <= q + q_offset), P~_k = exp(S_k - m) for allowed keys and 0 otherwise, l = sum_k P~_k.
- * exp is a fixed FP32 method: n = rint(x log2 e), r = (x - n ln2_hi) - n ln2_lo (ln 2 split at 16
- * significant bits), p = degree-7 Taylor polynomial of e^r in Horner form, result p 2^n (0 below -104).
+ * exp is a fixed FP32 method: n = rint(x log2 e), r = fma(n, -ln2_lo, fma(n, -ln2_hi, x)) (ln 2 split at
+ * 16 significant bits), p = degree-7 Taylor polynomial of e^r in Horner form with fused multiply-adds,
+ * result p 2^n (0 below -104).
  * P~ is ScaleSearch-quantized along the keys (window [f_lo, f_hi] of 1, 9 or 17 offsets) with the tensor
  * scale g = fl(1/2688): codes [batch, Tq, Tk/2], sf the tile layout of the [Tq, Tk] matrices
  * (nvfp4_sf_mma_bytes(Tq, Tk, batch) bytes), *gscale = g, row_max / row_sum [batch * Tq] (FP32; the

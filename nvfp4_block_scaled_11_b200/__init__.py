@@ -410,17 +410,18 @@ def msda_forward(value, shapes, loc: torch.Tensor, w: torch.Tensor, out: torch.T
 
 
 # ---- FP4 attention (ScaleSearchAttention numerics, unfused) ----
-def softmax_quantize_mma(s: torch.Tensor, causal: bool = False, q_offset: int = 0, f_lo: int = -2, f_hi: int = 6):
+def softmax_quantize_mma(s: torch.Tensor, causal: bool = False, q_offset: int = 0, f_lo: int = -2, f_hi: int = 6,
+                         codes=None, sf=None, g=None, m=None, l=None):
     """s float32 [batch, Tq, Tk] (or [Tq, Tk]).  Returns (codes [.., Tq, Tk/2], sf tile layout, gscale[1],
-    row_max [batch*Tq], row_sum [batch*Tq]) for the softmax numerators P~ = exp(S - m)."""
+    row_max [batch*Tq], row_sum [batch*Tq]) for the softmax numerators P~ = exp(S - m); outputs may be given."""
     _cuda(s, "s")
     batch, Tq, Tk = (1, *s.shape) if s.dim() == 2 else s.shape
     dev = s.device
-    codes = torch.empty((*s.shape[:-1], Tk // 2), dtype=torch.uint8, device=dev)
-    sf = torch.empty(max(sf_mma_bytes(Tq, Tk, batch), 1), dtype=torch.uint8, device=dev)
-    g = torch.empty(1, dtype=torch.float32, device=dev)
-    m = torch.empty(batch * Tq, dtype=torch.float32, device=dev)
-    l = torch.empty(batch * Tq, dtype=torch.float32, device=dev)
+    codes = torch.empty((*s.shape[:-1], Tk // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    sf = torch.empty(max(sf_mma_bytes(Tq, Tk, batch), 1), dtype=torch.uint8, device=dev) if sf is None else sf
+    g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
+    m = torch.empty(batch * Tq, dtype=torch.float32, device=dev) if m is None else m
+    l = torch.empty(batch * Tq, dtype=torch.float32, device=dev) if l is None else l
     _check(lib().nvfp4_softmax_quantize_mma(_ptr(s), batch, Tq, Tk, int(bool(causal)), q_offset, f_lo, f_hi,
                                             _ptr(codes), _ptr(sf), _ptr(g), _ptr(m), _ptr(l), _stream(s)))
     return codes, sf, g, m, l

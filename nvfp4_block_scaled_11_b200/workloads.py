@@ -124,6 +124,17 @@ def msda_inputs(device="cpu", nq: int = 10000, bs: int = 6, heads: int = 8, poin
     return loc.contiguous(), w.contiguous()
 
 
+def attn_inputs(device="cpu", Tq: int = 2048, scale: float = 1.0):
+    """FP4-attention inputs over the KV-cache keys: q [8, Tq, 128] ~ N(0,1) (seed 21), k = kv_bf16's keys
+    [8, 32768, 128] (seed 2), v [8, 32768, 128] ~ N(0,1) (seed 22), all BF16; `scale` shrinks the tokens."""
+    Tk = max(128, int(32768 * scale)) // 128 * 128
+    Tq = max(64, int(Tq * scale)) // 64 * 64
+    k = kv_bf16(device, scale=Tk / 32768)[0]
+    q = torch.randn((8, Tq, 128), generator=_gen(21, device), device=device).to(torch.bfloat16)
+    v = torch.randn((8, Tk, 128), generator=_gen(22, device), device=device).to(torch.bfloat16)
+    return q, k[:, :Tk].contiguous(), v
+
+
 def make(name: str, device="cpu", scale: float = 1.0, shard: int = 0) -> Workload:
     if name == "act_f32":
         return Workload(name, act_f32(device, scale), -2, 6, "quantize", "FP32 [1024,4096] N(0,1), seed 0")

@@ -473,15 +473,15 @@ float ref_exp_ss(float x) {
   const float ln2_hi = 0x1.62e4p-1f;                   /* ln 2 rounded to 16 significant bits */
   const float ln2_lo = 0x1.7f7d1cp-20f;                /* fl(ln 2 - ln2_hi) */
   const float n = rintf(x * log2e);
-  const float r = (x - n * ln2_hi) - n * ln2_lo;
-  float p = 0x1.a01a02p-13f;                           /* 1/7! */
-  p = p * r + 0x1.6c16c2p-10f;                         /* 1/6! */
-  p = p * r + 0x1.111112p-7f;                          /* 1/5! */
-  p = p * r + 0x1.555556p-5f;                          /* 1/4! */
-  p = p * r + 0x1.555556p-3f;                          /* 1/3! */
-  p = p * r + 0x1p-1f;                                 /* 1/2! */
-  p = p * r + 1.0f;
-  p = p * r + 1.0f;
+  const float r = fmaf(n, -ln2_lo, fmaf(n, -ln2_hi, x));  /* the first step is exact */
+  float p = 0x1.a01a02p-13f;                           /* 1/7!, then Horner with fused multiply-adds */
+  p = fmaf(p, r, 0x1.6c16c2p-10f);                     /* 1/6! */
+  p = fmaf(p, r, 0x1.111112p-7f);                      /* 1/5! */
+  p = fmaf(p, r, 0x1.555556p-5f);                      /* 1/4! */
+  p = fmaf(p, r, 0x1.555556p-3f);                      /* 1/3! */
+  p = fmaf(p, r, 0x1p-1f);                             /* 1/2! */
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
   const int k = (int)n;
   if (k >= -126) return p * pow2f(k);
   return (p * pow2f(k + 64)) * pow2f(-64);

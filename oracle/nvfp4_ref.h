@@ -128,9 +128,10 @@ int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* s
  * exp is ref_exp_ss below, so both implementations produce the same P~ bit for bit. */
 
 /* exp(x) in FP32 by Cody-Waite reduction and a degree-7 Taylor polynomial (published method, fixed
- * operation order, no FMA): n = rint(x * log2(e)), r = (x - n * ln2_hi) - n * ln2_lo with ln2 split at 16
- * significant bits (n * ln2_hi exact), p = Horner(1, 1, 1/2!, ..., 1/7!) at r, result p * 2^n (scaled in
- * two exact steps below 2^-126).  x < -104 gives 0; NaN gives NaN. */
+ * operation order): n = rint(x * log2(e)), r = fma(n, -ln2_lo, fma(n, -ln2_hi, x)) with ln2 split at 16
+ * significant bits (the inner step is exact), p = Horner(1, 1, 1/2!, ..., 1/7!) at r with fused
+ * multiply-adds, result p * 2^n (scaled in two exact steps below 2^-126).  x < -104 gives 0; NaN gives
+ * NaN.  (The one place the oracle uses FMA: it is part of this method's definition.) */
 float ref_exp_ss(float x);
 
 int ref_softmax_quantize(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
