@@ -91,6 +91,13 @@ int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, 
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n,
                      int out_dtype, void* out, void* stream);
 
+/* nvfp4_dequantize with a bound on the launch footprint: at most ctas_per_sm CTAs of 256 threads per
+ * SM (1..8; 0 = the default 8), so that the kernel can run beside another kernel that occupies most of
+ * each SM -- e.g. dequantizing a finished chunk on a second stream while the search of the next chunk
+ * is still running.  Outputs are identical to nvfp4_dequantize. */
+int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n,
+                        int out_dtype, void* out, int ctas_per_sm, void* stream);
+
 /* Hadamard-16 rotation ("Search your block floating-point scales!", ScaleSearchAttention >
  * incoherence processing): each contiguous group of 16 elements is multiplied by the Sylvester
  * Hadamard matrix H16 / 4, computed as butterflies with strides 1, 2, 4, 8 in FP32.

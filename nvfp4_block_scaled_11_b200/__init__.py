@@ -37,6 +37,7 @@ _SIGS = {
     "nvfp4_quantize": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P]),
     "nvfp4_quantize_ex": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
+    "nvfp4_dequantize_ex": (_I, [_P, _P, _P, _I64, _I, _P, _I, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_msda_forward_nvfp4": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
@@ -171,13 +172,14 @@ def quantize_ex(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,
-               out: torch.Tensor | None = None) -> torch.Tensor:
-    """Dequantize n = 16 * scales.numel() elements to out_dtype."""
+               out: torch.Tensor | None = None, ctas_per_sm: int = 0) -> torch.Tensor:
+    """Dequantize n = 16 * scales.numel() elements to out_dtype.  ctas_per_sm > 0 bounds the launch
+    footprint (to run beside another kernel on a second stream); 0 = default."""
     _cuda(codes, "codes"), _cuda(scales, "scales"), _cuda(gscale, "gscale")
     n = scales.numel() * 16
     out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
-    _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), _ptr(gscale), n, DTYPE_CODE[out.dtype], _ptr(out),
-                                  _stream(codes)))
+    _check(lib().nvfp4_dequantize_ex(_ptr(codes), _ptr(scales), _ptr(gscale), n, DTYPE_CODE[out.dtype], _ptr(out),
+                                     ctas_per_sm, _stream(codes)))
     return out
 
 

@@ -323,13 +323,18 @@ int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int
 
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,
                      void* out, void* stream) {
-  if (!dtype_ok(out_dtype) || gscale == nullptr) return NVFP4_ERR_ARG;
+  return nvfp4_dequantize_ex(codes, scales, gscale, n, out_dtype, out, 0, stream);
+}
+
+int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,
+                        void* out, int ctas_per_sm, void* stream) {
+  if (!dtype_ok(out_dtype) || gscale == nullptr || ctas_per_sm < 0 || ctas_per_sm > 8) return NVFP4_ERR_ARG;
   if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (codes == nullptr || scales == nullptr || out == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
   const int64_t nb = n / 16;
-  const int grid = grid_for(nb, 256, 8);
+  const int grid = grid_for(nb, 256, ctas_per_sm ? ctas_per_sm : 8);
   const int v8 = aligned(out, 32) ? 1 : 0;
   char* o = static_cast<char*>(out);
   cudaStream_t s = S(stream);
