@@ -52,3 +52,30 @@ def test_concurrent_streams_mma_layout_and_product():
         assert np.array_equal(ac.cpu().numpy().reshape(-1), rc) and np.array_equal(asf.cpu().numpy(), rsf)
         d_seq = nv.gemm_nt(ac, asf, ag, bc, bsf, bg)          # the same product, alone
         assert torch.equal(d, d_seq)
+
+
+def test_dequantize_footprint_and_chunked_overlap_are_identical():
+    g = torch.Generator().manual_seed(19)
+    x = (torch.randn(1 << 22, generator=g) * 3).cuda()
+    codes, scales, gs = nv.quantize(x)
+    ref = nv.dequantize(codes, scales, gs)
+    for cps in (1, 2, 8):
+        assert torch.equal(nv.dequantize(codes, scales, gs, ctas_per_sm=cps), ref)
+    with pytest.raises(nv.NVFP4Error):
+        nv.dequantize(codes, scales, gs, ctas_per_sm=9)
+    # search chunk i+1 on the main stream while chunk i is dequantized on a second one
+    n, nch = x.numel(), 4
+    c = n // nch
+    c2, s2, d2 = torch.empty_like(codes), torch.empty_like(scales), torch.empty_like(ref)
+    main, aux = torch.cuda.current_stream(), torch.cuda.Stream()
+    for i in range(nch):
+        nv.quantize_ex(x[i * c:(i + 1) * c], gscale_in=gs, want_f=False, want_sse=False,
+                       codes=c2[i * c // 2:(i + 1) * c // 2], scales=s2[i * c // 16:(i + 1) * c // 16], gscale=None)
+        ev = torch.cuda.Event()
+        ev.record(main)
+        aux.wait_event(ev)
+        with torch.cuda.stream(aux):
+            nv.dequantize(c2[i * c // 2:(i + 1) * c // 2], s2[i * c // 16:(i + 1) * c // 16], gs,
+                          out=d2[i * c:(i + 1) * c], ctas_per_sm=2)
+    torch.cuda.synchronize()
+    assert torch.equal(c2, codes) and torch.equal(s2, scales) and torch.equal(d2, ref)
