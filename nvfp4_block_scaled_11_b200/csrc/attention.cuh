@@ -85,8 +85,9 @@ constexpr int kSoftmaxDeferCap = 64;
 
 template <int NC>
 __global__ void __launch_bounds__(256) softmax_quantize_kernel(QuantParams p, SoftmaxParams a) {
-  __shared__ CandEntry tab[128];
+  __shared__ CandEntry tab_store[kTabSize];
   __shared__ float thr[128];
+  CandEntry* tab = tab_store + kTabPad;   // indexed by code
   __shared__ int defer[8][kSoftmaxDeferCap];
   const float g = __fdiv_rn(1.0f, kTensorDiv);   // the tensor scale of numerators whose maximum is 1
   build_cand_entries(tab, g);
