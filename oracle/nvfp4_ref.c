@@ -370,6 +370,25 @@ int ref_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype
   return 0;
 }
 
+/* Hadamard-16 with a random sign diagonal D (QuIP#-style incoherence processing, as cited on the
+ * ScaleSearchAttention page): forward out = (H16 / 4) D x, inverse (the transpose) out = D (H16 / 4) x.
+ * Bit i of `signs` set means element i of every group is negated; negation is exact.  signs = 0 and
+ * either direction give ref_hadamard16. */
+int ref_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_dtype, uint32_t signs, int inverse) {
+  if (n < 0 || n % 16 != 0 || signs > 0xFFFFu) return -2;
+  float blk[16];
+  for (int64_t b = 0; b < n / 16; ++b) {
+    for (int i = 0; i < 16; ++i) blk[i] = load_elem(x, dtype, 16 * b + i);
+    if (!inverse)
+      for (int i = 0; i < 16; ++i) if ((signs >> i) & 1u) blk[i] = -blk[i];
+    ref_fwht16_f32(blk);
+    if (inverse)
+      for (int i = 0; i < 16; ++i) if ((signs >> i) & 1u) blk[i] = -blk[i];
+    for (int i = 0; i < 16; ++i) store_elem(out, out_dtype, 16 * b + i, blk[i]);
+  }
+  return 0;
+}
+
 /* ---------------------------------------------------------------------------------------------
  * Attention-sink mixed-precision KV layout ([SS] page, ScaleSearchAttention > attention-sink-aware
  * mixed-precision caching): the first and last blocks of the cache stay at full precision, the

@@ -90,6 +90,9 @@ int ref_dequantize(const uint8_t* codes, const uint8_t* scales, float g, int64_t
 /* 16-point fast Walsh-Hadamard transform on each contiguous group of 16, times 1/4. */
 int ref_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype);
 void ref_fwht16_f32(float* a);
+/* The same with a sign diagonal D from the low 16 bits of `signs` (bit i negates element i):
+ * inverse = 0: out = (H16/4) D x; inverse = 1: out = D (H16/4) x.  -2 if signs > 0xFFFF. */
+int ref_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_dtype, uint32_t signs, int inverse);
 
 /* Mixed-precision KV layout for K[B,H,T,D] (BF16): tokens [0,sink) and [T-recent,T) copied verbatim,
  * the rest optionally rotated (FWHT-16 along D) and ScaleSearch-quantized along D with one tensor

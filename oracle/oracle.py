@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "ref_quantize_blocks": (None, [P, I, I64, I64, F, I, I, P, P, P, P]),
             "ref_dequantize": (I, [P, P, F, I64, I, P]),
             "ref_hadamard16": (I, [P, I64, I, P, I]),
+            "ref_hadamard16_ex": (I, [P, I64, I, P, I, ctypes.c_uint32, I]),
             "ref_fwht16_f32": (None, [P]),
             "ref_kv_mixed": (I, [P, I64, I64, I64, I64, I, I, I, I, I, P, P, P, P, P]),
             "ref_exp_ss": (F, [F]),
@@ -215,6 +216,18 @@ def hadamard16(x: np.ndarray, dtype: int | None = None, out_dtype: int = F32) ->
     rc = lib().ref_hadamard16(_p(x), x.size, dtype, _p(out), out_dtype)
     if rc != 0:
         raise ValueError(f"ref_hadamard16 returned {rc}")
+    return out
+
+
+def hadamard16_ex(x: np.ndarray, signs: int, inverse: bool = False, dtype: int | None = None,
+                  out_dtype: int = F32) -> np.ndarray:
+    """(H16/4) D x, or D (H16/4) x when inverse; D negates element i of each group when bit i of signs is set."""
+    x = np.ascontiguousarray(x)
+    dtype = _dtype_of(x) if dtype is None else dtype
+    out = np.empty(x.size, _NP_OF[out_dtype])
+    rc = lib().ref_hadamard16_ex(_p(x), x.size, dtype, _p(out), out_dtype, signs, int(inverse))
+    if rc != 0:
+        raise ValueError(f"ref_hadamard16_ex returned {rc}")
     return out
 
 

@@ -260,6 +260,26 @@ def test_hadamard16_matches_matrix_and_is_an_involution():
     assert np.array_equal(O.hadamard16(xb.view(np.uint16), dtype=O.BF16), O.hadamard16(xb.astype(np.float32)))
 
 
+def test_hadamard16_sign_diagonal():
+    """QuIP#-style H D: the forward map is (H/4) D, the inverse its transpose D (H/4)."""
+    H = _sylvester(16) / 4.0
+    Xi = RNG.integers(-64, 65, (256, 16)).astype(np.float32)
+    for signs in (0x0001, 0x8000, 0xA5C3, 0xFFFF, int(RNG.integers(0, 1 << 16))):
+        D = np.diag([-1.0 if (signs >> i) & 1 else 1.0 for i in range(16)])
+        fwd = O.hadamard16_ex(Xi.reshape(-1), signs).reshape(-1, 16)
+        assert np.array_equal(fwd, (Xi.astype(np.float64) @ (H @ D).T).astype(np.float32))
+        inv = O.hadamard16_ex(Xi.reshape(-1), signs, inverse=True).reshape(-1, 16)
+        assert np.array_equal(inv, (Xi.astype(np.float64) @ (D @ H).T).astype(np.float32))
+        # the inverse undoes the forward map, and dot products of rotated pairs are unchanged
+        assert np.array_equal(O.hadamard16_ex(fwd.reshape(-1), signs, inverse=True).reshape(-1, 16), Xi)
+        assert np.array_equal((fwd[:128].astype(np.float64) * fwd[128:]).sum(1),
+                              (Xi[:128].astype(np.float64) * Xi[128:]).sum(1))
+    assert np.array_equal(O.hadamard16_ex(Xi.reshape(-1), 0), O.hadamard16(Xi.reshape(-1)))
+    assert np.array_equal(O.hadamard16_ex(Xi.reshape(-1), 0, inverse=True), O.hadamard16(Xi.reshape(-1)))
+    with pytest.raises(ValueError):
+        O.hadamard16_ex(Xi.reshape(-1), 1 << 16)
+
+
 def test_kv_mixed_layout():
     rng = np.random.default_rng(3)
     B, H, T, D = 1, 2, 80, 128
