@@ -104,6 +104,15 @@ int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float
  * x and out: n elements (n % 16 == 0); out may alias x only when dtype == out_dtype. */
 int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype, void* stream);
 
+/* Hadamard-16 with a sign diagonal D, the random-sign form of QuIP#-style incoherence processing that
+ * the ScaleSearchAttention page cites: bit i of `signs` (0..0xFFFF) negates element i of every group
+ * of 16 (exact).  inverse = 0: out = (H16/4) D x; inverse = 1: out = D (H16/4) x, the transpose, so
+ * applying both returns x up to FP32 rounding.  Q and K rotated with the same signs keep their dot
+ * products.  signs = 0 gives nvfp4_hadamard16.  Other arguments and errors as nvfp4_hadamard16;
+ * NVFP4_ERR_ARG for signs > 0xFFFF or inverse not 0/1. */
+int nvfp4_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_dtype, uint32_t signs,
+                        int inverse, void* stream);
+
 /* Attention-sink mixed-precision KV layout ("Search your block floating-point scales!",
  * ScaleSearchAttention > attention-sink-aware mixed-precision caching).
  * k_bf16: K[B,H,T,D] BF16, contiguous.  D % 16 == 0, T >= sink_tokens + recent_tokens.

@@ -39,6 +39,7 @@ _SIGS = {
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_dequantize_ex": (_I, [_P, _P, _P, _I64, _I, _P, _I, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
+    "nvfp4_hadamard16_ex": (_I, [_P, _I64, _I, _P, _I, ctypes.c_uint32, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_msda_forward_nvfp4": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
     "nvfp4_msda_forward": (_I, [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
@@ -183,12 +184,18 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, 
     return out
 
 
-def hadamard16(x: torch.Tensor, out_dtype=None, out: torch.Tensor | None = None) -> torch.Tensor:
-    """FWHT-16 / 4 on every contiguous group of 16 elements."""
+def hadamard16(x: torch.Tensor, out_dtype=None, out: torch.Tensor | None = None, signs: int = 0,
+               inverse: bool = False) -> torch.Tensor:
+    """FWHT-16 / 4 on every contiguous group of 16 elements; with `signs` (16-bit mask) the sign diagonal
+    D goes first, (H/4) D x, or last for the inverse, D (H/4) x."""
     _cuda(x, "x")
     out_dtype = x.dtype if out_dtype is None else out_dtype
     out = torch.empty(x.shape, dtype=out_dtype, device=x.device) if out is None else out
-    _check(lib().nvfp4_hadamard16(_ptr(x), x.numel(), _dt(x), _ptr(out), DTYPE_CODE[out.dtype], _stream(x)))
+    if signs == 0 and not inverse:
+        _check(lib().nvfp4_hadamard16(_ptr(x), x.numel(), _dt(x), _ptr(out), DTYPE_CODE[out.dtype], _stream(x)))
+    else:
+        _check(lib().nvfp4_hadamard16_ex(_ptr(x), x.numel(), _dt(x), _ptr(out), DTYPE_CODE[out.dtype], signs,
+                                         int(inverse), _stream(x)))
     return out
 
 
@@ -438,10 +445,11 @@ def rows_divide(x: torch.Tensor, l: torch.Tensor) -> torch.Tensor:
 
 
 def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, rotate: bool = True,
-                  scale: float | None = None, f_lo: int = -2, f_hi: int = 6):
+                  scale: float | None = None, f_lo: int = -2, f_hi: int = 6, signs: int = 0):
     """Attention with every product in NVFP4 on the tensor cores ("Search your block floating-point
     scales!", ScaleSearchAttention; unfused): q [H, Tq, D], k and v [H, Tk, D].
-      rotate: Hadamard-16 along D on q and k (Q K^T unchanged, outliers spread);
+      rotate: Hadamard-16 along D on q and k (Q K^T unchanged, outliers spread), after the sign
+        diagonal given by the 16-bit mask `signs` (the same for both, so Q K^T is still unchanged);
       S = scale * Q K^T (NVFP4 x NVFP4, FP32 accumulation);  P~ = exp(S - rowmax) quantized with ScaleSearch;
       O = (P~ V) / rowsum with V quantized along the tokens.  Causal: query i sees keys <= i + Tk - Tq.
     Returns O [H, Tq, D] float32."""
@@ -449,8 +457,8 @@ def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
     Tk = k.shape[1]
     scale = D ** -0.5 if scale is None else scale
     if rotate:
-        q = hadamard16(q.contiguous(), out_dtype=torch.float32)
-        k = hadamard16(k.contiguous(), out_dtype=torch.float32)
+        q = hadamard16(q.contiguous(), out_dtype=torch.float32, signs=signs)
+        k = hadamard16(k.contiguous(), out_dtype=torch.float32, signs=signs)
     qc, qsf, qg = quantize_mma(q.contiguous(), f_lo, f_hi)
     kc, ksf, kg = quantize_mma(k.contiguous(), f_lo, f_hi)
     s = gemm_nt(qc, qsf, qg, kc, ksf, kg, alpha=scale)

@@ -380,18 +380,31 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 }
 
 // =================================================================================================
-// Hadamard-16: one thread per group of 16.
+// Hadamard-16: one thread per group of 16.  An optional sign diagonal D (bit i of `signs` negates
+// element i, exactly, by flipping its sign bit) goes before the butterflies (H D) or, for the inverse,
+// after them (D H).
 // =================================================================================================
+__device__ __forceinline__ void flip_signs(float (&a)[16], const uint32_t (&m)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(__float_as_uint(a[i]) ^ m[i]);
+}
+
 template <int DT, int OT>
 __global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict__ x, int64_t ngroups,
-                                                         char* __restrict__ out, int v8_in, int v8_out) {
+                                                         char* __restrict__ out, int v8_in, int v8_out,
+                                                         uint32_t signs, int inverse) {
   constexpr int ES = DT == DT_F32 ? 4 : 2;
   constexpr int OS = OT == DT_F32 ? 4 : 2;
+  uint32_t m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = ((signs >> i) & 1u) << 31;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < ngroups; b += stride) {
     float a[16];
     load_block<DT>(x + 16 * ES * b, v8_in != 0, a);
+    if (!inverse) flip_signs(a, m);
     fwht16(a);
+    if (inverse) flip_signs(a, m);
     char* o = out + 16 * OS * b;
     if (OT == DT_F32) {
       uint32_t w[16];

@@ -347,7 +347,13 @@ int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float
 }
 
 int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dtype, void* stream) {
-  if (!dtype_ok(dtype) || !dtype_ok(out_dtype)) return NVFP4_ERR_ARG;
+  return nvfp4_hadamard16_ex(x, n, dtype, out, out_dtype, 0u, 0, stream);
+}
+
+int nvfp4_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_dtype, uint32_t signs,
+                        int inverse, void* stream) {
+  if (!dtype_ok(dtype) || !dtype_ok(out_dtype) || signs > 0xFFFFu || (inverse != 0 && inverse != 1))
+    return NVFP4_ERR_ARG;
   if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (x == nullptr || out == nullptr) return NVFP4_ERR_ARG;
@@ -359,7 +365,7 @@ int nvfp4_hadamard16(const void* x, int64_t n, int dtype, void* out, int out_dty
   const char* xp = static_cast<const char*>(x);
   char* o = static_cast<char*>(out);
   cudaStream_t s = S(stream);
-#define NVFP4_H16(DI, DO) hadamard16_kernel<DI, DO><<<grid, 256, 0, s>>>(xp, ng, o, v8i, v8o)
+#define NVFP4_H16(DI, DO) hadamard16_kernel<DI, DO><<<grid, 256, 0, s>>>(xp, ng, o, v8i, v8o, signs, inverse)
   if (dtype == DT_F32) {
     if (out_dtype == DT_F32) NVFP4_H16(DT_F32, DT_F32);
     else if (out_dtype == DT_BF16) NVFP4_H16(DT_F32, DT_BF16);
@@ -500,11 +506,21 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
   p.sf_mat_bytes = ((Tq + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
   if ((Tq % 128 != 0 || bpr % 4 != 0) && cudaMemsetAsync(sf, 0, (size_t)(batch * p.sf_mat_bytes), st) != cudaSuccess)
     return NVFP4_ERR_CUDA;
-  SoftmaxParams a{s, rows, Tq, Tk, causal ? 1 : 0, q_offset, aligned(s, 32) ? 1 : 0, row_max, row_sum, gscale};
-  const int grid = grid_for(rows * 32, 256, 4);
-  if (nc == 9) softmax_quantize_kernel<9><<<grid, 256, 0, st>>>(p, a);
-  else if (nc == 1) softmax_quantize_kernel<1><<<grid, 256, 0, st>>>(p, a);
-  else softmax_quantize_kernel<17><<<grid, 256, 0, st>>>(p, a);
+  // warps per row: one while the rows alone give every SM its 32 resident warps (the kernel is bound by
+  // instruction issue, and warps that share a row wait for one another twice per row); for fewer, longer
+  // rows (decode) up to 8, each warp keeping at least 64 blocks (two rounds of its lanes)
+  int wpr = 1;
+  while (wpr < 8 && rows * wpr < (int64_t)sm_count() * 32 && bpr >= 128 * (int64_t)wpr) wpr *= 2;
+  SoftmaxParams a{s, rows, Tq, Tk, causal ? 1 : 0, q_offset, aligned(s, 32) ? 1 : 0, wpr, row_max, row_sum, gscale};
+  const int64_t groups = (rows + 8 / wpr - 1) / (8 / wpr);
+  const int grid = grid_for(groups * 256, 256, 4);
+#define NVFP4_SOFTMAX(NC) \
+  (wpr > 1 ? softmax_quantize_kernel<NC, true><<<grid, 256, 0, st>>>(p, a) \
+           : softmax_quantize_kernel<NC, false><<<grid, 256, 0, st>>>(p, a))
+  if (nc == 9) NVFP4_SOFTMAX(9);
+  else if (nc == 1) NVFP4_SOFTMAX(1);
+  else NVFP4_SOFTMAX(17);
+#undef NVFP4_SOFTMAX
   return last_error();
 }
 

@@ -68,6 +68,9 @@ def test_other_entry_point_errors(L):
     assert L.nvfp4_dequantize(fake, fake, fake, 32, 0, V(0x10004), None) == -3
     assert L.nvfp4_hadamard16(fake, 20, 0, fake, 0, None) == -2
     assert L.nvfp4_hadamard16(fake, 32, 0, fake, 1, None) == -1  # in place across dtypes
+    assert L.nvfp4_hadamard16_ex(fake, 32, 0, fake, 0, 0x10000, 0, None) == -1   # signs beyond 16 bits
+    assert L.nvfp4_hadamard16_ex(fake, 32, 0, fake, 0, 0x00FF, 2, None) == -1     # inverse not 0/1
+    assert L.nvfp4_hadamard16_ex(fake, 20, 0, fake, 0, 0x00FF, 1, None) == -2
     assert L.nvfp4_tensor_amax(fake, 10, 5, fake, None) == -1
     assert L.nvfp4_tensor_amax(V(0x10002), 10, 0, fake, None) == -3
     assert L.nvfp4_global_scale(None, fake, None) == -1

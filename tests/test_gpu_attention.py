@@ -24,7 +24,11 @@ def _scores(batch, Tq, Tk, seed, scale=2.5):
 
 @pytest.mark.parametrize("batch,Tq,Tk,causal,q_offset,window", [
     (2, 37, 96, False, 0, (-2, 6)), (1, 130, 2048, True, 1918, (-2, 6)), (3, 8, 64, True, 0, (-2, 6)),
-    (1, 64, 256, False, 0, (0, 0)), (1, 64, 256, True, 192, (-8, 8))])
+    (1, 64, 256, False, 0, (0, 0)), (1, 64, 256, True, 192, (-8, 8)),
+    # several warps per row: 8 (ragged 75-block chunks), 4 with an odd row count (the last CTA round has
+    # warps without a row), 8 with the causal limit inside a chunk, 2 with NC = 17
+    (1, 5, 9600, False, 0, (-2, 6)), (3, 7, 4800, True, 4790, (-2, 6)), (1, 33, 8192, True, 4000, (-2, 6)),
+    (2, 9, 2064, True, 1000, (-8, 8))])
 def test_softmax_quantize_matches_oracle(batch, Tq, Tk, causal, q_offset, window):
     s = _scores(batch, Tq, Tk, Tq + Tk)
     codes, sf, g, m, l = nv.softmax_quantize_mma(s.cuda(), causal, q_offset, *window)
@@ -97,3 +101,26 @@ def test_attention_fp4_pipeline_matches_oracle(causal):
     of = torch.einsum("hqk,hkd->hqd", torch.softmax(sf, -1), vf).numpy()
     nae = np.abs(o - of).mean() / np.abs(of).mean()
     assert nae < 0.25, nae
+
+
+def test_attention_fp4_sign_diagonal_keeps_the_product():
+    """Q and K rotated with the same random signs: the scores are those of the unrotated inputs up to
+    NVFP4 error, and the pipeline equals the oracle's with the same signs."""
+    H, Tq, Tk, D = 2, 64, 256, 64
+    g = torch.Generator().manual_seed(12)
+    q = torch.randn((H, Tq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
+    signs = 0x5A93
+    qr = nv.hadamard16(q.cuda(), out_dtype=torch.float32, signs=signs)
+    kr = nv.hadamard16(k.cuda(), out_dtype=torch.float32, signs=signs)
+    assert np.array_equal(qr.cpu().numpy().reshape(-1),
+                          O.hadamard16_ex(_u16(q).reshape(-1), signs, dtype=O.BF16, out_dtype=O.F32))
+    s_rot = torch.einsum("hqd,hkd->hqk", qr.double(), kr.double()).cpu()
+    s_ref = torch.einsum("hqd,hkd->hqk", q.double(), k.double())
+    assert torch.allclose(s_rot, s_ref, rtol=0, atol=1e-4)
+    o = nv.attention_fp4(q.cuda(), k.cuda(), v.cuda(), causal=True, signs=signs).cpu().double()
+    sf = (s_ref * D ** -0.5).masked_fill(torch.arange(Tk)[None, :] > torch.arange(Tq)[:, None] + (Tk - Tq),
+                                         float("-inf"))
+    of = torch.einsum("hqk,hkd->hqd", torch.softmax(sf, -1), v.double())
+    assert ((o - of).abs().mean() / of.abs().mean()).item() < 0.25

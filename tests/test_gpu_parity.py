@@ -136,6 +136,23 @@ def test_hadamard16(din, dout):
     assert same_f32(got, ref) if dout == torch.float32 else np.array_equal(got, ref)
 
 
+@pytest.mark.parametrize("din,dout", [(torch.float32, torch.float32), (torch.bfloat16, torch.float32),
+                                      (torch.float16, torch.bfloat16)])
+@pytest.mark.parametrize("signs", [0x0001, 0xA5C3, 0xFFFF])
+@pytest.mark.parametrize("inverse", [False, True])
+def test_hadamard16_signs(din, dout, signs, inverse):
+    x = (torch.randn(4096 * 16 + 16 * 7, generator=torch.Generator().manual_seed(signs)) * 3).to(din)
+    x[5] = float("nan")                          # a NaN group: all 16 outputs NaN (payloads may differ)
+    out = nv.hadamard16(x.cuda(), dout, signs=signs, inverse=inverse)
+    ref = O.hadamard16_ex(host_np(x), signs, inverse, dtype=DT_CODE[din], out_dtype=DT_CODE[dout])
+    got = host_np(out)
+    if dout == torch.float32:
+        assert same_f32(got, ref)
+    else:
+        nan_g, nan_r = (got & 0x7FFF) > 0x7F80, (ref & 0x7FFF) > 0x7F80
+        assert np.array_equal(nan_g, nan_r) and nan_r[:16].all() and np.array_equal(got[~nan_g], ref[~nan_r])
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("n", [0, 1, 7, 15, 16, 33, 1000, 4096 * 1024 + 13])
 def test_tensor_amax(dtype, n):
