@@ -120,15 +120,27 @@ __device__ __forceinline__ void softmax_block(const float* sr, int64_t j, float 
 }
 
 // The maximum over the allowed keys among [k0, k1) of a row (k0, k1 multiples of 16), warp-reduced.
+// Eight 16-byte loads per lane are issued before any is used, so a warp spends this pass waiting for
+// one round trip per 4 KB rather than per 512 bytes.
+__device__ __forceinline__ float row_max4(float m, const float4& v, int64_t k, int64_t lim) {
+  if (k + 3 <= lim) return fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+  if (k <= lim) m = fmaxf(m, v.x);
+  if (k + 1 <= lim) m = fmaxf(m, v.y);
+  if (k + 2 <= lim) m = fmaxf(m, v.z);
+  return m;
+}
+
 __device__ __forceinline__ float softmax_row_max(const float* sr, int64_t k0, int64_t k1, int64_t lim, int lane) {
   float m = -INFINITY;
-  for (int64_t k = k0 + 4 * (int64_t)lane; k < k1; k += 128) {
-    const float4 v = *reinterpret_cast<const float4*>(sr + k);
-    if (k <= lim) m = fmaxf(m, v.x);
-    if (k + 1 <= lim) m = fmaxf(m, v.y);
-    if (k + 2 <= lim) m = fmaxf(m, v.z);
-    if (k + 3 <= lim) m = fmaxf(m, v.w);
+  int64_t k = k0 + 4 * (int64_t)lane;
+  for (; k + 7 * 128 < k1; k += 8 * 128) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = *reinterpret_cast<const float4*>(sr + k + 128 * u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) m = row_max4(m, v[u], k + 128 * u, lim);
   }
+  for (; k < k1; k += 128) m = row_max4(m, *reinterpret_cast<const float4*>(sr + k), k, lim);
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   return m;
