@@ -130,6 +130,10 @@ __device__ __forceinline__ float row_max4(float m, const float4& v, int64_t k, i
   return m;
 }
 
+// One past the last key of the 16-key block that holds key lim (0 when no key is allowed): keys from
+// there on are masked, so the maximum pass need not read them.
+__device__ __forceinline__ int64_t allowed_end(int64_t lim) { return lim < 0 ? 0 : (lim & ~(int64_t)15) + 16; }
+
 __device__ __forceinline__ float softmax_row_max(const float* sr, int64_t k0, int64_t k1, int64_t lim, int lane) {
   float m = -INFINITY;
   int64_t k = k0 + 4 * (int64_t)lane;
@@ -177,7 +181,12 @@ __device__ __forceinline__ float softmax_row_blocks(const QuantParams& p, const 
   for (int64_t j0 = jb; j0 < je; j0 += 32) {   // warp-uniform rounds
     const int64_t j = j0 + lane;
     bool deferred = false;
-    if (j < je) {
+    if (j < je && 16 * j0 > lim) {
+      // the whole round lies past the last allowed key: every block is zero, which quantizes to scale 0
+      // and zero codes (what the full path computes for it), without exp or search
+      const u64 zero[8] = {0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull};
+      write_block<SRC_LINEAR, false>(p, row * bpr + j, zero, tab, 0, -128, 0.0f, false, 0.0f);
+    } else if (j < je) {
       float x[16];
       softmax_block(sr, j, m, lim, v8, x);
       u64 x2[8];
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(256, 4) softmax_quantize_kernel(QuantParams p,
     for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < a.rows; row += nwarps) {
       const int64_t lim = a.causal ? row % a.Tq + a.q_offset : a.Tk - 1;   // last allowed key
       const float* sr = a.s + row * a.Tk;
-      const float m = softmax_row_max(sr, 0, a.Tk, lim, lane);
+      const float m = softmax_row_max(sr, 0, min(a.Tk, allowed_end(lim)), lim, lane);
       const float l = softmax_row_blocks<NC>(p, tab, thr, inv6g, dlist, sr, row, bpr, 0, bpr, m, lim, v8, lane);
       if (lane == 0) {
         a.row_max[row] = m;
@@ -247,7 +256,7 @@ __global__ void __launch_bounds__(256, 4) softmax_quantize_kernel(QuantParams p,
       const bool live = row < a.rows;
       const int64_t lim = live && a.causal ? row % a.Tq + a.q_offset : a.Tk - 1;
       const float* sr = a.s + (live ? row : 0) * a.Tk;
-      float m = live ? softmax_row_max(sr, 16 * jb, 16 * je, lim, lane) : -INFINITY;
+      float m = live ? softmax_row_max(sr, 16 * jb, min(16 * je, allowed_end(lim)), lim, lane) : -INFINITY;
       if (lane == 0) red_max[warp] = m;
       __syncthreads();
       m = red_max[w0];

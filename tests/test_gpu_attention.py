@@ -28,7 +28,9 @@ def _scores(batch, Tq, Tk, seed, scale=2.5):
     # several warps per row: 8 (ragged 75-block chunks), 4 with an odd row count (the last CTA round has
     # warps without a row), 8 with the causal limit inside a chunk, 2 with NC = 17
     (1, 5, 9600, False, 0, (-2, 6)), (3, 7, 4800, True, 4790, (-2, 6)), (1, 33, 8192, True, 4000, (-2, 6)),
-    (2, 9, 2064, True, 1000, (-8, 8))])
+    (2, 9, 2064, True, 1000, (-8, 8)),
+    # square causal: whole 32-block rounds past the limit are written as zero blocks directly
+    (2, 64, 1024, True, 0, (-2, 6)), (1, 96, 2048, True, 0, (-2, 6)), (1, 40, 640, True, -100, (-2, 6))])
 def test_softmax_quantize_matches_oracle(batch, Tq, Tk, causal, q_offset, window):
     s = _scores(batch, Tq, Tk, Tq + Tk)
     codes, sf, g, m, l = nv.softmax_quantize_mma(s.cuda(), causal, q_offset, *window)
@@ -124,3 +126,30 @@ def test_attention_fp4_sign_diagonal_keeps_the_product():
                                          float("-inf"))
     of = torch.einsum("hqk,hkd->hqd", torch.softmax(sf, -1), v.double())
     assert ((o - of).abs().mean() / of.abs().mean()).item() < 0.25
+
+
+def test_softmax_quantize_full_size_sampled():
+    """The attention step's softmax shape (8 heads x 2048 queries x 32768 keys, causal, queries at the end)
+    in the benchmark's launch configuration (one warp per row): seeded scores made on the device, sampled
+    rows against the oracle run on those rows alone."""
+    H, Tq, Tk = 8, 2048, 32768
+    bpr = Tk // 16
+    gen = torch.Generator(device="cuda").manual_seed(23)
+    s = torch.randn((H, Tq, Tk), generator=gen, device="cuda") * 2.5
+    codes, sf, g, m, l = nv.softmax_quantize_mma(s, True, Tk - Tq)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(24)
+    picks = [(0, 0), (0, Tq - 1), (7, Tq - 1), (3, 777), (5, 1)] + [
+        (int(h), int(q)) for h, q in zip(rng.integers(0, H, 19), rng.integers(0, Tq, 19))]
+    codes_h = codes.view(H, Tq, Tk // 2)
+    sf_h = sf.cpu().numpy()
+    mat = O.sf_mma_bytes(Tq, bpr)
+    for h, q in picks:
+        row = s[h, q].cpu().numpy()[None, None, :]
+        rc, rs, rm, rl, rg = O.softmax_quantize(row, True, q + Tk - Tq)   # key k allowed iff k <= q + Tk - Tq
+        assert g.item() == rg
+        assert np.array_equal(codes_h[h, q].cpu().numpy(), rc.reshape(-1)), (h, q)
+        offs = [h * mat + O.sf_mma_offset(q, c, bpr) for c in range(bpr)]
+        assert np.array_equal(sf_h[offs], rs.reshape(-1)), (h, q)
+        assert m[h * Tq + q].item() == rm.item()
+        assert abs(l[h * Tq + q].item() - rl.item()) <= (Tk + 4) * U * rl.item()
