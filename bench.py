@@ -672,7 +672,8 @@ def attn_config(args, shape):
         "workload": f"attn_nvfp4 (q [{H},{Tq},{D}] N(0,1) seed 21; k = KV-cache keys [{H},{Tk},{D}] (N(0,1) + channel "
                     f"bias, seed 2); v [{H},{Tk},{D}] N(0,1) seed 22; BF16; causal, queries at the end)",
         "window": [args.f_lo, args.f_hi],
-        "step": "Hadamard-16 on q, k; ScaleSearch NVFP4 quantize of q, k (tile layout) and of v along tokens; "
+        "step": "ScaleSearch NVFP4 quantize of Hadamard-16-rotated q, k (rotation fused into amax and search; "
+                "tile layout) and of v along tokens; "
                 "S = Q K^T (FP4 tensor cores); softmax numerators quantized with ScaleSearch; O = P~ V^T "
                 "(FP4 tensor cores) / rowsum",
         "l2": "inputs and scores larger than L2 (S is 2.1 GB), no flush",
@@ -695,9 +696,9 @@ def run_attn(args, rank, world, dev):
     # every intermediate preallocated, so the step launches kernels only (no allocator calls)
     f32, u8 = torch.float32, torch.uint8
     E = lambda *shape, dt=f32: torch.empty(shape, dtype=dt, device=dev)
-    qr, kr = E(H, Tq, D), E(H, Tk, D)
     qc, qsf, qg = E(H, Tq, D // 2, dt=u8), E(nv.sf_mma_bytes(Tq, D, H), dt=u8), E(1)
     kc, ksf, kg = E(H, Tk, D // 2, dt=u8), E(nv.sf_mma_bytes(Tk, D, H), dt=u8), E(1)
+    q4, k4, qc4, kc4 = q[None], k[None], qc[None], kc[None]   # [1, H, T, D] views for the fused prologue
     vc, vsf, vg = E(H, D, Tk // 2, dt=u8), E(nv.sf_mma_bytes(D, Tk, H), dt=u8), E(1)
     s_buf = E(H, Tq, Tk)
     pc, psf, pg = E(H, Tq, Tk // 2, dt=u8), E(nv.sf_mma_bytes(Tq, Tk, H), dt=u8), E(1)
@@ -708,10 +709,9 @@ def run_attn(args, rank, world, dev):
             if evs:
                 evs[i].record(stream)
         mark(0)
-        nv.hadamard16(q, out=qr)
-        nv.hadamard16(k, out=kr)
-        nv.quantize_mma(qr, args.f_lo, args.f_hi, codes=qc, sf=qsf, gscale=qg)
-        nv.quantize_mma(kr, args.f_lo, args.f_hi, codes=kc, sf=ksf, gscale=kg)
+        # Hadamard-16 fused into the amax and search kernels of q and k (no FP32 copy)
+        nv.kv_mixed_mma(q4, 0, 0, True, args.f_lo, args.f_hi, codes=qc4, sf=qsf, gscale=qg)
+        nv.kv_mixed_mma(k4, 0, 0, True, args.f_lo, args.f_hi, codes=kc4, sf=ksf, gscale=kg)
         nv.quantize_mma_t(v, args.f_lo, args.f_hi, codes=vc, sf=vsf, gscale=vg)
         mark(1)
         nv.gemm_nt(qc, qsf, qg, kc, ksf, kg, alpha=scale, out=s_buf, alpha_work=aw1)
@@ -797,7 +797,7 @@ def run_attn(args, rank, world, dev):
         "breakdown_ms": {"rotate_and_quantize_qkv": stage[0], "qk_product": stage[1], "softmax_quantize": stage[2],
                          "pv_product": stage[3], "rows_divide": stage[4]},
         "normalised_abs_error_vs_fp64_attention": nae,
-        "gpu_launches": 20 * steps,
+        "gpu_launches": 18 * steps,   # 15 kernels + 3 memsets of the tensor-scale words
         "clocks": clocks,
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps},
     }

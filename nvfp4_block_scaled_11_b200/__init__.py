@@ -278,8 +278,11 @@ def quantize_mma_t(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: to
 
 
 def kv_mixed_mma(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = True, f_lo: int = -2,
-                 f_hi: int = 6):
+                 f_hi: int = 6, codes: torch.Tensor | None = None, sf: torch.Tensor | None = None,
+                 gscale: torch.Tensor | None = None):
     """kv_mixed with the middle-token scales of every (batch, head) in the tensor-core tile layout.
+    With sink = recent = 0 and rotate it is the rotated quantize of every token, fused (codes and scales
+    as quantize_mma of the FWHT-16-rotated FP32 tensor).  codes / sf / gscale: optional preallocated outputs.
 
     Returns (sink, recent, codes uint8[B,H,Tm,D/2], sf uint8[sf_mma_bytes(Tm, D, B*H)], gscale)."""
     _cuda(k, "k")
@@ -290,9 +293,14 @@ def kv_mixed_mma(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool
     dev = k.device
     so = torch.empty((B, H, sink, D), dtype=torch.bfloat16, device=dev)
     ro = torch.empty((B, H, recent, D), dtype=torch.bfloat16, device=dev)
-    codes = torch.empty((B, H, Tm, D // 2), dtype=torch.uint8, device=dev)
-    sf = torch.empty(max(sf_mma_bytes(Tm, D, B * H), 1), dtype=torch.uint8, device=dev)
-    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    codes = torch.empty((B, H, Tm, D // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    sf = torch.empty(max(sf_mma_bytes(Tm, D, B * H), 1), dtype=torch.uint8, device=dev) if sf is None else sf
+    gscale = torch.empty(1, dtype=torch.float32, device=dev) if gscale is None else gscale
+    for t, nm, need in ((codes, "codes", B * H * Tm * D // 2), (sf, "sf", sf_mma_bytes(Tm, D, B * H)),
+                        (gscale, "gscale", 1)):
+        _cuda(t, nm)
+        if t.numel() < need:
+            raise ValueError(f"{nm} holds {t.numel()} elements, {need} needed")
     _check(lib().nvfp4_kv_mixed_mma(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), f_lo, f_hi, _ptr(so),
                                     _ptr(ro), _ptr(codes), _ptr(sf), _ptr(gscale), _stream(k)))
     return so, ro, codes, sf, gscale
@@ -444,6 +452,19 @@ def rows_divide(x: torch.Tensor, l: torch.Tensor) -> torch.Tensor:
     return x
 
 
+def _prologue_operand(x: torch.Tensor, rotate: bool, signs: int, f_lo: int, f_hi: int):
+    """Q or K [H, T, D] as an NVFP4 tensor-core operand, Hadamard-rotated along D when `rotate`.  BF16
+    input without signs takes the fused path (rotation inside the amax and search kernels, no FP32 copy);
+    the result is bit-identical to quantize_mma(hadamard16(x, float32))."""
+    x = x.contiguous()
+    if rotate and signs == 0 and x.dtype == torch.bfloat16:
+        _, _, codes, sf, g = kv_mixed_mma(x[None], 0, 0, True, f_lo, f_hi)
+        return codes[0], sf, g
+    if rotate:
+        x = hadamard16(x, out_dtype=torch.float32, signs=signs)
+    return quantize_mma(x, f_lo, f_hi)
+
+
 def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, rotate: bool = True,
                   scale: float | None = None, f_lo: int = -2, f_hi: int = 6, signs: int = 0):
     """Attention with every product in NVFP4 on the tensor cores ("Search your block floating-point
@@ -456,11 +477,8 @@ def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: boo
     H, Tq, D = q.shape
     Tk = k.shape[1]
     scale = D ** -0.5 if scale is None else scale
-    if rotate:
-        q = hadamard16(q.contiguous(), out_dtype=torch.float32, signs=signs)
-        k = hadamard16(k.contiguous(), out_dtype=torch.float32, signs=signs)
-    qc, qsf, qg = quantize_mma(q.contiguous(), f_lo, f_hi)
-    kc, ksf, kg = quantize_mma(k.contiguous(), f_lo, f_hi)
+    qc, qsf, qg = _prologue_operand(q, rotate, signs, f_lo, f_hi)
+    kc, ksf, kg = _prologue_operand(k, rotate, signs, f_lo, f_hi)
     s = gemm_nt(qc, qsf, qg, kc, ksf, kg, alpha=scale)
     pc, psf, pg, _, l = softmax_quantize_mma(s, causal, Tk - Tq, f_lo, f_hi)
     vc, vsf, vg = quantize_mma_t(v.contiguous(), f_lo, f_hi)

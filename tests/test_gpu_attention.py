@@ -153,3 +153,14 @@ def test_softmax_quantize_full_size_sampled():
         assert np.array_equal(sf_h[offs], rs.reshape(-1)), (h, q)
         assert m[h * Tq + q].item() == rm.item()
         assert abs(l[h * Tq + q].item() - rl.item()) <= (Tk + 4) * U * rl.item()
+
+
+def test_fused_prologue_equals_rotate_then_quantize():
+    """attention_fp4's fused Q/K prologue (rotation inside the amax and search kernels) gives the same
+    operand bits as rotating into FP32 and quantizing that."""
+    g = torch.Generator().manual_seed(31)
+    x = (torch.randn((4, 192, 128), generator=g) * 3).to(torch.bfloat16).cuda()
+    x[1, 7, 5] = 40.0
+    c1, s1, g1 = nv._prologue_operand(x, True, 0, -2, 6)
+    c2, s2, g2 = nv.quantize_mma(nv.hadamard16(x, out_dtype=torch.float32), -2, 6)
+    assert torch.equal(g1, g2) and torch.equal(c1, c2) and torch.equal(s1, s2)
