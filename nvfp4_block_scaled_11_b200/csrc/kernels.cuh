@@ -165,6 +165,38 @@ __device__ __forceinline__ int64_t kv_block_elem(int64_t b, int64_t Tm, int64_t 
   return ((int64_t)bh * T + sink + t) * D + 16 * (int64_t)j;
 }
 
+// The split (bh, t, j) of KV block indices along a grid-stride loop: one division-based split at the
+// first block, then each step adds the stride, written as (qt head rows, qr tokens, rs block columns),
+// with at most one carry per level, so the loop itself divides nothing.
+struct KvCursor {
+  uint32_t bh, t, j;
+  uint32_t qt, qr, rs, Tm, bpr;
+  __device__ __forceinline__ void init(int64_t b, int64_t stride, int64_t Tm_, int64_t bpr_) {
+    Tm = (uint32_t)Tm_;
+    bpr = (uint32_t)bpr_;
+    kv_split(b, Tm_, bpr_, bh, t, j);
+    const uint32_t S = (uint32_t)stride, qs = S / bpr;
+    rs = S - qs * bpr;
+    qt = qs / Tm;
+    qr = qs - qt * Tm;
+  }
+  __device__ __forceinline__ void advance() {
+    j += rs;
+    const uint32_t c = j >= bpr ? 1u : 0u;
+    j -= c * bpr;
+    uint64_t tt = (uint64_t)t + qr + c;   // < 2 Tm
+    bh += qt;
+    if (tt >= Tm) {
+      tt -= Tm;
+      ++bh;
+    }
+    t = (uint32_t)tt;
+  }
+  __device__ __forceinline__ int64_t elem(int64_t T, int64_t sink, int64_t D) const {
+    return ((int64_t)bh * T + sink + t) * D + 16 * (int64_t)j;
+  }
+};
+
 // Output block index of block b (input order), fixed by the source mode at compile time: linear blocks
 // land where they are read; KV blocks land in rows out_t0.. of a cap-row cache when appending
 // (out_cap > 0); column blocks land in the transposed layout (row c of matrix l, block rb).
@@ -578,10 +610,12 @@ __global__ void __launch_bounds__(256) kv_amax_kernel(const char* __restrict__ k
                                                       uint32_t* __restrict__ out) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t m = 0;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < ngroups; b += stride) {
-    const int64_t elem = kv_block_elem(b, Tm, bpr, T, sink, D);
+  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  KvCursor kc;
+  if (b < ngroups) kc.init(b, stride, Tm, bpr);
+  for (; b < ngroups; b += stride, kc.advance()) {
     float x[16];
-    load_block<DT_BF16>(k + 2 * elem, v8 != 0, x);
+    load_block<DT_BF16>(k + 2 * kc.elem(T, sink, D), v8 != 0, x);
     if (ROT) fwht16(x);
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(x[i]) & 0x7FFFFFFFu);

@@ -501,8 +501,20 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const bool v8 = p.v8 != 0;
   int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  KvCursor kc;   // KV mode: the split of the block held in xn, carried along the loop
+  auto load_next = [&](int64_t bb, u64 (&dst)[8]) {
+    if constexpr (MODE == SRC_KV) {
+      constexpr int ES = DT == DT_F32 ? 4 : 2;
+      load_pairs<DT>(p.x + kc.elem(p.T, p.sink, p.D) * ES, v8, dst);
+    } else {
+      load_block_pairs<DT, MODE>(p, bb, v8, dst);
+    }
+  };
   u64 xn[8];
-  if (b < p.nblocks) load_block_pairs<DT, MODE>(p, b, v8, xn);  // in flight while the tables are built
+  if (b < p.nblocks) {
+    if constexpr (MODE == SRC_KV) kc.init(b, stride, p.Tm, p.bpr);
+    load_next(b, xn);  // in flight while the tables are built
+  }
   float g = *p.g_src;
   if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
   const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
@@ -531,7 +543,10 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
     u64 x2[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) x2[k] = xn[k];
-    if (b + stride < p.nblocks) load_block_pairs<DT, MODE>(p, b + stride, v8, xn);
+    if (b + stride < p.nblocks) {
+      if constexpr (MODE == SRC_KV) kc.advance();
+      load_next(b + stride, xn);
+    }
     const bool deferred = active && quantize_block_fast<MODE, ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
     if constexpr (NC > 1) {  // a single-offset window never needs the definition pass
       const unsigned m = __ballot_sync(0xFFFFFFFFu, deferred);
