@@ -81,6 +81,12 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+def library_path() -> str:
+    """Path of the loaded libnvfp4.so (for C programs that link it)."""
+    lib()
+    return _SO
+
+
 def status_str(status: int) -> str:
     return lib().nvfp4_status_str(status).decode()
 
