@@ -30,7 +30,9 @@
  * Errors: argument errors are reported synchronously as a negative status and nothing is enqueued.
  * A CUDA launch error is returned as NVFP4_ERR_CUDA.  With the environment variable NVFP4_CHECKED=1
  * the quantize / kv calls synchronise the stream and return NVFP4_ERR_NONFINITE when the tensor held a
- * NaN or Inf (the outputs are then poisoned in-band as described above).
+ * NaN or Inf (the outputs are then poisoned in-band as described above).  For tests of the CUDA error
+ * path, NVFP4_FAULT_INJECT=launch makes nvfp4_dequantize(_ex) request an invalid block size, which the
+ * CUDA runtime rejects on the host: the call returns NVFP4_ERR_CUDA and nothing reaches the GPU.
  * Alignment: element buffers must be 16-byte aligned (32-byte aligned inputs use 256-bit loads);
  * code buffers 8-byte aligned.  Sizes are element counts and must be multiples of 16 (one block).
  */

@@ -53,6 +53,19 @@ bool checked_mode() {
   return mode == 1;
 }
 
+// Host-side fault injection for tests of the CUDA error path: with NVFP4_FAULT_INJECT=launch in the
+// environment, nvfp4_dequantize(_ex) asks for blocks of 2048 threads, a configuration the CUDA runtime
+// rejects on the host (cudaErrorInvalidConfiguration, nothing reaches the GPU), so the call returns
+// NVFP4_ERR_CUDA and the context stays usable.
+bool inject_launch_fault() {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* e = getenv("NVFP4_FAULT_INJECT");
+    mode = (e && strcmp(e, "launch") == 0) ? 1 : 0;
+  }
+  return mode == 1;
+}
+
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline bool dtype_ok(int dt) { return dt == DT_F32 || dt == DT_BF16 || dt == DT_F16; }
@@ -338,10 +351,11 @@ int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float
   const int v8 = aligned(out, 32) ? 1 : 0;
   char* o = static_cast<char*>(out);
   cudaStream_t s = S(stream);
+  const int threads = inject_launch_fault() ? 2048 : 256;
   switch (out_dtype) {
-    case DT_F32: dequantize_kernel<DT_F32><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
-    case DT_BF16: dequantize_kernel<DT_BF16><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
-    default: dequantize_kernel<DT_F16><<<grid, 256, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+    case DT_F32: dequantize_kernel<DT_F32><<<grid, threads, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+    case DT_BF16: dequantize_kernel<DT_BF16><<<grid, threads, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
+    default: dequantize_kernel<DT_F16><<<grid, threads, 0, s>>>(codes, scales, gscale, nb, o, v8); break;
   }
   return last_error();
 }
