@@ -194,6 +194,27 @@ def time_oracle(name, f_lo, f_hi, budget_s, max_elems=1 << 25):
     return xs, code, n
 
 
+def quant_stats(nv, x, g, deq, f_lo, f_hi, elements_per_s):
+    """Secondary statistics of the timed input, computed once after the timed region: the histogram of
+    the chosen offsets f*, the total block SSE against max-scaling (window {0}) under the same g, and
+    the normalised absolute error of the dequantized tensor (sums in float64, in chunks)."""
+    import torch
+    _, _, _, f, sse = nv.quantize_ex(x, f_lo, f_hi, gscale_in=g)
+    _, _, _, _, sse0 = nv.quantize_ex(x, 0, 0, gscale_in=g, want_f=False)
+    counts = torch.bincount(f.to(torch.int64) + 128, minlength=256).cpu().tolist()
+    s, s0 = sse.double().sum().item(), sse0.double().sum().item()
+    num = den = 0.0
+    xf, df = x.reshape(-1), deq.reshape(-1)
+    for i in range(0, xf.numel(), 1 << 26):
+        a, b = xf[i:i + (1 << 26)].double(), df[i:i + (1 << 26)].double()
+        num += (a - b).abs().sum().item()
+        den += a.abs().sum().item()
+    return {"elements_per_s": elements_per_s, "blocks": f.numel(),
+            "f_star_hist": {str(i - 128): c for i, c in enumerate(counts) if c},
+            "sse_total": s, "sse_max_scaling": s0, "mse_reduction_pct": 100.0 * (1.0 - s / s0) if s0 > 0 else None,
+            "nae_dequant": num / den if den > 0 else None}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -1091,6 +1112,10 @@ def main():
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / args.steps},
         "overlap": overlap,
     }
+    if not kv:
+        line["stats"] = quant_stats(nv, x, g, deq, args.f_lo, args.f_hi, value / esz * 1e9)
+        if world > 1:
+            line["stats"]["scope"] = "rank 0's shard"
     if kv:
         args.no_e2e = True
     # end to end through the public API with host buffers: pinned H2D of the input, the step, and a
