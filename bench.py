@@ -990,6 +990,16 @@ def main():
         elapsed_ms = t0.elapsed_time(t1)
     else:  # the flushes are not part of the step
         elapsed_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+
+    def rmax(ms):
+        """A time as the maximum over ranks, so that every rank compares the same numbers."""
+        if world == 1:
+            return ms
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    elapsed_ms = rmax(elapsed_ms)
     eager_ms = elapsed_ms
     graph_used = False
     if world == 1 and not args.no_graph:
@@ -1061,20 +1071,89 @@ def main():
             step_overlap()
         ob.record(stream)
         torch.cuda.synchronize()
-        overlap_ms = oa.elapsed_time(ob)
+        overlap_ms = rmax(oa.elapsed_time(ob))
         overlap = {"chunks": OVERLAP_CHUNKS, "dequant_ctas_per_sm": OVERLAP_DEQ_CTAS_PER_SM,
                    "ms_per_step": overlap_ms / args.steps, "used_for_value": overlap_ms < elapsed_ms}
         if overlap_ms < elapsed_ms:
             elapsed_ms = overlap_ms
             graph_used = False
-    clocks = sampler.stop()   # sampled over the eager, graph and overlapped timings
+    # The same step with the quantize and the dequantize fused (nvfp4_quantize_dequantize: the search
+    # kernel writes each block's dequantized values as soon as its scale is chosen, so the codes are not
+    # read back): same outputs (tested), one pass fewer over HBM.
+    fused = None
+    if not kv:
+        def step_fused(ev=None):
+            nv.tensor_amax(x, out=amax)
+            if world > 1:
+                dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+            nv.global_scale(amax, out=g)
+            if ev:
+                ev[0].record(stream)
+            nv.quantize_dequantize(x, args.f_lo, args.f_hi, gscale_in=g, codes=codes, scales=scales, gscale=None,
+                                   out=deq)
+            if ev:
+                ev[1].record(stream)
+
+        for _ in range(args.warmup):
+            step_fused()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa.record(stream)
+        for k in range(args.steps):
+            if flush is not None:
+                flush.fill_(float(k + 0.5))
+            fev[k][2].record(stream)
+            step_fused(fev[k])
+            fev[k][3].record(stream)
+        fb.record(stream)
+        torch.cuda.synchronize()
+        fused_ms = fa.elapsed_time(fb) if flush is None else sum(e[2].elapsed_time(e[3]) for e in fev)
+        fused_ms = rmax(fused_ms)
+        fused_graph_ms = None
+        if world == 1 and not args.no_graph:
+            # the fused step replayed as a CUDA graph (the small configurations are launch-bound)
+            cgf = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step_fused()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(cgf, stream=side):
+                step_fused()
+            for _ in range(max(1, args.warmup)):
+                cgf.replay()
+            torch.cuda.synchronize()
+            gfe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+            fa.record(stream)
+            for k in range(args.steps):
+                if flush is not None:
+                    flush.fill_(float(k + 0.25))
+                gfe[k][0].record(stream)
+                cgf.replay()
+                gfe[k][1].record(stream)
+            fb.record(stream)
+            torch.cuda.synchronize()
+            fused_graph_ms = fa.elapsed_time(fb) if flush is None else sum(a.elapsed_time(b) for a, b in gfe)
+            del cgf
+        fused = {"ms_per_step": fused_ms / args.steps,
+                 "graph_ms_per_step": fused_graph_ms / args.steps if fused_graph_ms is not None else None,
+                 "kernel_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in fev)}
+        fused["graph_used"] = fused_graph_ms is not None and fused_graph_ms < fused_ms
+        if fused["graph_used"]:
+            fused_ms = fused_graph_ms
+        fused["used_for_value"] = fused_ms < elapsed_ms
+        if fused_ms < elapsed_ms:
+            elapsed_ms = fused_ms
+            graph_used = False
+            if overlap:
+                overlap["used_for_value"] = False
+    clocks = sampler.stop()   # sampled over the eager, graph, overlapped and fused timings
     amax_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     q_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     dq_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = t.item()
 
     bytes_in = n * esz
     value = world * bytes_in * args.steps / (elapsed_ms * 1e-3) / 1e9
@@ -1087,30 +1166,47 @@ def main():
         q_ms = amax_ms + q_ms
         amax_ms = 0.0
     q_gbs = (two_pass_bytes if kv else q_bytes) / (q_ms * 1e-3) / 1e9
+    f32_default = not kv and x.dtype == torch.float32 and (args.f_lo, args.f_hi) == (-2, 6)
+    search_roofline = {"bound": "hbm",
+                       "kernel": "kv_mixed (amax + search passes)" if kv else "quantize (ScaleSearch search + encode pass)",
+                       "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
+                       "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0>", n) if f32_default else None,
+                       "peak_source": peak_src, "bytes_per_launch": two_pass_bytes if kv else q_bytes}
+    roofline = search_roofline
+    if kv:
+        launches = 5
+    elif fused and fused["used_for_value"]:
+        # the step's dominant kernel is then the fused one: read x, write codes, scales and the values
+        launches = 3
+        f_bytes = n_q * esz + n_q // 2 + n_q // 16 + deq.element_size() * n_q
+        f_gbs = f_bytes / (fused["kernel_ms"] * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "quantize_dequantize (ScaleSearch search + encode + dequantized values)",
+                    "achieved": f_gbs, "peak": peak, "unit": "GB/s", "frac": f_gbs / peak,
+                    "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0,0>", n) if f32_default else None,
+                    "peak_source": peak_src, "bytes_per_launch": f_bytes}
+    elif overlap and overlap["used_for_value"]:
+        launches = 2 + 2 * OVERLAP_CHUNKS
+    else:
+        launches = 4
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
         "config": workload_config(args),
-        "roofline": {"bound": "hbm",
-                     "kernel": "kv_mixed (amax + search passes)" if kv else
-                     "quantize (ScaleSearch search + encode pass)",
-                     "achieved": q_gbs, "peak": peak, "unit": "GB/s", "frac": q_gbs / peak,
-                     "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0>", n)
-                     if (not kv and x.dtype == torch.float32 and (args.f_lo, args.f_hi) == (-2, 6)) else None,
-                     "peak_source": peak_src,
-                     "bytes_per_launch": two_pass_bytes if kv else q_bytes},
-        "breakdown_ms": {"amax_and_g": amax_ms, "quantize": q_ms, "dequantize": dq_ms},
+        "roofline": roofline,
+        "roofline_search_pass": search_roofline,
+        "breakdown_ms": {"amax_and_g": amax_ms, "quantize": q_ms, "dequantize": dq_ms,
+                         "fused_quantize_dequantize": fused["kernel_ms"] if fused else None},
         "quantize_two_pass": {"gbs_input": n_q * esz / ((amax_ms + q_ms) * 1e-3) / 1e9,
                               "gbs_moved": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 1e9,
                               "frac_of_8TBs": two_pass_bytes / ((amax_ms + q_ms) * 1e-3) / 8e12},
         "dequantize": {"gbs_moved": dq_bytes / (dq_ms * 1e-3) / 1e9},
-        "gpu_launches": (5 if kv else (2 + 2 * OVERLAP_CHUNKS if overlap and overlap["used_for_value"] else 4))
-                        * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks,
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / args.steps},
         "overlap": overlap,
+        "fused": fused,
     }
     if not kv:
         line["stats"] = quant_stats(nv, x, g, deq, args.f_lo, args.f_hi, value / esz * 1e9)

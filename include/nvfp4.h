@@ -93,6 +93,17 @@ int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, 
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n,
                      int out_dtype, void* out, void* stream);
 
+/* Quantize and dequantize in one pass (a fused round trip, e.g. simulated quantization): the outputs of
+ * nvfp4_quantize_ex (codes, scales, gscale; gscale_in as there) plus out = the dequantized tensor, n
+ * elements of `dtype` (the input's), bit-identical to nvfp4_dequantize(codes, scales, g, n, dtype, out)
+ * ("Search your block floating-point scales!", Method > ScaleSearch; NVFP4 page, the two-level scale).
+ * For windows of 1, 9 or 17 offsets the search kernel writes each block's values as soon as its scale
+ * is chosen, so the codes are not read back; other widths run the two passes.  out: 16-byte aligned;
+ * it may be x itself (each block is read before its own values are written) but must not overlap x
+ * otherwise.  Errors as nvfp4_quantize_ex, NVFP4_ERR_ARG for out == NULL with n > 0. */
+int nvfp4_quantize_dequantize(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const float* gscale_in,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* out, void* stream);
+
 /* nvfp4_dequantize with a bound on the launch footprint: at most ctas_per_sm CTAs of 256 threads per
  * SM (1..8; 0 = the default 8), so that the kernel can run beside another kernel that occupies most of
  * each SM -- e.g. dequantizing a finished chunk on a second stream while the search of the next chunk

@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
-    "dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
+    "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
     "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4",
 ]
@@ -38,6 +38,7 @@ _SIGS = {
     "nvfp4_quantize_ex": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_dequantize": (_I, [_P, _P, _P, _I64, _I, _P, _P]),
     "nvfp4_dequantize_ex": (_I, [_P, _P, _P, _I64, _I, _P, _I, _P]),
+    "nvfp4_quantize_dequantize": (_I, [_P, _I64, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_hadamard16_ex": (_I, [_P, _I64, _I, _P, _I, ctypes.c_uint32, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
@@ -176,6 +177,28 @@ def quantize_ex(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch
     _check(lib().nvfp4_quantize_ex(_ptr(x), n, _dt(x), block, f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
                                    _ptr(scales), _ptr(gscale), _ptr(block_f), _ptr(block_sse), _stream(x)))
     return codes, scales, gscale, block_f, block_sse
+
+
+def quantize_dequantize(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None,
+                        codes=None, scales=None, gscale=None, out: torch.Tensor | None = None):
+    """Fused round trip: quantize x with ScaleSearch and write its dequantized values (x's dtype) in the same
+    pass.  Returns (out, codes, scales, gscale); out equals dequantize(codes, scales, g, x.dtype) bit for bit.
+    out may be x itself (in-place simulated quantization)."""
+    _cuda(x, "x")
+    n = x.numel()
+    if gscale_in is not None:
+        _cuda(gscale_in, "gscale_in")
+    keep = gscale
+    codes, scales, gscale = _alloc_q(x, codes, scales, gscale)
+    if gscale_in is not None and keep is None:
+        gscale = None
+    out = torch.empty_like(x) if out is None else out
+    _cuda(out, "out")
+    if out.dtype != x.dtype or out.numel() != n:
+        raise ValueError("out must have x's dtype and size")
+    _check(lib().nvfp4_quantize_dequantize(_ptr(x), n, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes), _ptr(scales),
+                                           _ptr(gscale), _ptr(out), _stream(x)))
+    return out, codes, scales, gscale
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, out_dtype=torch.float32,

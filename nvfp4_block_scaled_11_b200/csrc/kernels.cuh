@@ -133,6 +133,10 @@ struct QuantParams {
   // rows of one column; tr_rb = rows / 16.  Blocks run column-fastest, so a warp reads rows of
   // consecutive columns; outputs are the transposed [batch, tr_cols, rows] layout.
   int64_t tr_cols, tr_rb;
+  // fused round trip (linear mode): when deq_out is set, each block's dequantized values (the input's
+  // dtype) are written there too, at the block's own position
+  char* deq_out;
+  int deq_v8;          // deq_out is 32-byte aligned
 };
 
 // Where the 16 elements of a block come from.
@@ -356,58 +360,63 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
 // =================================================================================================
 // Dequantize: one thread per block; the block step d = fl(E4M3(scale) * g) is applied by one multiply.
 // =================================================================================================
+// The 16 values of one block from its packed codes (cw_lo: elements 0..7, cw_hi: 8..15) and its step
+// d = fl(E4M3(scale) * g): out_i = fl(E2M1(q_i) * d), narrowed to OT by RNE, stored at o (64 bytes for
+// FP32, 32 otherwise; v8: o is 32-byte aligned).  Shared by the dequantize kernel and the fused round
+// trip, so the two agree bit for bit.
+template <int OT>
+__device__ __forceinline__ void store_dequantized(char* o, uint32_t cw_lo, uint32_t cw_hi, float d, bool v8) {
+  float v[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t byte = ((k < 4 ? cw_lo : cw_hi) >> (8 * (k & 3))) & 0xFFu;
+    const uint32_t h2 = e2m1x2_to_f16x2(byte);
+    v[2 * k] = __fmul_rn(f16lo(h2), d);
+    v[2 * k + 1] = __fmul_rn(f16hi(h2), d);
+  }
+  if (OT == DT_F32) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(v[i]);
+    if (v8) {
+      st_v8(o, static_cast<const uint32_t*>(w));
+      st_v8(o + 32, w + 8);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
+    }
+  } else {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (OT == DT_BF16) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&h);
+      } else {
+        __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&h);
+      }
+    }
+    if (v8) {
+      st_v8(o, w);
+    } else {
+      st_v4(o, w);
+      st_v4(o + 16, w + 4);
+    }
+  }
+}
+
 template <int OT>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes,
                                                          const uint8_t* __restrict__ scales,
                                                          const float* __restrict__ gsrc, int64_t nblocks,
                                                          char* __restrict__ out, int v8) {
+  constexpr int OS = OT == DT_F32 ? 4 : 2;
   const float g = *gsrc;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
     const uint2 cw = reinterpret_cast<const uint2*>(codes)[b];
-    const float d = __fmul_rn(e4m3_value(scales[b]), g);
-    float v[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xFFu;
-      const uint32_t h2 = e2m1x2_to_f16x2(byte);
-      v[2 * k] = __fmul_rn(f16lo(h2), d);
-      v[2 * k + 1] = __fmul_rn(f16hi(h2), d);
-    }
-    if (OT == DT_F32) {
-      char* o = out + 64 * b;
-      uint32_t w[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(v[i]);
-      if (v8) {
-        uint32_t a[8], c[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { a[i] = w[i]; c[i] = w[8 + i]; }
-        st_v8(o, a);
-        st_v8(o + 32, c);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) st_v4(o + 16 * k, w + 4 * k);
-      }
-    } else {
-      char* o = out + 32 * b;
-      uint32_t w[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (OT == DT_BF16) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-          w[k] = *reinterpret_cast<uint32_t*>(&h);
-        } else {
-          __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
-          w[k] = *reinterpret_cast<uint32_t*>(&h);
-        }
-      }
-      if (v8) st_v8(o, w);
-      else {
-        st_v4(o, w);
-        st_v4(o + 16, w + 4);
-      }
-    }
+    store_dequantized<OT>(out + 16 * OS * b, cw.x, cw.y, __fmul_rn(e4m3_value(scales[b]), g), v8 != 0);
   }
 }
 

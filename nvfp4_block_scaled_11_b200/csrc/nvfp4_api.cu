@@ -97,6 +97,12 @@ int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_
 template <int DT, int MODE, bool ROT, int NC>
 void launch_search(const QuantParams& p, cudaStream_t s) {
   const int grid = grid_for(p.nblocks, 256, NVFP4_SEARCH_CTAS_PER_SM);
+  if constexpr (MODE == SRC_LINEAR && !ROT) {
+    if (p.deq_out) {  // fused round trip: the dequantized values in the input's dtype
+      quantize_search_kernel<DT, MODE, ROT, NC, false, DT><<<grid, 256, 0, s>>>(p);
+      return;
+    }
+  }
   if (p.block_sse) quantize_search_kernel<DT, MODE, ROT, NC, true><<<grid, 256, 0, s>>>(p);
   else quantize_search_kernel<DT, MODE, ROT, NC, false><<<grid, 256, 0, s>>>(p);
 }
@@ -155,6 +161,8 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
   p.sf_mat_bytes = sf.sf_mat_bytes;
   p.tr_cols = sf.tr_cols;
   p.tr_rb = sf.tr_rb;
+  p.deq_out = sf.deq_out;
+  p.deq_v8 = sf.deq_v8;
   if (gscale_in == nullptr) {
     // gscale doubles as the amax accumulator: zero, reduce, quantize (reads it as amax), then g.
     if (cudaMemsetAsync(gscale, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -337,6 +345,26 @@ int nvfp4_quantize(const void* x, int64_t n, int dtype, int block, int f_lo, int
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,
                      void* out, void* stream) {
   return nvfp4_dequantize_ex(codes, scales, gscale, n, out_dtype, out, 0, stream);
+}
+
+int nvfp4_quantize_dequantize(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const float* gscale_in,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* out, void* stream) {
+  if (!dtype_ok(dtype) || !window_ok(f_lo, f_hi)) return NVFP4_ERR_ARG;
+  if (n > 0 && out == nullptr) return NVFP4_ERR_ARG;
+  if (n > 0 && !aligned(out, 16)) return NVFP4_ERR_ALIGN;
+  const int nc = f_hi - f_lo + 1;
+  cudaStream_t s = S(stream);
+  if (nc == 1 || nc == 9 || nc == 17) {
+    QuantParams sf{};
+    sf.deq_out = static_cast<char*>(out);
+    sf.deq_v8 = aligned(out, 32) ? 1 : 0;
+    return quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes, scales, gscale, nullptr, nullptr, sf, s);
+  }
+  // other window widths: the two passes, the dequantize reading the codes just written
+  QuantParams sf{};
+  if (int rc = quantize_impl(x, n, dtype, f_lo, f_hi, gscale_in, codes, scales, gscale, nullptr, nullptr, sf, s))
+    return rc;
+  return nvfp4_dequantize_ex(codes, scales, gscale_in ? gscale_in : gscale, n, dtype, out, 0, stream);
 }
 
 int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,

@@ -370,7 +370,8 @@ __device__ __forceinline__ void maybe_rotate(u64 (&x2)[8]) {
   }
 }
 
-template <int MODE, bool WANT_SSE>
+// DEQ >= 0 (a dtype): also write the block's dequantized values to p.deq_out (fused round trip).
+template <int MODE, bool WANT_SSE, int DEQ = -1>
 __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, const u64 (&x2)[8], const CandEntry* tab,
                                             int c0, int fstar, float sse, bool poisoned, float amax_b) {
   uint32_t wlo = 0u, whi = 0u;
@@ -404,10 +405,15 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
   p.scales[scale_index(p, ob)] = (uint8_t)scale;
   if (p.block_f) p.block_f[ob] = (int8_t)fstar;
   if (WANT_SSE) p.block_sse[ob] = sse;
+  if constexpr (DEQ >= 0) {
+    // the table's d of every scale byte 0..127 is fl(E4M3(c) * g), the dequantize kernel's step
+    constexpr int OS = DEQ == DT_F32 ? 4 : 2;
+    store_dequantized<DEQ>(p.deq_out + 16 * OS * ob, wlo, whi, tab[scale].d, p.deq_v8 != 0);
+  }
 }
 
 // Fast path for one block.  Returns true when the block needs the definition (outputs not written).
-template <int MODE, bool ROT, int NC, bool WANT_SSE>
+template <int MODE, bool ROT, int NC, bool WANT_SSE, int DEQ = -1>
 __device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const CandEntry* tab, const float* thr,
                                                     float inv6g, bool g_bad, int64_t b, u64 (&x2)[8]) {
   maybe_rotate<ROT>(x2);
@@ -427,13 +433,13 @@ __device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const 
       return true;
     }
   }
-  write_block<MODE, WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
   return false;
 }
 
 // The definition for one block already in registers (rotated if the path rotates): same outputs as the
 // fast path, every candidate scored in order.
-template <int MODE, bool WANT_SSE>
+template <int MODE, bool WANT_SSE, int DEQ = -1>
 __device__ __forceinline__ void quantize_block_def_x2(const QuantParams& p, const CandEntry* tab, const float* thr,
                                                       float inv6g, bool g_bad, int64_t b, const u64 (&x2)[8]) {
   const float amax_b = block_amax_nan(x2);
@@ -447,7 +453,7 @@ __device__ __forceinline__ void quantize_block_def_x2(const QuantParams& p, cons
     for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
     search_def(x, c0, p.f_lo, p.f_hi, tab, fstar, sse);
   }
-  write_block<MODE, WANT_SSE>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
 }
 
 // First element of block b (linear and KV modes: the 16 elements are contiguous).
@@ -475,13 +481,13 @@ __device__ __forceinline__ void load_block_pairs(const QuantParams& p, int64_t b
 }
 
 // The definition for one block (deferred blocks): reload, rotate, score every candidate in order.
-template <int DT, int MODE, bool ROT, bool WANT_SSE>
+template <int DT, int MODE, bool ROT, bool WANT_SSE, int DEQ = -1>
 __device__ __forceinline__ void quantize_block_def(const QuantParams& p, const CandEntry* tab, const float* thr,
                                                    float inv6g, bool g_bad, int64_t b, bool v8) {
   u64 x2[8];
   load_block_pairs<DT, MODE>(p, b, v8, x2);
   maybe_rotate<ROT>(x2);
-  quantize_block_def_x2<MODE, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
+  quantize_block_def_x2<MODE, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, b, x2);
 }
 
 // One thread per 16-element block, grid-stride in warp-uniform rounds, the next block's loads in flight
@@ -492,7 +498,7 @@ constexpr int kDeferCap = 64;
 #define NVFP4_SEARCH_CTAS_PER_SM 2
 #endif
 
-template <int DT, int MODE, bool ROT, int NC, bool WANT_SSE>
+template <int DT, int MODE, bool ROT, int NC, bool WANT_SSE, int DEQ = -1>
 __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search_kernel(QuantParams p) {
   __shared__ CandEntry tab_store[kTabSize];
   __shared__ float thr[128];
@@ -531,7 +537,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
     __syncwarp();
     for (int e = lane; e < dcount; e += 32) {
       const int64_t bd = dlist[e];
-      quantize_block_def<DT, MODE, ROT, WANT_SSE>(p, tab, thr, inv6g, g_bad, bd, p.v8 != 0);
+      quantize_block_def<DT, MODE, ROT, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, bd, p.v8 != 0);
     }
     __syncwarp();
     dcount = 0;
@@ -547,7 +553,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
       if constexpr (MODE == SRC_KV) kc.advance();
       load_next(b + stride, xn);
     }
-    const bool deferred = active && quantize_block_fast<MODE, ROT, NC, WANT_SSE>(p, tab, thr, inv6g, g_bad, b, x2);
+    const bool deferred = active && quantize_block_fast<MODE, ROT, NC, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, b, x2);
     if constexpr (NC > 1) {  // a single-offset window never needs the definition pass
       const unsigned m = __ballot_sync(0xFFFFFFFFu, deferred);
       if (m) {

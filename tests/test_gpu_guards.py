@@ -49,6 +49,13 @@ def test_quantize_dequantize_hadamard_guards():
     nv.dequantize(codes, scales, gs, torch.bfloat16, out=gd.out(n, torch.bfloat16), ctas_per_sm=1)
     nv.hadamard16(x, out=gd.out(n, torch.bfloat16))
     nv.hadamard16(x, out=gd.out(n, torch.float32), signs=0x3C3C, inverse=True)
+    # the fused round trip, with its own outputs guarded (and the same in place on a guarded copy)
+    nv.quantize_dequantize(x, codes=gd.out(n // 2, torch.uint8), scales=gd.out(n // 16, torch.uint8),
+                           gscale=gd.out(1, torch.float32), out=gd.out(n, torch.float32))
+    xi = gd.out(n, torch.float32)
+    xi.copy_(x)
+    nv.quantize_dequantize(xi, -8, 8, codes=gd.out(n // 2, torch.uint8), scales=gd.out(n // 16, torch.uint8),
+                           gscale=gd.out(1, torch.float32), out=xi)
     mc, ms = gd.out(n // 2, torch.uint8), gd.out(n // 32, torch.uint8)
     nv.mxfp4_quantize(x[: n // 32 * 32], codes=mc, scales=ms)
     nv.mxfp4_dequantize(mc, ms, torch.float16, out=gd.out(n // 32 * 32, torch.float16))

@@ -313,6 +313,14 @@ def test_full_size_sampled(name):
     out = nv.dequantize(codes, scales, g, torch.float32)
     rd = O.dequantize(codes.view(-1, 8)[ti].cpu().numpy().reshape(-1), rs, rg)
     assert same_f32(out.view(-1, 16)[ti].cpu().numpy(), rd)
+    del out
+    # the fused round trip in the same configuration: codes, scales and g byte-equal to the two passes;
+    # sampled blocks of its output equal the oracle's dequantize in the input's dtype
+    fo, fc, fs, fg = nv.quantize_dequantize(x, w.f_lo, w.f_hi)
+    assert torch.equal(fc, codes) and torch.equal(fs, scales) and torch.equal(fg, g)
+    rdx = O.dequantize(codes.view(-1, 8)[ti].cpu().numpy().reshape(-1), rs, rg, out_dtype=DT_CODE[x.dtype])
+    got = host_np(fo.view(-1, 16)[ti])
+    assert same_f32(got, rdx) if x.dtype == torch.float32 else np.array_equal(got.reshape(-1), rdx.reshape(-1))
 
 
 def test_many_blocks_with_natural_near_ties():
