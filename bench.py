@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--scale", type=float, default=1.0, help="fraction of the workload size (profiling runs)")
     ap.add_argument("--f-lo", type=int, default=-2)
     ap.add_argument("--f-hi", type=int, default=6)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1214,43 +1214,72 @@ def main():
             line["stats"]["scope"] = "rank 0's shard"
     if kv:
         args.no_e2e = True
-    # end to end through the public API with host buffers: pinned H2D of the input, the step, and a
-    # D2H read of the quantized result (codes, scales, g) every step.
+    # end to end through the public API with host buffers: every step copies its whole input in from
+    # pinned host memory, runs the step, and reads its quantized result (codes, scales, g) back.  The
+    # buffers are doubled and the copies run on their own streams, so step k's read-back overlaps step
+    # k+1's input copy (PCIe carries both directions at once); a buffer is reused only after the step
+    # that last used it has been computed and read back.
     if not args.no_e2e and args.e2e_steps > 0:
+        NB = 2
         hx = torch.empty(n, dtype=x.dtype, pin_memory=True)
         hx.copy_(x)
-        hc = torch.empty(n // 2, dtype=torch.uint8, pin_memory=True)
-        hs = torch.empty(n // 16, dtype=torch.uint8, pin_memory=True)
-        hg = torch.empty(1, dtype=torch.float32, pin_memory=True)
-        xin = torch.empty_like(x)
+        xin = [torch.empty_like(x) for _ in range(NB)]
+        cb = [codes] + [torch.empty_like(codes) for _ in range(NB - 1)]
+        sb = [scales] + [torch.empty_like(scales) for _ in range(NB - 1)]
+        gb = [g] + [torch.empty_like(g) for _ in range(NB - 1)]
+        hc = [torch.empty(n // 2, dtype=torch.uint8, pin_memory=True) for _ in range(NB)]
+        hs = [torch.empty(n // 16, dtype=torch.uint8, pin_memory=True) for _ in range(NB)]
+        hg = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(NB)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         fused_step = bool(fused and fused["used_for_value"])
+        computed, read_back = [None] * NB, [None] * NB
 
-        def e2e_step():
-            xin.copy_(hx, non_blocking=True)
-            nv.tensor_amax(xin, out=amax)
+        def e2e_step(k):
+            i = k % NB
+            if computed[i] is not None:
+                s_in.wait_event(computed[i])          # xin[i] was read by step k - NB
+            with torch.cuda.stream(s_in):
+                xin[i].copy_(hx, non_blocking=True)
+            arrived = torch.cuda.Event()
+            arrived.record(s_in)
+            stream.wait_event(arrived)
+            if read_back[i] is not None:
+                stream.wait_event(read_back[i])       # cb[i], sb[i], gb[i] were read back by step k - NB
+            nv.tensor_amax(xin[i], out=amax)
             if world > 1:
                 dist.all_reduce(amax, op=dist.ReduceOp.MAX)
-            nv.global_scale(amax, out=g)
+            nv.global_scale(amax, out=gb[i])
             if fused_step:   # the schedule that set `value`
-                nv.quantize_dequantize(xin, args.f_lo, args.f_hi, gscale_in=g, codes=codes, scales=scales,
+                nv.quantize_dequantize(xin[i], args.f_lo, args.f_hi, gscale_in=gb[i], codes=cb[i], scales=sb[i],
                                        gscale=None, out=deq)
             else:
-                nv.quantize_ex(xin, args.f_lo, args.f_hi, gscale_in=g, want_f=False, want_sse=False, codes=codes,
-                               scales=scales, gscale=None)
-                nv.dequantize(codes, scales, g, torch.float32, out=deq)
-            hc.copy_(codes, non_blocking=True)
-            hs.copy_(scales, non_blocking=True)
-            hg.copy_(g, non_blocking=True)
+                nv.quantize_ex(xin[i], args.f_lo, args.f_hi, gscale_in=gb[i], want_f=False, want_sse=False,
+                               codes=cb[i], scales=sb[i], gscale=None)
+                nv.dequantize(cb[i], sb[i], gb[i], torch.float32, out=deq)
+            done = torch.cuda.Event()
+            done.record(stream)
+            computed[i] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                hc[i].copy_(cb[i], non_blocking=True)
+                hs[i].copy_(sb[i], non_blocking=True)
+                hg[i].copy_(gb[i], non_blocking=True)
+            back = torch.cuda.Event()
+            back.record(s_out)
+            read_back[i] = back
 
-        e2e_step()
+        e2e_step(0)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        s_in.wait_event(a)
+        for k in range(1, args.e2e_steps + 1):
+            e2e_step(k)
+        for ev in read_back:
+            stream.wait_event(ev)
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b)
@@ -1260,8 +1289,9 @@ def main():
             e2e_ms = t.item()
         line["e2e"] = {"value": world * bytes_in * args.e2e_steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                        "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": n // 2 + n // 16 + 4,
-                       "schedule": "fused round trip" if fused_step else "quantize + dequantize"}
-        del hx, hc, hs, hg, xin
+                       "schedule": ("fused round trip" if fused_step else "quantize + dequantize")
+                       + ", input copy of step k+1 overlapping the read-back of step k"}
+        del hx, hc, hs, hg, xin, cb, sb, gb
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         xs, code, ns = time_oracle(args.workload, args.f_lo, args.f_hi, args.cpu_seconds)
