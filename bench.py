@@ -1081,8 +1081,15 @@ def main():
     # kernel writes each block's dequantized values as soon as its scale is chosen, so the codes are not
     # read back): same outputs (tested), one pass fewer over HBM.
     fused = None
-    if not kv:
+    if True:
         def step_fused(ev=None):
+            if kv:   # one call: copies + rotated amax + rotated search writing codes, scales and values
+                if ev:
+                    ev[0].record(stream)
+                nv.kv_mixed_dequantize(x, 16, 16, True, args.f_lo, args.f_hi, mid_out=deq)
+                if ev:
+                    ev[1].record(stream)
+                return
             nv.tensor_amax(x, out=amax)
             if world > 1:
                 dist.all_reduce(amax, op=dist.ReduceOp.MAX)
@@ -1173,7 +1180,14 @@ def main():
                        "traffic": captured_traffic("quantize_search_kernel<0,0,0,9,0>", n) if f32_default else None,
                        "peak_source": peak_src, "bytes_per_launch": two_pass_bytes if kv else q_bytes}
     roofline = search_roofline
-    if kv:
+    if kv and fused and fused["used_for_value"]:
+        launches = 4
+        f_bytes = two_pass_bytes + deq.element_size() * n_q
+        f_gbs = f_bytes / (fused["kernel_ms"] * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "kv_mixed_dequantize (copies + rotated amax + rotated search writing "
+                    "codes, scales and values)", "achieved": f_gbs, "peak": peak, "unit": "GB/s", "frac": f_gbs / peak,
+                    "traffic": None, "peak_source": peak_src, "bytes_per_launch": f_bytes}
+    elif kv:
         launches = 5
     elif fused and fused["used_for_value"]:
         # the step's dominant kernel is then the fused one: read x, write codes, scales and the values

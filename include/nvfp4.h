@@ -138,6 +138,16 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
 
+/* nvfp4_kv_mixed plus the middle tokens' dequantized values in the same pass (a fused round trip):
+ * mid_out receives BF16 [B,H,T-sink-recent,D], element-aligned with the codes, equal bit for bit to
+ * nvfp4_dequantize(codes, scales, gscale, n_mid, NVFP4_BF16) -- the rotated values when `rotate`.
+ * For windows of 1, 9 or 17 offsets the search kernel writes them as each block's scale is chosen;
+ * other widths dequantize after the search.  mid_out: 16-byte aligned, required when the middle is
+ * not empty (NVFP4_ERR_ARG).  Everything else as nvfp4_kv_mixed. */
+int nvfp4_kv_mixed_dequantize(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                              int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* mid_out, void* stream);
+
 /* ---- Multi-scale deformable attention forward on NVFP4 values ("自動運転モデル BEVFormer の NVIDIA Blackwell
  * B200 FP8/FP4 CUDAカーネル・チューニング", sections 5-7: only the value tensor is low precision; locations,
  * weights, interpolation and accumulation stay FP32) ----

@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
-    "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
+    "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "kv_mixed_dequantize", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
     "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4",
 ]
@@ -42,6 +42,7 @@ _SIGS = {
     "nvfp4_hadamard16": (_I, [_P, _I64, _I, _P, _I, _P]),
     "nvfp4_hadamard16_ex": (_I, [_P, _I64, _I, _P, _I, ctypes.c_uint32, _I, _P]),
     "nvfp4_kv_mixed": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_kv_mixed_dequantize": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_msda_forward_nvfp4": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
     "nvfp4_msda_forward": (_I, [_P, _I, _I64, _I64, _I64, _I64, _P, _I, _I, _I64, _P, _P, _P, _P]),
     "nvfp4_mxfp4_quantize": (_I, [_P, _I64, _I, _P, _P, _P]),
@@ -256,6 +257,32 @@ def sf_mma_bytes(rows: int, cols: int, batch: int = 1) -> int:
     if nb < 0:
         raise NVFP4Error(int(nb))
     return int(nb)
+
+
+def kv_mixed_dequantize(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = True, f_lo: int = -2,
+                        f_hi: int = 6, mid_out: torch.Tensor | None = None):
+    """kv_mixed plus the middle's dequantized values (BF16 [B,H,Tm,D], rotated when `rotate`) in the same
+    pass.  Returns (sink, recent, codes, scales, gscale, mid)."""
+    _cuda(k, "k")
+    if k.dtype != torch.bfloat16 or k.dim() != 4:
+        raise TypeError("k must be a 4-D bfloat16 tensor [B,H,T,D]")
+    B, H, T, D = k.shape
+    Tm = T - sink - recent
+    if Tm < 0:
+        raise ValueError("T < sink + recent")
+    dev = k.device
+    so = torch.empty((B, H, sink, D), dtype=torch.bfloat16, device=dev)
+    ro = torch.empty((B, H, recent, D), dtype=torch.bfloat16, device=dev)
+    codes = torch.empty((B, H, Tm, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((B, H, Tm, D // 16), dtype=torch.uint8, device=dev)
+    gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    mid = torch.empty((B, H, Tm, D), dtype=torch.bfloat16, device=dev) if mid_out is None else mid_out
+    _cuda(mid, "mid_out")
+    if mid.dtype != torch.bfloat16 or mid.numel() != B * H * Tm * D:
+        raise ValueError("mid_out must be bfloat16 with B*H*Tm*D elements")
+    _check(lib().nvfp4_kv_mixed_dequantize(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), f_lo, f_hi, _ptr(so),
+                                           _ptr(ro), _ptr(codes), _ptr(scales), _ptr(gscale), _ptr(mid), _stream(k)))
+    return so, ro, codes, scales, gscale, mid
 
 
 def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch.Tensor | None = None,

@@ -97,7 +97,7 @@ int launch_amax(const void* x, int64_t n, int dtype, uint32_t* word, cudaStream_
 template <int DT, int MODE, bool ROT, int NC>
 void launch_search(const QuantParams& p, cudaStream_t s) {
   const int grid = grid_for(p.nblocks, 256, NVFP4_SEARCH_CTAS_PER_SM);
-  if constexpr (MODE == SRC_LINEAR && !ROT) {
+  if constexpr ((MODE == SRC_LINEAR && !ROT) || MODE == SRC_KV) {
     if (p.deq_out) {  // fused round trip: the dequantized values in the input's dtype
       quantize_search_kernel<DT, MODE, ROT, NC, false, DT><<<grid, 256, 0, s>>>(p);
       return;
@@ -425,9 +425,13 @@ int nvfp4_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_
   return last_error();
 }
 
+// mid_out (optional, linear scales only): the middle's dequantized values, BF16 [BH, Tm, D] in the
+// codes' block order (the rotated values when rotating), written by the search kernel for windows of
+// 1, 9 or 17 offsets and by the dequantize kernel otherwise.
 static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
                          int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
-                         uint8_t* codes, uint8_t* scales, float* gscale, bool mma, void* stream) {
+                         uint8_t* codes, uint8_t* scales, float* gscale, bool mma, void* stream,
+                         void* mid_out = nullptr) {
   if (!window_ok(f_lo, f_hi) || gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
     return NVFP4_ERR_SIZE;
@@ -440,8 +444,11 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   if (ngroups > 0 && (codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
   if (ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if ((BH > 0 && !aligned(k_bf16, 16)) || (sink_bf16 && !aligned(sink_bf16, 16)) ||
-      (recent_bf16 && !aligned(recent_bf16, 16)) || (codes && !aligned(codes, 8)) || !aligned(gscale, 4))
+      (recent_bf16 && !aligned(recent_bf16, 16)) || (codes && !aligned(codes, 8)) || !aligned(gscale, 4) ||
+      (mid_out && !aligned(mid_out, 16)))
     return NVFP4_ERR_ALIGN;
+  const int nc = f_hi - f_lo + 1;
+  const bool fused = mid_out != nullptr && (nc == 1 || nc == 9 || nc == 17);
   cudaStream_t s = S(stream);
   const char* k = static_cast<const char*>(k_bf16);
   if (BH > 0 && sink_tokens + recent_tokens > 0) {
@@ -484,11 +491,18 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
           cudaMemsetAsync(scales, 0, (size_t)(BH * p.sf_mat_bytes), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     }
+    if (fused) {
+      p.deq_out = static_cast<char*>(mid_out);
+      p.deq_v8 = aligned(mid_out, 32) ? 1 : 0;
+    }
     int rc = rotate ? launch_quantize_t<SRC_KV, true>(DT_BF16, p, s) : launch_quantize_t<SRC_KV, false>(DT_BF16, p, s);
     if (rc) return rc;
   }
   global_scale_kernel<<<1, 32, 0, s>>>(gscale, gscale);
   if (int rc = last_error()) return rc;
+  if (mid_out != nullptr && !fused && ngroups > 0) {
+    if (int rc = nvfp4_dequantize_ex(codes, scales, gscale, ngroups * 16, DT_BF16, mid_out, 0, stream)) return rc;
+  }
   return check_finite_sync(gscale, s);
 }
 
@@ -685,6 +699,14 @@ int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t 
                    uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
   return kv_mixed_impl(k_bf16, B, H, T, D, sink_tokens, recent_tokens, rotate, f_lo, f_hi, sink_bf16, recent_bf16,
                        codes, scales, gscale, false, stream);
+}
+
+int nvfp4_kv_mixed_dequantize(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,
+                              int recent_tokens, int rotate, int f_lo, int f_hi, void* sink_bf16, void* recent_bf16,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* mid_out, void* stream) {
+  if (B > 0 && H > 0 && T > (int64_t)sink_tokens + recent_tokens && mid_out == nullptr) return NVFP4_ERR_ARG;
+  return kv_mixed_impl(k_bf16, B, H, T, D, sink_tokens, recent_tokens, rotate, f_lo, f_hi, sink_bf16, recent_bf16,
+                       codes, scales, gscale, false, stream, mid_out);
 }
 
 int nvfp4_kv_mixed_mma(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,

@@ -102,3 +102,28 @@ def test_round_trip_errors():
     assert L.nvfp4_quantize_dequantize(p(x), 64, 0, -2, 6, None, p(c), p(s), p(g), None, st) == -1
     assert L.nvfp4_quantize_dequantize(p(x), 60, 0, -2, 6, None, p(c), p(s), p(g), p(x), st) == -2
     assert L.nvfp4_quantize_dequantize(p(x), 64, 0, -2, 6, None, p(c), p(s), p(g), p(x) + 4, st) == -3
+
+
+@pytest.mark.parametrize("window", [(-2, 6), (0, 0), (-8, 8), (-1, 3)])
+@pytest.mark.parametrize("rotate,sink,recent", [(True, 16, 16), (False, 16, 16), (True, 0, 0), (True, 5, 27)])
+def test_kv_round_trip_matches_oracle(window, rotate, sink, recent):
+    """kv_mixed_dequantize: the KV layout's outputs equal the oracle's, and the middle's values equal the
+    oracle's dequantize of the oracle's codes (BF16, rotated space when rotating)."""
+    g = torch.Generator().manual_seed(41)
+    k = torch.randn((2, 3, 200, 64), generator=g)
+    k[..., 7] += 3.0                                     # an outlier channel, as in the KV recipe
+    k = k.to(torch.bfloat16)
+    kh = k.view(torch.int16).numpy().view(np.uint16)
+    rso, rro, rc, rs, rg = O.kv_mixed(kh, sink, recent, int(rotate), *window)
+    so, ro, c, s, gs, mid = nv.kv_mixed_dequantize(k.cuda(), sink, recent, rotate, *window)
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy().reshape(-1), rc.reshape(-1))
+    assert np.array_equal(s.cpu().numpy().reshape(-1), rs.reshape(-1))
+    assert gs.cpu().numpy().view(np.uint32)[0] == np.float32(rg).view(np.uint32)
+    assert np.array_equal(_bits(so), rso.reshape(-1)) and np.array_equal(_bits(ro), rro.reshape(-1))
+    want = O.dequantize(rc.reshape(-1), rs.reshape(-1), rg, out_dtype=O.BF16)
+    assert _same(_bits(mid), want, torch.bfloat16)
+    # and the same as the two calls it fuses
+    so2, ro2, c2, s2, g2 = nv.kv_mixed(k.cuda(), sink, recent, rotate, *window)
+    assert torch.equal(c, c2) and torch.equal(s, s2)
+    assert torch.equal(mid.view(torch.int16), nv.dequantize(c2, s2, g2, torch.bfloat16).view(mid.shape).view(torch.int16))
