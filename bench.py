@@ -71,7 +71,7 @@ def peaks():
 
 def captured_traffic(kernel_key: str, elements: int):
     """DRAM bytes per launch from the committed ncu record, scaled to `elements`; None when the kernel
-    sources changed since the capture (the counters then no longer describe this build)."""
+    sources changed since the capture (the counters then no longer describe the compiled kernel)."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
