@@ -11,6 +11,38 @@ namespace nvfp4 {
 
 enum : int { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
 
+// ---- packed FP32x2 arithmetic: each lane rounds exactly as the scalar operation ----
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 pk2(float lo, float hi) {
+  u64 r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(u64 v, float& lo, float& hi) {
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 add2(u64 a, u64 b) {
+  u64 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
+  u64 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 // ---- streaming loads: read-only path, no L1 allocation (every byte is read once per pass) ----
 __device__ __forceinline__ void ld_v8(const void* p, uint32_t (&v)[8]) {
   asm("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -147,6 +179,42 @@ __device__ __forceinline__ void fwht16(float (&a)[16]) {
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) a[i] = __fmul_rn(a[i], 0.25f);
+}
+
+// The same transform on 8 packed pairs (x2[k] = elements 2k, 2k+1), with the same additions in the same
+// order: stage 1 pairs the two lanes of one register (scalar), stages 2, 4 and 8 pair registers k and
+// k + h/2 lane by lane (one FP32x2 add and one subtract per register pair), then the packed x0.25.
+__device__ __forceinline__ void fwht16_x2(u64 (&x2)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float u, v;
+    upk2(x2[k], u, v);
+    x2[k] = pk2(__fadd_rn(u, v), __fsub_rn(u, v));
+  }
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if ((k & h) == 0) {
+        const u64 u = x2[k], v = x2[k + h];
+        x2[k] = add2(u, v);
+        x2[k + h] = sub2(u, v);
+      }
+    }
+  }
+  const u64 q = pk2(0.25f, 0.25f);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x2[k] = mul2(x2[k], q);
+}
+
+// fwht16_x2 on 16 values held as floats (packed and unpacked around it).
+__device__ __forceinline__ void fwht16_packed(float (&a)[16]) {
+  u64 x2[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x2[k] = pk2(a[2 * k], a[2 * k + 1]);
+  fwht16_x2(x2);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) upk2(x2[k], a[2 * k], a[2 * k + 1]);
 }
 
 }  // namespace nvfp4

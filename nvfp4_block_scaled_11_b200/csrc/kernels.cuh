@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(256) hadamard16_kernel(const char* __restrict_
     float a[16];
     load_block<DT>(x + 16 * ES * b, v8_in != 0, a);
     if (!inverse) flip_signs(a, m);
-    fwht16(a);
+    fwht16_packed(a);
     if (inverse) flip_signs(a, m);
     char* o = out + 16 * OS * b;
     if (OT == DT_F32) {
@@ -625,7 +625,7 @@ __global__ void __launch_bounds__(256) kv_amax_kernel(const char* __restrict__ k
   for (; b < ngroups; b += stride, kc.advance()) {
     float x[16];
     load_block<DT_BF16>(k + 2 * kc.elem(T, sink, D), v8 != 0, x);
-    if (ROT) fwht16(x);
+    if (ROT) fwht16_packed(x);
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(x[i]) & 0x7FFFFFFFu);
   }

@@ -28,31 +28,6 @@
 
 namespace nvfp4 {
 
-typedef unsigned long long u64;
-
-__device__ __forceinline__ u64 pk2(float lo, float hi) {
-  u64 r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void upk2(u64 v, float& lo, float& hi) {
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
-  u64 d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ u64 add2(u64 a, u64 b) {
-  u64 d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
-  u64 d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 // Exact E2M1 roundings of (lo, hi), returned as the f16 halves of one register (RNE, saturating).
 __device__ __forceinline__ uint32_t e2m1_round2(float lo, float hi) {
   uint32_t r;
@@ -360,14 +335,7 @@ __device__ __forceinline__ float block_amax_nan(const u64 (&x2)[8]) {
 
 template <bool ROT>
 __device__ __forceinline__ void maybe_rotate(u64 (&x2)[8]) {
-  if (ROT) {
-    float t[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) upk2(x2[k], t[2 * k], t[2 * k + 1]);
-    fwht16(t);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) x2[k] = pk2(t[2 * k], t[2 * k + 1]);
-  }
+  if (ROT) fwht16_x2(x2);
 }
 
 // DEQ >= 0 (a dtype): also write the block's dequantized values to p.deq_out (fused round trip).
