@@ -127,3 +127,17 @@ def test_kv_round_trip_matches_oracle(window, rotate, sink, recent):
     so2, ro2, c2, s2, g2 = nv.kv_mixed(k.cuda(), sink, recent, rotate, *window)
     assert torch.equal(c, c2) and torch.equal(s, s2)
     assert torch.equal(mid.view(torch.int16), nv.dequantize(c2, s2, g2, torch.bfloat16).view(mid.shape).view(torch.int16))
+
+
+@pytest.mark.parametrize("mag", [1e-44, 1e-40, 1e-36, 1e-20, 1e20, 1e35, 3e38])
+def test_round_trip_extreme_tensor_scales(mag):
+    """Tensor scales computed from extreme tensors: g subnormal or zero (tiny inputs, subnormal ones
+    included) and g near the top of the range; codes, scales, g and values against the oracle."""
+    g = torch.Generator().manual_seed(int(abs(np.log10(mag))) + 7)
+    x = (torch.randn(16 * 2003, generator=g, dtype=torch.float64) * mag).clamp(-3.4e38, 3.4e38).to(torch.float32)
+    _check(x, -2, 6)
+    _check(x, -8, 8)
+    xd = x.cuda()
+    c, s, gs = nv.quantize(xd)
+    rc, rs, rg, _, _ = O.quantize(x.numpy(), -2, 6)
+    assert np.array_equal(c.cpu().numpy(), rc) and np.array_equal(s.cpu().numpy(), rs)
