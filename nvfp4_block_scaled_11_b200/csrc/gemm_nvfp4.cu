@@ -106,6 +106,11 @@ int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs
   if (batch < 0 || M < 0 || N < 0 || K < 0) return NVFP4_ERR_ARG;
   const int64_t lim = (int64_t(1) << 31) - 1;
   if (K % 32 != 0 || batch > lim || M > lim || N > lim || K > lim) return NVFP4_ERR_SIZE;
+  int64_t t;   // every buffer's element count must fit in int64 (no wrapped size passes a later check)
+  if (__builtin_mul_overflow(batch, M, &t) || __builtin_mul_overflow(t, N, &t) || __builtin_mul_overflow(t, 4, &t) ||
+      __builtin_mul_overflow(batch, M, &t) || __builtin_mul_overflow(t, K, &t) ||
+      __builtin_mul_overflow(batch, N, &t) || __builtin_mul_overflow(t, K, &t))
+    return NVFP4_ERR_SIZE;
   if (batch == 0 || M == 0 || N == 0) return NVFP4_OK;
   if (d == nullptr) return NVFP4_ERR_ARG;
   const int esize = d_dtype == NVFP4_F32 ? 4 : 2;

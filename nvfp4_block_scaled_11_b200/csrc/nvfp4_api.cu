@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <initializer_list>
 #include <mutex>
 
 #include "../../include/nvfp4.h"
@@ -64,6 +65,16 @@ bool inject_launch_fault() {
     mode = (e && strcmp(e, "launch") == 0) ? 1 : 0;
   }
   return mode == 1;
+}
+
+// Product of sizes that must each be non-negative, or -1 when one is negative or the product does not
+// fit in int64 (so that no later size arithmetic can wrap round and pass a check).
+int64_t checked_prod(std::initializer_list<int64_t> v) {
+  int64_t p = 1;
+  for (int64_t a : v) {
+    if (a < 0 || __builtin_mul_overflow(p, a, &p)) return -1;
+  }
+  return p;
 }
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -207,6 +218,9 @@ int msda_setup(MsdaParams& p, int64_t bs, int64_t nkeys, int64_t heads, int64_t 
     keys += H * W;
   }
   if (keys != nkeys) return NVFP4_ERR_SIZE;
+  if (checked_prod({bs, nkeys, heads, ch}) < 0 || checked_prod({bs, nq, heads, (int64_t)L, (int64_t)P, 2}) < 0 ||
+      checked_prod({bs, nq, heads, ch}) < 0)
+    return NVFP4_ERR_SIZE;
   p.nkeys = nkeys;
   p.heads = heads;
   p.nq = nq;
@@ -285,15 +299,16 @@ int nvfp4_quantize_ex(const void* x, int64_t n, int dtype, int block, int f_lo, 
 int64_t nvfp4_sf_mma_bytes(int64_t rows, int64_t cols, int64_t batch) {
   if (rows < 0 || cols < 0 || batch < 0) return NVFP4_ERR_ARG;
   if (cols % 16 != 0) return NVFP4_ERR_SIZE;
-  return batch * ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
+  const int64_t b = checked_prod({batch, (rows + 127) / 128, 128, (cols / 16 + 3) / 4, 4});
+  return b < 0 ? NVFP4_ERR_SIZE : b;
 }
 
 int nvfp4_quantize_mma(const void* x, int64_t batch, int64_t rows, int64_t cols, int dtype, int f_lo, int f_hi,
                        const float* gscale_in, uint8_t* codes, uint8_t* sf, float* gscale, void* stream) {
   if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_ARG;
   if (cols % 16 != 0) return NVFP4_ERR_SIZE;
-  const int64_t n = batch * rows * cols;
-  if (n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  const int64_t n = checked_prod({batch, rows, cols});
+  if (n < 0 || n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
   if (n > 0 && sf == nullptr) return NVFP4_ERR_ARG;
   cudaStream_t s = S(stream);
   QuantParams lay{};
@@ -315,8 +330,8 @@ int nvfp4_quantize_mma_t(const void* x, int64_t batch, int64_t rows, int64_t col
                          const float* gscale_in, uint8_t* codes_t, uint8_t* sf_t, float* gscale, void* stream) {
   if (batch < 0 || rows < 0 || cols < 0) return NVFP4_ERR_ARG;
   if (rows % 16 != 0) return NVFP4_ERR_SIZE;
-  const int64_t n = batch * rows * cols;
-  if (n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  const int64_t n = checked_prod({batch, rows, cols});
+  if (n < 0 || n / 16 >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
   if (n > 0 && sf_t == nullptr) return NVFP4_ERR_ARG;
   cudaStream_t s = S(stream);
   QuantParams lay{};
@@ -435,6 +450,7 @@ static int kv_mixed_impl(const void* k_bf16, int64_t B, int64_t H, int64_t T, in
   if (!window_ok(f_lo, f_hi) || gscale == nullptr || sink_tokens < 0 || recent_tokens < 0) return NVFP4_ERR_ARG;
   if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
     return NVFP4_ERR_SIZE;
+  if (checked_prod({B, H, T, D}) < 0) return NVFP4_ERR_SIZE;
   const int64_t BH = B * H;
   const int64_t Tm = T - sink_tokens - recent_tokens;
   const int64_t ngroups = BH * Tm * (D / 16);
@@ -542,6 +558,7 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
   const int nc = f_hi - f_lo + 1;
   if (!window_ok(f_lo, f_hi) || (nc != 1 && nc != 9 && nc != 17) || gscale == nullptr) return NVFP4_ERR_ARG;
   if (batch < 0 || Tq < 0 || Tk < 0 || Tk % 16 != 0) return NVFP4_ERR_SIZE;
+  if (checked_prod({batch, Tq, Tk}) < 0) return NVFP4_ERR_SIZE;
   const int64_t rows = batch * Tq, bpr = Tk / 16;
   if (rows * bpr >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
   cudaStream_t st = S(stream);
@@ -581,7 +598,7 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
 }
 
 int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream) {
-  if (rows < 0 || cols < 0 || cols % 4 != 0) return NVFP4_ERR_SIZE;
+  if (rows < 0 || cols < 0 || cols % 4 != 0 || checked_prod({rows, cols}) < 0) return NVFP4_ERR_SIZE;
   if (rows == 0 || cols == 0) return NVFP4_OK;
   if (x == nullptr || l == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(x, 16) || !aligned(l, 4)) return NVFP4_ERR_ALIGN;
@@ -634,6 +651,7 @@ int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t
   if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 16 != 0 || T < (int64_t)sink_tokens + recent_tokens)
     return NVFP4_ERR_SIZE;
   const int64_t Tm = T - sink_tokens - recent_tokens;
+  if (checked_prod({B, H, T, D}) < 0) return NVFP4_ERR_SIZE;
   const int64_t ngroups = B * H * Tm * (D / 16);
   if (ngroups >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if (ngroups > 0 && k_bf16 == nullptr) return NVFP4_ERR_ARG;
@@ -659,7 +677,8 @@ int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, in
                     int scale_layout, void* stream) {
   if (!window_ok(f_lo, f_hi) || gscale == nullptr || (scale_layout != 0 && scale_layout != 1)) return NVFP4_ERR_ARG;
   if (BH < 0 || T < 0 || n < 0 || first < 0 || t0 < 0 || cap < 0 || D <= 0 || D % 16 != 0) return NVFP4_ERR_SIZE;
-  if (first + n > T || t0 + n > cap) return NVFP4_ERR_SIZE;
+  if (first > T - n || t0 > cap - n) return NVFP4_ERR_SIZE;
+  if (checked_prod({BH, T, D}) < 0 || checked_prod({BH, cap, D}) < 0) return NVFP4_ERR_SIZE;
   if (scale_layout == 1 && BH * cap * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
   if (BH * n * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
   if (BH == 0 || n == 0) return NVFP4_OK;

@@ -85,3 +85,18 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(TypeError):
         nv.quantize(torch.zeros(32))
+
+
+def test_size_products_that_overflow_are_rejected(L):
+    """Sizes whose products do not fit in 64 bits come back as NVFP4_ERR_SIZE before anything runs."""
+    fake, big = V(0x10000), 1 << 40
+    assert L.nvfp4_quantize_mma(fake, big, big, 16 * big, 0, -2, 6, None, fake, fake, fake, None) == -2
+    assert L.nvfp4_quantize_mma_t(fake, big, 16 * big, big, 0, -2, 6, None, fake, fake, fake, None) == -2
+    assert L.nvfp4_sf_mma_bytes(big, 16 * big, big) == -2
+    assert L.nvfp4_kv_mixed(fake, big, big, big, 128, 16, 16, 1, -2, 6, fake, fake, fake, fake, fake, None) == -2
+    assert L.nvfp4_kv_gscale(fake, big, big, big, 128, 16, 16, 1, fake, None) == -2
+    assert L.nvfp4_softmax_quantize_mma(fake, big, big, 16 * big, 1, 0, -2, 6, fake, fake, fake, fake, fake, None) == -2
+    assert L.nvfp4_rows_divide(fake, fake, big, 4 * big, None) == -2
+    assert L.nvfp4_kv_append(fake, big, big, 0, 16, 128, 1, -2, 6, fake, fake, fake, big, 0, 0, None) == -2
+    assert L.nvfp4_gemm_nt(fake, fake, fake, fake, fake, fake, 1 << 30, 1 << 30, 1 << 30, 32, 1.0, fake, 0, fake,
+                           None) == -2
