@@ -35,6 +35,9 @@
  * CUDA runtime rejects on the host: the call returns NVFP4_ERR_CUDA and nothing reaches the GPU.
  * Alignment: element buffers must be 16-byte aligned (32-byte aligned inputs use 256-bit loads);
  * code buffers 8-byte aligned.  Sizes are element counts and must be multiples of 16 (one block).
+ * Size limits (NVFP4_ERR_SIZE otherwise, before anything is enqueued): one-dimensional counts up to
+ * 2^60 elements; the products of multi-dimensional sizes must fit in int64; calls that split block
+ * indices in 32 bits (tile layouts, KV, softmax) say so and take fewer than 2^32 blocks.
  */
 #ifndef NVFP4_H
 #define NVFP4_H

@@ -67,6 +67,10 @@ bool inject_launch_fault() {
   return mode == 1;
 }
 
+// Largest element count of a one-dimensional call: byte offsets of any element type stay far from
+// int64 overflow.
+constexpr int64_t kMaxElems = int64_t(1) << 60;
+
 // Product of sizes that must each be non-negative, or -1 when one is negative or the product does not
 // fit in int64 (so that no later size arithmetic can wrap round and pass a check).
 int64_t checked_prod(std::initializer_list<int64_t> v) {
@@ -151,7 +155,7 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
                   cudaStream_t s) {
   if (!dtype_ok(dtype) || !window_ok(f_lo, f_hi)) return NVFP4_ERR_ARG;
   if (gscale_in == nullptr && gscale == nullptr) return NVFP4_ERR_ARG;
-  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n % 16 != 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_ARG;
   if ((n > 0 && !aligned(x, 16)) || (n > 0 && !aligned(codes, 8)) || (gscale && !aligned(gscale, 4)) ||
       (gscale_in && !aligned(gscale_in, 4)) || (block_sse && !aligned(block_sse, 4)))
@@ -273,7 +277,7 @@ int nvfp4_version(void) { return 100; }
 
 int nvfp4_tensor_amax(const void* x, int64_t n, int dtype, float* d_amax, void* stream) {
   if (!dtype_ok(dtype) || d_amax == nullptr || (n > 0 && x == nullptr)) return NVFP4_ERR_ARG;
-  if (n < 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if ((n > 0 && !aligned(x, 16)) || !aligned(d_amax, 4)) return NVFP4_ERR_ALIGN;
   cudaStream_t s = S(stream);
   if (cudaMemsetAsync(d_amax, 0, sizeof(float), s) != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -385,7 +389,7 @@ int nvfp4_quantize_dequantize(const void* x, int64_t n, int dtype, int f_lo, int
 int nvfp4_dequantize_ex(const uint8_t* codes, const uint8_t* scales, const float* gscale, int64_t n, int out_dtype,
                         void* out, int ctas_per_sm, void* stream) {
   if (!dtype_ok(out_dtype) || gscale == nullptr || ctas_per_sm < 0 || ctas_per_sm > 8) return NVFP4_ERR_ARG;
-  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n % 16 != 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (codes == nullptr || scales == nullptr || out == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
@@ -411,7 +415,7 @@ int nvfp4_hadamard16_ex(const void* x, int64_t n, int dtype, void* out, int out_
                         int inverse, void* stream) {
   if (!dtype_ok(dtype) || !dtype_ok(out_dtype) || signs > 0xFFFFu || (inverse != 0 && inverse != 1))
     return NVFP4_ERR_ARG;
-  if (n < 0 || n % 16 != 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n % 16 != 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (x == nullptr || out == nullptr) return NVFP4_ERR_ARG;
   if (x == out && dtype != out_dtype) return NVFP4_ERR_ARG;
@@ -608,7 +612,7 @@ int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void
 
 int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, uint8_t* scales, void* stream) {
   if (!dtype_ok(dtype)) return NVFP4_ERR_ARG;
-  if (n < 0 || n % 32 != 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n % 32 != 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (x == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(x, 16) || !aligned(codes, 16)) return NVFP4_ERR_ALIGN;
@@ -628,7 +632,7 @@ int nvfp4_mxfp4_quantize(const void* x, int64_t n, int dtype, uint8_t* codes, ui
 int nvfp4_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t n, int out_dtype, void* out,
                            void* stream) {
   if (!dtype_ok(out_dtype)) return NVFP4_ERR_ARG;
-  if (n < 0 || n % 32 != 0) return NVFP4_ERR_SIZE;
+  if (n < 0 || n % 32 != 0 || n > kMaxElems) return NVFP4_ERR_SIZE;
   if (n == 0) return NVFP4_OK;
   if (codes == nullptr || scales == nullptr || out == nullptr) return NVFP4_ERR_ARG;
   if (!aligned(codes, 16) || !aligned(out, 16)) return NVFP4_ERR_ALIGN;

@@ -100,3 +100,9 @@ def test_size_products_that_overflow_are_rejected(L):
     assert L.nvfp4_kv_append(fake, big, big, 0, 16, 128, 1, -2, 6, fake, fake, fake, big, 0, 0, None) == -2
     assert L.nvfp4_gemm_nt(fake, fake, fake, fake, fake, fake, 1 << 30, 1 << 30, 1 << 30, 32, 1.0, fake, 0, fake,
                            None) == -2
+    huge = 1 << 61
+    assert L.nvfp4_quantize(fake, huge, 0, 16, -2, 6, fake, fake, fake, None) == -2
+    assert L.nvfp4_dequantize(fake, fake, fake, huge, 0, fake, None) == -2
+    assert L.nvfp4_hadamard16(fake, huge, 0, fake, 0, None) == -2
+    assert L.nvfp4_tensor_amax(fake, huge, 0, fake, None) == -2
+    assert L.nvfp4_mxfp4_quantize(fake, huge, 0, fake, fake, None) == -2
