@@ -76,3 +76,37 @@ def test_two_rank_sharded_quantize_matches_single_process():
     codes = np.concatenate([out[r][2] for r in range(world)])
     scales = np.concatenate([out[r][3] for r in range(world)])
     assert np.array_equal(codes, rc) and np.array_equal(scales, rs)
+
+
+def _failing_worker(rank, world, port, x, out):
+    """Rank 1 fails before the exchange; rank 0 must learn of it on the host through its collective
+    (the peer closes its connection, or the short process-group timeout expires), not hang."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    try:
+        if rank == 1:
+            raise RuntimeError("injected failure before the amax exchange")
+        lo, hi = nvdist.shard_bounds(x.numel(), world, rank)
+        nvdist.sharded_quantize(x[lo:hi].contiguous(), -2, 6, ops=_oracle_ops())
+        out[rank] = "completed"
+    except Exception as e:  # recorded for the parent: the failure has to surface as an error
+        out[rank] = f"error: {type(e).__name__}: {e}"
+    finally:
+        if rank == 1:
+            dist.destroy_process_group()
+
+
+def test_failed_rank_is_detected_on_the_host():
+    import time
+    x = torch.from_numpy(np.random.default_rng(9).standard_normal(16 * 512).astype(np.float32))
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    t = time.monotonic()
+    mp.start_processes(_failing_worker, args=(world, _free_port(), x, out), nprocs=world, start_method="spawn",
+                       join=True)
+    assert time.monotonic() - t < 120
+    assert out[1].startswith("error: RuntimeError: injected failure")
+    assert out[0].startswith("error:"), out[0]
