@@ -106,6 +106,17 @@ def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
     return t
 
 
+def _out(t: torch.Tensor, name: str, dtype, need: int) -> torch.Tensor:
+    """A caller-provided buffer that a kernel reads or writes by size: a contiguous CUDA tensor of `dtype`
+    (None: any dtype) with at least `need` elements, so that no launch reaches past its end."""
+    _cuda(t, name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < need:
+        raise ValueError(f"{name} holds {t.numel()} elements, {need} needed")
+    return t
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -124,15 +135,15 @@ def _dt(t: torch.Tensor) -> int:
 def tensor_amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """max |x| as a 1-element float32 device tensor (NaN / Inf propagate)."""
     _cuda(x, "x")
-    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else _out(out, "out", torch.float32, 1)
     _check(lib().nvfp4_tensor_amax(_ptr(x), x.numel(), _dt(x), _ptr(out), _stream(x)))
     return out
 
 
 def global_scale(amax: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """g = amax / 2688 on the device."""
-    _cuda(amax, "amax")
-    out = torch.empty(1, dtype=torch.float32, device=amax.device) if out is None else out
+    _out(amax, "amax", torch.float32, 1)
+    out = torch.empty(1, dtype=torch.float32, device=amax.device) if out is None else _out(out, "out", torch.float32, 1)
     _check(lib().nvfp4_global_scale(_ptr(amax), _ptr(out), _stream(amax)))
     return out
 
@@ -140,9 +151,11 @@ def global_scale(amax: torch.Tensor, out: torch.Tensor | None = None) -> torch.T
 def _alloc_q(x, codes, scales, gscale):
     n = x.numel()
     dev = x.device
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev) if codes is None else codes
-    scales = torch.empty(n // 16, dtype=torch.uint8, device=dev) if scales is None else scales
-    gscale = torch.empty(1, dtype=torch.float32, device=dev) if gscale is None else gscale
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev) if codes is None else _out(codes, "codes", torch.uint8, n // 2)
+    scales = (torch.empty(n // 16, dtype=torch.uint8, device=dev) if scales is None
+              else _out(scales, "scales", torch.uint8, n // 16))
+    gscale = (torch.empty(1, dtype=torch.float32, device=dev) if gscale is None
+              else _out(gscale, "gscale", torch.float32, 1))
     return codes, scales, gscale
 
 
@@ -165,16 +178,20 @@ def quantize_ex(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torch
     Returns (codes, scales, gscale, block_f int8[n/16] or None, block_sse float32[n/16] or None)."""
     _cuda(x, "x")
     n = x.numel()
+    keep = gscale
     if gscale_in is not None:
-        _cuda(gscale_in, "gscale_in")
-        keep = gscale
+        _out(gscale_in, "gscale_in", torch.float32, 1)
     codes, scales, gscale = _alloc_q(x, codes, scales, gscale)
     if gscale_in is not None and keep is None:
         gscale = None  # g comes from gscale_in; no copy requested
     if want_f and block_f is None:
         block_f = torch.empty(n // 16, dtype=torch.int8, device=x.device)
+    elif block_f is not None:
+        _out(block_f, "block_f", torch.int8, n // 16)
     if want_sse and block_sse is None:
         block_sse = torch.empty(n // 16, dtype=torch.float32, device=x.device)
+    elif block_sse is not None:
+        _out(block_sse, "block_sse", torch.float32, n // 16)
     _check(lib().nvfp4_quantize_ex(_ptr(x), n, _dt(x), block, f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
                                    _ptr(scales), _ptr(gscale), _ptr(block_f), _ptr(block_sse), _stream(x)))
     return codes, scales, gscale, block_f, block_sse
@@ -188,7 +205,7 @@ def quantize_dequantize(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_i
     _cuda(x, "x")
     n = x.numel()
     if gscale_in is not None:
-        _cuda(gscale_in, "gscale_in")
+        _out(gscale_in, "gscale_in", torch.float32, 1)
     keep = gscale
     codes, scales, gscale = _alloc_q(x, codes, scales, gscale)
     if gscale_in is not None and keep is None:
@@ -206,9 +223,10 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor, 
                out: torch.Tensor | None = None, ctas_per_sm: int = 0) -> torch.Tensor:
     """Dequantize n = 16 * scales.numel() elements to out_dtype.  ctas_per_sm > 0 bounds the launch
     footprint (to run beside another kernel on a second stream); 0 = default."""
-    _cuda(codes, "codes"), _cuda(scales, "scales"), _cuda(gscale, "gscale")
+    _cuda(scales, "scales")
     n = scales.numel() * 16
-    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
+    _out(codes, "codes", torch.uint8, n // 2), _out(gscale, "gscale", torch.float32, 1)
+    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else _out(out, "out", None, n)
     _check(lib().nvfp4_dequantize_ex(_ptr(codes), _ptr(scales), _ptr(gscale), n, DTYPE_CODE[out.dtype], _ptr(out),
                                      ctas_per_sm, _stream(codes)))
     return out
@@ -220,7 +238,7 @@ def hadamard16(x: torch.Tensor, out_dtype=None, out: torch.Tensor | None = None,
     D goes first, (H/4) D x, or last for the inverse, D (H/4) x."""
     _cuda(x, "x")
     out_dtype = x.dtype if out_dtype is None else out_dtype
-    out = torch.empty(x.shape, dtype=out_dtype, device=x.device) if out is None else out
+    out = torch.empty(x.shape, dtype=out_dtype, device=x.device) if out is None else _out(out, "out", None, x.numel())
     if signs == 0 and not inverse:
         _check(lib().nvfp4_hadamard16(_ptr(x), x.numel(), _dt(x), _ptr(out), DTYPE_CODE[out.dtype], _stream(x)))
     else:
@@ -301,10 +319,10 @@ def quantize_mma(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: torc
         sf = torch.empty(sf_mma_bytes(rows, cols, batch), dtype=torch.uint8, device=dev)
     if gscale is None:
         gscale = torch.empty(1, dtype=torch.float32, device=dev)
-    if codes.numel() * 2 != x.numel() or sf.numel() < sf_mma_bytes(rows, cols, batch):
-        raise ValueError("codes / sf buffers are too small")
+    _out(codes, "codes", torch.uint8, x.numel() // 2), _out(gscale, "gscale", torch.float32, 1)
+    _out(sf, "sf", torch.uint8, sf_mma_bytes(rows, cols, batch))
     if gscale_in is not None:
-        _cuda(gscale_in, "gscale_in")
+        _out(gscale_in, "gscale_in", torch.float32, 1)
     _check(lib().nvfp4_quantize_mma(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
                                     _ptr(sf), _ptr(gscale), _stream(x)))
     return codes, sf, gscale
@@ -326,8 +344,10 @@ def quantize_mma_t(x: torch.Tensor, f_lo: int = -2, f_hi: int = 6, gscale_in: to
         sf = torch.empty(sf_mma_bytes(cols, rows, batch), dtype=torch.uint8, device=dev)
     if gscale is None:
         gscale = torch.empty(1, dtype=torch.float32, device=dev)
+    _out(codes, "codes", torch.uint8, x.numel() // 2), _out(gscale, "gscale", torch.float32, 1)
+    _out(sf, "sf", torch.uint8, sf_mma_bytes(cols, rows, batch))
     if gscale_in is not None:
-        _cuda(gscale_in, "gscale_in")
+        _out(gscale_in, "gscale_in", torch.float32, 1)
     _check(lib().nvfp4_quantize_mma_t(_ptr(x), batch, rows, cols, _dt(x), f_lo, f_hi, _ptr(gscale_in), _ptr(codes),
                                       _ptr(sf), _ptr(gscale), _stream(x)))
     return codes, sf, gscale
@@ -380,11 +400,19 @@ def gemm_nt(a_codes: torch.Tensor, a_sf: torch.Tensor, a_gscale: torch.Tensor, b
         raise ValueError("a_codes and b_codes disagree on batch or K")
     N, K = b3.shape[1], 2 * K2
     dev = a_codes.device
+    if a_codes.dtype != torch.uint8 or b_codes.dtype != torch.uint8:
+        raise TypeError("a_codes and b_codes must be uint8")
+    _out(a_sf, "a_sf", torch.uint8, sf_mma_bytes(M, K, batch) if M and K else 0)
+    _out(b_sf, "b_sf", torch.uint8, sf_mma_bytes(N, K, batch) if N and K else 0)
+    _out(a_gscale, "a_gscale", torch.float32, 1), _out(b_gscale, "b_gscale", torch.float32, 1)
     if out is None:
         out = torch.empty((batch, M, N), dtype=out_dtype, device=dev)
-    _cuda(out, "out")
+    _out(out, "out", None, batch * M * N)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
     if alpha_work is None:
         alpha_work = torch.empty(1, dtype=torch.float32, device=dev)
+    _out(alpha_work, "alpha_work", torch.float32, 1)
     _check(lib().nvfp4_gemm_nt(_ptr(a_codes), _ptr(a_sf), _ptr(a_gscale), _ptr(b_codes), _ptr(b_sf), _ptr(b_gscale),
                                batch, M, N, K, float(alpha), _ptr(out), DTYPE_CODE[out.dtype], _ptr(alpha_work),
                                _stream(a_codes)))
@@ -407,7 +435,7 @@ def kv_gscale(k: torch.Tensor, sink: int = 16, recent: int = 16, rotate: bool = 
     if k.dtype != torch.bfloat16 or k.dim() != 4:
         raise TypeError("k must be a 4-D bfloat16 tensor [B,H,T,D]")
     B, H, T, D = k.shape
-    out = torch.empty(1, dtype=torch.float32, device=k.device) if out is None else out
+    out = torch.empty(1, dtype=torch.float32, device=k.device) if out is None else _out(out, "out", torch.float32, 1)
     _check(lib().nvfp4_kv_gscale(_ptr(k), B, H, T, D, sink, recent, int(bool(rotate)), _ptr(out), _stream(k)))
     return out
 
@@ -425,6 +453,8 @@ def kv_append(k_rows: torch.Tensor, first: int, n: int, gscale: torch.Tensor, co
     T, D = k_rows.shape[-2], k_rows.shape[-1]
     BH = k_rows.numel() // max(T * D, 1)
     cap = codes.shape[-2]
+    _out(gscale, "gscale", torch.float32, 1), _out(codes, "codes", torch.uint8, BH * cap * (D // 2))
+    _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
     _check(lib().nvfp4_kv_append(_ptr(k_rows), BH, T, first, n, D, int(bool(rotate)), f_lo, f_hi, _ptr(gscale),
                                  _ptr(codes), _ptr(scales), cap, t0, 1 if tile_layout else 0, _stream(k_rows)))
 
@@ -434,17 +464,19 @@ def mxfp4_quantize(x: torch.Tensor, codes: torch.Tensor | None = None, scales: t
     """MXFP4 (32-element blocks, E8M0 power-of-two scales).  Returns (codes uint8[n/2], scales uint8[n/32])."""
     _cuda(x, "x")
     n = x.numel()
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=x.device) if codes is None else codes
-    scales = torch.empty(n // 32, dtype=torch.uint8, device=x.device) if scales is None else scales
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=x.device) if codes is None else _out(codes, "codes", torch.uint8, n // 2)
+    scales = (torch.empty(n // 32, dtype=torch.uint8, device=x.device) if scales is None
+              else _out(scales, "scales", torch.uint8, n // 32))
     _check(lib().nvfp4_mxfp4_quantize(_ptr(x), n, _dt(x), _ptr(codes), _ptr(scales), _stream(x)))
     return codes, scales
 
 
 def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, out_dtype=torch.float32,
                      out: torch.Tensor | None = None) -> torch.Tensor:
-    _cuda(codes, "codes"), _cuda(scales, "scales")
+    _cuda(scales, "scales")
     n = scales.numel() * 32
-    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else out
+    _out(codes, "codes", torch.uint8, n // 2)
+    out = torch.empty(n, dtype=out_dtype, device=codes.device) if out is None else _out(out, "out", None, n)
     _check(lib().nvfp4_mxfp4_dequantize(_ptr(codes), _ptr(scales), n, DTYPE_CODE[out.dtype], _ptr(out),
                                         _stream(codes)))
     return out
@@ -462,16 +494,18 @@ def msda_forward(value, shapes, loc: torch.Tensor, w: torch.Tensor, out: torch.T
     bs, nq, heads, L, P, _ = loc.shape
     if isinstance(value, (tuple, list)):
         codes, scales, gscale = value
-        for t, nm in ((codes, "codes"), (scales, "scales"), (gscale, "gscale")):
-            _cuda(t, nm)
         _, nkeys, _, ch2 = codes.shape
         ch = 2 * ch2
+        _out(codes, "codes", torch.uint8, bs * nkeys * heads * ch2)
+        _out(scales, "scales", torch.uint8, bs * nkeys * heads * (ch // 16)), _out(gscale, "gscale", torch.float32, 1)
     else:
         _cuda(value, "value")
         _, nkeys, _, ch = value.shape
+        _out(value, "value", None, bs * nkeys * heads * ch)
+    _out(loc, "loc", torch.float32, bs * nq * heads * L * P * 2), _out(w, "w", torch.float32, bs * nq * heads * L * P)
     if out is None:
         out = torch.empty((bs, nq, heads, ch), dtype=torch.float32, device=loc.device)
-    _cuda(out, "out")
+    _out(out, "out", torch.float32, bs * nq * heads * ch)
     shp = sh.ctypes.data
     if isinstance(value, (tuple, list)):
         _check(lib().nvfp4_msda_forward_nvfp4(_ptr(codes), _ptr(scales), _ptr(gscale), bs, nkeys, heads, ch, shp,
@@ -490,11 +524,15 @@ def softmax_quantize_mma(s: torch.Tensor, causal: bool = False, q_offset: int = 
     _cuda(s, "s")
     batch, Tq, Tk = (1, *s.shape) if s.dim() == 2 else s.shape
     dev = s.device
+    if s.dtype != torch.float32:
+        raise TypeError("s must be float32")
     codes = torch.empty((*s.shape[:-1], Tk // 2), dtype=torch.uint8, device=dev) if codes is None else codes
     sf = torch.empty(max(sf_mma_bytes(Tq, Tk, batch), 1), dtype=torch.uint8, device=dev) if sf is None else sf
     g = torch.empty(1, dtype=torch.float32, device=dev) if g is None else g
     m = torch.empty(batch * Tq, dtype=torch.float32, device=dev) if m is None else m
     l = torch.empty(batch * Tq, dtype=torch.float32, device=dev) if l is None else l
+    _out(codes, "codes", torch.uint8, batch * Tq * (Tk // 2)), _out(sf, "sf", torch.uint8, sf_mma_bytes(Tq, Tk, batch))
+    _out(g, "g", torch.float32, 1), _out(m, "m", torch.float32, batch * Tq), _out(l, "l", torch.float32, batch * Tq)
     _check(lib().nvfp4_softmax_quantize_mma(_ptr(s), batch, Tq, Tk, int(bool(causal)), q_offset, f_lo, f_hi,
                                             _ptr(codes), _ptr(sf), _ptr(g), _ptr(m), _ptr(l), _stream(s)))
     return codes, sf, g, m, l
@@ -502,8 +540,11 @@ def softmax_quantize_mma(s: torch.Tensor, causal: bool = False, q_offset: int = 
 
 def rows_divide(x: torch.Tensor, l: torch.Tensor) -> torch.Tensor:
     """In place: x[r, :] /= l[r] for x float32 [..., cols] viewed as rows."""
-    _cuda(x, "x"), _cuda(l, "l")
+    _cuda(x, "x")
+    if x.dtype != torch.float32:
+        raise TypeError("x must be float32")
     cols = x.shape[-1]
+    _out(l, "l", torch.float32, x.numel() // max(cols, 1))
     _check(lib().nvfp4_rows_divide(_ptr(x), _ptr(l), x.numel() // max(cols, 1), cols, _stream(x)))
     return x
 

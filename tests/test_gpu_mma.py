@@ -137,7 +137,7 @@ def test_gemm_nt_poisoned_block_gives_nan_row_only():
 
 def test_gemm_nt_zero_k_and_errors():
     z = torch.empty((4, 0), dtype=torch.uint8, device="cuda")
-    sf = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    sf = torch.zeros(4096, dtype=torch.uint8, device="cuda")    # room for every shape below: the C statuses are tested
     g = torch.ones(1, device="cuda")
     d = nv.gemm_nt(z, sf, g, torch.empty((8, 0), dtype=torch.uint8, device="cuda"), sf, g)
     assert d.shape == (4, 8) and not d.any()
