@@ -31,8 +31,22 @@ try:
     print("no error")
 except nv.NVFP4Error as e:
     print("status", e.status)
+k = torch.randn(1, 2, 64, 32, device="cuda").to(torch.bfloat16)
+nv.kv_mixed(k)                                   # finite: no error
+k[0, 1, 30, 3] = float("inf")                    # a middle token
+try:
+    nv.kv_mixed(k)
+    print("kv no error")
+except nv.NVFP4Error as e:
+    print("kv status", e.status)
+try:
+    nv.quantize_dequantize(x)
+    print("fused no error")
+except nv.NVFP4Error as e:
+    print("fused status", e.status)
 """, NVFP4_CHECKED="1")
     assert "finite ok True" in out and "status -5" in out, out
+    assert "kv status -5" in out and "fused status -5" in out, out
 
 
 def test_injected_launch_error_is_reported_and_recoverable():
