@@ -684,6 +684,192 @@ def run_msda_reference(args, rank, world):
 # ------------------------------------------------------------------------------------------------
 # FP4 attention (ScaleSearchAttention numerics, unfused)
 # ------------------------------------------------------------------------------------------------
+KVD_METRIC = ("KV-cache decode: tokens appended per second (16-token groups of new keys quantized into the "
+              "NVFP4 middle of the cache, 8 heads x 128)")
+
+
+def kvd_config(args, n_new):
+    return {
+        "workload": f"kv_decode (cache = kv_bf16 keys [1,8,32768,128] with the prefill's tensor scale; {n_new} newly "
+                    f"decoded keys [8,{n_new},128] BF16, N(0,1) + the same channel bias, seed 4)",
+        "window": [args.f_lo, args.f_hi],
+        "step": "one 16-token group of new keys, Hadamard-rotated and ScaleSearch-quantized with the prefill's "
+                "tensor scale into the next 16 rows of the NVFP4 middle (nvfp4_kv_append)",
+        "l2": "each group's 32 KB of keys is read once; latency-bound (1024 blocks per launch)",
+        "heads": 8, "head_dim": 128, "group": 16,
+    }
+
+
+def run_kv_decode(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    k = W.kv_bf16(dev)
+    B, H, T, D = k.shape
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    e2e_steps = max(0, args.e2e_steps) if not args.no_e2e else 0
+    n_new = 16 * (steps + warmup + e2e_steps + 9)
+    cap = (T - 32) + n_new
+    g = nv.kv_gscale(k)                                   # the prefill's tensor scale (rotated middle)
+    codes = torch.empty((H, cap, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((H, cap, D // 16), dtype=torch.uint8, device=dev)
+    nv.kv_append(k[0], 16, T - 32, g, codes, scales, 0)   # prefill of the middle (not timed)
+    new = W.kv_decode_keys(dev, n_new)
+    stream = torch.cuda.current_stream(dev)
+    group = [0]
+
+    def step():
+        i = group[0]
+        nv.kv_append(new, 16 * i, 16, g, codes, scales, (T - 32) + 16 * i, f_lo=args.f_lo, f_hi=args.f_hi)
+        group[0] += 1
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    call_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    eager_ms = elapsed_ms
+    graph_used = False
+    if world == 1 and not args.no_graph and steps >= 8:
+        # a decode loop runs as a CUDA graph: 8 consecutive group appends captured once and replayed, every
+        # replay quantizing the same 8 groups into the same rows again (the same work per group)
+        base = group[0]
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+
+        def eight():
+            for j in range(8):
+                nv.kv_append(new, 16 * (base + j), 16, g, codes, scales, (T - 32) + 16 * (base + j),
+                             f_lo=args.f_lo, f_hi=args.f_hi)
+
+        with torch.cuda.stream(side):
+            eight()
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=side):
+            eight()
+        cg.replay()
+        torch.cuda.synchronize()
+        ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ga.record(stream)
+        for _ in range(steps // 8):
+            cg.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ga.elapsed_time(gb) * steps / (8 * (steps // 8))   # per `steps` groups
+        del cg
+        group[0] += 8
+        if graph_ms < elapsed_ms:
+            elapsed_ms, graph_used = graph_ms, True
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    peak, psrc = peaks()
+    nbytes = 16 * H * D * 2 + 16 * H * (D // 2) + 16 * H * (D // 16)
+    launch_ms = elapsed_ms / steps if graph_used else call_ms     # one launch per group
+    line = {
+        "metric": KVD_METRIC, "value": world * 16 * steps / (elapsed_ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": elapsed_ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, nvfp4 out",
+        "data": SOURCE_NOTE, "config": kvd_config(args, n_new),
+        "roofline": {"bound": "hbm", "kernel": "quantize_search_kernel (KV append, 1024 blocks per launch)",
+                     "achieved": nbytes / (launch_ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": nbytes / (launch_ms * 1e-3) / 1e9 / peak, "traffic": None, "peak_source": psrc,
+                     "bytes_per_launch": nbytes,
+                     "note": "latency-bound: one block per thread on 4 CTAs; the bytes are far below HBM's"},
+        "gpu_launches": steps,
+        "clocks": clocks,
+        "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps},
+    }
+    if e2e_steps > 0:
+        # every step: the group's new keys from pinned host memory, the append, and the group's codes and
+        # scales read back
+        hk = torch.empty((H, 16 * e2e_steps, D), dtype=torch.bfloat16, pin_memory=True)
+        hk.copy_(new[:, 16 * group[0]:16 * (group[0] + e2e_steps)])
+        dk = torch.empty((H, 16, D), dtype=torch.bfloat16, device=dev)
+        hc = torch.empty((H, 16, D // 2), dtype=torch.uint8, pin_memory=True)
+        hs = torch.empty((H, 16, D // 16), dtype=torch.uint8, pin_memory=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for j in range(e2e_steps):
+            row = (T - 32) + 16 * group[0]
+            dk.copy_(hk[:, 16 * j:16 * (j + 1)], non_blocking=True)
+            nv.kv_append(dk, 0, 16, g, codes, scales, row, f_lo=args.f_lo, f_hi=args.f_hi)
+            hc.copy_(codes[:, row:row + 16], non_blocking=True)
+            hs.copy_(scales[:, row:row + 16], non_blocking=True)
+            group[0] += 1
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * 16 * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": 16 * H * D * 2, "d2h_bytes_per_step": 16 * H * (D // 2 + D // 16)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = kvd_oracle_baseline(args)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def kvd_oracle_baseline(args, groups=20):
+    """The oracle's append of `groups` 16-token groups (single-threaded C), as tokens/s."""
+    import numpy as np
+    import torch
+    from nvfp4_block_scaled_11_b200 import workloads as W
+    from oracle import oracle as O
+    new = W.kv_decode_keys("cpu", 16 * groups).view(torch.int16).numpy().view(np.uint16)
+    H, _, D = new.shape
+    codes = np.zeros((H, 16 * groups, D // 2), np.uint8)
+    scales = np.zeros((H, 16 * groups, D // 16), np.uint8)
+    g = 0.0015   # a tensor scale of the prefill's magnitude (the oracle's cost does not depend on its value)
+    t = time.perf_counter()
+    for i in range(groups):
+        O.kv_append(new, 16 * i, 16, g, codes, scales, 16 * i, 1, args.f_lo, args.f_hi)
+    el = time.perf_counter() - t
+    return {"value": 16 * groups / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{groups} groups of 16 new keys x 8 heads, oracle kv_append (C, 1 thread), {el:.2f} s"}
+
+
+def run_kvd_reference(args, rank, world):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        kvd_oracle_baseline(args, groups=4)
+    cb = kvd_oracle_baseline(args, groups=max(4, min(200, 4 * max(1, args.steps))))
+    line = {
+        "impl": "reference", "metric": KVD_METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 16e3 / cb["value"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, nvfp4 out", "data": SOURCE_NOTE,
+        "config": kvd_config(args, 16 * max(1, args.steps)), "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 ATTN_METRIC = "FP4 attention TFLOP/s (4*H*Tq*Tk*D per step; NVFP4 Q K^T and P V^T on the tensor cores)"
 
 
@@ -924,6 +1110,8 @@ def main():
             run_msda_reference(args, rank, world)
         elif args.workload == "attn_nvfp4":
             run_attn_reference(args, rank, world)
+        elif args.workload == "kv_decode":
+            run_kvd_reference(args, rank, world)
         else:
             run_reference(args, rank, world)
         return
@@ -949,6 +1137,9 @@ def main():
         return
     if args.workload == "attn_nvfp4":
         run_attn(args, rank, world, dev)
+        return
+    if args.workload == "kv_decode":
+        run_kv_decode(args, rank, world, dev)
         return
     w = W.make(args.workload, dev, args.scale, shard=rank)
     x = w.x.contiguous()

@@ -124,6 +124,20 @@ def msda_inputs(device="cpu", nq: int = 10000, bs: int = 6, heads: int = 8, poin
     return loc.contiguous(), w.contiguous()
 
 
+def kv_decode_keys(device="cpu", n: int = 4096, heads: int = 8, head_dim: int = 128) -> torch.Tensor:
+    """Keys of n newly decoded tokens for the `kv_bf16` cache, [heads, n, head_dim] BF16: the same recipe
+    (N(0,1) plus the bias of the same 4 channels, from seed 2's channel draw) with their own seed, 4."""
+    g = _gen(4, device)
+    k = torch.randn((heads, n, head_dim), generator=g, device=device, dtype=torch.float32)
+    gc = torch.Generator(device="cpu")
+    gc.manual_seed(2)
+    chans = torch.randperm(head_dim, generator=gc)[:4]
+    bias = torch.randn((4,), generator=gc) * math.sqrt(2.0)
+    for c, b in zip(chans.tolist(), bias.tolist()):
+        k[..., c] += b
+    return k.to(torch.bfloat16).contiguous()
+
+
 def attn_inputs(device="cpu", Tq: int = 2048, scale: float = 1.0):
     """FP4-attention inputs over the KV-cache keys: q [8, Tq, 128] ~ N(0,1) (seed 21), k = kv_bf16's keys
     [8, 32768, 128] (seed 2), v [8, 32768, 128] ~ N(0,1) (seed 22), all BF16; `scale` shrinks the tokens."""
