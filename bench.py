@@ -791,11 +791,12 @@ def run_kv_decode(args, rank, world, dev):
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": elapsed_ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, nvfp4 out",
         "data": SOURCE_NOTE, "config": kvd_config(args, n_new),
-        "roofline": {"bound": "hbm", "kernel": "quantize_search_kernel (KV append, 1024 blocks per launch)",
+        "roofline": {"bound": "hbm", "kernel": "quantize_lanes_kernel (KV append, 1024 blocks per launch)",
                      "achieved": nbytes / (launch_ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": nbytes / (launch_ms * 1e-3) / 1e9 / peak, "traffic": None, "peak_source": psrc,
                      "bytes_per_launch": nbytes,
-                     "note": "latency-bound: one block per thread on 4 CTAs; the bytes are far below HBM's"},
+                     "note": "latency-bound: a half warp per block (one offset per lane) on 64 CTAs, one "
+                             "block's load-search-store chain per launch; the bytes are far below HBM's"},
         "gpu_launches": steps,
         "clocks": clocks,
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps},

@@ -65,6 +65,15 @@ const char* nvfp4_status_str(int status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int nvfp4_version(void);
 
+/* Launch policy of every ScaleSearch quantize (nvfp4_quantize*, the KV calls, nvfp4_quantize_mma_t):
+ * a launch of at most `limit` blocks whose window has at most 32 offsets runs the lane-group search
+ * (a half warp or a warp per block, one offset per lane, the definition scored directly), a larger
+ * one the thread-per-block certified search.  Both write the same bytes; the choice only moves time.
+ * max_blocks >= 0 sets the process-wide limit and returns the previous one; -1 returns the current
+ * limit unchanged; anything else returns NVFP4_ERR_ARG.  Host only (no device call); the default is
+ * the crossover measured on B200.  The pages have no counterpart: it is a launch-shape choice. */
+int64_t nvfp4_lane_search_limit(int64_t max_blocks);
+
 /* Tensor amax (the FP32 per-tensor scale's input; NVFP4 page, second-level FP32 scale).
  * x: n elements of `dtype`.  d_amax: one device float, overwritten with max |x_i| (NaN if any x_i is
  * NaN, else Inf if any is infinite; 0 for n == 0).  n need not be a multiple of 16. */

@@ -18,7 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "kv_mixed_dequantize", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
-    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4",
+    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "lane_search_limit",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -32,6 +32,7 @@ _P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _SIGS = {
     "nvfp4_status_str": (ctypes.c_char_p, [_I]),
     "nvfp4_version": (_I, []),
+    "nvfp4_lane_search_limit": (_I64, [_I64]),
     "nvfp4_tensor_amax": (_I, [_P, _I64, _I, _P, _P]),
     "nvfp4_global_scale": (_I, [_P, _P, _P]),
     "nvfp4_quantize": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P]),
@@ -96,6 +97,16 @@ def status_str(status: int) -> str:
 def _check(rc: int) -> None:
     if rc != 0:
         raise NVFP4Error(rc)
+
+
+def lane_search_limit(max_blocks: int | None = None) -> int:
+    """Launch policy of the ScaleSearch quantizers: launches of at most this many blocks (windows of at
+    most 32 offsets) run the lane-group search, larger ones the thread-per-block search (same bytes).
+    With `max_blocks` set, installs it and returns the previous limit; without, returns the current one."""
+    rc = lib().nvfp4_lane_search_limit(-1 if max_blocks is None else int(max_blocks))
+    if rc < 0 and max_blocks is not None and max_blocks < 0:
+        raise NVFP4Error(int(rc))
+    return int(rc)
 
 
 def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:

@@ -185,7 +185,7 @@ __device__ __forceinline__ float softmax_row_blocks(const QuantParams& p, const 
       // the whole round lies past the last allowed key: every block is zero, which quantizes to scale 0
       // and zero codes (what the full path computes for it), without exp or search
       const u64 zero[8] = {0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull, 0ull};
-      write_block<SRC_LINEAR, false>(p, row * bpr + j, zero, tab, 0, -128, 0.0f, false, 0.0f);
+      write_block<SRC_LINEAR, false>(p, row * bpr + j, zero, TableScales{tab}, 0, -128, 0.0f, false, 0.0f);
     } else if (j < je) {
       float x[16];
       softmax_block(sr, j, m, lim, v8, x);

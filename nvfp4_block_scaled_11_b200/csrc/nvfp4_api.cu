@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <initializer_list>
 #include <mutex>
 
@@ -122,9 +123,33 @@ void launch_search(const QuantParams& p, cudaStream_t s) {
   else quantize_search_kernel<DT, MODE, ROT, NC, false><<<grid, 256, 0, s>>>(p);
 }
 
+// Launches of at most this many blocks (and windows of at most 32 offsets) take the lane-group search:
+// below it a thread-per-block launch leaves SMs idle and lasts one thread's chain (crossover measured).
+constexpr int64_t kLaneSearchDefaultLimit = 16384;
+std::atomic<int64_t> g_lane_limit{kLaneSearchDefaultLimit};
+
+template <int DT, int MODE, bool ROT, int G>
+void launch_lanes(const QuantParams& p, cudaStream_t s) {
+  const int grid = (int)((p.nblocks * G + 255) / 256);
+  if constexpr ((MODE == SRC_LINEAR && !ROT) || MODE == SRC_KV) {
+    if (p.deq_out) {
+      quantize_lanes_kernel<DT, MODE, ROT, G, false, DT><<<grid, 256, 0, s>>>(p);
+      return;
+    }
+  }
+  if (p.block_sse) quantize_lanes_kernel<DT, MODE, ROT, G, true><<<grid, 256, 0, s>>>(p);
+  else quantize_lanes_kernel<DT, MODE, ROT, G, false><<<grid, 256, 0, s>>>(p);
+}
+
 template <int DT, int MODE, bool ROT>
 void launch_quantize_dt(const QuantParams& p, cudaStream_t s) {
-  switch (p.f_hi - p.f_lo + 1) {
+  const int nc = p.f_hi - p.f_lo + 1;
+  if (nc <= 32 && p.nblocks <= g_lane_limit.load(std::memory_order_relaxed)) {
+    if (nc <= 16) launch_lanes<DT, MODE, ROT, 16>(p, s);
+    else launch_lanes<DT, MODE, ROT, 32>(p, s);
+    return;
+  }
+  switch (nc) {
     case 1: launch_search<DT, MODE, ROT, 1>(p, s); break;
     case 9: launch_search<DT, MODE, ROT, 9>(p, s); break;
     case 17: launch_search<DT, MODE, ROT, 17>(p, s); break;
@@ -274,6 +299,12 @@ const char* nvfp4_status_str(int status) {
 }
 
 int nvfp4_version(void) { return 100; }
+
+int64_t nvfp4_lane_search_limit(int64_t max_blocks) {
+  if (max_blocks < -1) return NVFP4_ERR_ARG;
+  if (max_blocks == -1) return g_lane_limit.load();
+  return g_lane_limit.exchange(max_blocks);
+}
 
 int nvfp4_tensor_amax(const void* x, int64_t n, int dtype, float* d_amax, void* stream) {
   if (!dtype_ok(dtype) || d_amax == nullptr || (n > 0 && x == nullptr)) return NVFP4_ERR_ARG;

@@ -338,9 +338,22 @@ __device__ __forceinline__ void maybe_rotate(u64 (&x2)[8]) {
   if (ROT) fwht16_x2(x2);
 }
 
+// Where write_block finds the chosen scale code's r (to encode) and d (to dequantize): the launch's
+// candidate table, or one lane's own candidate (d of any code computed as the table would hold it).
+struct TableScales {
+  const CandEntry* tab;
+  __device__ __forceinline__ float r(int c) const { return tab[c].r; }
+  __device__ __forceinline__ float d(int c) const { return tab[c].d; }
+};
+struct LaneScales {
+  float rw, g;  // r of the lane's candidate (the only code it encodes with); the tensor scale
+  __device__ __forceinline__ float r(int) const { return rw; }
+  __device__ __forceinline__ float d(int c) const { return __fmul_rn(e4m3_value((uint32_t)c), g); }
+};
+
 // DEQ >= 0 (a dtype): also write the block's dequantized values to p.deq_out (fused round trip).
-template <int MODE, bool WANT_SSE, int DEQ = -1>
-__device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, const u64 (&x2)[8], const CandEntry* tab,
+template <int MODE, bool WANT_SSE, int DEQ = -1, class SC>
+__device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, const u64 (&x2)[8], const SC& sc,
                                             int c0, int fstar, float sse, bool poisoned, float amax_b) {
   uint32_t wlo = 0u, whi = 0u;
   int scale;
@@ -349,7 +362,7 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
     sse = __uint_as_float(0x7FFFFFFFu);
   } else if (fstar != -128) {
     scale = c0 + fstar;
-    encode_pairs(x2, tab[scale].r, wlo, whi);
+    encode_pairs(x2, sc.r(scale), wlo, whi);
   } else {
     // all-zero block or no usable candidate: sign-only zero codes, scale 0, sse = sum of x^2
     scale = 0;
@@ -374,9 +387,9 @@ __device__ __forceinline__ void write_block(const QuantParams& p, int64_t b, con
   if (p.block_f) p.block_f[ob] = (int8_t)fstar;
   if (WANT_SSE) p.block_sse[ob] = sse;
   if constexpr (DEQ >= 0) {
-    // the table's d of every scale byte 0..127 is fl(E4M3(c) * g), the dequantize kernel's step
+    // d of every scale byte 0..127 is fl(E4M3(c) * g), the dequantize kernel's step
     constexpr int OS = DEQ == DT_F32 ? 4 : 2;
-    store_dequantized<DEQ>(p.deq_out + 16 * OS * ob, wlo, whi, tab[scale].d, p.deq_v8 != 0);
+    store_dequantized<DEQ>(p.deq_out + 16 * OS * ob, wlo, whi, sc.d(scale), p.deq_v8 != 0);
   }
 }
 
@@ -401,7 +414,7 @@ __device__ __forceinline__ bool quantize_block_fast(const QuantParams& p, const 
       return true;
     }
   }
-  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, TableScales{tab}, c0, fstar, sse, poisoned, amax_b);
   return false;
 }
 
@@ -421,7 +434,7 @@ __device__ __forceinline__ void quantize_block_def_x2(const QuantParams& p, cons
     for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
     search_def(x, c0, p.f_lo, p.f_hi, tab, fstar, sse);
   }
-  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, tab, c0, fstar, sse, poisoned, amax_b);
+  write_block<MODE, WANT_SSE, DEQ>(p, b, x2, TableScales{tab}, c0, fstar, sse, poisoned, amax_b);
 }
 
 // First element of block b (linear and KV modes: the 16 elements are contiguous).
@@ -534,6 +547,53 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   if constexpr (NC > 1) {
     if (dcount) flush();
   }
+}
+
+// Small launches (a decode step's few thousand blocks): a thread per block leaves most SMs idle and the
+// launch lasts one thread's long chain (table build, barrier, nine candidates scored in turn).  Here a
+// group of G lanes takes one block: every lane loads the whole block (one transaction per group),
+// derives c0 itself and scores one offset, f_lo + j, with the definition; the group's smallest
+// (SSE, visiting rank) wins, rank 0, 1, 2, 3, ... for f = 0, -1, +1, -2, ..., which is the definition's
+// "first strictly smaller SSE in that order".  The winner lane writes the block; when no candidate is
+// usable (or the block is zero or poisoned), lane 0 does.  Needs f_hi - f_lo < G.
+template <int DT, int MODE, bool ROT, int G, bool WANT_SSE, int DEQ = -1>
+__global__ void __launch_bounds__(256) quantize_lanes_kernel(QuantParams p) {
+  static_assert(G == 16 || G == 32, "a block group is a half warp or a warp");
+  const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
+  if (b >= p.nblocks) return;   // whole groups leave together
+  const int j = threadIdx.x & (G - 1);
+  const unsigned gmask = G == 32 ? 0xFFFFFFFFu : (0xFFFFu << (threadIdx.x & 16));
+  u64 x2[8];
+  load_block_pairs<DT, MODE>(p, b, p.v8 != 0, x2);
+  float g = *p.g_src;
+  if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
+  const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
+  maybe_rotate<ROT>(x2);
+  const float amax_b = block_amax_nan(x2);
+  const bool poisoned = g_bad || !(amax_b <= FLT_MAX);
+  const int f = p.f_lo + j;
+  int c0 = 0;
+  float r = 0.0f, s = 0.0f;
+  u64 key = ~0ull;
+  if (!poisoned && amax_b != 0.0f) {
+    c0 = c0_exact(amax_b, g);
+    const int c = c0 + f;
+    if (f <= p.f_hi && c >= 1 && c <= 126) {
+      const float d = __fmul_rn(e4m3_value((uint32_t)c), g);
+      r = __frcp_rn(d);
+      if (d != 0.0f && fabsf(r) <= FLT_MAX) {
+        s = block_sse_def_pairs(x2, d, r);   // never NaN: x finite, v d finite
+        const uint32_t rank = f < 0 ? 2u * (uint32_t)(-f) - 1u : 2u * (uint32_t)f;
+        key = ((u64)__float_as_uint(s) << 8) | rank;
+      }
+    }
+  }
+  u64 kmin = key;
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(gmask, kmin, o));
+  const bool found = kmin != ~0ull;
+  if (found ? key == kmin : j == 0)
+    write_block<MODE, WANT_SSE, DEQ>(p, b, x2, LaneScales{r, g}, c0, found ? f : -128, s, poisoned, amax_b);
 }
 
 }  // namespace nvfp4
