@@ -65,14 +65,19 @@ const char* nvfp4_status_str(int status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int nvfp4_version(void);
 
-/* Launch policy of every ScaleSearch quantize (nvfp4_quantize*, the KV calls, nvfp4_quantize_mma_t):
- * a launch of at most `limit` blocks whose window has at most 32 offsets runs the lane-group search
- * (a half warp or a warp per block, one offset per lane, the definition scored directly), a larger
- * one the thread-per-block certified search.  Both write the same bytes; the choice only moves time.
- * max_blocks >= 0 sets the process-wide limit and returns the previous one; -1 returns the current
- * limit unchanged; anything else returns NVFP4_ERR_ARG.  Host only (no device call); the default is
- * the crossover measured on B200.  The pages have no counterpart: it is a launch-shape choice. */
-int64_t nvfp4_lane_search_limit(int64_t max_blocks);
+/* Launch policy of every ScaleSearch quantize (nvfp4_quantize*, the KV calls, nvfp4_quantize_mma_t).
+ * A launch of n blocks whose window has at most 32 offsets takes the first shape that fits:
+ *   n * G1 <= lane1_max:  G1 = 16 lanes per block (windows up to 16 offsets) or 32, one offset per lane,
+ *                         each scored with the definition, the winner found by a shuffle reduction;
+ *   n * G2 <= lanes_max:  G2 = 4 lanes per block with 3 offsets each (up to 12 offsets) or 8 with 4;
+ *   otherwise:            a thread per block with the certified fast score.
+ * The bounds count threads (blocks x lanes per block).  Wider windows always take a thread per block.
+ * Every shape writes the same bytes; the choice only moves time (defaults 65536 and 393216 threads:
+ * the crossovers measured on B200).  A bound >= 0 is installed, -1 keeps the current one; the previous
+ * bounds are stored through old_lane1_max / old_lanes_max when those are not NULL (host pointers).
+ * Process-wide, host only (no device call).  Returns NVFP4_OK, or NVFP4_ERR_ARG for a bound below -1.
+ * The pages have no counterpart: it is a launch-shape choice. */
+int nvfp4_search_policy(int64_t lane1_max, int64_t lanes_max, int64_t* old_lane1_max, int64_t* old_lanes_max);
 
 /* Tensor amax (the FP32 per-tensor scale's input; NVFP4 page, second-level FP32 scale).
  * x: n elements of `dtype`.  d_amax: one device float, overwritten with max |x_i| (NaN if any x_i is

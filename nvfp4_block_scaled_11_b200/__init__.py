@@ -18,7 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "kv_mixed_dequantize", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
-    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "lane_search_limit",
+    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "search_policy",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -32,7 +32,7 @@ _P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _SIGS = {
     "nvfp4_status_str": (ctypes.c_char_p, [_I]),
     "nvfp4_version": (_I, []),
-    "nvfp4_lane_search_limit": (_I64, [_I64]),
+    "nvfp4_search_policy": (_I, [_I64, _I64, _P, _P]),
     "nvfp4_tensor_amax": (_I, [_P, _I64, _I, _P, _P]),
     "nvfp4_global_scale": (_I, [_P, _P, _P]),
     "nvfp4_quantize": (_I, [_P, _I64, _I, _I, _I, _I, _P, _P, _P, _P]),
@@ -99,14 +99,15 @@ def _check(rc: int) -> None:
         raise NVFP4Error(rc)
 
 
-def lane_search_limit(max_blocks: int | None = None) -> int:
-    """Launch policy of the ScaleSearch quantizers: launches of at most this many blocks (windows of at
-    most 32 offsets) run the lane-group search, larger ones the thread-per-block search (same bytes).
-    With `max_blocks` set, installs it and returns the previous limit; without, returns the current one."""
-    rc = lib().nvfp4_lane_search_limit(-1 if max_blocks is None else int(max_blocks))
-    if rc < 0 and max_blocks is not None and max_blocks < 0:
-        raise NVFP4Error(int(rc))
-    return int(rc)
+def search_policy(lane1_max: int | None = None, lanes_max: int | None = None) -> tuple[int, int]:
+    """Launch policy of the ScaleSearch quantizers (windows of at most 32 offsets), bounds in threads
+    (blocks x lanes per block): up to `lane1_max`, one offset per lane (16 or 32 lanes per block); up to
+    `lanes_max`, a few offsets per lane (4 or 8 lanes per block); beyond, a thread per block.  All write
+    the same bytes.  None keeps a bound; returns the previous bounds."""
+    a, b = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().nvfp4_search_policy(-1 if lane1_max is None else int(lane1_max),
+                                     -1 if lanes_max is None else int(lanes_max), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
 
 
 def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:

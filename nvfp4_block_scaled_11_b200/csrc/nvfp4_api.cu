@@ -123,31 +123,44 @@ void launch_search(const QuantParams& p, cudaStream_t s) {
   else quantize_search_kernel<DT, MODE, ROT, NC, false><<<grid, 256, 0, s>>>(p);
 }
 
-// Launches of at most this many blocks (and windows of at most 32 offsets) take the lane-group search:
-// below it a thread-per-block launch leaves SMs idle and lasts one thread's chain (crossover measured).
-constexpr int64_t kLaneSearchDefaultLimit = 16384;
-std::atomic<int64_t> g_lane_limit{kLaneSearchDefaultLimit};
+// Launch shapes of the search (windows of at most 32 offsets; wider ones always take a thread per block),
+// chosen by the threads a lane-group launch would start (blocks x lanes per block): up to g_lane1_max,
+// a half warp / warp per block with one offset per lane (shortest chain); up to g_lanes_max, 4 / 8
+// lanes per block with 3 / 4 offsets each (fewer instructions per block); beyond, a thread per block
+// with the certified fast score.  Defaults: the crossovers measured on B200, which fall at about the
+// same thread counts for both group sizes of a shape.
+constexpr int64_t kLane1DefaultMax = 65536;
+constexpr int64_t kLanesDefaultMax = 393216;
+std::atomic<int64_t> g_lane1_max{kLane1DefaultMax};
+std::atomic<int64_t> g_lanes_max{kLanesDefaultMax};
 
-template <int DT, int MODE, bool ROT, int G>
+template <int DT, int MODE, bool ROT, int G, int CPL>
 void launch_lanes(const QuantParams& p, cudaStream_t s) {
   const int grid = (int)((p.nblocks * G + 255) / 256);
   if constexpr ((MODE == SRC_LINEAR && !ROT) || MODE == SRC_KV) {
     if (p.deq_out) {
-      quantize_lanes_kernel<DT, MODE, ROT, G, false, DT><<<grid, 256, 0, s>>>(p);
+      quantize_lanes_kernel<DT, MODE, ROT, G, CPL, false, DT><<<grid, 256, 0, s>>>(p);
       return;
     }
   }
-  if (p.block_sse) quantize_lanes_kernel<DT, MODE, ROT, G, true><<<grid, 256, 0, s>>>(p);
-  else quantize_lanes_kernel<DT, MODE, ROT, G, false><<<grid, 256, 0, s>>>(p);
+  if (p.block_sse) quantize_lanes_kernel<DT, MODE, ROT, G, CPL, true><<<grid, 256, 0, s>>>(p);
+  else quantize_lanes_kernel<DT, MODE, ROT, G, CPL, false><<<grid, 256, 0, s>>>(p);
 }
 
 template <int DT, int MODE, bool ROT>
 void launch_quantize_dt(const QuantParams& p, cudaStream_t s) {
   const int nc = p.f_hi - p.f_lo + 1;
-  if (nc <= 32 && p.nblocks <= g_lane_limit.load(std::memory_order_relaxed)) {
-    if (nc <= 16) launch_lanes<DT, MODE, ROT, 16>(p, s);
-    else launch_lanes<DT, MODE, ROT, 32>(p, s);
-    return;
+  if (nc <= 32) {   // nblocks < 2^56, so the thread counts fit in int64
+    if (p.nblocks * (nc <= 16 ? 16 : 32) <= g_lane1_max.load(std::memory_order_relaxed)) {
+      if (nc <= 16) launch_lanes<DT, MODE, ROT, 16, 1>(p, s);
+      else launch_lanes<DT, MODE, ROT, 32, 1>(p, s);
+      return;
+    }
+    if (p.nblocks * (nc <= 12 ? 4 : 8) <= g_lanes_max.load(std::memory_order_relaxed)) {
+      if (nc <= 12) launch_lanes<DT, MODE, ROT, 4, 3>(p, s);
+      else launch_lanes<DT, MODE, ROT, 8, 4>(p, s);
+      return;
+    }
   }
   switch (nc) {
     case 1: launch_search<DT, MODE, ROT, 1>(p, s); break;
@@ -300,10 +313,13 @@ const char* nvfp4_status_str(int status) {
 
 int nvfp4_version(void) { return 100; }
 
-int64_t nvfp4_lane_search_limit(int64_t max_blocks) {
-  if (max_blocks < -1) return NVFP4_ERR_ARG;
-  if (max_blocks == -1) return g_lane_limit.load();
-  return g_lane_limit.exchange(max_blocks);
+int nvfp4_search_policy(int64_t lane1_max, int64_t lanes_max, int64_t* old_lane1_max, int64_t* old_lanes_max) {
+  if (lane1_max < -1 || lanes_max < -1) return NVFP4_ERR_ARG;
+  const int64_t a = lane1_max == -1 ? g_lane1_max.load() : g_lane1_max.exchange(lane1_max);
+  const int64_t b = lanes_max == -1 ? g_lanes_max.load() : g_lanes_max.exchange(lanes_max);
+  if (old_lane1_max) *old_lane1_max = a;
+  if (old_lanes_max) *old_lanes_max = b;
+  return NVFP4_OK;
 }
 
 int nvfp4_tensor_amax(const void* x, int64_t n, int dtype, float* d_amax, void* stream) {

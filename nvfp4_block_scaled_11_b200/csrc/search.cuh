@@ -552,17 +552,18 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
 // Small launches (a decode step's few thousand blocks): a thread per block leaves most SMs idle and the
 // launch lasts one thread's long chain (table build, barrier, nine candidates scored in turn).  Here a
 // group of G lanes takes one block: every lane loads the whole block (one transaction per group),
-// derives c0 itself and scores one offset, f_lo + j, with the definition; the group's smallest
-// (SSE, visiting rank) wins, rank 0, 1, 2, 3, ... for f = 0, -1, +1, -2, ..., which is the definition's
-// "first strictly smaller SSE in that order".  The winner lane writes the block; when no candidate is
-// usable (or the block is zero or poisoned), lane 0 does.  Needs f_hi - f_lo < G.
-template <int DT, int MODE, bool ROT, int G, bool WANT_SSE, int DEQ = -1>
+// derives c0 itself and scores the offsets f_lo + j, f_lo + j + G, ... (CPL of them, independent
+// chains) with the definition; the group's smallest (SSE, visiting rank) wins, rank 0, 1, 2, 3, ... for
+// f = 0, -1, +1, -2, ..., which is the definition's "first strictly smaller SSE in that order".  The
+// lane holding the winner writes the block; when no candidate is usable (or the block is zero or
+// poisoned), lane 0 does.  Needs f_hi - f_lo < G * CPL.
+template <int DT, int MODE, bool ROT, int G, int CPL, bool WANT_SSE, int DEQ = -1>
 __global__ void __launch_bounds__(256) quantize_lanes_kernel(QuantParams p) {
-  static_assert(G == 16 || G == 32, "a block group is a half warp or a warp");
+  static_assert(G == 4 || G == 8 || G == 16 || G == 32, "a block group is 4, 8, 16 or 32 lanes");
   const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
   if (b >= p.nblocks) return;   // whole groups leave together
-  const int j = threadIdx.x & (G - 1);
-  const unsigned gmask = G == 32 ? 0xFFFFFFFFu : (0xFFFFu << (threadIdx.x & 16));
+  const int lane = threadIdx.x & 31, j = lane & (G - 1);
+  const unsigned gmask = G == 32 ? 0xFFFFFFFFu : (((1u << G) - 1u) << (lane & ~(G - 1)));
   u64 x2[8];
   load_block_pairs<DT, MODE>(p, b, p.v8 != 0, x2);
   float g = *p.g_src;
@@ -571,20 +572,27 @@ __global__ void __launch_bounds__(256) quantize_lanes_kernel(QuantParams p) {
   maybe_rotate<ROT>(x2);
   const float amax_b = block_amax_nan(x2);
   const bool poisoned = g_bad || !(amax_b <= FLT_MAX);
-  const int f = p.f_lo + j;
-  int c0 = 0;
-  float r = 0.0f, s = 0.0f;
+  int c0 = 0, fw = -128;
+  float rw = 0.0f, sw = 0.0f;
   u64 key = ~0ull;
   if (!poisoned && amax_b != 0.0f) {
     c0 = c0_exact(amax_b, g);
-    const int c = c0 + f;
-    if (f <= p.f_hi && c >= 1 && c <= 126) {
-      const float d = __fmul_rn(e4m3_value((uint32_t)c), g);
-      r = __frcp_rn(d);
-      if (d != 0.0f && fabsf(r) <= FLT_MAX) {
-        s = block_sse_def_pairs(x2, d, r);   // never NaN: x finite, v d finite
-        const uint32_t rank = f < 0 ? 2u * (uint32_t)(-f) - 1u : 2u * (uint32_t)f;
-        key = ((u64)__float_as_uint(s) << 8) | rank;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      // every slot is scored (no branch, so the CPL chains interleave); unusable ones get key ~0
+      const int f = p.f_lo + j + G * i, c = c0 + f;
+      const bool in = f <= p.f_hi && c >= 1 && c <= 126;
+      const float d = in ? __fmul_rn(e4m3_value((uint32_t)c & 0x7Fu), g) : 0.0f;
+      const float r = __frcp_rn(d);
+      const bool ok = d != 0.0f && fabsf(r) <= FLT_MAX;
+      const float s = block_sse_def_pairs(x2, d, ok ? r : 0.0f);   // usable: never NaN (x, v d finite)
+      const uint32_t rank = f < 0 ? 2u * (uint32_t)(-f) - 1u : 2u * (uint32_t)f;
+      const u64 k = ok ? (((u64)__float_as_uint(s) << 8) | rank) : ~0ull;
+      if (k < key) {
+        key = k;
+        rw = r;
+        sw = s;
+        fw = f;
       }
     }
   }
@@ -593,7 +601,7 @@ __global__ void __launch_bounds__(256) quantize_lanes_kernel(QuantParams p) {
   for (int o = G / 2; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(gmask, kmin, o));
   const bool found = kmin != ~0ull;
   if (found ? key == kmin : j == 0)
-    write_block<MODE, WANT_SSE, DEQ>(p, b, x2, LaneScales{r, g}, c0, found ? f : -128, s, poisoned, amax_b);
+    write_block<MODE, WANT_SSE, DEQ>(p, b, x2, LaneScales{rw, g}, c0, found ? fw : -128, sw, poisoned, amax_b);
 }
 
 }  // namespace nvfp4

@@ -106,3 +106,19 @@ def test_size_products_that_overflow_are_rejected(L):
     assert L.nvfp4_hadamard16(fake, huge, 0, fake, 0, None) == -2
     assert L.nvfp4_tensor_amax(fake, huge, 0, fake, None) == -2
     assert L.nvfp4_mxfp4_quantize(fake, huge, 0, fake, fake, None) == -2
+
+
+def test_search_policy_is_host_only_and_restorable():
+    """The launch-policy call touches no device: its defaults, set / restore and argument errors."""
+    default = nv.search_policy()
+    assert default == (65536, 393216)
+    try:
+        assert nv.search_policy(10, 20) == default
+        assert nv.search_policy(None, 30) == (10, 20)
+        assert nv.search_policy() == (10, 30)
+        with pytest.raises(nv.NVFP4Error):
+            nv.search_policy(-5, None)
+        assert nv.search_policy() == (10, 30)
+    finally:
+        nv.search_policy(*default)
+    assert nv.search_policy() == default

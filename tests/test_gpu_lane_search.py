@@ -1,9 +1,8 @@
-"""The two launch shapes of the ScaleSearch quantizers -- the lane-group search (a half warp or a warp
-per block, one offset per lane, small launches) and the thread-per-block certified search -- each
-checked bit-exactly against the oracle on the same inputs, through every source mode that reaches
-them (linear, KV with and without rotation, appended KV rows, transposed columns, fused round trips).
-The launch policy is forced with `lane_search_limit`: 0 sends every launch to the thread-per-block
-kernel, a huge limit sends every eligible launch (windows of at most 32 offsets) to the lane groups."""
+"""The three launch shapes of the ScaleSearch quantizers -- one offset per lane (a half warp or a warp
+per block), a few offsets per lane (4 or 8 lanes per block) and a thread per block (the certified fast
+score) -- each checked bit-exactly against the oracle on the same inputs, through every source mode
+that reaches them (linear, KV with and without rotation, appended KV rows, transposed columns, fused
+round trips).  The shape is forced with `search_policy` (bounds on the block count of each shape)."""
 import contextlib
 
 import numpy as np
@@ -16,17 +15,19 @@ from oracle import oracle as O
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"lanes": 1 << 40, "wide": 0}
+HUGE = 1 << 40
+PATHS = {"lane1": (HUGE, HUGE), "lanes": (0, HUGE), "wide": (0, 0)}
+SHAPES = list(PATHS)
 DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 
 @contextlib.contextmanager
 def path(name):
-    prev = nv.lane_search_limit(PATHS[name])
+    prev = nv.search_policy(*PATHS[name])
     try:
         yield
     finally:
-        nv.lane_search_limit(prev)
+        nv.search_policy(*prev)
 
 
 def _host(t):
@@ -90,7 +91,7 @@ def _check_quantize(x, f_lo, f_hi, gscale_in=None):
     assert same_f32(bs.cpu().numpy(), rbs)
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
+@pytest.mark.parametrize("name", SHAPES)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("window", [(0, 0), (-2, 6), (-8, 8), (-3, 3), (-15, 16), (-20, 20)])
 def test_linear_both_paths(name, dtype, window):
@@ -101,11 +102,11 @@ def test_linear_both_paths(name, dtype, window):
         _check_quantize(sp.cuda(), *window, gscale_in=0.01)
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
-@pytest.mark.parametrize("nblocks", [1, 7, 15, 17, 33, 1003])
+@pytest.mark.parametrize("name", SHAPES)
+@pytest.mark.parametrize("nblocks", [1, 7, 15, 17, 33, 63, 65, 1003])
 def test_ragged_group_counts(name, nblocks):
-    """Launches whose block count leaves a CTA partly empty (16 blocks per CTA for half-warp groups,
-    8 for warp groups)."""
+    """Launches whose block count leaves a CTA partly empty (a 256-thread CTA holds 16 blocks in
+    half-warp groups, 8 in warp groups, 64 in groups of 4 lanes, 32 in groups of 8)."""
     g = torch.Generator().manual_seed(nblocks)
     x = torch.randn(nblocks * 16, generator=g) * 3.0
     with path(name):
@@ -113,7 +114,7 @@ def test_ragged_group_counts(name, nblocks):
             _check_quantize(x.cuda(), *window)
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
+@pytest.mark.parametrize("name", SHAPES)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("window", [(0, 0), (-2, 6), (-8, 8)])
 def test_fused_round_trip_both_paths(name, dtype, window):
@@ -138,7 +139,7 @@ def _u16(t):
     return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
+@pytest.mark.parametrize("name", SHAPES)
 @pytest.mark.parametrize("rotate", [True, False])
 @pytest.mark.parametrize("window", [(-2, 6), (-8, 8), (0, 0)])
 def test_kv_mixed_and_fused_both_paths(name, rotate, window):
@@ -156,7 +157,7 @@ def test_kv_mixed_and_fused_both_paths(name, rotate, window):
         assert np.array_equal(_u16(mid).reshape(-1), rd.reshape(-1))
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
+@pytest.mark.parametrize("name", SHAPES)
 @pytest.mark.parametrize("rotate", [True, False])
 @pytest.mark.parametrize("tile", [False, True])
 def test_kv_append_both_paths(name, rotate, tile):
@@ -186,7 +187,7 @@ def test_kv_append_both_paths(name, rotate, tile):
         assert np.array_equal(scales.cpu().numpy(), rs.reshape(-1))
 
 
-@pytest.mark.parametrize("name", ["lanes", "wide"])
+@pytest.mark.parametrize("name", SHAPES)
 def test_transposed_columns_both_paths(name):
     g = torch.Generator().manual_seed(3)
     x = (torch.randn(2, 48, 40, generator=g) * torch.linspace(0.1, 10, 40)).to(torch.bfloat16)
@@ -199,19 +200,23 @@ def test_transposed_columns_both_paths(name):
     assert np.array_equal(sf.cpu().numpy().reshape(-1), rsf.reshape(-1))
 
 
-def test_limit_boundary_and_default():
-    """A launch of exactly `limit` blocks takes the lane groups, one more block the other kernel; the
-    bytes are the same either way, and the policy call restores what it replaced."""
-    default = nv.lane_search_limit()
-    assert default > 0
+def test_policy_boundaries_and_defaults():
+    """A launch of exactly a bound's thread count takes that shape, one thread less sends it on to the
+    next one; the bytes are the same either way, and the policy call restores what it replaced."""
+    default = nv.search_policy()
+    assert 0 < default[0] <= default[1]
     x = torch.randn(64 * 16, generator=torch.Generator().manual_seed(1)).cuda()
     outs = []
-    for lim in (64, 63):
-        prev = nv.lane_search_limit(lim)
+    for bounds in ((64 * 16, 0), (64 * 16 - 1, 64 * 4), (0, 64 * 4 - 1)):   # 64 blocks, window [-2, 6]
+        prev = nv.search_policy(*bounds)
         try:
             outs.append([t.cpu() for t in nv.quantize_ex(x, -2, 6)])
         finally:
-            assert nv.lane_search_limit(prev) == lim
-    for a, b in zip(*outs):
-        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
-    assert nv.lane_search_limit() == default
+            assert nv.search_policy(*prev) == bounds
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert nv.search_policy() == default
+    with pytest.raises(nv.NVFP4Error):
+        nv.search_policy(-2, 5)
+    assert nv.search_policy() == default
