@@ -219,6 +219,29 @@ int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, in
                     int f_lo, int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
                     int scale_layout, void* stream);
 
+/* One KV append of a batch: the arguments of nvfp4_kv_append (same meaning, layout, alignment and size
+ * rules), as a plain struct so that several appends can be passed at once. */
+typedef struct nvfp4_kv_append_desc {
+  const void* k_bf16;     /* BF16 rows [BH, T, D], device, 16-byte aligned */
+  const float* gscale;    /* device float: this cache's tensor scale */
+  uint8_t* codes;         /* [BH, cap, D/2], device, 8-byte aligned */
+  uint8_t* scales;        /* [BH, cap, D/16], or the tile layout when scale_layout == 1 */
+  int64_t BH, T, first, n, D, cap, t0;
+  int32_t rotate, scale_layout;
+} nvfp4_kv_append_desc;
+
+#define NVFP4_KV_APPEND_BATCH_MAX 64
+
+/* Several KV appends in one launch (e.g. the K and V groups of every layer of a decode step, each
+ * flushing its window into its own cache): descs is a HOST array of `count` descriptors (read before
+ * the call returns; count <= NVFP4_KV_APPEND_BATCH_MAX), all quantized with the window [f_lo, f_hi]
+ * (at most 32 offsets, NVFP4_ERR_ARG otherwise).  Each item writes exactly the bytes nvfp4_kv_append
+ * would; items must not write overlapping outputs.  Every descriptor is validated before anything is
+ * launched (the first failing item's status is returned); items with BH == 0 or n == 0 are skipped.
+ * The launch always takes lane groups (16 or 32 lanes per block while the batch is small, 4 or 8 with
+ * several offsets each beyond nvfp4_search_policy's first bound): it is meant for decode-sized groups. */
+int nvfp4_kv_append_batch(const nvfp4_kv_append_desc* descs, int count, int f_lo, int f_hi, void* stream);
+
 /* ---- Tensor-core consumer ("Search your block floating-point scales!", ScaleSearchAttention: QK^T and
  * PV run as NVFP4 products on the tensor cores with FP32 accumulation) ----
  *

@@ -18,7 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "kv_mixed_dequantize", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
-    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "search_policy",
+    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "search_policy", "kv_append_batch",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -50,6 +50,7 @@ _SIGS = {
     "nvfp4_mxfp4_dequantize": (_I, [_P, _P, _I64, _I, _P, _P]),
     "nvfp4_kv_gscale": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P]),
     "nvfp4_kv_append": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _P]),
+    "nvfp4_kv_append_batch": (_I, [_P, _I, _I, _I, _P]),
     "nvfp4_sf_mma_bytes": (_I64, [_I64, _I64, _I64]),
     "nvfp4_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "nvfp4_quantize_mma_t": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
@@ -469,6 +470,43 @@ def kv_append(k_rows: torch.Tensor, first: int, n: int, gscale: torch.Tensor, co
     _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
     _check(lib().nvfp4_kv_append(_ptr(k_rows), BH, T, first, n, D, int(bool(rotate)), f_lo, f_hi, _ptr(gscale),
                                  _ptr(codes), _ptr(scales), cap, t0, 1 if tile_layout else 0, _stream(k_rows)))
+
+
+class _KvAppendDesc(ctypes.Structure):
+    """nvfp4_kv_append_desc (include/nvfp4.h)."""
+    _fields_ = [("k_bf16", _P), ("gscale", _P), ("codes", _P), ("scales", _P), ("BH", _I64), ("T", _I64),
+                ("first", _I64), ("n", _I64), ("D", _I64), ("cap", _I64), ("t0", _I64),
+                ("rotate", ctypes.c_int32), ("scale_layout", ctypes.c_int32)]
+
+
+KV_APPEND_BATCH_MAX = 64
+
+
+def kv_append_batch(items, f_lo: int = -2, f_hi: int = 6) -> None:
+    """Several kv_append calls in one launch.  `items`: a sequence of tuples
+    (k_rows, first, n, gscale, codes, scales, t0, rotate, tile_layout) with kv_append's meanings; all use
+    the window [f_lo, f_hi] (at most 32 offsets).  Outputs of different items must not overlap."""
+    items = list(items)
+    if len(items) > KV_APPEND_BATCH_MAX:
+        raise ValueError(f"at most {KV_APPEND_BATCH_MAX} items per batch")
+    descs = (_KvAppendDesc * max(len(items), 1))()
+    stream = None
+    for i, (k_rows, first, n, gscale, codes, scales, t0, rotate, tile_layout) in enumerate(items):
+        for t, nm in ((k_rows, "k_rows"), (gscale, "gscale"), (codes, "codes"), (scales, "scales")):
+            _cuda(t, nm)
+        if k_rows.dtype != torch.bfloat16:
+            raise TypeError("k_rows must be bfloat16")
+        T, D = k_rows.shape[-2], k_rows.shape[-1]
+        BH = k_rows.numel() // max(T * D, 1)
+        cap = codes.shape[-2]
+        _out(gscale, "gscale", torch.float32, 1), _out(codes, "codes", torch.uint8, BH * cap * (D // 2))
+        _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
+        descs[i] = _KvAppendDesc(k_rows.data_ptr(), gscale.data_ptr(), codes.data_ptr(), scales.data_ptr(), BH, T,
+                                 first, n, D, cap, t0, int(bool(rotate)), 1 if tile_layout else 0)
+        stream = stream or _stream(k_rows)
+    if not items:
+        return
+    _check(lib().nvfp4_kv_append_batch(ctypes.cast(descs, _P), len(items), f_lo, f_hi, stream))
 
 
 # ---- MXFP4 (comparison format) ----

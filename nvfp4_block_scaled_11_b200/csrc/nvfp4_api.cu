@@ -10,6 +10,7 @@
 
 #include "../../include/nvfp4.h"
 #include "attention.cuh"
+#include "lanes.cuh"
 #include "msda.cuh"
 #include "search.cuh"
 
@@ -243,6 +244,46 @@ int quantize_impl(const void* x, int64_t n, int dtype, int f_lo, int f_hi, const
       return NVFP4_ERR_CUDA;
   }
   return check_finite_sync(gscale_in, s);
+}
+
+// Validation and launch parameters of one KV append (nvfp4_kv_append and each item of the batch call);
+// p.nblocks == 0 when there is nothing to do.
+int kv_append_params(const void* k_bf16, int64_t BH, int64_t T, int64_t first, int64_t n, int64_t D, int f_lo,
+                     int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
+                     int scale_layout, QuantParams& p) {
+  if (!window_ok(f_lo, f_hi) || gscale == nullptr || (scale_layout != 0 && scale_layout != 1)) return NVFP4_ERR_ARG;
+  if (BH < 0 || T < 0 || n < 0 || first < 0 || t0 < 0 || cap < 0 || D <= 0 || D % 16 != 0) return NVFP4_ERR_SIZE;
+  if (first > T - n || t0 > cap - n) return NVFP4_ERR_SIZE;
+  if (checked_prod({BH, T, D}) < 0 || checked_prod({BH, cap, D}) < 0) return NVFP4_ERR_SIZE;
+  if (scale_layout == 1 && BH * cap * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
+  if (BH * n * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
+  p = QuantParams{};
+  if (BH == 0 || n == 0) return NVFP4_OK;
+  if (k_bf16 == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
+  if (!aligned(k_bf16, 16) || !aligned(codes, 8) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
+  p.x = static_cast<const char*>(k_bf16);
+  p.nblocks = BH * n * (D / 16);
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.g_src = gscale;
+  p.g_is_amax = 0;
+  p.codes = codes;
+  p.scales = scales;
+  p.v8 = aligned(k_bf16, 32) ? 1 : 0;
+  p.T = T;
+  p.Tm = n;
+  p.sink = first;
+  p.D = D;
+  p.bpr = D / 16;
+  p.out_cap = cap;
+  p.out_t0 = t0;
+  if (scale_layout == 1) {
+    p.sf_bpr = (uint32_t)(D / 16);
+    p.sf_rows = (uint32_t)cap;
+    p.sf_ctiles = (uint32_t)((D / 16 + 3) / 4);
+    p.sf_mat_bytes = ((cap + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
+  }
+  return NVFP4_OK;
 }
 
 // Validation shared by the two deformable-attention entry points; fills the level fields of p.
@@ -726,42 +767,56 @@ int nvfp4_kv_gscale(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t
 int nvfp4_kv_append(const void* k_bf16, int64_t BH, int64_t T, int64_t first, int64_t n, int64_t D, int rotate,
                     int f_lo, int f_hi, const float* gscale, uint8_t* codes, uint8_t* scales, int64_t cap, int64_t t0,
                     int scale_layout, void* stream) {
-  if (!window_ok(f_lo, f_hi) || gscale == nullptr || (scale_layout != 0 && scale_layout != 1)) return NVFP4_ERR_ARG;
-  if (BH < 0 || T < 0 || n < 0 || first < 0 || t0 < 0 || cap < 0 || D <= 0 || D % 16 != 0) return NVFP4_ERR_SIZE;
-  if (first > T - n || t0 > cap - n) return NVFP4_ERR_SIZE;
-  if (checked_prod({BH, T, D}) < 0 || checked_prod({BH, cap, D}) < 0) return NVFP4_ERR_SIZE;
-  if (scale_layout == 1 && BH * cap * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;
-  if (BH * n * (D / 16) >= (int64_t(1) << 32)) return NVFP4_ERR_SIZE;  // KV block indices are split in 32 bits
-  if (BH == 0 || n == 0) return NVFP4_OK;
-  if (k_bf16 == nullptr || codes == nullptr || scales == nullptr) return NVFP4_ERR_ARG;
-  if (!aligned(k_bf16, 16) || !aligned(codes, 8) || !aligned(gscale, 4)) return NVFP4_ERR_ALIGN;
   QuantParams p{};
-  p.x = static_cast<const char*>(k_bf16);
-  p.nblocks = BH * n * (D / 16);
-  p.f_lo = f_lo;
-  p.f_hi = f_hi;
-  p.g_src = gscale;
-  p.g_is_amax = 0;
-  p.codes = codes;
-  p.scales = scales;
-  p.v8 = aligned(k_bf16, 32) ? 1 : 0;
-  p.T = T;
-  p.Tm = n;
-  p.sink = first;
-  p.D = D;
-  p.bpr = D / 16;
-  p.out_cap = cap;
-  p.out_t0 = t0;
-  if (scale_layout == 1) {
-    p.sf_bpr = (uint32_t)(D / 16);
-    p.sf_rows = (uint32_t)cap;
-    p.sf_ctiles = (uint32_t)((D / 16 + 3) / 4);
-    p.sf_mat_bytes = ((cap + 127) / 128) * 128 * (int64_t)p.sf_ctiles * 4;
-  }
+  if (int rc = kv_append_params(k_bf16, BH, T, first, n, D, f_lo, f_hi, gscale, codes, scales, cap, t0, scale_layout, p))
+    return rc;
+  if (p.nblocks == 0) return NVFP4_OK;
   cudaStream_t s = S(stream);
   const int rc = rotate ? launch_quantize_t<SRC_KV, true>(DT_BF16, p, s) : launch_quantize_t<SRC_KV, false>(DT_BF16, p, s);
   if (rc) return rc;
   return check_finite_sync(gscale, s);
+}
+
+int nvfp4_kv_append_batch(const nvfp4_kv_append_desc* descs, int count, int f_lo, int f_hi, void* stream) {
+  if (count < 0 || count > NVFP4_KV_APPEND_BATCH_MAX || (count > 0 && descs == nullptr)) return NVFP4_ERR_ARG;
+  if (!window_ok(f_lo, f_hi) || f_hi - f_lo + 1 > 32) return NVFP4_ERR_ARG;
+  static_assert(NVFP4_KV_APPEND_BATCH_MAX == kKvBatchMax, "batch bound");
+  KvBatchParams bp{};
+  int m = 0;
+  int64_t total = 0;
+  for (int k = 0; k < count; ++k) {
+    const nvfp4_kv_append_desc& d = descs[k];
+    QuantParams p{};
+    if (d.rotate != 0 && d.rotate != 1) return NVFP4_ERR_ARG;
+    if (int rc = kv_append_params(d.k_bf16, d.BH, d.T, d.first, d.n, d.D, f_lo, f_hi, d.gscale, d.codes, d.scales,
+                                  d.cap, d.t0, d.scale_layout, p))
+      return rc;
+    if (p.nblocks == 0) continue;
+    bp.q[m] = p;
+    bp.rot[m] = d.rotate;
+    bp.start[m] = total;
+    total += p.nblocks;   // each item < 2^32 blocks, at most 64 items
+    ++m;
+  }
+  if (m == 0) return NVFP4_OK;
+  bp.count = m;
+  bp.start[m] = total;
+  cudaStream_t s = S(stream);
+  const int nc = f_hi - f_lo + 1;
+  if (total * (nc <= 16 ? 16 : 32) <= g_lane1_max.load(std::memory_order_relaxed)) {
+    const int grid = (int)((total * (nc <= 16 ? 16 : 32) + 255) / 256);
+    if (nc <= 16) kv_append_batch_kernel<16, 1><<<grid, 256, 0, s>>>(bp);
+    else kv_append_batch_kernel<32, 1><<<grid, 256, 0, s>>>(bp);
+  } else {
+    const int grid = (int)((total * (nc <= 12 ? 4 : 8) + 255) / 256);
+    if (nc <= 12) kv_append_batch_kernel<4, 3><<<grid, 256, 0, s>>>(bp);
+    else kv_append_batch_kernel<8, 4><<<grid, 256, 0, s>>>(bp);
+  }
+  if (int rc = last_error()) return rc;
+  for (int k = 0; k < m; ++k) {
+    if (int rc = check_finite_sync(bp.q[k].g_src, s)) return rc;
+  }
+  return NVFP4_OK;
 }
 
 int nvfp4_kv_mixed(const void* k_bf16, int64_t B, int64_t H, int64_t T, int64_t D, int sink_tokens,

@@ -549,59 +549,4 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   }
 }
 
-// Small launches (a decode step's few thousand blocks): a thread per block leaves most SMs idle and the
-// launch lasts one thread's long chain (table build, barrier, nine candidates scored in turn).  Here a
-// group of G lanes takes one block: every lane loads the whole block (one transaction per group),
-// derives c0 itself and scores the offsets f_lo + j, f_lo + j + G, ... (CPL of them, independent
-// chains) with the definition; the group's smallest (SSE, visiting rank) wins, rank 0, 1, 2, 3, ... for
-// f = 0, -1, +1, -2, ..., which is the definition's "first strictly smaller SSE in that order".  The
-// lane holding the winner writes the block; when no candidate is usable (or the block is zero or
-// poisoned), lane 0 does.  Needs f_hi - f_lo < G * CPL.
-template <int DT, int MODE, bool ROT, int G, int CPL, bool WANT_SSE, int DEQ = -1>
-__global__ void __launch_bounds__(256) quantize_lanes_kernel(QuantParams p) {
-  static_assert(G == 4 || G == 8 || G == 16 || G == 32, "a block group is 4, 8, 16 or 32 lanes");
-  const int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  if (b >= p.nblocks) return;   // whole groups leave together
-  const int lane = threadIdx.x & 31, j = lane & (G - 1);
-  const unsigned gmask = G == 32 ? 0xFFFFFFFFu : (((1u << G) - 1u) << (lane & ~(G - 1)));
-  u64 x2[8];
-  load_block_pairs<DT, MODE>(p, b, p.v8 != 0, x2);
-  float g = *p.g_src;
-  if (p.g_is_amax) g = __fdiv_rn(g, kTensorDiv);
-  const bool g_bad = !(g >= 0.0f) || !(g <= FLT_MAX);
-  maybe_rotate<ROT>(x2);
-  const float amax_b = block_amax_nan(x2);
-  const bool poisoned = g_bad || !(amax_b <= FLT_MAX);
-  int c0 = 0, fw = -128;
-  float rw = 0.0f, sw = 0.0f;
-  u64 key = ~0ull;
-  if (!poisoned && amax_b != 0.0f) {
-    c0 = c0_exact(amax_b, g);
-#pragma unroll
-    for (int i = 0; i < CPL; ++i) {
-      // every slot is scored (no branch, so the CPL chains interleave); unusable ones get key ~0
-      const int f = p.f_lo + j + G * i, c = c0 + f;
-      const bool in = f <= p.f_hi && c >= 1 && c <= 126;
-      const float d = in ? __fmul_rn(e4m3_value((uint32_t)c & 0x7Fu), g) : 0.0f;
-      const float r = __frcp_rn(d);
-      const bool ok = d != 0.0f && fabsf(r) <= FLT_MAX;
-      const float s = block_sse_def_pairs(x2, d, ok ? r : 0.0f);   // usable: never NaN (x, v d finite)
-      const uint32_t rank = f < 0 ? 2u * (uint32_t)(-f) - 1u : 2u * (uint32_t)f;
-      const u64 k = ok ? (((u64)__float_as_uint(s) << 8) | rank) : ~0ull;
-      if (k < key) {
-        key = k;
-        rw = r;
-        sw = s;
-        fw = f;
-      }
-    }
-  }
-  u64 kmin = key;
-#pragma unroll
-  for (int o = G / 2; o > 0; o >>= 1) kmin = min(kmin, __shfl_xor_sync(gmask, kmin, o));
-  const bool found = kmin != ~0ull;
-  if (found ? key == kmin : j == 0)
-    write_block<MODE, WANT_SSE, DEQ>(p, b, x2, LaneScales{rw, g}, c0, found ? fw : -128, sw, poisoned, amax_b);
-}
-
 }  // namespace nvfp4

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import torch
 
-from . import kv_append, kv_gscale, sf_mma_bytes
+from . import KV_APPEND_BATCH_MAX, kv_append, kv_append_batch, kv_gscale, sf_mma_bytes
 
 
 class NVFP4KVCache:
@@ -84,26 +84,67 @@ class NVFP4KVCache:
         """Append tokens K_new[B, H, n, D] (BF16) in order."""
         if not self.prefilled:
             raise RuntimeError("prefill first")
-        r = self.recent
         for i in range(k_new.shape[2]):
-            if self.n_window == 2 * r:
-                self._flush_group()
-            slot = (self.head + self.n_window) % (2 * r)
-            self.window[:, :, slot].copy_(k_new[:, :, i])
-            self.n_window += 1
+            if self._full():
+                kv_append(*self._flush_args()[:7], self.rotate, self.f_lo, self.f_hi, self.tile_layout)
+                self._flushed()
+            self._push(k_new[:, :, i])
 
-    def _flush_group(self) -> None:
+    def _full(self) -> bool:
+        return self.n_window == 2 * self.recent
+
+    def _flush_args(self):
+        """kv_append's arguments for the oldest `recent` window tokens (the contiguous slots head ..
+        head + recent - 1) going to rows n_mid .. of the middle, as a kv_append_batch item."""
         r = self.recent
         if self.n_mid + r > self.capacity:
             raise RuntimeError("NVFP4 cache capacity exceeded")
-        # the oldest `recent` window tokens are the contiguous slots head .. head + recent - 1
-        kv_append(self.window, self.head, r, self.gscale, self.codes, self.scales, self.n_mid, self.rotate,
-                  self.f_lo, self.f_hi, self.tile_layout)
+        return (self.window, self.head, r, self.gscale, self.codes, self.scales, self.n_mid, self.rotate,
+                self.tile_layout)
+
+    def _flushed(self) -> None:
+        r = self.recent
         self.n_mid += r
         self.head = (self.head + r) % (2 * r)
         self.n_window -= r
+
+    def _push(self, token: torch.Tensor) -> None:
+        slot = (self.head + self.n_window) % (2 * self.recent)
+        self.window[:, :, slot].copy_(token)
+        self.n_window += 1
 
     def recent_tokens(self) -> torch.Tensor:
         """The BF16 window in token order, [B, H, n_window, D]."""
         idx = [(self.head + i) % (2 * self.recent) for i in range(self.n_window)]
         return self.window[:, :, idx]
+
+
+def append_many(caches, ks) -> None:
+    """Append one decode step's new tokens to several caches at once (e.g. the K and V caches of every
+    layer): ks[i] [B, H, n, D] (BF16) goes to caches[i], token by token; whenever windows are full, all
+    of them flush together in one nvfp4_kv_append_batch launch (up to 64 per launch) instead of one
+    launch per cache.  The caches must share the ScaleSearch window [f_lo, f_hi]; the result is the
+    same as calling append on each cache."""
+    caches, ks = list(caches), list(ks)
+    if len(caches) != len(ks):
+        raise ValueError("one token tensor per cache")
+    if not caches:
+        return
+    for c in caches:
+        if not c.prefilled:
+            raise RuntimeError("prefill first")
+    if len({(c.f_lo, c.f_hi) for c in caches}) != 1:
+        raise ValueError("caches in one call must share the offset window")
+    n = ks[0].shape[2]
+    if any(k.shape[2] != n for k in ks):
+        raise ValueError("every cache receives the same number of tokens")
+    f_lo, f_hi = caches[0].f_lo, caches[0].f_hi
+    for i in range(n):
+        full = [c for c in caches if c._full()]
+        for j in range(0, len(full), KV_APPEND_BATCH_MAX):
+            part = full[j:j + KV_APPEND_BATCH_MAX]
+            kv_append_batch([c._flush_args() for c in part], f_lo, f_hi)
+            for c in part:
+                c._flushed()
+        for c, k in zip(caches, ks):
+            c._push(k[:, :, i])

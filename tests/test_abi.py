@@ -122,3 +122,22 @@ def test_search_policy_is_host_only_and_restorable():
     finally:
         nv.search_policy(*default)
     assert nv.search_policy() == default
+
+
+def test_kv_append_batch_validates_on_the_host(L):
+    """Argument errors of the batched KV append come back before any device call: too many items, a
+    window wider than 32 offsets, an item with a bad head_dim or rows past the cache."""
+    D = nv._KvAppendDesc
+    fake = 1 << 20   # never dereferenced: every case fails validation first
+    ok = D(fake, fake, fake, fake, 2, 32, 0, 16, 64, 64, 0, 1, 0)
+    arr = (D * 65)(*([ok] * 65))
+    assert L.nvfp4_kv_append_batch(ctypes.cast(arr, ctypes.c_void_p), 65, -2, 6, None) == -1
+    assert L.nvfp4_kv_append_batch(ctypes.cast(arr, ctypes.c_void_p), 1, -16, 16, None) == -1
+    assert L.nvfp4_kv_append_batch(None, 1, -2, 6, None) == -1
+    assert L.nvfp4_kv_append_batch(None, 0, -2, 6, None) == 0
+    bad_d = D(fake, fake, fake, fake, 2, 32, 0, 16, 60, 64, 0, 1, 0)
+    past = D(fake, fake, fake, fake, 2, 32, 0, 16, 64, 64, 50, 1, 0)
+    badrot = D(fake, fake, fake, fake, 2, 32, 0, 16, 64, 64, 0, 2, 0)
+    for d, want in ((bad_d, -2), (past, -2), (badrot, -1)):
+        arr2 = (D * 2)(ok, d)
+        assert L.nvfp4_kv_append_batch(ctypes.cast(arr2, ctypes.c_void_p), 2, -2, 6, None) == want

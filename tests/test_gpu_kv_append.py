@@ -103,3 +103,94 @@ def test_decode_cache_matches_oracle_sequence(tile):
         assert np.array_equal(cache.scales.cpu().numpy().reshape(B * H, 256, D // 16)[:, :n_mid], rs[:, :n_mid])
     assert torch.equal(cache.sink.cpu(), full[:, :, :16])
     assert torch.equal(cache.recent_tokens().cpu(), full[:, :, Tfull - cache.n_window:])
+
+
+def _append_item(k, first, n, g, cap, t0, rotate, tile):
+    """Device buffers (prefilled with 0xAA) and the oracle's expected bytes for one KV append."""
+    BH, T, D = k.shape
+    codes = torch.full((BH, cap, D // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    nsf = nv.sf_mma_bytes(cap, D, BH) if tile else BH * cap * (D // 16)
+    scales = torch.full((nsf,), 0xAA, dtype=torch.uint8, device="cuda")
+    rc = np.full((BH, cap, D // 2), 0xAA, np.uint8)
+    rs = np.full((BH, cap, D // 16), 0xAA, np.uint8)
+    O.kv_append(_u16(k), first, n, g, rc, rs, t0, rotate=int(rotate))
+    if tile:
+        want = np.full(nsf, 0xAA, np.uint8)
+        per = O.sf_mma_bytes(cap, D // 16)
+        for l in range(BH):
+            for r in range(t0, t0 + n):
+                for c in range(D // 16):
+                    want[l * per + O.sf_mma_offset(r, c, D // 16)] = rs[l, r, c]
+    else:
+        want = rs.reshape(-1)
+    item = (k.cuda(), first, n, torch.tensor([g], dtype=torch.float32, device="cuda"), codes, scales, t0, rotate, tile)
+    return item, rc, want
+
+
+@pytest.mark.parametrize("policy", [None, (0, None)])     # small batch: 16 lanes per block; or 4 x 3
+def test_kv_append_batch_matches_oracle(policy):
+    """Heterogeneous items (heads, head_dim, rotation, scale layout, rows, tensor scale) in one launch:
+    each item's bytes equal the oracle's kv_append; an empty item is skipped."""
+    specs = [(3, 64, 128, True, False, 5, 16, 100, 7, 0.0021), (2, 40, 64, True, True, 0, 16, 300, 120, 0.0033),
+             (1, 33, 128, False, False, 17, 16, 64, 48, 0.0017), (4, 20, 32, False, True, 2, 3, 130, 127, 0.004),
+             (2, 16, 128, True, False, 0, 0, 16, 16, 0.002)]
+    items, want = [], []
+    for i, (BH, T, D, rot, tile, first, n, cap, t0, g) in enumerate(specs):
+        k = W.kv_decode_keys("cpu", n=T, heads=BH, head_dim=D) * (1.0 + i)
+        item, rc, rs = _append_item(k.to(torch.bfloat16), first, n, g, cap, t0, rot, tile)
+        items.append(item)
+        want.append((rc, rs))
+    prev = nv.search_policy(*policy) if policy else None
+    try:
+        nv.kv_append_batch(items)
+        torch.cuda.synchronize()
+    finally:
+        if prev:
+            nv.search_policy(*prev)
+    for item, (rc, rs) in zip(items, want):
+        assert np.array_equal(item[4].cpu().numpy(), rc)
+        assert np.array_equal(item[5].cpu().numpy(), rs)
+
+
+def test_kv_append_batch_errors_launch_nothing():
+    k = W.kv_decode_keys("cpu", n=32, heads=2, head_dim=64)
+    good, _, _ = _append_item(k, 0, 16, 0.002, 64, 0, True, False)
+    bad = (good[0], 0, 16, good[3], good[4], good[5], 60, True, False)       # rows 60..75 exceed cap 64
+    before = good[4].clone()
+    with pytest.raises(nv.NVFP4Error) as e:
+        nv.kv_append_batch([good, bad])
+    assert e.value.status == -2
+    with pytest.raises(nv.NVFP4Error) as e:
+        nv.kv_append_batch([good], -16, 16)                                     # 33 offsets
+    assert e.value.status == -1
+    with pytest.raises(ValueError):
+        nv.kv_append_batch([good] * 65)
+    torch.cuda.synchronize()
+    assert torch.equal(good[4], before)                                         # nothing was launched
+    nv.kv_append_batch([])
+
+
+@pytest.mark.parametrize("tile", [False, True])
+def test_append_many_equals_separate_appends(tile):
+    """Several caches (the K and V of three layers, different head counts) stepped together with one
+    batched flush per step give the same state as appending to each cache on its own."""
+    from nvfp4_block_scaled_11_b200.kvcache import append_many
+    B, D, T0, steps = 1, 128, 40, 45
+    shapes = [2, 2, 3, 3, 1, 1]
+    seqs = [W.kv_decode_keys("cpu", n=T0 + steps, heads=h, head_dim=D)[None] * (1 + 0.5 * i)
+            for i, h in enumerate(shapes)]
+    seqs = [s.to(torch.bfloat16) for s in seqs]
+    a = [NVFP4KVCache(B, h, D, capacity=128, tile_layout=tile, rotate=(i % 2 == 0)) for i, h in enumerate(shapes)]
+    b = [NVFP4KVCache(B, h, D, capacity=128, tile_layout=tile, rotate=(i % 2 == 0)) for i, h in enumerate(shapes)]
+    for c1, c2, s in zip(a, b, seqs):
+        c1.prefill(s[:, :, :T0].cuda())
+        c2.prefill(s[:, :, :T0].cuda())
+    for t in range(T0, T0 + steps):
+        append_many(a, [s[:, :, t:t + 1].cuda() for s in seqs])
+        for c, s in zip(b, seqs):
+            c.append(s[:, :, t:t + 1].cuda())
+    torch.cuda.synchronize()
+    for c1, c2 in zip(a, b):
+        assert (c1.n_mid, c1.n_window, c1.head) == (c2.n_mid, c2.n_window, c2.head) and c1.n_mid > 16
+        assert torch.equal(c1.codes, c2.codes) and torch.equal(c1.scales, c2.scales)
+        assert torch.equal(c1.window, c2.window)
