@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time the eager step only (no CUDA graph replay)")
+    ap.add_argument("--kv-layers", type=int, default=32, help="kv_decode_layers: layers flushed per step (K and V each)")
     return ap.parse_args()
 
 
@@ -871,6 +872,193 @@ def run_kvd_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+KVDL_METRIC = ("KV-cache decode, whole model: tokens appended per second (every step one 16-token group of new "
+               "keys and values leaves the BF16 window of each of L layers' K and V caches, 8 heads x 128 each, "
+               "quantized in one batched launch)")
+
+
+def kvdl_config(args, n_new):
+    L = args.kv_layers
+    return {
+        "workload": f"kv_decode_layers ({2 * L} caches = K and V of {L} layers, each 8 heads x 128 with the kv_bf16 "
+                    f"prefill's tensor scale; per cache {n_new} new rows [8,{n_new},128] BF16 = kv_decode_keys x "
+                    f"(1 + 0.01 j) for cache j)",
+        "window": [args.f_lo, args.f_hi], "layers": L, "caches": 2 * L,
+        "step": f"one decode flush: {2 * L} 16-token groups (Hadamard-rotated, ScaleSearch with the tensor scale) "
+                f"into the next 16 rows of each cache's NVFP4 middle, one nvfp4_kv_append_batch launch",
+        "l2": f"{2 * L} x 32 KB of window keys read once per step; latency-bound",
+    }
+
+
+def run_kv_decode_layers(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_11_b200 as nv
+    from nvfp4_block_scaled_11_b200 import workloads as W
+
+    L = max(1, min(args.kv_layers, nv.KV_APPEND_BATCH_MAX // 2))
+    args.kv_layers = L
+    C = 2 * L
+    k = W.kv_bf16(dev)
+    _, H, _, D = k.shape
+    g = nv.kv_gscale(k)
+    del k
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    e2e_steps = max(0, args.e2e_steps) if not args.no_e2e else 0
+    n_new = 16 * (steps + warmup + e2e_steps + 9)
+    base = W.kv_decode_keys(dev, n_new)
+    srcs = [(base.float() * (1.0 + 0.01 * j)).to(torch.bfloat16) for j in range(C)]
+    codes = [torch.empty((H, n_new, D // 2), dtype=torch.uint8, device=dev) for _ in range(C)]
+    scales = [torch.empty((H, n_new, D // 16), dtype=torch.uint8, device=dev) for _ in range(C)]
+    stream = torch.cuda.current_stream(dev)
+    group = [0]
+
+    def items(i):
+        return [(srcs[j], 16 * i, 16, g, codes[j], scales[j], 16 * i, True, False) for j in range(C)]
+
+    def step():
+        nv.kv_append_batch(items(group[0]), args.f_lo, args.f_hi)
+        group[0] += 1
+
+    def separate(i):
+        for j in range(C):
+            nv.kv_append(srcs[j], 16 * i, 16, g, codes[j], scales[j], 16 * i, f_lo=args.f_lo, f_hi=args.f_hi)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    sampler.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = eager_ms = t0.elapsed_time(t1)
+    graph_used, sep_ms = False, None
+    if world == 1 and not args.no_graph and steps >= 8:
+        # the decode loop as a CUDA graph: 8 consecutive flushes captured once and replayed (the same rows
+        # rewritten, the same work per flush); the same 8 flushes as 2L launches each, timed beside it
+        g0 = group[0]
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+
+        def graph_ms(fn):
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.synchronize()
+            cg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(cg, stream=side):
+                fn()
+            cg.replay()
+            torch.cuda.synchronize()
+            ga, gb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ga.record(stream)
+            for _ in range(steps // 8):
+                cg.replay()
+            gb.record(stream)
+            torch.cuda.synchronize()
+            del cg
+            return ga.elapsed_time(gb) * steps / (8 * (steps // 8))
+
+        batched = graph_ms(lambda: [nv.kv_append_batch(items(g0 + j), args.f_lo, args.f_hi) for j in range(8)])
+        sep_ms = graph_ms(lambda: [separate(g0 + j) for j in range(8)]) / steps
+        group[0] += 8
+        if batched < elapsed_ms:
+            elapsed_ms, graph_used = batched, True
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = t.item()
+    peak, psrc = peaks()
+    nbytes = C * (16 * H * D * 2 + 16 * H * (D // 2) + 16 * H * (D // 16))
+    launch_ms = elapsed_ms / steps
+    line = {
+        "metric": KVDL_METRIC, "value": world * 16 * steps / (elapsed_ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": elapsed_ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, nvfp4 out",
+        "data": SOURCE_NOTE, "config": kvdl_config(args, n_new),
+        "roofline": {"bound": "hbm", "kernel": f"kv_append_batch_kernel ({C} items, {C * 1024} blocks per launch)",
+                     "achieved": nbytes / (launch_ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": nbytes / (launch_ms * 1e-3) / 1e9 / peak, "traffic": None, "peak_source": psrc,
+                     "bytes_per_launch": nbytes,
+                     "note": "latency-bound: one launch per step; lane groups (16 lanes per block while the "
+                             "batch has at most 4096 blocks, then 4 lanes x 3 offsets)"},
+        "gpu_launches": steps,
+        "clocks": clocks,
+        "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps,
+                       "separate_launches_ms_per_step": sep_ms},
+    }
+    if e2e_steps > 0:
+        # every step: the C windows' 16 new rows from pinned host memory, one batched flush, and the C
+        # groups' codes and scales read back
+        hk = torch.empty((C, H, 16 * e2e_steps, D), dtype=torch.bfloat16, pin_memory=True)
+        for j in range(C):
+            hk[j].copy_(srcs[j][:, 16 * group[0]:16 * (group[0] + e2e_steps)])
+        dk = torch.empty((C, H, 16, D), dtype=torch.bfloat16, device=dev)
+        hc = torch.empty((C, H, 16, D // 2), dtype=torch.uint8, pin_memory=True)
+        hs = torch.empty((C, H, 16, D // 16), dtype=torch.uint8, pin_memory=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(e2e_steps):
+            row = 16 * group[0]
+            dk.copy_(hk[:, :, 16 * i:16 * (i + 1)], non_blocking=True)
+            nv.kv_append_batch([(dk[j], 0, 16, g, codes[j], scales[j], row, True, False) for j in range(C)],
+                               args.f_lo, args.f_hi)
+            for j in range(C):
+                hc[j].copy_(codes[j][:, row:row + 16], non_blocking=True)
+                hs[j].copy_(scales[j][:, row:row + 16], non_blocking=True)
+            group[0] += 1
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * 16 * e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": C * 16 * H * D * 2, "d2h_bytes_per_step": C * 16 * H * (D // 2 + D // 16)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = kvdl_oracle_baseline(args)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def kvdl_oracle_baseline(args, steps=4):
+    """The oracle appending `steps` flushes of 2L 16-token groups (single-threaded C), as tokens/s."""
+    cb = kvd_oracle_baseline(args, groups=steps * 2 * args.kv_layers)
+    value = cb["value"] / (2 * args.kv_layers)      # one sequence token = a row in each of the 2L caches
+    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{steps} flushes of {2 * args.kv_layers} groups of 16 new keys x 8 heads, oracle kv_append "
+                      f"(C, 1 thread)"}
+
+
+def run_kvdl_reference(args, rank, world):
+    if rank != 0:
+        return
+    args.kv_layers = max(1, min(args.kv_layers, 32))
+    for _ in range(args.warmup):
+        kvdl_oracle_baseline(args, steps=1)
+    cb = kvdl_oracle_baseline(args, steps=max(1, min(8, args.steps)))
+    line = {
+        "impl": "reference", "metric": KVDL_METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 16e3 / cb["value"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, nvfp4 out", "data": SOURCE_NOTE,
+        "config": kvdl_config(args, 16 * max(1, args.steps)), "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 ATTN_METRIC = "FP4 attention TFLOP/s (4*H*Tq*Tk*D per step; NVFP4 Q K^T and P V^T on the tensor cores)"
 
 
@@ -1113,6 +1301,8 @@ def main():
             run_attn_reference(args, rank, world)
         elif args.workload == "kv_decode":
             run_kvd_reference(args, rank, world)
+        elif args.workload == "kv_decode_layers":
+            run_kvdl_reference(args, rank, world)
         else:
             run_reference(args, rank, world)
         return
@@ -1141,6 +1331,9 @@ def main():
         return
     if args.workload == "kv_decode":
         run_kv_decode(args, rank, world, dev)
+        return
+    if args.workload == "kv_decode_layers":
+        run_kv_decode_layers(args, rank, world, dev)
         return
     w = W.make(args.workload, dev, args.scale, shard=rank)
     x = w.x.contiguous()
