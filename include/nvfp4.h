@@ -23,7 +23,8 @@
  * codes 0, f* = -128, sse NaN.
  *
  * Memory: every pointer argument is device memory owned by the caller unless stated otherwise; the
- * library allocates nothing and keeps no state between calls except cached device properties.
+ * library allocates nothing and keeps no state between calls except cached device properties and the
+ * launch policy set by nvfp4_search_policy (which changes no result).
  * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls enqueue
  * work and return without synchronising; outputs are valid once the stream reaches that point.
  * Overlapping calls on different streams that write the same outputs race, as with any kernel.
