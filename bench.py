@@ -909,16 +909,16 @@ def run_kv_decode_layers(args, rank, world, dev):
     n_new = 16 * (steps + warmup + e2e_steps + 9)
     base = W.kv_decode_keys(dev, n_new)
     srcs = [(base.float() * (1.0 + 0.01 * j)).to(torch.bfloat16) for j in range(C)]
-    codes = [torch.empty((H, n_new, D // 2), dtype=torch.uint8, device=dev) for _ in range(C)]
-    scales = [torch.empty((H, n_new, D // 16), dtype=torch.uint8, device=dev) for _ in range(C)]
+    codes_all = torch.empty((C, H, n_new, D // 2), dtype=torch.uint8, device=dev)
+    scales_all = torch.empty((C, H, n_new, D // 16), dtype=torch.uint8, device=dev)
+    codes, scales = list(codes_all), list(scales_all)
     stream = torch.cuda.current_stream(dev)
     group = [0]
-
-    def items(i):
-        return [(srcs[j], 16 * i, 16, g, codes[j], scales[j], 16 * i, True, False) for j in range(C)]
+    # the caches' descriptors are prepared once; each flush sets only the rows
+    batch = nv.KvAppendBatch([(srcs[j], g, codes[j], scales[j], True, False) for j in range(C)], args.f_lo, args.f_hi)
 
     def step():
-        nv.kv_append_batch(items(group[0]), args.f_lo, args.f_hi)
+        batch(16 * group[0], 16, 16 * group[0])
         group[0] += 1
 
     def separate(i):
@@ -967,7 +967,7 @@ def run_kv_decode_layers(args, rank, world, dev):
             del cg
             return ga.elapsed_time(gb) * steps / (8 * (steps // 8))
 
-        batched = graph_ms(lambda: [nv.kv_append_batch(items(g0 + j), args.f_lo, args.f_hi) for j in range(8)])
+        batched = graph_ms(lambda: [batch(16 * (g0 + j), 16, 16 * (g0 + j)) for j in range(8)])
         sep_ms = graph_ms(lambda: [separate(g0 + j) for j in range(8)]) / steps
         group[0] += 8
         if batched < elapsed_ms:
@@ -996,24 +996,24 @@ def run_kv_decode_layers(args, rank, world, dev):
                        "separate_launches_ms_per_step": sep_ms},
     }
     if e2e_steps > 0:
-        # every step: the C windows' 16 new rows from pinned host memory, one batched flush, and the C
-        # groups' codes and scales read back
+        # every step: the C windows' 16 new rows from pinned host memory (one copy), one batched flush,
+        # and the C groups' codes and scales read back (one copy each)
         hk = torch.empty((C, H, 16 * e2e_steps, D), dtype=torch.bfloat16, pin_memory=True)
         for j in range(C):
             hk[j].copy_(srcs[j][:, 16 * group[0]:16 * (group[0] + e2e_steps)])
         dk = torch.empty((C, H, 16, D), dtype=torch.bfloat16, device=dev)
         hc = torch.empty((C, H, 16, D // 2), dtype=torch.uint8, pin_memory=True)
         hs = torch.empty((C, H, 16, D // 16), dtype=torch.uint8, pin_memory=True)
+        ebatch = nv.KvAppendBatch([(dk[j], g, codes[j], scales[j], True, False) for j in range(C)],
+                                  args.f_lo, args.f_hi)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for i in range(e2e_steps):
             row = 16 * group[0]
             dk.copy_(hk[:, :, 16 * i:16 * (i + 1)], non_blocking=True)
-            nv.kv_append_batch([(dk[j], 0, 16, g, codes[j], scales[j], row, True, False) for j in range(C)],
-                               args.f_lo, args.f_hi)
-            for j in range(C):
-                hc[j].copy_(codes[j][:, row:row + 16], non_blocking=True)
-                hs[j].copy_(scales[j][:, row:row + 16], non_blocking=True)
+            ebatch(0, 16, row)
+            hc.copy_(codes_all[:, :, row:row + 16], non_blocking=True)
+            hs.copy_(scales_all[:, :, row:row + 16], non_blocking=True)
             group[0] += 1
         b.record(stream)
         torch.cuda.synchronize()

@@ -18,7 +18,7 @@ __all__ = [
     "NVFP4Error", "lib", "status_str", "tensor_amax", "global_scale", "quantize", "quantize_ex",
     "dequantize", "quantize_dequantize", "hadamard16", "kv_mixed", "kv_mixed_dequantize", "DTYPE_CODE", "sf_mma_bytes", "quantize_mma", "quantize_mma_t", "kv_mixed_mma",
     "gemm_nt", "gemm_sf_offsets", "kv_gscale", "kv_append", "mxfp4_quantize", "mxfp4_dequantize",
-    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "search_policy", "kv_append_batch",
+    "msda_forward", "softmax_quantize_mma", "rows_divide", "attention_fp4", "search_policy", "kv_append_batch", "KvAppendBatch",
 ]
 
 _SO = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
@@ -482,6 +482,50 @@ class _KvAppendDesc(ctypes.Structure):
 KV_APPEND_BATCH_MAX = 64
 
 
+class KvAppendBatch:
+    """A prepared nvfp4_kv_append_batch over fixed caches: `caches` is a sequence of tuples
+    (k_rows, gscale, codes, scales, rotate, tile_layout) with kv_append's meanings, validated once (at most
+    64; the tensors are kept alive).  Each call sets only the rows: first, n and t0 (an int for every item,
+    or one value per item; n = 0 skips an item) and launches once.  Outputs of different items must not
+    overlap."""
+
+    def __init__(self, caches, f_lo: int = -2, f_hi: int = 6):
+        caches = list(caches)
+        if len(caches) > KV_APPEND_BATCH_MAX:
+            raise ValueError(f"at most {KV_APPEND_BATCH_MAX} items per batch")
+        self._keep, self.f_lo, self.f_hi = caches, f_lo, f_hi
+        self._descs = (_KvAppendDesc * max(len(caches), 1))()
+        self._device = None
+        for i, (k_rows, gscale, codes, scales, rotate, tile_layout) in enumerate(caches):
+            for t, nm in ((k_rows, "k_rows"), (gscale, "gscale"), (codes, "codes"), (scales, "scales")):
+                _cuda(t, nm)
+            if k_rows.dtype != torch.bfloat16:
+                raise TypeError("k_rows must be bfloat16")
+            T, D = k_rows.shape[-2], k_rows.shape[-1]
+            BH = k_rows.numel() // max(T * D, 1)
+            cap = codes.shape[-2]
+            _out(gscale, "gscale", torch.float32, 1), _out(codes, "codes", torch.uint8, BH * cap * (D // 2))
+            _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
+            self._descs[i] = _KvAppendDesc(k_rows.data_ptr(), gscale.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                           BH, T, 0, 0, D, cap, 0, int(bool(rotate)), 1 if tile_layout else 0)
+            self._device = self._device or k_rows.device
+        self._count = len(caches)
+
+    def __len__(self) -> int:
+        return self._count
+
+    def __call__(self, first, n, t0) -> None:
+        if self._count == 0:
+            return
+        d = self._descs
+        for i in range(self._count):
+            d[i].first = first if isinstance(first, int) else first[i]
+            d[i].n = n if isinstance(n, int) else n[i]
+            d[i].t0 = t0 if isinstance(t0, int) else t0[i]
+        _check(lib().nvfp4_kv_append_batch(ctypes.cast(d, _P), self._count, self.f_lo, self.f_hi,
+                                           ctypes.c_void_p(torch.cuda.current_stream(self._device).cuda_stream)))
+
+
 def kv_append_batch(items, f_lo: int = -2, f_hi: int = 6) -> None:
     """Several kv_append calls in one launch.  `items`: a sequence of tuples
     (k_rows, first, n, gscale, codes, scales, t0, rotate, tile_layout) with kv_append's meanings; all use
@@ -489,24 +533,10 @@ def kv_append_batch(items, f_lo: int = -2, f_hi: int = 6) -> None:
     items = list(items)
     if len(items) > KV_APPEND_BATCH_MAX:
         raise ValueError(f"at most {KV_APPEND_BATCH_MAX} items per batch")
-    descs = (_KvAppendDesc * max(len(items), 1))()
-    stream = None
-    for i, (k_rows, first, n, gscale, codes, scales, t0, rotate, tile_layout) in enumerate(items):
-        for t, nm in ((k_rows, "k_rows"), (gscale, "gscale"), (codes, "codes"), (scales, "scales")):
-            _cuda(t, nm)
-        if k_rows.dtype != torch.bfloat16:
-            raise TypeError("k_rows must be bfloat16")
-        T, D = k_rows.shape[-2], k_rows.shape[-1]
-        BH = k_rows.numel() // max(T * D, 1)
-        cap = codes.shape[-2]
-        _out(gscale, "gscale", torch.float32, 1), _out(codes, "codes", torch.uint8, BH * cap * (D // 2))
-        _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
-        descs[i] = _KvAppendDesc(k_rows.data_ptr(), gscale.data_ptr(), codes.data_ptr(), scales.data_ptr(), BH, T,
-                                 first, n, D, cap, t0, int(bool(rotate)), 1 if tile_layout else 0)
-        stream = stream or _stream(k_rows)
     if not items:
         return
-    _check(lib().nvfp4_kv_append_batch(ctypes.cast(descs, _P), len(items), f_lo, f_hi, stream))
+    b = KvAppendBatch([(it[0], it[3], it[4], it[5], it[7], it[8]) for it in items], f_lo, f_hi)
+    b([it[1] for it in items], [it[2] for it in items], [it[6] for it in items])
 
 
 # ---- MXFP4 (comparison format) ----

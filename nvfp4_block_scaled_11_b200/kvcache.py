@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import torch
 
-from . import KV_APPEND_BATCH_MAX, kv_append, kv_append_batch, kv_gscale, sf_mma_bytes
+from . import KV_APPEND_BATCH_MAX, KvAppendBatch, kv_append, kv_gscale, sf_mma_bytes
 
 
 class NVFP4KVCache:
@@ -119,32 +119,55 @@ class NVFP4KVCache:
         return self.window[:, :, idx]
 
 
+class NVFP4KVCacheGroup:
+    """Caches that advance together, e.g. the K and V caches of every layer of a model: append() steps all
+    of them token by token, and whenever windows are full they flush together in one
+    nvfp4_kv_append_batch launch per 64 caches, through descriptors prepared once (each flush only sets
+    the rows).  The caches must share the ScaleSearch window [f_lo, f_hi]; the result is the same as
+    calling append on each cache."""
+
+    def __init__(self, caches):
+        self.caches = list(caches)
+        if len({(c.f_lo, c.f_hi) for c in self.caches}) > 1:
+            raise ValueError("caches in one group must share the offset window")
+        self._parts = []
+        for j in range(0, len(self.caches), KV_APPEND_BATCH_MAX):
+            part = self.caches[j:j + KV_APPEND_BATCH_MAX]
+            batch = KvAppendBatch([(c.window, c.gscale, c.codes, c.scales, c.rotate, c.tile_layout) for c in part],
+                                  part[0].f_lo, part[0].f_hi)
+            self._parts.append((part, batch))
+
+    def append(self, ks) -> None:
+        """Append ks[i] [B, H, n, D] (BF16) to caches[i], the same n for every cache."""
+        ks = list(ks)
+        if len(ks) != len(self.caches):
+            raise ValueError("one token tensor per cache")
+        if not ks:
+            return
+        for c in self.caches:
+            if not c.prefilled:
+                raise RuntimeError("prefill first")
+        n = ks[0].shape[2]
+        if any(k.shape[2] != n for k in ks):
+            raise ValueError("every cache receives the same number of tokens")
+        for i in range(n):
+            for part, batch in self._parts:
+                full = [c._full() for c in part]
+                if any(full):
+                    for c, f in zip(part, full):
+                        if f and c.n_mid + c.recent > c.capacity:
+                            raise RuntimeError("NVFP4 cache capacity exceeded")
+                    # full windows flush their oldest `recent` slots (head ..) into rows n_mid ..; others skip
+                    batch([c.head for c in part], [c.recent if f else 0 for c, f in zip(part, full)],
+                          [c.n_mid for c in part])
+                    for c, f in zip(part, full):
+                        if f:
+                            c._flushed()
+            for c, k in zip(self.caches, ks):
+                c._push(k[:, :, i])
+
+
 def append_many(caches, ks) -> None:
-    """Append one decode step's new tokens to several caches at once (e.g. the K and V caches of every
-    layer): ks[i] [B, H, n, D] (BF16) goes to caches[i], token by token; whenever windows are full, all
-    of them flush together in one nvfp4_kv_append_batch launch (up to 64 per launch) instead of one
-    launch per cache.  The caches must share the ScaleSearch window [f_lo, f_hi]; the result is the
-    same as calling append on each cache."""
-    caches, ks = list(caches), list(ks)
-    if len(caches) != len(ks):
-        raise ValueError("one token tensor per cache")
-    if not caches:
-        return
-    for c in caches:
-        if not c.prefilled:
-            raise RuntimeError("prefill first")
-    if len({(c.f_lo, c.f_hi) for c in caches}) != 1:
-        raise ValueError("caches in one call must share the offset window")
-    n = ks[0].shape[2]
-    if any(k.shape[2] != n for k in ks):
-        raise ValueError("every cache receives the same number of tokens")
-    f_lo, f_hi = caches[0].f_lo, caches[0].f_hi
-    for i in range(n):
-        full = [c for c in caches if c._full()]
-        for j in range(0, len(full), KV_APPEND_BATCH_MAX):
-            part = full[j:j + KV_APPEND_BATCH_MAX]
-            kv_append_batch([c._flush_args() for c in part], f_lo, f_hi)
-            for c in part:
-                c._flushed()
-        for c, k in zip(caches, ks):
-            c._push(k[:, :, i])
+    """Append one decode step's new tokens to several caches at once (a one-off NVFP4KVCacheGroup; keep a
+    group for a decode loop, so that its descriptors are prepared once)."""
+    NVFP4KVCacheGroup(caches).append(ks)

@@ -171,26 +171,39 @@ def test_kv_append_batch_errors_launch_nothing():
 
 
 @pytest.mark.parametrize("tile", [False, True])
-def test_append_many_equals_separate_appends(tile):
-    """Several caches (the K and V of three layers, different head counts) stepped together with one
-    batched flush per step give the same state as appending to each cache on its own."""
-    from nvfp4_block_scaled_11_b200.kvcache import append_many
+def test_cache_group_equals_separate_appends(tile):
+    """Several caches (the K and V of three layers, different head counts, rotated or not) stepped
+    together -- through a persistent NVFP4KVCacheGroup, and through append_many -- with one batched flush
+    per step give the same state as appending to each cache on its own; a cache whose window is not full
+    is skipped within the batch (one layer starts a token later)."""
+    from nvfp4_block_scaled_11_b200.kvcache import NVFP4KVCacheGroup, append_many
     B, D, T0, steps = 1, 128, 40, 45
     shapes = [2, 2, 3, 3, 1, 1]
-    seqs = [W.kv_decode_keys("cpu", n=T0 + steps, heads=h, head_dim=D)[None] * (1 + 0.5 * i)
+    ahead = [0, 0, 1, 1, 0, 0]                   # layer 1's windows hold one more token: they fill earlier
+    seqs = [W.kv_decode_keys("cpu", n=T0 + 1 + steps, heads=h, head_dim=D)[None] * (1 + 0.5 * i)
             for i, h in enumerate(shapes)]
     seqs = [s.to(torch.bfloat16) for s in seqs]
-    a = [NVFP4KVCache(B, h, D, capacity=128, tile_layout=tile, rotate=(i % 2 == 0)) for i, h in enumerate(shapes)]
-    b = [NVFP4KVCache(B, h, D, capacity=128, tile_layout=tile, rotate=(i % 2 == 0)) for i, h in enumerate(shapes)]
-    for c1, c2, s in zip(a, b, seqs):
-        c1.prefill(s[:, :, :T0].cuda())
-        c2.prefill(s[:, :, :T0].cuda())
-    for t in range(T0, T0 + steps):
-        append_many(a, [s[:, :, t:t + 1].cuda() for s in seqs])
-        for c, s in zip(b, seqs):
-            c.append(s[:, :, t:t + 1].cuda())
+
+    def make():
+        cs = [NVFP4KVCache(B, h, D, capacity=128, tile_layout=tile, rotate=(i % 2 == 0))
+              for i, h in enumerate(shapes)]
+        for c, s, ah in zip(cs, seqs, ahead):
+            c.prefill(s[:, :, :T0].cuda())
+            if ah:
+                c.append(s[:, :, T0:T0 + ah].cuda())
+        return cs
+
+    a, b, c3 = make(), make(), make()
+    group = NVFP4KVCacheGroup(a)
+    for step in range(steps):
+        rows = [s[:, :, T0 + ah + step:T0 + ah + step + 1].cuda() for s, ah in zip(seqs, ahead)]
+        group.append(rows)
+        append_many(c3, rows)
+        for c, r in zip(b, rows):
+            c.append(r)
     torch.cuda.synchronize()
-    for c1, c2 in zip(a, b):
-        assert (c1.n_mid, c1.n_window, c1.head) == (c2.n_mid, c2.n_window, c2.head) and c1.n_mid > 16
-        assert torch.equal(c1.codes, c2.codes) and torch.equal(c1.scales, c2.scales)
-        assert torch.equal(c1.window, c2.window)
+    for c1, c2, c4 in zip(a, b, c3):
+        for c in (c1, c4):
+            assert (c.n_mid, c.n_window, c.head) == (c2.n_mid, c2.n_window, c2.head) and c.n_mid > 16
+            assert torch.equal(c.codes, c2.codes) and torch.equal(c.scales, c2.scales)
+            assert torch.equal(c.window, c2.window)
