@@ -18,10 +18,10 @@
 // both F and P are perturbations of the real sum of (x_i - v_i d)^2 by the roundings of r, y, the
 // products and the sums, and |x_i - v_i d| <= d * max(1, y_max - 6) bounds the cross terms.  When the
 // runner-up's score exceeds the best score by more than twice that bound, the best candidate of the
-// score is the best candidate of the definition and no exact work is needed.  Otherwise every
-// candidate that is not so separated is re-scored with the definition, and the definition's tie rule
-// decides.  Blocks outside the covered range, or whose window leaves the codes 1..126, are scored with
-// the definition throughout.
+// score is the best candidate of the definition and no exact work is needed.  Otherwise the block is
+// deferred and every candidate is re-scored with the definition, whose tie rule decides.  Blocks outside
+// the covered range, or whose window leaves the codes 1..126 (narrow windows; wide ones score the part
+// inside), are scored with the definition throughout.
 #pragma once
 
 #include "kernels.cuh"
@@ -35,14 +35,6 @@ __device__ __forceinline__ uint32_t e2m1_round2(float lo, float hi) {
       : "=r"(r)
       : "f"(lo), "f"(hi));
   return r;
-}
-// (v_lo - y_lo, v_hi - y_hi) with v the f16 halves of h2 (exact values): one rounding each.
-__device__ __forceinline__ u64 vsub2(uint32_t h2, float ylo, float yhi) {
-  float lo, hi;
-  asm("{ .reg .b16 l, h; mov.b32 {l,h}, %2; sub.rn.f32.f16 %0, l, %3; sub.rn.f32.f16 %1, h, %4; }"
-      : "=f"(lo), "=f"(hi)
-      : "r"(h2), "f"(ylo), "f"(yhi));
-  return pk2(lo, hi);
 }
 // E2M1 codes of 8 values packed into a word, value 2k in the low nibble of byte k.
 __device__ __forceinline__ uint32_t e2m1_pack8(u64 p0, u64 p1, u64 p2, u64 p3) {

@@ -64,3 +64,22 @@ def test_tile_layout_gemm_and_attention_buffers_are_checked():
     g = nv.kv_gscale(k[None], 0, 0)
     with pytest.raises(ValueError):
         nv.kv_append(k, 0, 16, g, E((2, 20, 31)), E((2, 20, 4)), 0)
+
+
+def test_kv_append_batch_buffers_are_checked():
+    k = torch.randn(2, 32, 64, device="cuda").to(torch.bfloat16)
+    g = torch.ones(1, device="cuda")
+    ok = (k, g, E((2, 16, 32)), E((2, 16, 4)), True, False)
+    with pytest.raises(ValueError):
+        nv.KvAppendBatch([(k, g, E((2, 16, 31)), E((2, 16, 4)), True, False)])        # codes short
+    with pytest.raises(ValueError):
+        nv.KvAppendBatch([(k, g, E((2, 16, 32)), E(nv.sf_mma_bytes(16, 64, 2) - 1), True, True)])
+    with pytest.raises(TypeError):
+        nv.KvAppendBatch([(k.float(), g, E((2, 16, 32)), E((2, 16, 4)), True, False)])
+    with pytest.raises(ValueError):
+        nv.KvAppendBatch([ok] * 65)
+    b = nv.KvAppendBatch([ok, ok[:2] + (E((2, 16, 32)), E((2, 16, 4))) + ok[4:]])
+    b([0, 16], 16, [0, 0])                                  # per-item rows, one n for both
+    with pytest.raises(nv.NVFP4Error):
+        b(0, 16, 1)                                          # rows 1..16 exceed the 16-row caches
+    torch.cuda.synchronize()
