@@ -45,3 +45,12 @@ def test_reference_arm_line():
     d = _run("--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", "act_f32", timeout=300)
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("workload,extra", [("kv_decode", []), ("kv_decode_layers", ["--kv-layers", "2"])])
+def test_decode_reference_arm_lines(workload, extra):
+    """The decode workloads' reference arms (the oracle's appends on the host) keep the same contract."""
+    d = _run("--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", workload, *extra, timeout=300)
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"].startswith(workload)
