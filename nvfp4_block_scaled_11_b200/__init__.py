@@ -10,6 +10,7 @@ Element types: torch.float32, torch.bfloat16, torch.float16.
 from __future__ import annotations
 
 import ctypes
+import numbers
 import os
 
 import torch
@@ -518,10 +519,11 @@ class KvAppendBatch:
         if self._count == 0:
             return
         d = self._descs
+        one = [isinstance(v, numbers.Integral) for v in (first, n, t0)]
         for i in range(self._count):
-            d[i].first = first if isinstance(first, int) else first[i]
-            d[i].n = n if isinstance(n, int) else n[i]
-            d[i].t0 = t0 if isinstance(t0, int) else t0[i]
+            d[i].first = int(first if one[0] else first[i])
+            d[i].n = int(n if one[1] else n[i])
+            d[i].t0 = int(t0 if one[2] else t0[i])
         _check(lib().nvfp4_kv_append_batch(ctypes.cast(d, _P), self._count, self.f_lo, self.f_hi,
                                            ctypes.c_void_p(torch.cuda.current_stream(self._device).cuda_stream)))
 
