@@ -1,0 +1,88 @@
+"""Host logic of the decode caches, without a GPU: which caches of a group flush when, with which rows,
+and the errors raised before anything is launched.  The batched launch is replaced by a recorder."""
+import pytest
+import torch
+
+import nvfp4_block_scaled_11_b200.kvcache as kc
+
+
+class Recorder:
+    """Stands in for KvAppendBatch: remembers the caches it was built over and every (first, n, t0)."""
+    made = []
+
+    def __init__(self, items, f_lo, f_hi):
+        self.items, self.window, self.calls = list(items), (f_lo, f_hi), []
+        Recorder.made.append(self)
+
+    def __call__(self, first, n, t0):
+        self.calls.append((list(first), list(n), list(t0)))
+
+
+@pytest.fixture
+def fake_batch(monkeypatch):
+    Recorder.made = []
+    monkeypatch.setattr(kc, "KvAppendBatch", Recorder)
+    return Recorder
+
+
+def _cache(H=2, D=32, capacity=64, recent=16, window=16, f=(-2, 6)):
+    """A cache in the state prefill leaves (sink full, `window` tokens in the ring), on the CPU."""
+    c = kc.NVFP4KVCache(1, H, D, capacity=capacity, recent=recent, f_lo=f[0], f_hi=f[1], device="cpu")
+    c.prefilled, c.n_sink, c.n_window = True, 16, window
+    return c
+
+
+def _tok(c, v=0.0):
+    return torch.full((1, c.H, 1, c.D), v, dtype=torch.bfloat16)
+
+
+def test_group_flushes_full_windows_only(fake_batch):
+    cs = [_cache(), _cache(window=17), _cache(H=3)]
+    g = kc.NVFP4KVCacheGroup(cs)
+    (b,) = fake_batch.made
+    assert [it[0] is c.window and it[2] is c.codes for it, c in zip(b.items, cs)] == [True] * 3
+    for step in range(40):
+        g.append([_tok(c, step) for c in cs])
+    # cache 1 fills a token earlier; the others are items with n = 0 in its flush and vice versa
+    assert b.calls == [([0, 0, 0], [0, 16, 0], [0, 0, 0]),
+                       ([0, 16, 0], [16, 0, 16], [0, 16, 0]),
+                       ([16, 16, 16], [0, 16, 0], [16, 16, 16]),
+                       ([16, 0, 16], [16, 0, 16], [16, 32, 16])]
+    assert [(c.n_mid, c.n_window, c.head) for c in cs] == [(32, 24, 0), (32, 25, 0), (32, 24, 0)]
+    # the window ring holds the newest tokens in order
+    assert [v.item() for v in cs[0].recent_tokens()[0, 0, :, 0]] == [float(v) for v in range(16, 40)]
+
+
+def test_group_splits_into_batches_of_64(fake_batch):
+    cs = [_cache(H=1, D=16) for _ in range(70)]
+    g = kc.NVFP4KVCacheGroup(cs)
+    assert [len(b.items) for b in fake_batch.made] == [64, 6]
+    for step in range(17):
+        g.append([_tok(c) for c in cs])
+    assert [len(b.calls) for b in fake_batch.made] == [1, 1]
+
+
+def test_group_errors_before_any_launch(fake_batch):
+    with pytest.raises(ValueError):
+        kc.NVFP4KVCacheGroup([_cache(), _cache(f=(-8, 8))])          # windows differ
+    cs = [_cache(capacity=16), _cache(capacity=8)]
+    g = kc.NVFP4KVCacheGroup(cs)
+    with pytest.raises(RuntimeError):                                # the second cache has no room
+        g.append([torch.zeros((1, 2, 17, 32), dtype=torch.bfloat16)] * 2)
+    assert fake_batch.made[-1].calls == [] and cs[0].n_mid == 0
+    with pytest.raises(ValueError):
+        g.append([torch.zeros((1, 2, 1, 32), dtype=torch.bfloat16)])  # one tensor for two caches
+    with pytest.raises(ValueError):
+        g.append([torch.zeros((1, 2, 1, 32), dtype=torch.bfloat16), torch.zeros((1, 2, 2, 32), dtype=torch.bfloat16)])
+    fresh = kc.NVFP4KVCache(1, 2, 32, capacity=16, device="cpu")
+    with pytest.raises(RuntimeError):
+        kc.NVFP4KVCacheGroup([fresh]).append([torch.zeros((1, 2, 1, 32), dtype=torch.bfloat16)])
+
+
+def test_append_many_is_a_one_off_group(fake_batch):
+    cs = [_cache(), _cache()]
+    for step in range(20):
+        kc.append_many(cs, [_tok(c, step) for c in cs])
+    flushes = [call for b in fake_batch.made for call in b.calls]
+    assert flushes == [([0, 0], [16, 16], [0, 0])]
+    assert [(c.n_mid, c.n_window, c.head) for c in cs] == [(16, 20, 16)] * 2
