@@ -141,3 +141,21 @@ def test_kv_append_batch_validates_on_the_host(L):
     for d, want in ((bad_d, -2), (past, -2), (badrot, -1)):
         arr2 = (D * 2)(ok, d)
         assert L.nvfp4_kv_append_batch(ctypes.cast(arr2, ctypes.c_void_p), 2, -2, 6, None) == want
+
+
+def test_kv_append_desc_layout_matches_the_header(tmp_path):
+    """The binding's ctypes mirror of nvfp4_kv_append_desc has the C struct's size and field offsets
+    (a C program built against the header prints them)."""
+    import subprocess
+    fields = [f for f, _ in nv._KvAppendDesc._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "nvfp4.h"\nint main(void) {\n'
+                   '  printf("%zu", sizeof(nvfp4_kv_append_desc));\n'
+                   + "".join(f'  printf(" %zu", offsetof(nvfp4_kv_append_desc, {f}));\n' for f in fields)
+                   + '  printf("\\n");\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(nv._KvAppendDesc)] + [getattr(nv._KvAppendDesc, f).offset for f in fields]
+    assert got == want
