@@ -159,3 +159,29 @@ def test_kv_append_desc_layout_matches_the_header(tmp_path):
     got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
     want = [ctypes.sizeof(nv._KvAppendDesc)] + [getattr(nv._KvAppendDesc, f).offset for f in fields]
     assert got == want
+
+
+def _ctype_of(decl: str):
+    """ctypes class the binding must use for one C parameter or return declaration."""
+    d = " ".join(decl.replace("const", " ").split())
+    if "*" in d:
+        return ctypes.c_char_p if d.startswith("char") else ctypes.c_void_p
+    base = d.rsplit(" ", 1)[0] if " " in d else d
+    return {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "int32_t": ctypes.c_int, "uint32_t": ctypes.c_uint32,
+            "float": ctypes.c_float}[base]
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype's return type and parameter types (pointer, int64, int, uint32, float) equal the
+    ctypes signature the binding installs, so no argument is passed with the wrong width."""
+    src = re.sub(r"/\*.*?\*/", "", open(HDR).read(), flags=re.S)
+    src = "\n".join(ln for ln in src.splitlines() if not ln.lstrip().startswith("#"))
+    protos = re.findall(r"([A-Za-z_][\w\s\*]*?)\b(nvfp4_\w+)\s*\(([^)]*)\)\s*;", src)
+    assert len(protos) == len(_declared())
+    for ret, name, params in protos:
+        ret = ret.strip().splitlines()[-1]      # the return type sits on the prototype's first line
+        res, args = nv._SIGS[name]
+        want_ret = ctypes.c_char_p if "char" in ret else _ctype_of(ret.strip() + " r")
+        assert res is want_ret, name
+        ps = [p.strip() for p in params.split(",")] if params.strip() not in ("", "void") else []
+        assert [_ctype_of(p) for p in ps] == list(args), name
