@@ -38,3 +38,21 @@ def test_clock_sampler_without_the_tool(tmp_path, monkeypatch):
     s.start()
     c = s.stop()
     assert c["samples"] == 0 and c["sm_mhz"] is None and c["reasons"]
+
+
+def test_captured_traffic_scales_and_expires(tmp_path, monkeypatch):
+    """The committed DRAM record is scaled to a launch by elements, and reads as None once any of the
+    kernel's sources differs from what was hashed at capture time."""
+    import hashlib
+    import json
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cuh").write_text("kernel source v1\n")
+    h = hashlib.sha256(b"kernel source v1\n").hexdigest()
+    rec = {"K": {"source_sha256": h, "source_files": ["k.cuh"], "captured_elements": 1000,
+                 "dram_bytes_read": 3000, "dram_bytes_write": 1000}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic("K", 5000) == 20000
+    assert bench.captured_traffic("other", 5000) is None
+    (tmp_path / "k.cuh").write_text("kernel source v2\n")
+    assert bench.captured_traffic("K", 5000) is None
