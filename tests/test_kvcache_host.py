@@ -86,3 +86,29 @@ def test_append_many_is_a_one_off_group(fake_batch):
     flushes = [call for b in fake_batch.made for call in b.calls]
     assert flushes == [([0, 0], [16, 16], [0, 0])]
     assert [(c.n_mid, c.n_window, c.head) for c in cs] == [(16, 20, 16)] * 2
+
+
+def test_single_cache_argument_errors_and_window_order():
+    """Errors a cache raises before any launch, and the ring's token order after wrap-around."""
+    with pytest.raises(ValueError):
+        kc.NVFP4KVCache(1, 2, 30, capacity=8, device="cpu")                    # D not a multiple of 16
+    c = kc.NVFP4KVCache(1, 2, 32, capacity=8, device="cpu")
+    with pytest.raises(RuntimeError):
+        c.append(torch.zeros((1, 2, 1, 32), dtype=torch.bfloat16))            # no prefill yet
+    with pytest.raises(ValueError):
+        c.prefill(torch.zeros((1, 2, 40, 32), dtype=torch.float32))           # not BF16
+    with pytest.raises(ValueError):
+        c.prefill(torch.zeros((1, 3, 40, 32), dtype=torch.bfloat16))          # heads differ
+    with pytest.raises(ValueError):
+        c.prefill(torch.zeros((1, 2, 31, 32), dtype=torch.bfloat16))          # fewer than sink + recent
+    with pytest.raises(ValueError):
+        c.prefill(torch.zeros((1, 2, 41, 32), dtype=torch.bfloat16))          # middle of 9 > capacity 8
+    w = _cache(H=1, D=16, window=16)
+    w.head = 16                                                               # the ring has wrapped once
+    for i in range(16):
+        w.window[0, 0, (16 + i) % 32, 0] = float(i)
+    for i in range(5):
+        w._push(torch.full((1, 1, 16), 100.0 + i, dtype=torch.bfloat16))
+    got = [v.item() for v in w.recent_tokens()[0, 0, :, 0]]
+    assert got == [float(i) for i in range(16)] + [100.0 + i for i in range(5)]
+    assert w.length == 16 + 0 + 21
