@@ -233,12 +233,21 @@ def run_reference(args, rank, world):
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
+        "scaling": "weak", "vs_baseline": None, "dtype": workload_dtype(args.workload), "data": SOURCE_NOTE,
         "config": workload_config(args),
         "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+WORKLOAD_DTYPE = {"stream_f32": "f32", "act_f32": "f32", "act_bf16": "bf16", "kv_bf16": "bf16", "bev_f16": "f16"}
+
+
+def workload_dtype(name: str) -> str:
+    """The element type the quantize path reads and computes its dequantized values in (the search itself
+    runs in FP32 on the widened values)."""
+    return WORKLOAD_DTYPE.get(name, "f32")
 
 
 def workload_config(args):
@@ -1625,7 +1634,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": SOURCE_NOTE,
+        "scaling": "weak", "vs_baseline": None, "dtype": workload_dtype(args.workload), "data": SOURCE_NOTE,
         "config": workload_config(args),
         "roofline": roofline,
         "roofline_search_pass": search_roofline,

@@ -239,6 +239,8 @@ typedef struct nvfp4_kv_append_desc {
  * (at most 32 offsets, NVFP4_ERR_ARG otherwise).  Each item writes exactly the bytes nvfp4_kv_append
  * would; items must not write overlapping outputs.  Every descriptor is validated before anything is
  * launched (the first failing item's status is returned); items with BH == 0 or n == 0 are skipped.
+ * A batch whose blocks together need more thread blocks than one grid holds (2^31 - 1 CTAs of 256
+ * threads) returns NVFP4_ERR_SIZE, also before any launch.
  * The launch always takes lane groups (16 or 32 lanes per block while the batch is small, 4 or 8 with
  * several offsets each beyond nvfp4_search_policy's first bound): it is meant for decode-sized groups. */
 int nvfp4_kv_append_batch(const nvfp4_kv_append_desc* descs, int count, int f_lo, int f_hi, void* stream);

@@ -486,7 +486,7 @@ KV_APPEND_BATCH_MAX = 64
 class KvAppendBatch:
     """A prepared nvfp4_kv_append_batch over fixed caches: `caches` is a sequence of tuples
     (k_rows, gscale, codes, scales, rotate, tile_layout) with kv_append's meanings, validated once (at most
-    64; the tensors are kept alive).  Each call sets only the rows: first, n and t0 (an int for every item,
+    64, every tensor on one device; the tensors are kept alive).  Each call sets only the rows: first, n and t0 (an int for every item,
     or one value per item; n = 0 skips an item) and launches once.  Outputs of different items must not
     overlap."""
 
@@ -500,6 +500,10 @@ class KvAppendBatch:
         for i, (k_rows, gscale, codes, scales, rotate, tile_layout) in enumerate(caches):
             for t, nm in ((k_rows, "k_rows"), (gscale, "gscale"), (codes, "codes"), (scales, "scales")):
                 _cuda(t, nm)
+                # one launch on one device's stream reads and writes every item: all on that device
+                self._device = self._device or t.device
+                if t.device != self._device:
+                    raise ValueError(f"item {i}: {nm} is on {t.device}, the batch runs on {self._device}")
             if k_rows.dtype != torch.bfloat16:
                 raise TypeError("k_rows must be bfloat16")
             T, D = k_rows.shape[-2], k_rows.shape[-1]
@@ -509,7 +513,6 @@ class KvAppendBatch:
             _out(scales, "scales", torch.uint8, sf_mma_bytes(cap, D, BH) if tile_layout else BH * cap * (D // 16))
             self._descs[i] = _KvAppendDesc(k_rows.data_ptr(), gscale.data_ptr(), codes.data_ptr(), scales.data_ptr(),
                                            BH, T, 0, 0, D, cap, 0, int(bool(rotate)), 1 if tile_layout else 0)
-            self._device = self._device or k_rows.device
         self._count = len(caches)
 
     def __len__(self) -> int:

@@ -1,5 +1,6 @@
 // nvfp4_api.cu -- the libnvfp4 C ABI (include/nvfp4.h): argument validation and kernel launches.
 #include <cuda_runtime.h>
+#include <limits.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -801,14 +802,18 @@ int nvfp4_kv_append_batch(const nvfp4_kv_append_desc* descs, int count, int f_lo
   if (m == 0) return NVFP4_OK;
   bp.count = m;
   bp.start[m] = total;
-  cudaStream_t s = S(stream);
   const int nc = f_hi - f_lo + 1;
-  if (total * (nc <= 16 ? 16 : 32) <= g_lane1_max.load(std::memory_order_relaxed)) {
-    const int grid = (int)((total * (nc <= 16 ? 16 : 32) + 255) / 256);
+  const bool one_per_lane = total * (nc <= 16 ? 16 : 32) <= g_lane1_max.load(std::memory_order_relaxed);
+  const int64_t lanes = one_per_lane ? (nc <= 16 ? 16 : 32) : (nc <= 12 ? 4 : 8);
+  // every item is below 2^32 blocks, but 64 of them can ask for more CTAs than a grid holds
+  const int64_t ctas = (total * lanes + 255) / 256;
+  if (ctas > INT_MAX) return NVFP4_ERR_SIZE;
+  const int grid = (int)ctas;
+  cudaStream_t s = S(stream);
+  if (one_per_lane) {
     if (nc <= 16) kv_append_batch_kernel<16, 1><<<grid, 256, 0, s>>>(bp);
     else kv_append_batch_kernel<32, 1><<<grid, 256, 0, s>>>(bp);
   } else {
-    const int grid = (int)((total * (nc <= 12 ? 4 : 8) + 255) / 256);
     if (nc <= 12) kv_append_batch_kernel<4, 3><<<grid, 256, 0, s>>>(bp);
     else kv_append_batch_kernel<8, 4><<<grid, 256, 0, s>>>(bp);
   }

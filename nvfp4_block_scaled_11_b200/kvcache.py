@@ -123,13 +123,15 @@ class NVFP4KVCacheGroup:
     """Caches that advance together, e.g. the K and V caches of every layer of a model: append() steps all
     of them token by token, and whenever windows are full they flush together in one
     nvfp4_kv_append_batch launch per 64 caches, through descriptors prepared once (each flush only sets
-    the rows).  The caches must share the ScaleSearch window [f_lo, f_hi]; the result is the same as
+    the rows).  The caches must share the ScaleSearch window [f_lo, f_hi] and one device; the result is the same as
     calling append on each cache."""
 
     def __init__(self, caches):
         self.caches = list(caches)
         if len({(c.f_lo, c.f_hi) for c in self.caches}) > 1:
             raise ValueError("caches in one group must share the offset window")
+        if len({c.codes.device for c in self.caches}) > 1:
+            raise ValueError("caches in one group must live on one device (each flush is one launch)")
         self._parts = []
         for j in range(0, len(self.caches), KV_APPEND_BATCH_MAX):
             part = self.caches[j:j + KV_APPEND_BATCH_MAX]

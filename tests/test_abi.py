@@ -143,6 +143,18 @@ def test_kv_append_batch_validates_on_the_host(L):
         assert L.nvfp4_kv_append_batch(ctypes.cast(arr2, ctypes.c_void_p), 2, -2, 6, None) == want
 
 
+def test_kv_append_batch_rejects_a_grid_too_large(L):
+    """Each item stays below 2^32 blocks, but 64 such items need more CTAs than a grid holds: the call
+    returns NVFP4_ERR_SIZE on the host (the fake pointers are never dereferenced)."""
+    D = nv._KvAppendDesc
+    fake = 1 << 20
+    # BH = 1, D = 16: n rows are n blocks; 2^32 - 1 blocks per item, 64 items
+    big = D(fake, fake, fake, fake, 1, (1 << 32) - 1, 0, (1 << 32) - 1, 16, (1 << 32) - 1, 0, 0, 0)
+    arr = (D * 64)(*([big] * 64))
+    for lo, hi in ((-2, 6), (-1, 1), (-8, 8), (-16, 15)):   # 4, 4, 8 and 8 lanes per block
+        assert L.nvfp4_kv_append_batch(ctypes.cast(arr, ctypes.c_void_p), 64, lo, hi, None) == -2
+
+
 def test_kv_append_desc_layout_matches_the_header(tmp_path):
     """The binding's ctypes mirror of nvfp4_kv_append_desc has the C struct's size and field offsets
     (a C program built against the header prints them)."""

@@ -38,6 +38,16 @@ def test_default_workload_line():
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
     assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
     assert d["gpu_launches"] > 0
+    assert d["dtype"] == "f32"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("workload,dtype", [("act_bf16", "bf16"), ("bev_f16", "f16")])
+def test_line_dtype_follows_the_workload(workload, dtype):
+    """The line's dtype is the element type of the workload it measured."""
+    d = _run("--workload", workload, "--scale", "0.05", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+             "--no-e2e")
+    assert d["dtype"] == dtype and d["config"]["workload"].startswith(workload)
 
 
 def test_reference_arm_line():
@@ -45,6 +55,15 @@ def test_reference_arm_line():
     d = _run("--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", "act_f32", timeout=300)
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["dtype"] == "f32"
+
+
+def test_workload_dtypes():
+    """Both arms label a line with its workload's element type."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert [bench.workload_dtype(w) for w in ("stream_f32", "act_f32", "act_bf16", "kv_bf16", "bev_f16")] == \
+        ["f32", "f32", "bf16", "bf16", "f16"]
 
 
 @pytest.mark.parametrize("workload,extra", [("kv_decode", []), ("kv_decode_layers", ["--kv-layers", "2"])])

@@ -112,3 +112,34 @@ def test_single_cache_argument_errors_and_window_order():
     got = [v.item() for v in w.recent_tokens()[0, 0, :, 0]]
     assert got == [float(i) for i in range(16)] + [100.0 + i for i in range(5)]
     assert w.length == 16 + 0 + 21
+
+
+def test_group_refuses_caches_on_two_devices(fake_batch):
+    """One flush is one launch on one device: a group over caches on different devices is refused before
+    any batch is built (here a CPU cache and a meta-device cache stand in for two GPUs)."""
+    a = _cache()
+    b = kc.NVFP4KVCache(1, 2, 32, capacity=64, device="meta")
+    with pytest.raises(ValueError, match="one device"):
+        kc.NVFP4KVCacheGroup([a, b])
+    assert fake_batch.made == []
+
+
+def test_batch_refuses_items_on_two_devices(monkeypatch):
+    """KvAppendBatch checks every tensor of every item against the first item's device before it builds a
+    descriptor (the CUDA-tensor check is relaxed here so that CPU and meta tensors can stand in for two
+    GPUs; nothing is launched)."""
+    import nvfp4_block_scaled_11_b200 as nv
+    monkeypatch.setattr(nv, "_cuda", lambda t, name: t)
+
+    def item(dev, gdev=None):
+        k = torch.zeros(2, 32, 32, dtype=torch.bfloat16, device=dev)
+        g = torch.zeros(1, dtype=torch.float32, device=gdev or dev)
+        codes = torch.zeros(2, 64, 16, dtype=torch.uint8, device=dev)
+        scales = torch.zeros(2, 64, 2, dtype=torch.uint8, device=dev)
+        return (k, g, codes, scales, True, False)
+
+    with pytest.raises(ValueError, match="item 1: k_rows is on meta"):
+        nv.KvAppendBatch([item("cpu"), item("meta")])
+    with pytest.raises(ValueError, match="item 0: gscale is on meta"):
+        nv.KvAppendBatch([item("cpu", gdev="meta")])
+    assert len(nv.KvAppendBatch([item("cpu"), item("cpu")])) == 2
