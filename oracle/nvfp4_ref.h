@@ -134,7 +134,10 @@ int ref_msda_forward(const float* value, const int64_t* shapes, const int64_t* s
  * operation order): n = rint(x * log2(e)), r = fma(n, -ln2_lo, fma(n, -ln2_hi, x)) with ln2 split at 16
  * significant bits (the inner step is exact), p = Horner(1, 1, 1/2!, ..., 1/7!) at r with fused
  * multiply-adds, result p * 2^n (scaled in two exact steps below 2^-126).  x < -104 gives 0; NaN gives
- * NaN.  (The one place the oracle uses FMA: it is part of this method's definition.) */
+ * NaN.  (The one place the oracle uses FMA: it is part of this method's definition.)  The pages do not
+ * fix an exp; this fused form replaced an earlier one with separate multiplies and adds, and its exact
+ * bits are pinned by an evaluation of the same method on exact rationals, rounded once per operation,
+ * with the constants derived from ln 2 and the factorials (tests/test_oracle_attention.py). */
 float ref_exp_ss(float x);
 
 int ref_softmax_quantize(const float* s, int64_t batch, int64_t Tq, int64_t Tk, int causal, int64_t q_offset,
