@@ -24,7 +24,8 @@
  * brute-force search, closed forms, invariants); the exact f* histogram shape on Gaussian data is
  * qualitative on the pages (bimodal) and is "parity unpinned" beyond that shape.  The block-scale tile
  * layout is pinned by an independent reshape construction of the documented tile array, hand-checked
- * offsets, padding and bijectivity; the NVFP4 product (oracle.py) by exact rational arithmetic.
+ * offsets, padding and bijectivity; the NVFP4 product (oracle.py) by exact rational arithmetic; the
+ * softmax exp (ref_exp_ss) bit for bit by the same method evaluated on exact rationals.
  */
 #ifndef NVFP4_REF_H
 #define NVFP4_REF_H

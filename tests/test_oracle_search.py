@@ -313,3 +313,31 @@ def test_tensor_amax_and_global_scale():
     assert O.tensor_amax(np.zeros(0, np.float32)) == 0.0
     h = x.astype(np.float16)
     assert O.tensor_amax(h.view(np.uint16), O.F16) == np.abs(h).max().astype(np.float32)
+
+
+def test_fullsize_harness_counts_planted_mismatches(tmp_path):
+    """The whole-tensor comparison harness (spawned oracle workers over memory-mapped files) reports 0
+    mismatches when the "device" outputs are the oracle's own, and exactly the planted ones otherwise."""
+    from tests import fullsize as FS
+    rng = np.random.default_rng(5)
+    n = 16 * 3000
+    x = (rng.standard_normal(n) * 2).astype(np.float32)
+    xpath = str(tmp_path / "x.bin")
+    x.tofile(xpath)
+    g = O.global_scale(O.tensor_amax(x))
+    rc, rs, rf, rse = O.quantize_blocks(x, 0, n // 16, g, -2, 6)
+    rd = O.dequantize(rc, rs, g)
+    paths = {}
+    for k, a in (("codes", rc), ("scales", rs), ("f", rf), ("sse", rse), ("deq", rd)):
+        paths[k] = str(tmp_path / (k + ".bin"))
+        a.tofile(paths[k])
+    tot = FS.oracle_compare(xpath, 0, n, g, -2, 6, paths, processes=3)
+    assert tot["blocks"] == n // 16 and all(tot[k] == 0 for k in ("codes", "scales", "f", "sse", "deq"))
+    assert np.array_equal(tot["hist"], np.bincount(rf.astype(np.int64) + 128, minlength=256))
+    bad_c, bad_d = rc.copy(), rd.copy()
+    bad_c[8 * 1234 + 3] ^= 0x10
+    bad_d[16 * 2500 + 7] = np.nextafter(bad_d[16 * 2500 + 7], np.float32(np.inf))
+    bad_c.tofile(paths["codes"])
+    bad_d.tofile(paths["deq"])
+    tot = FS.oracle_compare(xpath, 0, n, g, -2, 6, paths, processes=3)
+    assert (tot["codes"], tot["codes_first"], tot["deq"], tot["deq_first"], tot["scales"]) == (1, 1234, 1, 2500, 0)
