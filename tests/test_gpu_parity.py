@@ -341,3 +341,30 @@ def test_exact_ties_on_dyadic_blocks():
     for gin in (2.0 ** -6, 2.0 ** -8, 3.0 * 2.0 ** -9):
         check_quantize(x, -2, 6, gscale_in=gin)
         check_quantize(x, -8, 8, gscale_in=gin)
+
+
+def test_certificate_blocks_on_the_thread_per_block_kernel():
+    """The adversarial blocks of tests/golden/certificate_blocks.txt (the fast score orders the two best
+    candidates against the definition, or breaks a definition tie, or sits at the edge of the covered
+    magnitude range) through the thread-per-block kernel (launch policy forced), each group of blocks
+    sharing a tensor scale and window interleaved with ordinary blocks so that they sit in warps whose
+    other lanes are decided by the fast score: codes, scales, offsets and SSE bit-exact."""
+    from tests import certblocks
+    rows = certblocks.load()
+    groups = {}
+    for kind, g, f_lo, nc, x in rows:
+        groups.setdefault((float(g), f_lo, nc), []).append(x)
+    prev = nv.search_policy(0, 0)
+    try:
+        rng = np.random.default_rng(9)
+        for (g, f_lo, nc), blocks in groups.items():
+            adv = np.stack(blocks)
+            fill = (rng.standard_normal((31 * len(blocks), 16)) * np.abs(adv).max() / 3).astype(np.float32)
+            allb = np.empty((32 * len(blocks), 16), np.float32)
+            allb[::32] = adv
+            rest = np.ones(len(allb), bool)
+            rest[::32] = False
+            allb[rest] = fill
+            check_quantize(torch.from_numpy(allb.reshape(-1)), f_lo, f_lo + nc - 1, gscale_in=g)
+    finally:
+        nv.search_policy(*prev)

@@ -341,3 +341,34 @@ def test_fullsize_harness_counts_planted_mismatches(tmp_path):
     bad_d.tofile(paths["deq"])
     tot = FS.oracle_compare(xpath, 0, n, g, -2, 6, paths, processes=3)
     assert (tot["codes"], tot["codes_first"], tot["deq"], tot["deq_first"], tot["scales"]) == (1, 1234, 1, 2500, 0)
+
+
+def test_certificate_blocks_are_adversarial_and_never_certified_wrongly():
+    """tests/golden/certificate_blocks.txt: every "flip" block has its two best candidates ordered one way
+    by the definition (oracle) and the other way by the kernel's fast score (exact emulation), every "tie"
+    block has two best candidates with equal definition scores that the fast score tells apart, and the
+    emulated certificate defers all of them; "edge" blocks, when certified, get the definition's winner.
+    At least a few hundred such blocks (the GPU runs them in test_gpu_certificate_blocks)."""
+    from tests import certblocks, fastscore as FSC
+    rows = certblocks.load()
+    kinds = {k: sum(1 for r in rows if r[0] == k) for k in ("flip", "tie", "edge")}
+    assert kinds["flip"] >= 200 and kinds["tie"] >= 50 and kinds["edge"] >= 40, kinds
+    for kind, g, f_lo, nc, x in rows:
+        P = FSC.scores(x, g, f_lo, nc)
+        F = {}
+        for f in P:
+            _, _, fs, sse = O.search_block(x, g, f, f)
+            if fs == f:
+                F[f] = float(sse)
+        st, fc = FSC.certificate(x, g, f_lo, nc)
+        win = min(F, key=lambda f: (F[f], abs(f), f)) if F else None
+        if kind in ("flip", "tie"):
+            a, b = sorted(F, key=lambda f: (F[f], abs(f), f))[:2]
+            if kind == "flip":
+                assert F[a] < F[b] and P[a] > P[b], (x, g)
+            else:
+                assert F[a] == F[b] and P[a] != P[b], (x, g)
+            assert st == "deferred", (kind, x, g)
+        elif st == "certified":
+            assert fc == win, (x, g)
+        assert O.search_block(x, g, f_lo, f_lo + nc - 1)[2] == (win if win is not None else -128)
