@@ -57,6 +57,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time the eager step only (no CUDA graph replay)")
     ap.add_argument("--kv-layers", type=int, default=32, help="kv_decode_layers: layers flushed per step (K and V each)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="default workload: skip the per-configuration lines of the other four workloads")
+    ap.add_argument("--config-steps", type=int, default=50, help="timed steps of each per-configuration run")
+    ap.add_argument("--with-configs", action="store_true", help="add the per-configuration lines at any --scale")
     return ap.parse_args()
 
 
@@ -1585,7 +1589,76 @@ def main():
             graph_used = False
             if overlap:
                 overlap["used_for_value"] = False
-    clocks = sampler.stop()   # sampled over the eager, graph, overlapped and fused timings
+    # Steady-state stream of tensors: the amax pass of step k+1 (HBM-bound) runs on a second stream beside the
+    # fused search of step k (bound by the FP32 pipes), each step with its own g word.  Every step still
+    # computes its own amax before its own search; only consecutive steps overlap.
+    pipelined = None
+    if not kv and world == 1 and flush is None and fused is not None:
+        aux = torch.cuda.Stream(dev)
+        amax2 = torch.empty(2, dtype=torch.float32, device=dev)
+        g2 = torch.empty(2, dtype=torch.float32, device=dev)
+
+        def run_pipelined(nsteps):
+            done = [None, None]
+            nv.tensor_amax(x, out=amax2[0:1])
+            nv.global_scale(amax2[0:1], out=g2[0:1])
+            ready = torch.cuda.Event()
+            ready.record(stream)
+            for k in range(nsteps):
+                nxt = None
+                if k + 1 < nsteps:
+                    j = (k + 1) % 2
+                    if done[j] is not None:
+                        aux.wait_event(done[j])      # step k-1's search has read g2[j]
+                    with torch.cuda.stream(aux):
+                        nv.tensor_amax(x, out=amax2[j:j + 1])
+                        nv.global_scale(amax2[j:j + 1], out=g2[j:j + 1])
+                    nxt = torch.cuda.Event()
+                    nxt.record(aux)
+                stream.wait_event(ready)
+                i = k % 2
+                nv.quantize_dequantize(x, args.f_lo, args.f_hi, gscale_in=g2[i:i + 1], codes=codes, scales=scales,
+                                       gscale=None, out=deq)
+                d = torch.cuda.Event()
+                d.record(stream)
+                done[i] = d
+                ready = nxt
+
+        run_pipelined(max(2, args.warmup))
+        torch.cuda.synchronize()
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pa.record(stream)
+        run_pipelined(args.steps)
+        pb.record(stream)
+        torch.cuda.synchronize()
+        pipe_ms = pa.elapsed_time(pb)
+        pipelined = {"ms_per_step": pipe_ms / args.steps, "streams": 2,
+                     "schedule": "amax of step k+1 beside the fused search of step k (separate g words)",
+                     "used_for_value": pipe_ms < elapsed_ms}
+        if pipe_ms < elapsed_ms:
+            elapsed_ms = pipe_ms
+            graph_used = False
+            fused["used_for_value"] = False
+            if overlap:
+                overlap["used_for_value"] = False
+    # the window sweep of the streaming configuration: the search pass alone for {0}, the default window
+    # and [-8,8], with the same g (CUDA events, mean of a few launches)
+    sweep = None
+    if not kv and world == 1:
+        sweep = {}
+        for lo, hi in ((0, 0), (args.f_lo, args.f_hi), (-8, 8)):
+            nv.quantize_ex(x, lo, hi, gscale_in=g, want_f=False, want_sse=False, codes=codes, scales=scales, gscale=None)
+            evs_s = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+            for a_, b_ in evs_s:
+                if flush is not None:
+                    flush.fill_(1.0)
+                a_.record(stream)
+                nv.quantize_ex(x, lo, hi, gscale_in=g, want_f=False, want_sse=False, codes=codes, scales=scales,
+                               gscale=None)
+                b_.record(stream)
+            torch.cuda.synchronize()
+            sweep[f"[{lo},{hi}]"] = statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs_s)
+    clocks = sampler.stop()   # sampled over the eager, graph, overlapped, fused and pipelined timings
     amax_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     q_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     dq_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -1617,7 +1690,7 @@ def main():
                     "traffic": None, "peak_source": peak_src, "bytes_per_launch": f_bytes}
     elif kv:
         launches = 5
-    elif fused and fused["used_for_value"]:
+    elif (fused and fused["used_for_value"]) or (pipelined and pipelined["used_for_value"]):
         # the step's dominant kernel is then the fused one: read x, write codes, scales and the values
         launches = 3
         f_bytes = n_q * esz + n_q // 2 + n_q // 16 + deq.element_size() * n_q
@@ -1649,7 +1722,12 @@ def main():
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / args.steps},
         "overlap": overlap,
         "fused": fused,
+        "pipelined": pipelined,
     }
+    if sweep:
+        base = amax_ms + sweep["[0,0]"]
+        line["window_sweep_ms"] = {"amax_and_g": amax_ms, "search": sweep,
+                                   "two_pass_over_max_scaling": {w: (amax_ms + t) / base for w, t in sweep.items()}}
     if not kv:
         line["stats"] = quant_stats(nv, x, g, deq, args.f_lo, args.f_hi, value / esz * 1e9)
         if world > 1:
@@ -1673,7 +1751,7 @@ def main():
         hs = [torch.empty(n // 16, dtype=torch.uint8, pin_memory=True) for _ in range(NB)]
         hg = [torch.empty(1, dtype=torch.float32, pin_memory=True) for _ in range(NB)]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        fused_step = bool(fused and fused["used_for_value"])
+        fused_step = bool((fused and fused["used_for_value"]) or (pipelined and pipelined["used_for_value"]))
         computed, read_back = [None] * NB, [None] * NB
 
         def e2e_step(k):
@@ -1745,11 +1823,47 @@ def main():
             "sample": f"{ns} elements of the {args.workload} recipe (CPU generator), one quantize + dequantize, "
                       f"{el:.1f} s single-threaded C",
         }
+    if (rank == 0 and world == 1 and args.workload == "stream_f32" and (args.scale == 1.0 or args.with_configs)
+            and not args.no_configs):
+        line["configs"] = config_lines(args)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+CONFIG_KEYS = ("value", "unit", "ms_per_step", "dtype", "roofline", "cpu_baseline", "quantize_two_pass", "breakdown_ms",
+               "clocks", "gpu_launches", "stats")
+
+
+def config_lines(args):
+    """The other four workloads (C1 act_f32, C2 act_bf16, C3 kv_bf16, C5 bev_f16), each measured by its own
+    run of this script (same metric: input GB/s of amax + g + ScaleSearch + dequantize), so that one default
+    run reports every configuration with its roofline and CPU baseline.  Each entry keeps the sub-run's
+    keys that describe its number; a failed sub-run is recorded as such."""
+    out = {}
+    for name in ("act_f32", "act_bf16", "kv_bf16", "bev_f16"):
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(args.config_steps),
+               "--warmup", str(max(3, args.warmup)), "--no-e2e", "--cpu-seconds", "2", "--no-configs",
+               "--f-lo", str(args.f_lo), "--f-hi", str(args.f_hi)]
+        try:
+            r = subprocess.run(cmd, capture_output=True, text=True, timeout=600,
+                               env={k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")})
+            rows = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+            d = json.loads(rows[-1]) if r.returncode == 0 and rows else None
+        except (subprocess.TimeoutExpired, ValueError):
+            d = None
+        if d is None:
+            out[name] = {"error": "sub-run failed"}
+            continue
+        e = {k: d[k] for k in CONFIG_KEYS if k in d}
+        e["workload"] = d["config"]["workload"]
+        e["steps"] = d["steps"]
+        if "roofline" in e and "quantize_two_pass" in d:
+            e["frac_of_8TBs_two_pass_quantize"] = d["quantize_two_pass"]["frac_of_8TBs"]
+        out[name] = e
+    return out
 
 
 if __name__ == "__main__":

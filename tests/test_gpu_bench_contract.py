@@ -42,6 +42,22 @@ def test_default_workload_line():
 
 
 @pytest.mark.gpu
+def test_default_line_carries_every_configuration():
+    """The default workload's line also reports C1, C2, C3 and C5 (each from its own run of the script) with
+    their roofline and CPU baseline, and the streaming window sweep ({0}, [-2,6], [-8,8])."""
+    d = _run("--scale", "0.01", "--steps", "3", "--warmup", "3", "--cpu-seconds", "0.3", "--no-e2e",
+             "--with-configs", "--config-steps", "3", timeout=900)
+    assert set(d["configs"]) == {"act_f32", "act_bf16", "kv_bf16", "bev_f16"}
+    for name, e in d["configs"].items():
+        assert "error" not in e, name
+        assert e["value"] > 0 and e["unit"] == "GB/s" and e["roofline"]["frac"] > 0
+        assert e["cpu_baseline"]["kind"] == "oracle" and e["workload"].startswith(name)
+    assert e["dtype"] == "f16" and d["configs"]["act_bf16"]["dtype"] == "bf16"
+    sw = d["window_sweep_ms"]
+    assert set(sw["search"]) == {"[0,0]", "[-2,6]", "[-8,8]"} and sw["two_pass_over_max_scaling"]["[0,0]"] == 1.0
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("workload,dtype", [("act_bf16", "bf16"), ("bev_f16", "f16")])
 def test_line_dtype_follows_the_workload(workload, dtype):
     """The line's dtype is the element type of the workload it measured."""
