@@ -263,7 +263,7 @@ def workload_config(args):
         "kv_bf16": "BF16 K [1,8,32768,128], N(0,1) + N(0,2) bias on 4 channels, seed 2",
         "bev_f16": "FP16 [6,30825,8,32] N(0,1) x level gain 1,2,4,8, seed 5",
     }
-    big = args.workload == "stream_f32"
+    big = args.workload == "stream_f32" and args.scale >= 0.125   # 512 MiB and more: no flush needed
     name = f"{args.workload} ({notes.get(args.workload, '')})"
     if args.scale != 1.0:
         name += f" scaled by {args.scale}"
@@ -273,7 +273,7 @@ def workload_config(args):
         "step": ("kv_mixed (sink/recent copy + FWHT-16 + amax + ScaleSearch) + dequantize BF16"
                  if args.workload == "kv_bf16" else
                  "amax + [allreduce max] + g + ScaleSearch quantize + dequantize"),
-        "l2": ("inputs larger than L2 (4 GiB per step per GPU), no flush" if big and args.scale == 1.0 else
+        "l2": ("inputs larger than L2 (at least 512 MiB per step per GPU), no flush" if big else
                "L2 flushed between steps by a 256 MiB write (not timed)"),
         "block": 16,
     }
