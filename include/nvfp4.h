@@ -297,6 +297,25 @@ int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs
                   const uint8_t* b_sf, const float* b_gscale, int64_t batch, int64_t M, int64_t N, int64_t K,
                   float alpha, void* d, int d_dtype, float* alpha_work, void* stream);
 
+/* nvfp4_gemm_nt for callers that cannot allocate device memory -- code running where cudaMalloc is not
+ * available to it or not allowed (a host framework that owns every device allocation through its own
+ * pool, a runtime that has reserved all device memory up front, code that must not allocate between
+ * setup and teardown) and so cannot provide the alpha_work word.  The paper has no counterpart: this is
+ * an interface choice of the library.
+ * Same arguments, results and errors as nvfp4_gemm_nt, without alpha_work: the scale word lives in a
+ * device array compiled into the library (one FP32 word, 256-byte aligned), present on every GPU that
+ * loads the library until the process exits.  The word does not grow with the sizes, so no size is too
+ * large for it; sizes are checked exactly as nvfp4_gemm_nt checks them.
+ * The first call on a device looks up that array's address (cudaGetSymbolAddress, no allocation) and
+ * returns NVFP4_ERR_CUDA if that fails; make that first call before any stream capture.  Nothing here
+ * calls cudaMalloc or cudaFree.  Each call overwrites the word before its product reads it, so nothing
+ * carries over from the previous call; but all calls on one device share the word, so two calls that can
+ * run at the same time on the GPU (different streams without ordering) race on it and may use each
+ * other's scale. */
+int nvfp4_gemm_nt_noalloc(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gscale,
+                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gscale, int64_t batch,
+                          int64_t M, int64_t N, int64_t K, float alpha, void* d, int d_dtype, void* stream);
+
 /* Softmax numerators for the P V^T product of FP4 attention ([SS] ScaleSearchAttention; the pages do
  * not say how P is formed, this is the flash-attention form).  s: scores [batch, Tq, Tk] FP32 (16-byte
  * aligned, Tk % 16 == 0).  For each row (b, q): m = max over the allowed keys (causal != 0: key k is

@@ -57,6 +57,7 @@ _SIGS = {
     "nvfp4_quantize_mma_t": (_I, [_P, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "nvfp4_kv_mixed_mma": (_I, [_P, _I64, _I64, _I64, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_gemm_nt": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P, _P]),
+    "nvfp4_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P]),
     "nvfp4_softmax_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_rows_divide": (_I, [_P, _P, _I64, _I64, _P]),
     "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),

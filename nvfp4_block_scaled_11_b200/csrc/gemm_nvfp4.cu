@@ -15,6 +15,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "cutlass/cutlass.h"
 #include "cute/tensor.hpp"
 #include "cutlass/detail/sm100_blockscaled_layout.hpp"
@@ -93,6 +95,30 @@ __global__ void gemm_alpha_kernel(const float* ga, const float* gb, float alpha,
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// The epilogue's scale word for nvfp4_gemm_nt_noalloc, in memory the library itself carries: a
+// file-scope device array, created on every GPU that loads the library and kept until the process exits.
+// It holds one FP32 word (padded to 256 bytes); the product needs that word whatever its sizes.
+constexpr int kAlphaScratchFloats = 1;
+static __device__ __align__(256) float g_alpha_scratch[kAlphaScratchFloats];
+
+// Device address of g_alpha_scratch on the current device, looked up once per device (host code sees only
+// a host-side stand-in under that name, so the address has to come from the runtime).
+constexpr int kMaxDevices = 64;
+int alpha_scratch_address(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  static std::mutex mu;
+  static float* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_alpha_scratch) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return NVFP4_OK;
+}
+
 }  // namespace nvfp4_consumer
 
 using namespace nvfp4_consumer;
@@ -129,6 +155,15 @@ int nvfp4_gemm_nt(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gs
     return Nvfp4Gemm<float>::run(a_codes, a_sf, b_codes, b_sf, (int)batch, (int)M, (int)N, (int)K, alpha_work, d, s);
   return Nvfp4Gemm<cutlass::bfloat16_t>::run(a_codes, a_sf, b_codes, b_sf, (int)batch, (int)M, (int)N, (int)K,
                                              alpha_work, d, s);
+}
+
+int nvfp4_gemm_nt_noalloc(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_gscale,
+                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_gscale, int64_t batch,
+                          int64_t M, int64_t N, int64_t K, float alpha, void* d, int d_dtype, void* stream) {
+  float* work = nullptr;
+  if (int rc = alpha_scratch_address(&work)) return rc;
+  return nvfp4_gemm_nt(a_codes, a_sf, a_gscale, b_codes, b_sf, b_gscale, batch, M, N, K, alpha, d, d_dtype, work,
+                       stream);
 }
 
 int nvfp4_gemm_sf_offsets(int64_t rows, int64_t K, int64_t batch, int64_t* out) {
