@@ -477,27 +477,34 @@ __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// Linear 16-bit sources: each thread's next block (32 bytes) is copied by cp.async into the thread's own
-// shared-memory slot while the current block is searched, and widened only when it is used.  This keeps
-// the prefetched block out of registers (the register copy of a widened block costs 16 moves per block;
-// measured on B200 with the C2 BF16 activations: search 130 -> 120 us, fused round trip 140 -> 130 us).
-// Two slots per thread; the two 16-byte chunks of threads 4..7 of each group of 8 are swapped so that
-// a quarter-warp's 16-byte accesses fall in distinct banks.
-template <int DT, int NC, bool WANT_SSE, int DEQ>
-__device__ __forceinline__ void search_linear_staged(const QuantParams& p, const CandEntry* tab, const float* thr,
-                                                     float inv6g, bool g_bad, int64_t (*defer)[kDeferCap]) {
-  static_assert(DT != DT_F32, "16-bit sources: a block is two 16-byte chunks");
+// 16-bit sources whose blocks are 32 contiguous bytes (linear tensors and the KV layout's middle tokens):
+// each thread's next block is copied by cp.async into the thread's own shared-memory slot while the
+// current block is searched, and widened (and rotated, when the path rotates) only when it is used.  This
+// keeps the prefetched block out of registers (the register copy of a widened block costs 16 moves per
+// block; measured on B200 with the C2 BF16 activations: search 130 -> 120 us, fused round trip 140 ->
+// 130 us).  Two slots per thread; the two 16-byte chunks of threads 4..7 of each group of 8 are swapped
+// so that a quarter-warp's 16-byte accesses fall in distinct banks.
+template <int DT, int MODE, bool ROT, int NC, bool WANT_SSE, int DEQ>
+__device__ __forceinline__ void search_staged(const QuantParams& p, const CandEntry* tab, const float* thr,
+                                              float inv6g, bool g_bad, int64_t (*defer)[kDeferCap]) {
+  static_assert(DT != DT_F32 && (MODE == SRC_LINEAR || MODE == SRC_KV), "32-byte contiguous blocks");
   __shared__ uint4 stage[2][256 * 2];
   const int t = threadIdx.x;
   const int sw = (t >> 2) & 1;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   int64_t b = (int64_t)blockIdx.x * blockDim.x + t;
+  KvCursor kc;   // KV mode: the split of the block being prefetched, carried along the loop
   auto issue = [&](int64_t bb, int buf) {
-    const char* src = p.x + bb * 32;
+    const char* src;
+    if constexpr (MODE == SRC_KV) src = p.x + kc.elem(p.T, p.sink, p.D) * 2;
+    else src = p.x + bb * 32;
     cp_async16((uint32_t)__cvta_generic_to_shared(&stage[buf][2 * t + sw]), src);
     cp_async16((uint32_t)__cvta_generic_to_shared(&stage[buf][2 * t + (sw ^ 1)]), src + 16);
   };
-  if (b < p.nblocks) issue(b, 0);
+  if (b < p.nblocks) {
+    if constexpr (MODE == SRC_KV) kc.init(b, stride, p.Tm, p.bpr);
+    issue(b, 0);
+  }
   cp_async_commit();
   const int lane = t & 31, warp = t >> 5;
   const unsigned lanes_below = (1u << lane) - 1u;
@@ -506,14 +513,17 @@ __device__ __forceinline__ void search_linear_staged(const QuantParams& p, const
   auto flush = [&]() {
     __syncwarp();
     for (int e = lane; e < dcount; e += 32)
-      quantize_block_def<DT, SRC_LINEAR, false, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, dlist[e], p.v8 != 0);
+      quantize_block_def<DT, MODE, ROT, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, dlist[e], p.v8 != 0);
     __syncwarp();
     dcount = 0;
   };
   int buf = 0;
   for (int64_t wb = b - lane; wb < p.nblocks; wb += stride, b += stride) {
     const bool active = b < p.nblocks;
-    if (b + stride < p.nblocks) issue(b + stride, buf ^ 1);
+    if (b + stride < p.nblocks) {
+      if constexpr (MODE == SRC_KV) kc.advance();
+      issue(b + stride, buf ^ 1);
+    }
     cp_async_commit();
     cp_async_wait1();   // this thread's copy of block b has landed
     u64 x2[8];
@@ -526,8 +536,7 @@ __device__ __forceinline__ void search_linear_staged(const QuantParams& p, const
       for (int k = 0; k < 8; ++k) x2[k] = pk2(x[2 * k], x[2 * k + 1]);
     }
     buf ^= 1;
-    const bool deferred = active && quantize_block_fast<SRC_LINEAR, false, NC, WANT_SSE, DEQ>(p, tab, thr, inv6g,
-                                                                                               g_bad, b, x2);
+    const bool deferred = active && quantize_block_fast<MODE, ROT, NC, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, b, x2);
     if constexpr (NC > 1) {
       const unsigned m = __ballot_sync(0xFFFFFFFFu, deferred);
       if (m) {
@@ -542,9 +551,9 @@ __device__ __forceinline__ void search_linear_staged(const QuantParams& p, const
   }
 }
 
-// Linear 16-bit sources take the shared-memory staged loop above; the others prefetch into registers.
+// 16-bit linear and KV sources take the shared-memory staged loop above; the others prefetch into registers.
 template <int DT, int MODE, bool ROT>
-constexpr bool kStaged = MODE == SRC_LINEAR && DT != DT_F32 && !ROT;
+constexpr bool kStaged = (MODE == SRC_LINEAR || MODE == SRC_KV) && DT != DT_F32;
 
 template <int DT, int MODE, bool ROT, int NC, bool WANT_SSE, int DEQ = -1>
 __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search_kernel(QuantParams p) {
@@ -577,7 +586,7 @@ __global__ void __launch_bounds__(256, NVFP4_SEARCH_CTAS_PER_SM) quantize_search
   __syncthreads();
   const float inv6g = __frcp_rn(__fmul_rn(6.0f, g));
   if constexpr (kStaged<DT, MODE, ROT>) {
-    search_linear_staged<DT, NC, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, defer);
+    search_staged<DT, MODE, ROT, NC, WANT_SSE, DEQ>(p, tab, thr, inv6g, g_bad, defer);
     return;
   }
 
