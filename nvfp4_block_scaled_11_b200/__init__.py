@@ -60,6 +60,8 @@ _SIGS = {
     "nvfp4_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _P, _I, _P]),
     "nvfp4_softmax_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_rows_divide": (_I, [_P, _P, _I64, _I64, _P]),
+    "nvfp4_attention_fused": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _I,
+                                   _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),
 }
 
@@ -646,6 +648,52 @@ def _prologue_operand(x: torch.Tensor, rotate: bool, signs: int, f_lo: int, f_hi
     if rotate:
         x = hadamard16(x, out_dtype=torch.float32, signs=signs)
     return quantize_mma(x, f_lo, f_hi)
+
+
+def attention_fused(qc, qsf, qg, kc, ksf, kg, vc_t, vsf_t, vg, causal: bool = False, q_offset: int = 0,
+                    alpha: float = 1.0, f_lo: int = -2, f_hi: int = 6, verify: bool = False):
+    """nvfp4_attention_fused on NVFP4 operands: q (codes [H, Tq, D/2], tile-layout scales, g), k likewise for
+    [H, Tk, D], v transposed (codes [H, D, Tk/2] and the tile layout of [D, Tk] matrices, as quantize_mma_t
+    gives them).  Returns (O [H, Tq, D] float32, row_max, row_sum), and with verify=True also the scores
+    [H, Tq, Tk] and P~ (codes, tile-layout scales)."""
+    for t_, nm in ((qc, "q codes"), (qsf, "q scales"), (qg, "q g"), (kc, "k codes"), (ksf, "k scales"), (kg, "k g"),
+                   (vc_t, "v codes"), (vsf_t, "v scales"), (vg, "v g")):
+        _cuda(t_, nm)
+    H, Tq, D = qc.shape[0], qc.shape[1], 2 * qc.shape[2]
+    Tk = kc.shape[1]
+    dev = qc.device
+    out = torch.empty((H, Tq, D), dtype=torch.float32, device=dev)
+    m = torch.empty(H * Tq, dtype=torch.float32, device=dev)
+    l = torch.empty(H * Tq, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    s_out = p_codes = p_sf = None
+    if verify:
+        s_out = torch.zeros((H, Tq, Tk), dtype=torch.float32, device=dev)
+        p_codes = torch.full((H, Tq, Tk // 2), 0xEE, dtype=torch.uint8, device=dev)   # every byte is written
+        p_sf = torch.full((max(sf_mma_bytes(Tq, Tk, H), 1),), 0xEE, dtype=torch.uint8, device=dev)
+    _check(lib().nvfp4_attention_fused(_ptr(qc), _ptr(qsf), _ptr(qg), _ptr(kc), _ptr(ksf), _ptr(kg), _ptr(vc_t),
+                                       _ptr(vsf_t), _ptr(vg), H, Tq, Tk, D, float(alpha), int(bool(causal)), q_offset,
+                                       f_lo, f_hi, _ptr(out), _ptr(m), _ptr(l), _ptr(s_out), _ptr(p_codes),
+                                       _ptr(p_sf), _ptr(status), _stream(qc)))
+    if verify:
+        return out, m, l, s_out, p_codes, p_sf, status
+    return out, m, l
+
+
+def attention_fp4_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, rotate: bool = True,
+                        scale: float | None = None, f_lo: int = -2, f_hi: int = 6, signs: int = 0):
+    """attention_fp4 with the scores kept on chip: the same NVFP4 prologue (Q and K rotated and quantized into
+    the tile layout, V quantized along the tokens), then nvfp4_attention_fused.  q [H, Tq, D], k and v
+    [H, Tk, D] with D = 128, Tq % 128 == 0, Tk % 64 == 0.  Returns O [H, Tq, D] float32."""
+    H, Tq, D = q.shape
+    Tk = k.shape[1]
+    scale = D ** -0.5 if scale is None else scale
+    qc, qsf, qg = _prologue_operand(q, rotate, signs, f_lo, f_hi)
+    kc, ksf, kg = _prologue_operand(k, rotate, signs, f_lo, f_hi)
+    vc, vsf, vg = quantize_mma_t(v.contiguous(), f_lo, f_hi)
+    o, _, _ = attention_fused(qc.view(H, Tq, D // 2), qsf, qg, kc.view(H, Tk, D // 2), ksf, kg,
+                              vc.view(H, D, Tk // 2), vsf, vg, causal, Tk - Tq, scale, f_lo, f_hi)
+    return o
 
 
 def attention_fp4(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, rotate: bool = True,

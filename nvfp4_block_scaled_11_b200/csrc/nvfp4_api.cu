@@ -11,6 +11,7 @@
 
 #include "../../include/nvfp4.h"
 #include "attention.cuh"
+#include "attn_fused.cuh"
 #include "lanes.cuh"
 #include "msda.cuh"
 #include "search.cuh"
@@ -688,6 +689,52 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
   else NVFP4_SOFTMAX(17);
 #undef NVFP4_SOFTMAX
   return last_error();
+}
+
+}  // extern "C"
+
+// One launch of the fused attention kernel for window width NC; its shared-memory limit is raised once per
+// instantiation (each kernel has its own attribute).
+template <int NC>
+int launch_attn_fused(const AttnFusedParams& a, dim3 grid, cudaStream_t st) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(attn_fused_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAfSmemBytes);
+  });
+  if (attr != cudaSuccess) return NVFP4_ERR_CUDA;
+  attn_fused_kernel<NC><<<grid, kAfThreads, kAfSmemBytes, st>>>(a);
+  return last_error();
+}
+
+extern "C" {
+
+int nvfp4_attention_fused(const uint8_t* q_codes, const uint8_t* q_sf, const float* q_gscale, const uint8_t* k_codes,
+                          const uint8_t* k_sf, const float* k_gscale, const uint8_t* v_codes_t, const uint8_t* v_sf_t,
+                          const float* v_gscale, int64_t H, int64_t Tq, int64_t Tk, int64_t D, float alpha, int causal,
+                          int64_t q_offset, int f_lo, int f_hi, float* out, float* row_max, float* row_sum,
+                          float* s_out, uint8_t* p_codes, uint8_t* p_sf, int* status, void* stream) {
+  const int nc = f_hi - f_lo + 1;
+  if (!window_ok(f_lo, f_hi) || (nc != 1 && nc != 9 && nc != 17)) return NVFP4_ERR_ARG;
+  if (H < 0 || Tq < 0 || Tk < 0 || D != kAfD || Tq % kAfBM != 0 || Tk % kAfBN != 0) return NVFP4_ERR_SIZE;
+  if (H > 65535 || checked_prod({H, Tq, Tk}) < 0 || checked_prod({H, Tq, D}) < 0) return NVFP4_ERR_SIZE;
+  if (H == 0 || Tq == 0) return NVFP4_OK;
+  if (Tk == 0) return NVFP4_ERR_SIZE;   // no keys: nothing to attend to
+  if (!q_codes || !q_sf || !q_gscale || !k_codes || !k_sf || !k_gscale || !v_codes_t || !v_sf_t || !v_gscale ||
+      !out || !row_max || !row_sum || ((p_codes == nullptr) != (p_sf == nullptr)))
+    return NVFP4_ERR_ARG;
+  if (!aligned(q_codes, 8) || !aligned(k_codes, 8) || !aligned(v_codes_t, 8) || !aligned(out, 16) ||
+      !aligned(q_gscale, 4) || !aligned(k_gscale, 4) || !aligned(v_gscale, 4) || !aligned(row_max, 4) ||
+      !aligned(row_sum, 4) || (s_out && !aligned(s_out, 16)) || (p_codes && !aligned(p_codes, 8)) ||
+      (status && !aligned(status, 4)))
+    return NVFP4_ERR_ALIGN;
+  AttnFusedParams a{q_codes, q_sf, q_gscale, k_codes, k_sf, k_gscale, v_codes_t, v_sf_t, v_gscale, H, Tq, Tk,
+                    alpha, causal ? 1 : 0, q_offset, f_lo, f_hi, out, row_max, row_sum, s_out, p_codes, p_sf, status};
+  const dim3 grid((unsigned)(Tq / kAfBM), (unsigned)H);
+  cudaStream_t st = S(stream);
+  if (nc == 9) return launch_attn_fused<9>(a, grid, st);
+  if (nc == 1) return launch_attn_fused<1>(a, grid, st);
+  return launch_attn_fused<17>(a, grid, st);
 }
 
 int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream) {

@@ -1,0 +1,122 @@
+"""The fused FP4-attention kernel (nvfp4_attention_fused) against the oracle, stage by stage, on the
+kernel's own intermediate values (returned only when asked for, for verification):
+* S: each score within the FP32-accumulation bound (D + 4) 2^-24 |alpha g_q g_k| sum_d |q_d k_d| of the
+  exact product of the same NVFP4 operands;
+* P~: the oracle's softmax quantizer applied to the kernel's scores gives the kernel's codes, tile-layout
+  scales and row maxima bit for bit, and its row sums within the FP32 summation bound;
+* O: each element within (Tk + 4) 2^-24 g_p g_v sum_k |p_k v_k| / l of the exact product of the oracle's
+  P~ and V divided by the kernel's row sum, plus the division's rounding."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_11_b200 as nv
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+U = 2.0 ** -24
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _inputs(H, Tq, Tk, seed, D=128):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((H, Tq, D), generator=g).to(torch.bfloat16)
+    k = (torch.randn((H, Tk, D), generator=g) * 1.3).to(torch.bfloat16)
+    v = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+def _check(H, Tq, Tk, causal, q_offset, window, seed):
+    D = 128
+    q, k, v = _inputs(H, Tq, Tk, seed)
+    f_lo, f_hi = window
+    qc, qsf, qg = nv._prologue_operand(q.cuda(), True, 0, f_lo, f_hi)
+    kc, ksf, kg = nv._prologue_operand(k.cuda(), True, 0, f_lo, f_hi)
+    vc, vsf, vg = nv.quantize_mma_t(v.cuda(), f_lo, f_hi)
+    alpha = D ** -0.5
+    out, m, l, s, pc, psf, status = nv.attention_fused(
+        qc.view(H, Tq, D // 2), qsf, qg, kc.view(H, Tk, D // 2), ksf, kg, vc.view(H, D, Tk // 2), vsf, vg,
+        causal, q_offset, alpha, f_lo, f_hi, verify=True)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    # operands from the oracle (linear scales), to form the exact products
+    rq = O.hadamard16(_u16(q).reshape(-1), dtype=O.BF16, out_dtype=O.F32)
+    rk = O.hadamard16(_u16(k).reshape(-1), dtype=O.BF16, out_dtype=O.F32)
+    rqc, rqs, rqg, _, _ = O.quantize(rq, f_lo, f_hi)
+    rkc, rks, rkg, _, _ = O.quantize(rk, f_lo, f_hi)
+    vt = np.ascontiguousarray(np.swapaxes(_u16(v).reshape(H, Tk, D), 1, 2)).reshape(-1)
+    rvc, rvs, rvg, _, _ = O.quantize(vt, f_lo, f_hi, dtype=O.BF16)
+    assert qg.item() == rqg and kg.item() == rkg and vg.item() == rvg
+    assert np.array_equal(qc.cpu().numpy().reshape(-1), rqc) and np.array_equal(kc.cpu().numpy().reshape(-1), rkc)
+    # S on the tiles the kernel forms (every tile holding an allowed key of some row of the CTA)
+    s_h = s.cpu().numpy().astype(np.float64)
+    s_ref = O.gemm_nt(rqc, rqs, rqg, rkc, rks, rkg, Tq, Tk, D, alpha, H)
+    mag = np.stack([np.abs(O.block_values(rqc.reshape(H, -1)[h], rqs.reshape(H, -1)[h], Tq, D)) @
+                    np.abs(O.block_values(rkc.reshape(H, -1)[h], rks.reshape(H, -1)[h], Tk, D)).T for h in range(H)])
+    bound = (D + 4) * U * abs(alpha * float(rqg) * float(rkg)) * mag + 1e-37
+    qi = np.arange(Tq)[:, None]
+    cta_last = (qi // 128) * 128 + 127 + q_offset if causal else np.full_like(qi, Tk - 1)
+    formed = (np.arange(Tk)[None, :] // 64) * 64 <= cta_last
+    err = np.abs(s_h - s_ref)
+    assert (err[:, formed] <= bound[:, formed]).all()
+    # P~ from the kernel's scores
+    rc, rs, rm, rl, rg = O.softmax_quantize(s.cpu().numpy(), causal, q_offset, f_lo, f_hi)
+    assert np.array_equal(pc.cpu().numpy().reshape(-1), rc.reshape(-1))
+    assert np.array_equal(psf.cpu().numpy(), O.scales_to_mma(rs, H, Tq, Tk // 16))
+    assert np.array_equal(m.cpu().numpy(), rm.reshape(-1))
+    l_g = l.cpu().numpy().astype(np.float64).reshape(H, Tq)
+    assert (np.abs(l_g - rl) <= (Tk + 4) * U * rl).all()
+    # O
+    d_ref = O.gemm_nt(rc, rs, rg, rvc, rvs, rvg, Tq, D, Tk, 1.0, H)
+    pmag = np.stack([np.abs(O.block_values(rc.reshape(H, -1)[h], rs.reshape(H, -1)[h], Tq, Tk)) @
+                     np.abs(O.block_values(rvc.reshape(H, -1)[h], rvs.reshape(H, -1)[h], D, Tk)).T for h in range(H)])
+    o_h = out.cpu().numpy().astype(np.float64)
+    want = d_ref / l_g[..., None]
+    tol = (Tk + 4) * U * float(rg) * float(rvg) * pmag / l_g[..., None] + U * np.abs(o_h) + 1e-37
+    assert (np.abs(o_h - want) <= tol).all()
+    return out
+
+
+@pytest.mark.parametrize("H,Tq,Tk,causal,q_offset,window", [
+    (2, 128, 256, False, 0, (-2, 6)),
+    (1, 256, 512, True, 256, (-2, 6)),     # queries at the end of the keys
+    (1, 256, 256, True, 0, (-2, 6)),       # square causal: the first CTA skips the keys past its last row
+    (2, 128, 192, True, 64, (-8, 8)),
+    (1, 128, 64, False, 0, (0, 0)),        # one tile, max-scaling
+])
+def test_fused_attention_stages_match_oracle(H, Tq, Tk, causal, q_offset, window):
+    _check(H, Tq, Tk, causal, q_offset, window, seed=H * 1000 + Tk + Tq)
+
+
+def test_fused_attention_end_to_end_entry_point():
+    """attention_fp4_fused (prologue + fused kernel) returns the fused kernel's O for the prologue's
+    operands, and stays as close to float64 attention on the unquantized inputs as the unfused chain."""
+    H, Tq, Tk, D = 2, 128, 512, 128
+    q, k, v = _inputs(H, Tq, Tk, 7)
+    o_f = nv.attention_fp4_fused(q.cuda(), k.cuda(), v.cuda(), causal=True).cpu().double()
+    o_u = nv.attention_fp4(q.cuda(), k.cuda(), v.cuda(), causal=True).cpu().double()
+    sf = torch.einsum("hqd,hkd->hqk", q.double(), k.double()) * D ** -0.5
+    sf = sf.masked_fill(torch.arange(Tk)[None, :] > torch.arange(Tq)[:, None] + (Tk - Tq), float("-inf"))
+    of = torch.einsum("hqk,hkd->hqd", torch.softmax(sf, -1), v.double())
+    nae_f = ((o_f - of).abs().mean() / of.abs().mean()).item()
+    nae_u = ((o_u - of).abs().mean() / of.abs().mean()).item()
+    assert abs(nae_f - nae_u) < 0.01 * nae_u, (nae_f, nae_u)
+
+
+def test_fused_attention_argument_errors():
+    dev = "cuda"
+    z8 = torch.zeros(64, dtype=torch.uint8, device=dev)
+    g = torch.ones(1, dtype=torch.float32, device=dev)
+    L = nv.lib()
+    import ctypes
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    o = torch.zeros(128 * 128, dtype=torch.float32, device=dev)
+    args = lambda Tq, Tk, D, lo, hi: (P(z8), P(z8), P(g), P(z8), P(z8), P(g), P(z8), P(z8), P(g), 1, Tq, Tk, D,
+                                      ctypes.c_float(1.0), 0, 0, lo, hi, P(o), P(g), P(g), None, None, None, None, None)
+    assert L.nvfp4_attention_fused(*args(100, 64, 128, -2, 6)) == -2     # Tq % 128
+    assert L.nvfp4_attention_fused(*args(128, 48, 128, -2, 6)) == -2     # Tk % 64
+    assert L.nvfp4_attention_fused(*args(128, 64, 64, -2, 6)) == -2      # D != 128
+    assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 5)) == -1     # 8 offsets
