@@ -1209,6 +1209,72 @@ def run_attn(args, rank, world, dev):
         if graph_ms < elapsed_ms:
             elapsed_ms, graph_used = graph_ms, True
     stage = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(5)]
+    chain_o = o.clone()
+
+    # The same attention with the scores kept on chip: the prologue, then nvfp4_attention_fused (Q K^T,
+    # row maxima, numerators, their ScaleSearch and P~ V^T in one kernel).  Timed eagerly (per-stage events)
+    # and as a CUDA graph; the faster of the chain and this schedule sets `value`.
+    fo, fm, fl, fst = E(H, Tq, D), E(H * Tq), E(H * Tq), torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step_fused(evs=None):
+        if evs:
+            evs[0].record(stream)
+        nv.kv_mixed_mma(q4, 0, 0, True, args.f_lo, args.f_hi, codes=qc4, sf=qsf, gscale=qg)
+        nv.kv_mixed_mma(k4, 0, 0, True, args.f_lo, args.f_hi, codes=kc4, sf=ksf, gscale=kg)
+        nv.quantize_mma_t(v, args.f_lo, args.f_hi, codes=vc, sf=vsf, gscale=vg)
+        if evs:
+            evs[1].record(stream)
+        nv.attention_fused(qc, qsf, qg, kc, ksf, kg, vc, vsf, vg, True, Tk - Tq, scale, args.f_lo, args.f_hi,
+                           out=fo, m=fm, l=fl, status=fst)
+        if evs:
+            evs[2].record(stream)
+        return fo
+
+    fused = None
+    if world == 1 and Tq % 128 == 0 and Tk % 64 == 0 and D == 128:
+        for _ in range(args.warmup):
+            step_fused()
+        torch.cuda.synchronize()
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fa.record(stream)
+        for i in range(steps):
+            step_fused(fev[i])
+        fb.record(stream)
+        torch.cuda.synchronize()
+        fused_ms = fa.elapsed_time(fb)
+        fused_graph_ms = None
+        if not args.no_graph:
+            cgf = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step_fused()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(cgf, stream=side):
+                step_fused()
+            for _ in range(max(1, args.warmup)):
+                cgf.replay()
+            torch.cuda.synchronize()
+            fa.record(stream)
+            for _ in range(steps):
+                cgf.replay()
+            fb.record(stream)
+            torch.cuda.synchronize()
+            fused_graph_ms = fa.elapsed_time(fb)
+            del cgf
+        best_f = min(fused_ms, fused_graph_ms) if fused_graph_ms is not None else fused_ms
+        fused = {"ms_per_step": fused_ms / steps,
+                 "graph_ms_per_step": fused_graph_ms / steps if fused_graph_ms is not None else None,
+                 "prologue_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in fev),
+                 "kernel_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in fev),
+                 "status": int(fst.item()),
+                 "max_abs_diff_vs_chain": float((fo - chain_o).abs().max().item()),
+                 "used_for_value": best_f < elapsed_ms and fst.item() == 0}
+        if fused["used_for_value"]:
+            elapsed_ms = best_f
+            graph_used = fused_graph_ms is not None and fused_graph_ms <= fused_ms
+            o = fo
     if world > 1:
         t = torch.tensor([elapsed_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -1218,6 +1284,12 @@ def run_attn(args, rank, world, dev):
     fp4_peak = bf16_peak * FP4_PER_BF16
     hbm_peak, hsrc = peaks()
     sm_bytes = H * Tq * Tk * 4 + H * Tq * Tk // 2 + H * Tq * Tk // 16 + 2 * H * Tq * 4
+    # the fused kernel's arithmetic roofline: the certified fast score costs 3 FP32-pipe operations per
+    # candidate and element (multiply, mixed-precision subtract, square-accumulate); P~ has one element per
+    # allowed (query, key) pair and args.f_hi - args.f_lo + 1 candidates per block
+    allowed = sum(min(Tk, q_ + (Tk - Tq) + 1) for q_ in range(Tq)) * H
+    fused_fp32_ops = 3.0 * (args.f_hi - args.f_lo + 1) * allowed / 1e12 * 1e12
+    fp32_peak = 128 * 148 * 1.965e9 / 1e12
     # accuracy against full-precision attention on the last 64 queries of head 0
     qf, kf, vf = q[0, -64:].double(), k[0].double(), v[0].double()
     sref = (qf @ kf.T) * scale
@@ -1229,17 +1301,26 @@ def run_attn(args, rank, world, dev):
         "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 operands, f32 accumulation", "data": SOURCE_NOTE, "config": attn_config(args, (H, Tq, Tk, D)),
-        "roofline": {"bound": "hbm", "kernel": "softmax_quantize_kernel (reads the FP32 scores, writes NVFP4 P)",
-                     "achieved": sm_bytes / (stage[2] * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": sm_bytes / (stage[2] * 1e-3) / 1e9 / hbm_peak, "traffic": None, "peak_source": hsrc,
-                     "bytes_per_launch": sm_bytes},
+        "roofline": ({"bound": "alu", "kernel": "attn_fused_kernel (Q K^T, row maxima, numerators, ScaleSearch of "
+                      "P~ and P~ V^T in one kernel)",
+                      "achieved": fused_fp32_ops / (fused["kernel_ms"] * 1e-3) / 1e12,
+                      "peak": fp32_peak, "unit": "TFLOP/s", "frac": fused_fp32_ops / (fused["kernel_ms"] * 1e-3) / 1e12 / fp32_peak,
+                      "traffic": None, "peak_source": "FP32 pipes: 128 lanes x 148 SMs x 1.965 GHz (one operation per lane per cycle)",
+                      "ops_per_launch": fused_fp32_ops,
+                      "ops": "3 FP32-pipe operations per scored candidate and element of P~ (9 candidates, allowed keys)"}
+                     if fused and fused["used_for_value"] else
+                     {"bound": "hbm", "kernel": "softmax_quantize_kernel (reads the FP32 scores, writes NVFP4 P)",
+                      "achieved": sm_bytes / (stage[2] * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                      "frac": sm_bytes / (stage[2] * 1e-3) / 1e9 / hbm_peak, "traffic": None, "peak_source": hsrc,
+                      "bytes_per_launch": sm_bytes}),
+        "fused": fused,
         "products": {"qk_tflops": 2.0 * H * Tq * Tk * D / (stage[1] * 1e-3) / 1e12,
                      "pv_tflops": 2.0 * H * Tq * Tk * D / (stage[3] * 1e-3) / 1e12,
                      "fp4_peak": fp4_peak, "peak_source": f"{src} bf16 burst x {FP4_PER_BF16:g}"},
         "breakdown_ms": {"rotate_and_quantize_qkv": stage[0], "qk_product": stage[1], "softmax_quantize": stage[2],
                          "pv_product": stage[3], "rows_divide": stage[4]},
         "normalised_abs_error_vs_fp64_attention": nae,
-        "gpu_launches": 18 * steps,   # 15 kernels + 3 memsets of the tensor-scale words
+        "gpu_launches": (10 if fused and fused["used_for_value"] else 18) * steps,   # kernels + tensor-scale memsets
         "clocks": clocks,
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps,
                        "v_quantize_on_second_stream": v_overlap_used},

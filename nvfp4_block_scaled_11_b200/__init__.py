@@ -651,7 +651,8 @@ def _prologue_operand(x: torch.Tensor, rotate: bool, signs: int, f_lo: int, f_hi
 
 
 def attention_fused(qc, qsf, qg, kc, ksf, kg, vc_t, vsf_t, vg, causal: bool = False, q_offset: int = 0,
-                    alpha: float = 1.0, f_lo: int = -2, f_hi: int = 6, verify: bool = False):
+                    alpha: float = 1.0, f_lo: int = -2, f_hi: int = 6, verify: bool = False, out=None, m=None, l=None,
+                    status=None):
     """nvfp4_attention_fused on NVFP4 operands: q (codes [H, Tq, D/2], tile-layout scales, g), k likewise for
     [H, Tk, D], v transposed (codes [H, D, Tk/2] and the tile layout of [D, Tk] matrices, as quantize_mma_t
     gives them).  Returns (O [H, Tq, D] float32, row_max, row_sum), and with verify=True also the scores
@@ -662,10 +663,12 @@ def attention_fused(qc, qsf, qg, kc, ksf, kg, vc_t, vsf_t, vg, causal: bool = Fa
     H, Tq, D = qc.shape[0], qc.shape[1], 2 * qc.shape[2]
     Tk = kc.shape[1]
     dev = qc.device
-    out = torch.empty((H, Tq, D), dtype=torch.float32, device=dev)
-    m = torch.empty(H * Tq, dtype=torch.float32, device=dev)
-    l = torch.empty(H * Tq, dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty((H, Tq, D), dtype=torch.float32, device=dev) if out is None else out
+    m = torch.empty(H * Tq, dtype=torch.float32, device=dev) if m is None else m
+    l = torch.empty(H * Tq, dtype=torch.float32, device=dev) if l is None else l
+    status = torch.zeros(1, dtype=torch.int32, device=dev) if status is None else status
+    _out(out, "out", torch.float32, H * Tq * D), _out(m, "m", torch.float32, H * Tq)
+    _out(l, "l", torch.float32, H * Tq), _out(status, "status", torch.int32, 1)
     s_out = p_codes = p_sf = None
     if verify:
         s_out = torch.zeros((H, Tq, Tk), dtype=torch.float32, device=dev)

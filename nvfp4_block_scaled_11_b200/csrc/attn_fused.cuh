@@ -155,8 +155,51 @@ __device__ __forceinline__ void af_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void af_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void af_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// One P~ block: ScaleSearch with the tensor scale of the table (the block's codes, scale byte and chosen
-// offset, as write_block would store them), without writing anything.
+// The definition for the blocks of a warp that the fast score left undecided, one block at a time with the
+// whole warp: lane j scores offset f_lo + j of the block (broadcast from its owner), and the smallest
+// (SSE, visiting rank) wins -- rank 0, 1, 2, 3, ... for f = 0, -1, +1, -2, ..., which is the definition's
+// "first strictly smaller SSE in that order" (the lane-group search's rule).  Called by all 32 lanes.
+template <int NC>
+__device__ __forceinline__ void af_resolve_deferred(unsigned mask, const u64 (&x2)[8], int c0, int f_lo, int f_hi,
+                                                    const CandEntry* tab, int& fstar) {
+  const int lane = threadIdx.x & 31;
+  while (mask) {
+    const int src = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    float xb[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float lo, hi;
+      upk2(x2[k], lo, hi);
+      xb[2 * k] = __shfl_sync(0xFFFFFFFFu, lo, src);
+      xb[2 * k + 1] = __shfl_sync(0xFFFFFFFFu, hi, src);
+    }
+    const int cb0 = __shfl_sync(0xFFFFFFFFu, c0, src);
+    const int f = f_lo + lane, c = cb0 + f;
+    u64 key = ~0ull;
+    if (lane < NC && f <= f_hi && c >= 1 && c <= 126) {
+      const CandEntry e = tab[c];
+      if (e.r != 0.0f) {
+        const float sse = block_sse_def(xb, e.d, e.r);
+        const uint32_t rank = f < 0 ? 2u * (uint32_t)(-f) - 1u : 2u * (uint32_t)f;
+        key = ((u64)__float_as_uint(sse) << 8) | rank;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) key = min(key, __shfl_xor_sync(0xFFFFFFFFu, key, o));
+    if (lane == src) {
+      if (key == ~0ull) {
+        fstar = -128;
+      } else {
+        const uint32_t rank = (uint32_t)(key & 0xFFu);
+        fstar = (rank & 1u) ? -(int)((rank + 1u) >> 1) : (int)(rank >> 1);
+      }
+    }
+  }
+}
+
+// One P~ block per lane: ScaleSearch with the tensor scale of the table (each lane's codes, scale byte, as
+// write_block would store them), without writing anything.  Called by all 32 lanes of a warp.
 template <int NC>
 __device__ __forceinline__ void af_quantize_block(const u64 (&x2)[8], const CandEntry* tab, const float* thr,
                                                   float inv6g, int f_lo, int f_hi, uint32_t& wlo, uint32_t& whi,
@@ -165,17 +208,19 @@ __device__ __forceinline__ void af_quantize_block(const u64 (&x2)[8], const Cand
   const bool poisoned = !(amax_b <= FLT_MAX);
   int c0 = 0, fstar = -128;
   float best = 0.0f;
+  bool deferred = false;
   if (!poisoned && amax_b != 0.0f) {
     c0 = c0_from_thresholds(thr, amax_b, inv6g);
     if (NC == 1) {
       const int c = c0 + f_lo;
       if (c >= 1 && c <= 126 && tab[c].r != 0.0f) fstar = f_lo;
-    } else if (!search_fast<NC, false>(x2, amax_b, c0, f_lo, tab, fstar, best)) {
-      float x[16];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) upk2(x2[k], x[2 * k], x[2 * k + 1]);
-      search_def(x, c0, f_lo, f_hi, tab, fstar, best);
+    } else {
+      deferred = !search_fast<NC, false>(x2, amax_b, c0, f_lo, tab, fstar, best);
     }
+  }
+  if constexpr (NC > 1) {
+    const unsigned dm = __ballot_sync(0xFFFFFFFFu, deferred);
+    if (dm) af_resolve_deferred<NC>(dm, x2, c0, f_lo, f_hi, tab, fstar);
   }
   wlo = whi = 0u;
   if (poisoned) {
@@ -202,7 +247,7 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
   __shared__ CandEntry tab_store[kTabSize];
   __shared__ float thr[128];
   __shared__ float red[4][kAfBM];
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) uint64_t bars[3];   // S buffer 0, S buffer 1, O
   __shared__ uint32_t tmem_slot;
   __shared__ int s_err;
   CandEntry* tab = tab_store + kTabPad;
@@ -229,8 +274,7 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (t == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(af_smem(&bars[0])));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(af_smem(&bars[1])));
+    for (int i = 0; i < 3; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(af_smem(&bars[i])));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_err = 0;
   }
@@ -251,33 +295,54 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
   af_fence_after();
   const uint32_t tmem = tmem_slot;
   const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
-  const uint32_t bar_s = af_smem(&bars[0]), bar_o = af_smem(&bars[1]);
-  uint32_t ph_s = 0, ph_o = 0;
+  // one completion barrier per S buffer (up to two products in flight, each buffer's phase tracked on its
+  // own) and one for O
+  const uint32_t bar_s[2] = {af_smem(&bars[0]), af_smem(&bars[1])}, bar_o = af_smem(&bars[2]);
+  uint32_t ph_s[2] = {0u, 0u}, ph_o = 0;
 
   const int64_t lim = a.causal ? q + a.q_offset : a.Tk - 1;                   // this row's last allowed key
   const int64_t lim_cta = a.causal ? q0 + kAfBM - 1 + a.q_offset : a.Tk - 1;  // the CTA's last
   const int64_t ntiles = a.Tk / kAfBN;
   const int64_t live = lim_cta < 0 ? 0 : min(ntiles, lim_cta / kAfBN + 1);    // tiles with an allowed key
 
-  // K tile j (64 keys x 8 blocks: one block per thread) into buffer b
-  auto load_k = [&](int64_t j, int b) {
-    const int key = t >> 3, kb = t & 7;
-    const int64_t kr = j * kAfBN + key;
-    uint4 lo, hi;
-    const uint2 cw = *reinterpret_cast<const uint2*>(a.k_codes + ((h * a.Tk + kr) * bpr_k + kb) * 8);
-    af_dequant_block(cw, a.k_sf[af_sf_index(h, kr, kb, a.Tk, bpr_k)], lo, hi);
-    af_store_block(sK(b), key, kb, kSboD, lo, hi);
+  // K tile j: 64 keys x 8 blocks, one block per thread (fetched into registers ahead of its use, then
+  // dequantized into buffer b); a tile past the end fetches nothing
+  struct RawBlock {
+    uint2 cw;
+    uint32_t sf;
   };
-  // V^T tile j (128 head-dimension rows x 4 key blocks: one block per thread) into buffer b
-  auto load_v = [&](int64_t j, int b) {
-    const int d = t >> 2, kb = t & 3;
-    const int64_t c = j * (kAfBN / 16) + kb;
-    uint4 lo, hi;
-    const uint2 cw = *reinterpret_cast<const uint2*>(a.v_codes + ((h * kAfD + d) * bpr_v + c) * 8);
-    af_dequant_block(cw, a.v_sf[af_sf_index(h, d, c, kAfD, bpr_v)], lo, hi);
-    af_store_block(sV(b), d, kb, kSboN, lo, hi);
+  auto fetch_k = [&](int64_t j) {
+    RawBlock rb{make_uint2(0u, 0u), 0u};
+    if (j < live) {
+      const int key = t >> 3, kb = t & 7;
+      const int64_t kr = j * kAfBN + key;
+      rb.cw = *reinterpret_cast<const uint2*>(a.k_codes + ((h * a.Tk + kr) * bpr_k + kb) * 8);
+      rb.sf = a.k_sf[af_sf_index(h, kr, kb, a.Tk, bpr_k)];
+    }
+    return rb;
   };
-  // S = Q K_j^T into TMEM columns 64 b .. 64 b + 63 (issued by thread 0, completion on bar_s)
+  auto store_k = [&](const RawBlock& rb, int b) {
+    uint4 lo, hi;
+    af_dequant_block(rb.cw, rb.sf, lo, hi);
+    af_store_block(sK(b), t >> 3, t & 7, kSboD, lo, hi);
+  };
+  // V^T tile j: 128 head-dimension rows x 4 key blocks, one block per thread
+  auto fetch_v = [&](int64_t j) {
+    RawBlock rb{make_uint2(0u, 0u), 0u};
+    if (j < live) {
+      const int d = t >> 2, kb = t & 3;
+      const int64_t c = j * (kAfBN / 16) + kb;
+      rb.cw = *reinterpret_cast<const uint2*>(a.v_codes + ((h * kAfD + d) * bpr_v + c) * 8);
+      rb.sf = a.v_sf[af_sf_index(h, d, c, kAfD, bpr_v)];
+    }
+    return rb;
+  };
+  auto store_v = [&](const RawBlock& rb, int b) {
+    uint4 lo, hi;
+    af_dequant_block(rb.cw, rb.sf, lo, hi);
+    af_store_block(sV(b), t >> 2, t & 3, kSboN, lo, hi);
+  };
+  // S = Q K_j^T into TMEM columns 64 b .. 64 b + 63 (issued by thread 0, completion on bar_s[b])
   auto mma_s = [&](int b) {
     if (t == 0) {
       af_fence_after();
@@ -286,7 +351,7 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
       for (int s = 0; s < kAfD / 16; ++s)
         af_mma(tmem + kAfBN * b, af_desc(af_smem(sQ) + 256 * s, kSboD), af_desc(af_smem(sK(b)) + 256 * s, kSboD),
                idesc, s > 0 ? 1u : 0u);
-      af_commit(bar_s);
+      af_commit(b ? bar_s[1] : bar_s[0]);
     }
   };
   // every thread waits; a wait that runs out stops the whole CTA (the flag is read after a barrier)
@@ -307,15 +372,24 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
 
   bool ok = true;
   // ---- sweep 1: row maxima over the allowed keys ----
+  // two products in flight: S(j + 1) runs while tile j's scores are read, and S(j + 2) is issued into
+  // tile j's buffers as soon as they are read; each K tile is fetched into registers two tiles ahead
   float m = -INFINITY;
-  for (int64_t j = 0; j < live && ok; ++j) {
-    const int b = (int)(j & 1);
-    load_k(j, b);
+  RawBlock kn = fetch_k(0), kn2 = fetch_k(1);
+  if (live > 0) {
+    store_k(kn, 0);
+    if (live > 1) store_k(kn2, 1);
+    kn = fetch_k(2);
+    kn2 = fetch_k(3);
     af_proxy_fence();
     af_fence_before();
     __syncthreads();
-    mma_s(b);
-    ok = wait_all(bar_s, ph_s);
+    mma_s(0);
+    if (live > 1) mma_s(1);
+  }
+  for (int64_t j = 0; j < live; ++j) {
+    const int b = (int)(j & 1);
+    ok = b ? wait_all(bar_s[1], ph_s[1]) : wait_all(bar_s[0], ph_s[0]);   // S(j) complete
     if (!ok) break;
     float s[16];
     scores(b, s);
@@ -323,6 +397,15 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (k0 + i <= lim) m = fmaxf(m, s[i]);
+    if (j + 2 < live) {
+      store_k(kn, b);                          // K(j + 2) into the buffer S(j) has finished reading
+      kn = kn2;
+      kn2 = fetch_k(j + 4);
+      af_proxy_fence();
+      af_fence_before();
+      __syncthreads();                         // K(j + 2) visible; every thread has read S(j)
+      mma_s(b);
+    }
   }
   if (ok) {
     red[cb][r] = m;
@@ -332,17 +415,35 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
   }
 
   // ---- sweep 2: numerators, their quantization, O += P~ V^T ----
+  // software-pipelined: S(j + 1) is formed while tile j's numerators are quantized, O += P~(j) V(j) runs
+  // while the next tiles are stored, and the raw K and V blocks are fetched a tile ahead of their store
   float l = 0.0f;
-  for (int64_t j = 0; j < live && ok; ++j) {
-    const int b = (int)(j & 1);
-    load_k(j, b);
-    load_v(j, b);
+  RawBlock kf = fetch_k(1), vf = fetch_v(1);
+  if (ok && live > 0) {
+    af_fence_before();
+    __syncthreads();          // every thread has read its last S of sweep 1
+    store_k(fetch_k(0), 0);
+    store_v(fetch_v(0), 0);
     af_proxy_fence();
     af_fence_before();
     __syncthreads();
-    mma_s(b);
-    ok = wait_all(bar_s, ph_s);
+    mma_s(0);
+  }
+  for (int64_t j = 0; j < live && ok; ++j) {
+    const int b = (int)(j & 1);
+    if (j + 1 < live) store_k(kf, b ^ 1);     // that buffer's last reader, S(j - 1), has completed
+    if (j > 0) {
+      ok = wait_all(bar_o, ph_o);              // O(j - 1) complete: its V and P~ buffers are free
+      if (!ok) break;
+    }
+    if (j + 1 < live) store_v(vf, b ^ 1);
+    kf = fetch_k(j + 2);
+    vf = fetch_v(j + 2);
+    af_proxy_fence();
+    af_fence_before();
+    ok = b ? wait_all(bar_s[1], ph_s[1]) : wait_all(bar_s[0], ph_s[0]);   // S(j) complete; K(j + 1), V(j + 1) visible
     if (!ok) break;
+    if (j + 1 < live) mma_s(b ^ 1);
     float s[16], x[16];
     scores(b, s);
     const int64_t k0 = j * kAfBN + 16 * cb;
@@ -394,8 +495,8 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
                idesc, (j > 0 || s2 > 0) ? 1u : 0u);
       af_commit(bar_o);
     }
-    ok = wait_all(bar_o, ph_o);
   }
+  if (ok && live > 0) ok = wait_all(bar_o, ph_o);   // the last O += P~ V^T
 
   // tiles past every row's last allowed key: P~ is a zero block there (scale 0, zero codes), which is what
   // the verification outputs receive; the products skip those tiles
