@@ -1215,6 +1215,9 @@ def run_attn(args, rank, world, dev):
     # row maxima, numerators, their ScaleSearch and P~ V^T in one kernel).  Timed eagerly (per-stage events)
     # and as a CUDA graph; the faster of the chain and this schedule sets `value`.
     fo, fm, fl, fst = E(H, Tq, D), E(H * Tq), E(H * Tq), torch.zeros(1, dtype=torch.int32, device=dev)
+    fused_ok = world == 1 and Tq % 128 == 0 and Tk % 64 == 0 and D == 128
+    f_splits = nv.attention_fused_splits(H, Tq, Tk) if fused_ok else 1
+    f_ws = nv.attention_fused_workspace(H, Tq, Tk, f_splits, dev) if fused_ok else None
 
     def step_fused(evs=None):
         if evs:
@@ -1225,13 +1228,13 @@ def run_attn(args, rank, world, dev):
         if evs:
             evs[1].record(stream)
         nv.attention_fused(qc, qsf, qg, kc, ksf, kg, vc, vsf, vg, True, Tk - Tq, scale, args.f_lo, args.f_hi,
-                           out=fo, m=fm, l=fl, status=fst)
+                           out=fo, m=fm, l=fl, status=fst, splits=f_splits, workspace=f_ws)
         if evs:
             evs[2].record(stream)
         return fo
 
     fused = None
-    if world == 1 and Tq % 128 == 0 and Tk % 64 == 0 and D == 128:
+    if fused_ok:
         for _ in range(args.warmup):
             step_fused()
         torch.cuda.synchronize()
@@ -1268,6 +1271,7 @@ def run_attn(args, rank, world, dev):
                  "graph_ms_per_step": fused_graph_ms / steps if fused_graph_ms is not None else None,
                  "prologue_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in fev),
                  "kernel_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in fev),
+                 "splits": f_splits,
                  "status": int(fst.item()),
                  "max_abs_diff_vs_chain": float((fo - chain_o).abs().max().item()),
                  "used_for_value": best_f < elapsed_ms and fst.item() == 0}
@@ -1301,8 +1305,8 @@ def run_attn(args, rank, world, dev):
         "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 operands, f32 accumulation", "data": SOURCE_NOTE, "config": attn_config(args, (H, Tq, Tk, D)),
-        "roofline": ({"bound": "alu", "kernel": "attn_fused_kernel (Q K^T, row maxima, numerators, ScaleSearch of "
-                      "P~ and P~ V^T in one kernel)",
+        "roofline": ({"bound": "alu", "kernel": "nvfp4_attention_fused (row maxima, numerators with their "
+                      "ScaleSearch and P~ V^T, combine; timed together)",
                       "achieved": fused_fp32_ops / (fused["kernel_ms"] * 1e-3) / 1e12,
                       "peak": fp32_peak, "unit": "TFLOP/s", "frac": fused_fp32_ops / (fused["kernel_ms"] * 1e-3) / 1e12 / fp32_peak,
                       "traffic": None, "peak_source": "FP32 pipes: 128 lanes x 148 SMs x 1.965 GHz (one operation per lane per cycle)",
@@ -1320,7 +1324,9 @@ def run_attn(args, rank, world, dev):
         "breakdown_ms": {"rotate_and_quantize_qkv": stage[0], "qk_product": stage[1], "softmax_quantize": stage[2],
                          "pv_product": stage[3], "rows_divide": stage[4]},
         "normalised_abs_error_vs_fp64_attention": nae,
-        "gpu_launches": (10 if fused and fused["used_for_value"] else 18) * steps,   # kernels + tensor-scale memsets
+        # kernels + tensor-scale memsets: 9 in the prologue, then the row maxima, the numerators and (with
+        # more than one key range) the combine; the chain: 18
+        "gpu_launches": ((11 + (f_splits > 1)) if fused and fused["used_for_value"] else 18) * steps,
         "clocks": clocks,
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps,
                        "v_quantize_on_second_stream": v_overlap_used},

@@ -335,31 +335,52 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
 /* x[r, c] = fl(x[r, c] / l[r]) for an FP32 [rows, cols] matrix (cols % 4 == 0, 16-byte aligned). */
 int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream);
 
-/* FP4 attention in one kernel ([SS] ScaleSearchAttention > native NVFP4 execution): the same result as
+/* FP4 attention with the scores kept on chip ([SS] ScaleSearchAttention > native NVFP4 execution): the
+ * same result as
  *   S = nvfp4_gemm_nt(Q, K, alpha);  nvfp4_softmax_quantize_mma(S, causal, q_offset, f_lo, f_hi);
  *   O = nvfp4_gemm_nt(P~, V^T);  nvfp4_rows_divide(O, row_sum)
- * without the scores leaving the chip: per head h and each 128 query rows, S is formed on the tensor cores
- * tile by tile (64 keys) in tensor memory, a first sweep takes the row maxima over the allowed keys, a
- * second forms the numerators, quantizes them (window [f_lo, f_hi] of 1, 9 or 17 offsets, tensor scale
- * fl(1/2688)) and accumulates P~ V^T.  Both products are FP32 sums of the exact products of the NVFP4
- * operands (the summation order differs from nvfp4_gemm_nt's); P~'s codes are those of
- * nvfp4_softmax_quantize_mma applied to this kernel's scores.
+ * without the scores leaving the SMs.  Per head and 128 query rows, the 64-key tiles holding an allowed key
+ * are cut into `splits` contiguous ranges.  Kernels run on `stream`: one forms S tile by tile on the
+ * tensor cores (in tensor memory) and takes each range's row maxima; one forms S again, the numerators
+ * exp(S - m) with m the maximum over all ranges, quantizes them (window [f_lo, f_hi] of 1, 9 or 17 offsets,
+ * tensor scale fl(1/2688)) and accumulates P~ V^T per range; with splits > 1 a third adds the ranges'
+ * accumulators and row sums and divides.  A first kernel writes K and V^T into the workspace as FP16 tiles.  Both products are FP32 sums of the exact products of the NVFP4
+ * operands (the summation order differs from nvfp4_gemm_nt's and depends on splits); P~'s codes are those
+ * of nvfp4_softmax_quantize_mma applied to this call's scores.
  * Operands (device, from the library's quantizers): q_codes [H, Tq, D/2] with q_sf the tile layout of the
  * H [Tq, D] matrices (nvfp4_quantize_mma / nvfp4_kv_mixed_mma) and q_gscale; k_* likewise for [H, Tk, D];
  * v_codes_t [H, D, Tk/2] with v_sf_t the tile layout of the H [D, Tk] matrices (nvfp4_quantize_mma_t).
+ * Code arrays 8-byte aligned, k_sf 4-byte aligned (NVFP4_ERR_ALIGN otherwise).
  * alpha multiplies the scores (with the two tensor scales, rounded as nvfp4_gemm_nt rounds them); causal:
- * key k allowed for query q iff k <= q + q_offset.  Outputs: out [H, Tq, D] FP32 (16-byte aligned), row_max
- * and row_sum [H * Tq].  Optional (NULL to skip; for verification): s_out [H, Tq, Tk] FP32 scores
- * (16-byte aligned; the 64-key tiles past the last allowed key of all 128 rows of a CTA are not formed and
- * not written), p_codes [H, Tq, Tk/2] and p_sf (tile layout of the H [Tq, Tk] matrices; zero blocks on
- * those tiles) -- both or neither; status: set nonzero if a wait
- * for the tensor cores ran out (that CTA's outputs are then not written).
- * Sizes: D == 128, Tq % 128 == 0, Tk % 64 == 0, Tk > 0, H <= 65535 (NVFP4_ERR_SIZE otherwise). */
+ * key k allowed for query q iff k <= q + q_offset.
+ * splits: 1 .. 64 (nvfp4_attention_fused_splits gives the count that fills the current device; any count
+ * gives a valid result).  workspace: caller-owned device memory, 16-byte aligned, at least
+ * nvfp4_attention_fused_workspace_bytes(H, Tq, Tk, splits) bytes (NVFP4_ERR_SIZE otherwise); it holds K
+ * and V^T expanded to FP16 tiles (exact) and the ranges' row maxima, row sums and accumulators between the
+ * kernels, so calls that share a workspace must be ordered on one stream.
+ * Outputs: out [H, Tq, D] FP32 (16-byte aligned), row_max and row_sum [H * Tq].  Optional (NULL to skip;
+ * for verification): s_out [H, Tq, Tk] FP32 scores (16-byte aligned; the 64-key tiles past the last
+ * allowed key of all 128 rows of a query tile are not formed and not written), p_codes [H, Tq, Tk/2] and
+ * p_sf (tile layout of the H [Tq, Tk] matrices; zero blocks on those tiles) -- both or neither; status: set
+ * nonzero if a wait for the tensor cores ran out (the outputs are then not valid).
+ * Sizes: D == 128, Tq % 128 == 0, Tk % 64 == 0, 0 < Tk < 2^26, H <= 65535 (NVFP4_ERR_SIZE otherwise). */
 int nvfp4_attention_fused(const uint8_t* q_codes, const uint8_t* q_sf, const float* q_gscale, const uint8_t* k_codes,
                           const uint8_t* k_sf, const float* k_gscale, const uint8_t* v_codes_t, const uint8_t* v_sf_t,
                           const float* v_gscale, int64_t H, int64_t Tq, int64_t Tk, int64_t D, float alpha, int causal,
-                          int64_t q_offset, int f_lo, int f_hi, float* out, float* row_max, float* row_sum,
-                          float* s_out, uint8_t* p_codes, uint8_t* p_sf, int* status, void* stream);
+                          int64_t q_offset, int f_lo, int f_hi, int splits, void* workspace, size_t workspace_bytes,
+                          float* out, float* row_max, float* row_sum, float* s_out, uint8_t* p_codes, uint8_t* p_sf,
+                          int* status, void* stream);
+
+/* The number of key ranges for nvfp4_attention_fused that fills the current device with equal waves of
+ * CTAs (from its SM count and the kernel's occupancy; ranges of at least 8 tiles), into *splits.  Host only
+ * (queries the device).  Sizes as nvfp4_attention_fused's (NVFP4_ERR_SIZE otherwise). */
+int nvfp4_attention_fused_splits(int64_t H, int64_t Tq, int64_t Tk, int* splits);
+
+/* Bytes of workspace nvfp4_attention_fused needs for H heads, Tq query rows, Tk keys and `splits` ranges:
+ * the ranges' row maxima (4 H Tq splits bytes) and, when splits > 1, row sums and O accumulators
+ * (4 H Tq splits (D + 1)), rounded up to 256, plus K and V^T in FP16 (2 H Tk D 2 bytes); 0 for invalid
+ * arguments.  Host only. */
+size_t nvfp4_attention_fused_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int splits);
 
 /* Host only, for verification: the byte offsets at which nvfp4_gemm_nt reads the scale of (matrix l,
  * row r, block column c), for l < batch, r < rows, c < K/16 in that (row-major) order, into out

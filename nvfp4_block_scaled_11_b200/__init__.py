@@ -61,7 +61,9 @@ _SIGS = {
     "nvfp4_softmax_quantize_mma": (_I, [_P, _I64, _I64, _I64, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
     "nvfp4_rows_divide": (_I, [_P, _P, _I64, _I64, _P]),
     "nvfp4_attention_fused": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_float, _I,
-                                   _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+                                   _I64, _I, _I, _I, _P, ctypes.c_size_t, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "nvfp4_attention_fused_splits": (_I, [_I64, _I64, _I64, _P]),
+    "nvfp4_attention_fused_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I]),
     "nvfp4_gemm_sf_offsets": (_I, [_I64, _I64, _I64, _P]),
 }
 
@@ -650,19 +652,40 @@ def _prologue_operand(x: torch.Tensor, rotate: bool, signs: int, f_lo: int, f_hi
     return quantize_mma(x, f_lo, f_hi)
 
 
+def attention_fused_splits(H: int, Tq: int, Tk: int) -> int:
+    """The key-range count nvfp4_attention_fused_splits chooses for the current device."""
+    s = ctypes.c_int(0)
+    _check(lib().nvfp4_attention_fused_splits(H, Tq, Tk, ctypes.byref(s)))
+    return s.value
+
+
+def attention_fused_workspace(H: int, Tq: int, Tk: int, splits: int, device) -> torch.Tensor:
+    """A workspace for nvfp4_attention_fused (uint8, nvfp4_attention_fused_workspace_bytes long)."""
+    n = lib().nvfp4_attention_fused_workspace_bytes(H, Tq, Tk, splits)
+    if n == 0:
+        raise NVFP4Error(-2)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
 def attention_fused(qc, qsf, qg, kc, ksf, kg, vc_t, vsf_t, vg, causal: bool = False, q_offset: int = 0,
                     alpha: float = 1.0, f_lo: int = -2, f_hi: int = 6, verify: bool = False, out=None, m=None, l=None,
-                    status=None):
+                    status=None, splits: int | None = None, workspace=None):
     """nvfp4_attention_fused on NVFP4 operands: q (codes [H, Tq, D/2], tile-layout scales, g), k likewise for
     [H, Tk, D], v transposed (codes [H, D, Tk/2] and the tile layout of [D, Tk] matrices, as quantize_mma_t
-    gives them).  Returns (O [H, Tq, D] float32, row_max, row_sum), and with verify=True also the scores
-    [H, Tq, Tk] and P~ (codes, tile-layout scales)."""
+    gives them).  splits: key ranges per query tile (None: attention_fused_splits); workspace: a uint8 tensor
+    of attention_fused_workspace's size (None: allocated here).  Returns (O [H, Tq, D] float32, row_max,
+    row_sum), and with verify=True also the scores [H, Tq, Tk] and P~ (codes, tile-layout scales)."""
     for t_, nm in ((qc, "q codes"), (qsf, "q scales"), (qg, "q g"), (kc, "k codes"), (ksf, "k scales"), (kg, "k g"),
                    (vc_t, "v codes"), (vsf_t, "v scales"), (vg, "v g")):
         _cuda(t_, nm)
     H, Tq, D = qc.shape[0], qc.shape[1], 2 * qc.shape[2]
     Tk = kc.shape[1]
     dev = qc.device
+    if splits is None:
+        splits = attention_fused_splits(H, Tq, Tk)
+    if workspace is None:
+        workspace = attention_fused_workspace(H, Tq, Tk, splits, dev)
+    _cuda(workspace, "workspace")
     out = torch.empty((H, Tq, D), dtype=torch.float32, device=dev) if out is None else out
     m = torch.empty(H * Tq, dtype=torch.float32, device=dev) if m is None else m
     l = torch.empty(H * Tq, dtype=torch.float32, device=dev) if l is None else l
@@ -676,8 +699,9 @@ def attention_fused(qc, qsf, qg, kc, ksf, kg, vc_t, vsf_t, vg, causal: bool = Fa
         p_sf = torch.full((max(sf_mma_bytes(Tq, Tk, H), 1),), 0xEE, dtype=torch.uint8, device=dev)
     _check(lib().nvfp4_attention_fused(_ptr(qc), _ptr(qsf), _ptr(qg), _ptr(kc), _ptr(ksf), _ptr(kg), _ptr(vc_t),
                                        _ptr(vsf_t), _ptr(vg), H, Tq, Tk, D, float(alpha), int(bool(causal)), q_offset,
-                                       f_lo, f_hi, _ptr(out), _ptr(m), _ptr(l), _ptr(s_out), _ptr(p_codes),
-                                       _ptr(p_sf), _ptr(status), _stream(qc)))
+                                       f_lo, f_hi, int(splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _ptr(out), _ptr(m), _ptr(l), _ptr(s_out), _ptr(p_codes), _ptr(p_sf),
+                                       _ptr(status), _stream(qc)))
     if verify:
         return out, m, l, s_out, p_codes, p_sf, status
     return out, m, l

@@ -1,17 +1,20 @@
-// attn_fused.cuh -- ScaleSearchAttention in one kernel on the sm_100a tensor cores.
+// attn_fused.cuh -- ScaleSearchAttention with the scores kept on chip, on the sm_100a tensor cores.
 //
 // "Search your block floating-point scales!" (gist.science summary of arXiv 2605.12464),
 // ScaleSearchAttention > native NVFP4 execution: Q K^T and P V^T run as NVFP4 products with FP32
 // accumulation and the softmax numerators P~ are ScaleSearch-quantized before the second product.  The
-// unfused chain writes the FP32 scores to HBM and reads them twice; here a CTA keeps its 128 query rows'
-// scores on chip:
-//   sweep 1: for each 64-key tile, S = alpha g_q g_k (Q K^T) into tensor memory (TMEM), row maxima over the
-//            allowed keys;
-//   sweep 2: S again, P~ = exp(S - m) (the same exp method as the oracle), ScaleSearch of every 16-key
-//            block with the tensor scale fl(1/2688) (the library's certified fast score, the definition
-//            where it cannot decide), the quantized block written to shared memory as the A operand of
-//            O += P~ V^T, accumulated in TMEM;
-//   epilogue: O = fl(fl(acc * fl(g_p g_v)) / l), l the FP32 sum of the numerators.
+// unfused chain writes the FP32 scores to HBM and reads them twice; here they never leave the SM.  The
+// 64-key tiles that hold an allowed key of a 128-row query tile are cut into `splits` contiguous ranges,
+// one CTA per (query tile, range, head), so that the grid fills every SM whatever the number of query
+// tiles, and three kernels run in turn:
+//   row maxima:  per range, S = alpha g_q g_k (Q K^T) tile by tile into tensor memory (TMEM) and the
+//                maximum over each row's allowed keys, written per range;
+//   numerators:  per range, S again, m = the maximum over the ranges, P~ = exp(S - m) (the same exp
+//                method as the oracle), ScaleSearch of every 16-key block with the tensor scale
+//                fl(1/2688) (the library's certified fast score, the definition where it cannot decide),
+//                the quantized block written to shared memory as the A operand of O += P~ V^T in TMEM;
+//                the range's O accumulator and row sum l are written out (or, with one range, the result);
+//   combine:     O = fl(fl(sum of the ranges' accumulators * fl(g_p g_v)) / l), l the sum of the ranges'.
 // Every result is the unfused chain's formula: P~'s codes are those of the definition applied to this
 // kernel's own scores, and both products are sums of exact terms accumulated in FP32.
 //
@@ -27,6 +30,12 @@
 //   (r mod 8) * 16 + (r div 8) * SBO + c * 128,   SBO = 128 * K / 8,
 // so one MMA instruction (K = 16: chunks 2s and 2s+1) reads from start + 256 s with LBO = 128 and that SBO.
 //
+// Schedule of the numerator kernel (one CTA barrier per tile): the products of tile j + 1 were issued a tile
+// earlier; a thread waits for S(j), reads its 16 scores, forms and quantizes its block of P~(j), waits for
+// O += P~(j-1) V(j-1) (long finished), stores its block of P~(j), of V(j) and of K(j+2); after the barrier
+// one thread issues O += P~(j) V(j) and S(j+2).  P~ and V have one buffer each, K and S two, so that the CTA
+// needs 96 KB of shared memory and 256 TMEM columns and two CTAs share an SM.
+//
 // Waits on the MMA completion barriers are bounded; a wait that runs out sets a status word, every thread
 // of the CTA leaves, the TMEM allocation is released and the outputs of that CTA are left unwritten.
 #pragma once
@@ -35,19 +44,26 @@
 
 namespace nvfp4 {
 
-constexpr int kAfBM = 128;        // query rows per CTA (the MMA's M)
-constexpr int kAfBN = 64;         // keys per tile (the first MMA's N, the second's K)
-constexpr int kAfD = 128;         // head dimension (the first MMA's K, the second's N)
-constexpr int kAfThreads = 512;   // 16 warps: 4 per TMEM lane quadrant, one 16-key block each per tile
-constexpr int kAfTmemCols = 256;  // S double buffer (2 x 64 columns) + O (128 columns)
-constexpr uint32_t kAfWaitLimit = 1u << 22;
+constexpr int kAfBM = 128;         // query rows per CTA (the MMA's M)
+constexpr int kAfBN = 64;          // keys per tile (the first MMA's N, the second's K)
+constexpr int kAfD = 128;          // head dimension (the first MMA's K, the second's N)
+constexpr int kAfThreads = 512;    // a half: 16 warps, 4 per TMEM lane quadrant, one 16-key block each per tile
+constexpr int kAfCtaThreads = 2 * kAfThreads;   // two halves, one key range each
+constexpr int kAfMaxSplits = 64;   // key ranges per query tile
+constexpr int kAfMaxStages = 4;       // row-max kernel: K tiles and S buffers per half
+constexpr int kAfTmemColsMax = 512;   // row-max kernel: per half four S buffers (4 x 64 columns)
+constexpr int kAfTmemCols = 512;      // numerator kernel: per half an S double buffer and O (128 columns)
 
-// dynamic shared memory: Q (128 x 128 FP16), K tiles (64 x 128) x 2, V^T tiles (128 x 64) x 2, P~ (128 x 64) x 2
+// dynamic shared memory: Q (128 x 128 FP16), shared by the halves, then per half
+//   row maxima:  K tiles (64 x 128) x 4;
+//   numerators:  K tiles x 2, V^T tiles (128 x 64) x 2 and a P~ tile (128 x 64)
 constexpr int kAfQBytes = kAfBM * kAfD * 2;
 constexpr int kAfKBytes = kAfBN * kAfD * 2;
 constexpr int kAfVBytes = kAfD * kAfBN * 2;
 constexpr int kAfPBytes = kAfBM * kAfBN * 2;
-constexpr int kAfSmemBytes = kAfQBytes + 2 * kAfKBytes + 2 * kAfVBytes + 2 * kAfPBytes;
+constexpr int kAfHalfBytes = 2 * kAfKBytes + 2 * kAfVBytes + kAfPBytes;
+constexpr int kAfMaxSmemBytes = kAfQBytes + 2 * kAfMaxStages * kAfKBytes;
+constexpr int kAfSmemBytes = kAfQBytes + 2 * kAfHalfBytes;
 
 struct AttnFusedParams {
   // operands: codes row-major (16-element blocks along the rows), scales in the tile layout, tensor scale
@@ -65,6 +81,12 @@ struct AttnFusedParams {
   int causal;               // key k allowed for query q iff k <= q + q_offset
   int64_t q_offset;
   int f_lo, f_hi;
+  int splits;               // key ranges per query tile
+  float* ws_max;            // [splits, H * Tq] the ranges' row maxima
+  float* ws_l;              // [splits, H * Tq] the ranges' row sums (splits > 1)
+  float* ws_o;              // [splits, H * Tq, D] the ranges' O accumulators (splits > 1)
+  uint8_t* kx;              // [H, Tk / 64] K tiles in FP16, the MMA's shared-memory layout (16 KB each)
+  uint8_t* vx;              // [H, Tk / 64] V^T tiles likewise
   float* out;               // [H, Tq, D]
   float* row_max;           // [H * Tq]
   float* row_sum;           // [H * Tq]
@@ -73,6 +95,20 @@ struct AttnFusedParams {
   uint8_t* p_sf;            // nullable: H matrices [Tq, Tk/16] P~ scales, tile layout (verification)
   int* status;              // set to a nonzero value when a wait ran out
 };
+
+// The tiles of query tile q0 that hold an allowed key of one of its rows, and range s of them.
+__device__ __forceinline__ int af_live_tiles(const AttnFusedParams& a, int64_t q0) {
+  const int64_t lim_cta = a.causal ? q0 + kAfBM - 1 + a.q_offset : a.Tk - 1;
+  return lim_cta < 0 ? 0 : (int)min(a.Tk / kAfBN, lim_cta / kAfBN + 1);
+}
+__device__ __forceinline__ void af_range(int live, int s, int ns, int& t0, int& t1) {
+  t0 = (int)((int64_t)live * s / ns);
+  t1 = (int)((int64_t)live * (s + 1) / ns);
+}
+// A row's last allowed key, clamped to [-1, Tk - 1].
+__device__ __forceinline__ int af_row_limit(const AttnFusedParams& a, int64_t q) {
+  return a.causal ? (int)max((int64_t)-1, min(q + a.q_offset, a.Tk - 1)) : (int)(a.Tk - 1);
+}
 
 __device__ __forceinline__ uint32_t af_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -130,11 +166,17 @@ __device__ __forceinline__ void af_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// Wait for the phase of parity `parity` of an mbarrier to complete.  Each try suspends the thread until the
+// phase completes or kAfWaitHintNs pass (the hint keeps waiting threads from spinning on the barrier, which
+// would fill the memory-instruction queue the other warps need); after kAfWaitTries tries (about a second)
+// the wait gives up and returns false.
+constexpr uint32_t kAfWaitHintNs = 10000;
+constexpr uint32_t kAfWaitTries = 100000;
 __device__ __forceinline__ bool af_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kAfWaitLimit; ++i) {
+  for (uint32_t i = 0; i < kAfWaitTries; ++i) {
     uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "n"(kAfWaitHintNs) : "memory");
     if (ok) return true;
   }
   return false;
@@ -241,232 +283,287 @@ __device__ __forceinline__ void af_quantize_block(const u64 (&x2)[8], const Cand
   }
 }
 
+
+constexpr uint32_t kAfSboD = 128 * kAfD / 8;    // tiles whose K is the head dimension (Q, K)
+constexpr uint32_t kAfSboN = 128 * kAfBN / 8;   // tiles whose K is a key tile (P~, V^T)
+constexpr uint32_t kAfTileBytes = 16384;        // a K tile (64 x 128) or a V^T tile (128 x 64) in FP16
+
+// ---------------------------------------------------------------------------------------------------------
+// K and V^T as FP16 tiles in the MMA's shared-memory layout (exact: v * E4M3(s), no tensor scale), once per
+// call: kx[h][j] the 64 x 128 K tile j, vx[h][j] the 128 x 64 V^T tile j, 16 KB each, so that the kernels
+// below fetch a tile with one bulk copy.  Grid (Tk / 64, H, 2), 512 threads: one 16-element block each, the
+// eight rows of a core matrix in consecutive threads (128 contiguous bytes per chunk column).
+// ---------------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kAfThreads) attn_expand_kernel(const AttnFusedParams a) {
+  const int t = threadIdx.x;
+  const int64_t j = blockIdx.x, h = blockIdx.y, tiles = a.Tk / kAfBN;
+  uint4 lo, hi;
+  if (blockIdx.z == 0) {   // K: 64 keys (8 row groups of 8) x 8 blocks
+    const int r = (t >> 6) * 8 + (t & 7), kb = (t >> 3) & 7;
+    const int64_t key = j * kAfBN + r;
+    const uint2 cw = *reinterpret_cast<const uint2*>(a.k_codes + ((h * a.Tk + key) * (kAfD / 16) + kb) * 8);
+    af_dequant_block(cw, a.k_sf[af_sf_index(h, key, kb, a.Tk, kAfD / 16)], lo, hi);
+    af_store_block(a.kx + (h * tiles + j) * kAfTileBytes, r, kb, kAfSboD, lo, hi);
+  } else {                 // V^T: 128 head-dimension rows (16 row groups of 8) x 4 key blocks
+    const int d = (t >> 5) * 8 + (t & 7), kb = (t >> 3) & 3;
+    const int64_t c = j * (kAfBN / 16) + kb;
+    const uint2 cw = *reinterpret_cast<const uint2*>(a.v_codes + ((h * kAfD + d) * (a.Tk / 16) + c) * 8);
+    af_dequant_block(cw, a.v_sf[af_sf_index(h, d, c, kAfD, a.Tk / 16)], lo, hi);
+    af_store_block(a.vx + (h * tiles + j) * kAfTileBytes, d, kb, kAfSboN, lo, hi);
+  }
+}
+
+// One tile (16 KB) from global into shared memory by the bulk-copy engine, its bytes counted on mbarrier
+// `bar` (which one thread arms with the byte count in the same call).  Issued by one thread.
+__device__ __forceinline__ void af_fetch_tile(uint32_t dst, const uint8_t* src, uint32_t bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "n"(kAfTileBytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "n"(kAfTileBytes), "r"(bar) : "memory");
+}
+
+// The CTA's 128 Q rows: 1024 blocks, one per thread of the CTA.
+__device__ __forceinline__ void af_load_q(const AttnFusedParams& a, uint8_t* sq, int64_t h, int64_t q0, int tid) {
+  const int row = tid >> 3, kb = tid & 7;
+  const int64_t qr = q0 + row;
+  uint4 lo, hi;
+  const uint2 cw = *reinterpret_cast<const uint2*>(a.q_codes + ((h * a.Tq + qr) * (kAfD / 16) + kb) * 8);
+  af_dequant_block(cw, a.q_sf[af_sf_index(h, qr, kb, a.Tq, kAfD / 16)], lo, hi);
+  af_store_block(sq, row, kb, kAfSboD, lo, hi);
+}
+
+// Barrier of one half (named barrier 1 + half, 512 threads); the _or form also returns whether p was set
+// in any of its threads.
+__device__ __forceinline__ bool af_half_sync_or(int half, bool p) {
+  uint32_t r;
+  asm volatile("{ .reg .pred a, b; setp.ne.u32 a, %1, 0; bar.red.or.pred b, %2, %3, a; selp.u32 %0, 1, 0, b; }"
+               : "=r"(r)
+               : "r"((uint32_t)p), "r"(1 + half), "n"(kAfThreads)
+               : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void af_half_sync(int half) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(kAfThreads) : "memory");
+}
+
+// S = Q K^T (64 columns of TMEM from tmem_d), completion on bar; issued by one thread.
+__device__ __forceinline__ void af_issue_s(uint32_t tmem_d, uint32_t sq, uint32_t sk, uint32_t bar) {
+  const uint32_t idesc = af_idesc(kAfBN);
+#pragma unroll
+  for (int s = 0; s < kAfD / 16; ++s)
+    af_mma(tmem_d, af_desc(sq + 256 * s, kAfSboD), af_desc(sk + 256 * s, kAfSboD), idesc, s > 0 ? 1u : 0u);
+  af_commit(bar);
+}
+// O (+)= P~ V^T (128 columns of TMEM from tmem_d), completion on bar; issued by one thread.
+__device__ __forceinline__ void af_issue_o(uint32_t tmem_d, uint32_t sp, uint32_t sv, bool acc, uint32_t bar) {
+  const uint32_t idesc = af_idesc(kAfD);
+#pragma unroll
+  for (int s = 0; s < kAfBN / 16; ++s)
+    af_mma(tmem_d, af_desc(sp + 256 * s, kAfSboN), af_desc(sv + 256 * s, kAfSboN), idesc, (acc || s > 0) ? 1u : 0u);
+  af_commit(bar);
+}
+
+// ---------------------------------------------------------------------------------------------------------
+// Row maxima of two key ranges per CTA (one per half): grid (Tq / 128, ceil(splits / 2), H), 1024 threads.
+// Per half: four K tiles in shared memory and four S buffers in TMEM; K(j + 4) is fetched once S(j) has
+// read its buffer, S(j + 2) is issued after the half's barrier of tile j (its K fetched two tiles earlier).
+// ---------------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kAfCtaThreads, 1) attn_rowmax_kernel(const AttnFusedParams a) {
+  extern __shared__ __align__(1024) uint8_t af_dyn[];
+  __shared__ float red[2][4][kAfBM];
+  __shared__ __align__(8) uint64_t bars[2][2][kAfMaxStages];   // per half: S complete, K landed
+  __shared__ uint32_t tmem_slot;
+
+  const int tid = threadIdx.x, half = tid / kAfThreads, t = tid % kAfThreads, w = t >> 5, lane = t & 31;
+  const int qd = w & 3, cb = w >> 2;          // TMEM lane quadrant; 16-key block of the tile
+  const int r = 32 * qd + lane;               // this thread's query row within the CTA
+  const int split = 2 * blockIdx.y + half;
+  const int64_t h = blockIdx.z, q0 = (int64_t)blockIdx.x * kAfBM, q = q0 + r;
+  const int live = af_live_tiles(a, q0);
+  int t0 = 0, t1 = 0;
+  if (split < a.splits) af_range(live, split, a.splits, t0, t1);
+  uint8_t* const sQ = af_dyn;
+  uint8_t* const sK0 = af_dyn + kAfQBytes + half * kAfMaxStages * kAfKBytes;
+  const uint8_t* const kx = a.kx + h * (a.Tk / kAfBN) * kAfTileBytes;
+
+  if (tid < 32) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(af_smem(&tmem_slot)),
+                 "r"(kAfTmemColsMax));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  const uint32_t bar_s0 = af_smem(&bars[half][0][0]), bar_k0 = af_smem(&bars[half][1][0]);
+  const uint32_t sq = af_smem(sQ), sk0 = af_smem(sK0);
+  if (t == 0) {
+    for (int i = 0; i < 2 * kAfMaxStages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_s0 + 8 * i));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int i = 0; i < kAfMaxStages && t0 + i < t1; ++i)
+      af_fetch_tile(sk0 + i * kAfKBytes, kx + (int64_t)(t0 + i) * kAfTileBytes, bar_k0 + 8 * i);
+  }
+  if (live > 0) af_load_q(a, sQ, h, q0, tid);
+  const float sc_s = __fmul_rn(__fmul_rn(a.alpha, *a.q_g), *a.k_g);
+  af_proxy_fence();
+  af_fence_before();
+  __syncthreads();
+  af_fence_after();
+  const uint32_t tmem = tmem_slot + (uint32_t)(half * kAfMaxStages * kAfBN), t_lane = (uint32_t)(32 * qd) << 16;
+  uint32_t ph_s = 0, ph_k = 0;   // parity bit per stage: S complete (all threads), K landed (thread 0)
+  bool ok = true;
+  if (t == 0) {
+    for (int i = 0; i < 2 && t0 + i < t1; ++i) {
+      ok = af_wait(bar_k0 + 8 * i, 0u) && ok;
+      ph_k ^= 1u << i;
+      af_issue_s(tmem + kAfBN * i, sq, sk0 + i * kAfKBytes, bar_s0 + 8 * i);
+    }
+  }
+
+  const int lim = af_row_limit(a, q);   // this row's last allowed key
+  float m = -INFINITY;
+  for (int j = t0; j < t1; ++j) {
+    const int b = (j - t0) % kAfMaxStages, b2 = (j + 2 - t0) % kAfMaxStages;
+    ok = af_wait(bar_s0 + 8 * b, (ph_s >> b) & 1u) && ok;   // S(j) complete: K buffer b free
+    ph_s ^= 1u << b;
+    af_fence_after();
+    if (t == 0 && j + kAfMaxStages < t1)
+      af_fetch_tile(sk0 + b * kAfKBytes, kx + (int64_t)(j + kAfMaxStages) * kAfTileBytes, bar_k0 + 8 * b);
+    float s[16];
+    af_ld16(tmem + t_lane + kAfBN * b + 16 * cb, s);
+    af_fence_before();
+    const int rem = lim - (j * kAfBN + 16 * cb);   // keys of the block at or below the row's limit
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i <= rem) m = fmaxf(m, __fmul_rn(s[i], sc_s));
+    if (af_half_sync_or(half, !ok)) {   // every thread has read S(j - 2)'s buffer, which S(j + 2) reuses
+      ok = false;
+      break;
+    }
+    if (t == 0 && j + 2 < t1) {
+      ok = af_wait(bar_k0 + 8 * b2, (ph_k >> b2) & 1u) && ok;   // K(j + 2) landed
+      ph_k ^= 1u << b2;
+      af_fence_after();
+      af_issue_s(tmem + kAfBN * b2, sq, sk0 + b2 * kAfKBytes, bar_s0 + 8 * b2);
+    }
+  }
+  ok = !af_half_sync_or(half, !ok);   // thread 0's waits after the last barrier included
+  if (ok && split < a.splits) {
+    red[half][cb][r] = m;
+    af_half_sync(half);
+    if (cb == 0)
+      a.ws_max[((int64_t)split * a.H + h) * a.Tq + q] =
+          fmaxf(fmaxf(red[half][0][r], red[half][1][r]), fmaxf(red[half][2][r], red[half][3][r]));
+  }
+  if (!ok && t == 0 && a.status) atomicExch(a.status, 1);
+  af_fence_before();
+  __syncthreads();
+  if (tid < 32) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "r"(kAfTmemColsMax));
+}
+
+// ---------------------------------------------------------------------------------------------------------
+// Numerators, their quantization and O += P~ V^T over two key ranges per CTA (one per half):
+// grid (Tq / 128, ceil(splits / 2), H), 1024 threads.  Per half: K and V^T tiles double-buffered and fetched
+// by bulk copies (K(j + 2) once S(j) has read its buffer, V(j + 1) once O(j - 1) has read its buffer), one
+// P~ tile written by the threads, S double-buffered and O in TMEM.
+// ---------------------------------------------------------------------------------------------------------
 template <int NC>
-__global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFusedParams a) {
+__global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const AttnFusedParams a) {
   extern __shared__ __align__(1024) uint8_t af_dyn[];
   __shared__ CandEntry tab_store[kTabSize];
   __shared__ float thr[128];
-  __shared__ float red[4][kAfBM];
-  __shared__ __align__(8) uint64_t bars[3];   // S buffer 0, S buffer 1, O
+  __shared__ float red[2][4][kAfBM];
+  __shared__ __align__(8) uint64_t bars[2][7];   // per half: S 0, S 1, O, K landed 0, 1, V landed 0, 1
   __shared__ uint32_t tmem_slot;
-  __shared__ int s_err;
   CandEntry* tab = tab_store + kTabPad;
-  uint8_t* const sQ = af_dyn;
-  auto sK = [&](int b) { return af_dyn + kAfQBytes + b * kAfKBytes; };
-  auto sV = [&](int b) { return af_dyn + kAfQBytes + 2 * kAfKBytes + b * kAfVBytes; };
-  auto sP = [&](int b) { return af_dyn + kAfQBytes + 2 * kAfKBytes + 2 * kAfVBytes + b * kAfPBytes; };
-  constexpr uint32_t kSboD = 128 * kAfD / 8;    // tiles whose K is the head dimension (Q, K)
-  constexpr uint32_t kSboN = 128 * kAfBN / 8;   // tiles whose K is a key tile (P~, V^T)
 
-  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int tid = threadIdx.x, half = tid / kAfThreads, t = tid % kAfThreads, w = t >> 5, lane = t & 31;
   const int qd = w & 3, cb = w >> 2;          // TMEM lane quadrant; 16-key block of the tile
   const int r = 32 * qd + lane;               // this thread's query row within the CTA
-  const int64_t h = blockIdx.y, q0 = (int64_t)blockIdx.x * kAfBM, q = q0 + r;
-  const int64_t bpr_k = kAfD / 16, bpr_v = a.Tk / 16;
+  const int split = 2 * blockIdx.y + half;
+  const int64_t h = blockIdx.z, q0 = (int64_t)blockIdx.x * kAfBM, q = q0 + r;
+  const int64_t row = h * a.Tq + q, bpr_v = a.Tk / 16;
+  const int live = af_live_tiles(a, q0);
+  int t0 = 0, t1 = 0;
+  if (split < a.splits) af_range(live, split, a.splits, t0, t1);
+  uint8_t* const sQ = af_dyn;
+  uint8_t* const sK0 = af_dyn + kAfQBytes + half * kAfHalfBytes;
+  uint8_t* const sV0 = sK0 + 2 * kAfKBytes;
+  uint8_t* const sP = sV0 + 2 * kAfVBytes;
+  const uint8_t* const kx = a.kx + h * (a.Tk / kAfBN) * kAfTileBytes;
+  const uint8_t* const vx = a.vx + h * (a.Tk / kAfBN) * kAfTileBytes;
 
   const float gp = __fdiv_rn(1.0f, kTensorDiv);   // P~'s tensor scale: every row's largest numerator is 1
   build_cand_entries(tab, gp);
   build_c0_thresholds(thr, gp);
   const float inv6g = __frcp_rn(__fmul_rn(6.0f, gp));
-  if (w == 0) {
+  if (tid < 32) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(af_smem(&tmem_slot)),
                  "r"(kAfTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  const uint32_t bar_s0 = af_smem(&bars[half][0]), bar_o = af_smem(&bars[half][2]);
+  const uint32_t bar_k0 = af_smem(&bars[half][3]), bar_v0 = af_smem(&bars[half][5]);
+  const uint32_t sq = af_smem(sQ), sk0 = af_smem(sK0), sv0 = af_smem(sV0), sp = af_smem(sP);
   if (t == 0) {
-    for (int i = 0; i < 3; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(af_smem(&bars[i])));
+    for (int i = 0; i < 7; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_s0 + 8 * i));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_err = 0;
+    for (int i = 0; i < 2 && t0 + i < t1; ++i)
+      af_fetch_tile(sk0 + i * kAfKBytes, kx + (int64_t)(t0 + i) * kAfTileBytes, bar_k0 + 8 * i);
+    if (t0 < t1) af_fetch_tile(sv0, vx + (int64_t)t0 * kAfTileBytes, bar_v0);
   }
-  // the CTA's Q rows (two blocks per thread)
-  for (int i = t; i < kAfBM * (kAfD / 16); i += kAfThreads) {
-    const int row = i >> 3, kb = i & 7;
-    const int64_t qr = q0 + row;
-    uint4 lo, hi;
-    const uint2 cw = *reinterpret_cast<const uint2*>(a.q_codes + ((h * a.Tq + qr) * bpr_k + kb) * 8);
-    af_dequant_block(cw, a.q_sf[af_sf_index(h, qr, kb, a.Tq, bpr_k)], lo, hi);
-    af_store_block(sQ, row, kb, kSboD, lo, hi);
-  }
+  // the row maximum over all ranges (the row-max kernel's)
+  float m = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) m = fmaxf(m, a.ws_max[(int64_t)s * a.H * a.Tq + row]);
+  if (live > 0) af_load_q(a, sQ, h, q0, tid);
   const float sc_s = __fmul_rn(__fmul_rn(a.alpha, *a.q_g), *a.k_g);
-  const float sc_o = __fmul_rn(gp, *a.v_g);
   af_proxy_fence();
   af_fence_before();
   __syncthreads();
   af_fence_after();
-  const uint32_t tmem = tmem_slot;
-  const uint32_t t_lane = (uint32_t)(32 * qd) << 16;
-  // one completion barrier per S buffer (up to two products in flight, each buffer's phase tracked on its
-  // own) and one for O
-  const uint32_t bar_s[2] = {af_smem(&bars[0]), af_smem(&bars[1])}, bar_o = af_smem(&bars[2]);
-  uint32_t ph_s[2] = {0u, 0u}, ph_o = 0;
-
-  const int64_t lim = a.causal ? q + a.q_offset : a.Tk - 1;                   // this row's last allowed key
-  const int64_t lim_cta = a.causal ? q0 + kAfBM - 1 + a.q_offset : a.Tk - 1;  // the CTA's last
-  const int64_t ntiles = a.Tk / kAfBN;
-  const int64_t live = lim_cta < 0 ? 0 : min(ntiles, lim_cta / kAfBN + 1);    // tiles with an allowed key
-
-  // K tile j: 64 keys x 8 blocks, one block per thread (fetched into registers ahead of its use, then
-  // dequantized into buffer b); a tile past the end fetches nothing
-  struct RawBlock {
-    uint2 cw;
-    uint32_t sf;
-  };
-  auto fetch_k = [&](int64_t j) {
-    RawBlock rb{make_uint2(0u, 0u), 0u};
-    if (j < live) {
-      const int key = t >> 3, kb = t & 7;
-      const int64_t kr = j * kAfBN + key;
-      rb.cw = *reinterpret_cast<const uint2*>(a.k_codes + ((h * a.Tk + kr) * bpr_k + kb) * 8);
-      rb.sf = a.k_sf[af_sf_index(h, kr, kb, a.Tk, bpr_k)];
-    }
-    return rb;
-  };
-  auto store_k = [&](const RawBlock& rb, int b) {
-    uint4 lo, hi;
-    af_dequant_block(rb.cw, rb.sf, lo, hi);
-    af_store_block(sK(b), t >> 3, t & 7, kSboD, lo, hi);
-  };
-  // V^T tile j: 128 head-dimension rows x 4 key blocks, one block per thread
-  auto fetch_v = [&](int64_t j) {
-    RawBlock rb{make_uint2(0u, 0u), 0u};
-    if (j < live) {
-      const int d = t >> 2, kb = t & 3;
-      const int64_t c = j * (kAfBN / 16) + kb;
-      rb.cw = *reinterpret_cast<const uint2*>(a.v_codes + ((h * kAfD + d) * bpr_v + c) * 8);
-      rb.sf = a.v_sf[af_sf_index(h, d, c, kAfD, bpr_v)];
-    }
-    return rb;
-  };
-  auto store_v = [&](const RawBlock& rb, int b) {
-    uint4 lo, hi;
-    af_dequant_block(rb.cw, rb.sf, lo, hi);
-    af_store_block(sV(b), t >> 2, t & 3, kSboN, lo, hi);
-  };
-  // S = Q K_j^T into TMEM columns 64 b .. 64 b + 63 (issued by thread 0, completion on bar_s[b])
-  auto mma_s = [&](int b) {
-    if (t == 0) {
-      af_fence_after();
-      const uint32_t idesc = af_idesc(kAfBN);
-#pragma unroll
-      for (int s = 0; s < kAfD / 16; ++s)
-        af_mma(tmem + kAfBN * b, af_desc(af_smem(sQ) + 256 * s, kSboD), af_desc(af_smem(sK(b)) + 256 * s, kSboD),
-               idesc, s > 0 ? 1u : 0u);
-      af_commit(b ? bar_s[1] : bar_s[0]);
-    }
-  };
-  // every thread waits; a wait that runs out stops the whole CTA (the flag is read after a barrier)
-  auto wait_all = [&](uint32_t bar, uint32_t& ph) -> bool {
-    const bool ok = af_wait(bar, ph);
-    ph ^= 1u;
-    if (!ok) s_err = 1;
-    __syncthreads();
-    af_fence_after();
-    return s_err == 0;
-  };
-  // this thread's 16 scores of tile j (buffer b), scaled
-  auto scores = [&](int b, float (&s)[16]) {
-    af_ld16(tmem + t_lane + kAfBN * b + 16 * cb, s);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = __fmul_rn(s[i], sc_s);
-  };
-
+  const uint32_t tmem = tmem_slot + (uint32_t)(half * 4 * kAfBN), t_lane = (uint32_t)(32 * qd) << 16;
+  // parity bits: bits 0, 1 S buffers and bit 2 O (all threads); bits 3, 4 K and 5, 6 V landed (thread 0)
+  uint32_t ph = 0;
   bool ok = true;
-  // ---- sweep 1: row maxima over the allowed keys ----
-  // two products in flight: S(j + 1) runs while tile j's scores are read, and S(j + 2) is issued into
-  // tile j's buffers as soon as they are read; each K tile is fetched into registers two tiles ahead
-  float m = -INFINITY;
-  RawBlock kn = fetch_k(0), kn2 = fetch_k(1);
-  if (live > 0) {
-    store_k(kn, 0);
-    if (live > 1) store_k(kn2, 1);
-    kn = fetch_k(2);
-    kn2 = fetch_k(3);
-    af_proxy_fence();
-    af_fence_before();
-    __syncthreads();
-    mma_s(0);
-    if (live > 1) mma_s(1);
-  }
-  for (int64_t j = 0; j < live; ++j) {
-    const int b = (int)(j & 1);
-    ok = b ? wait_all(bar_s[1], ph_s[1]) : wait_all(bar_s[0], ph_s[0]);   // S(j) complete
-    if (!ok) break;
-    float s[16];
-    scores(b, s);
-    const int64_t k0 = j * kAfBN + 16 * cb;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (k0 + i <= lim) m = fmaxf(m, s[i]);
-    if (j + 2 < live) {
-      store_k(kn, b);                          // K(j + 2) into the buffer S(j) has finished reading
-      kn = kn2;
-      kn2 = fetch_k(j + 4);
-      af_proxy_fence();
-      af_fence_before();
-      __syncthreads();                         // K(j + 2) visible; every thread has read S(j)
-      mma_s(b);
+  if (t == 0) {
+    for (int i = 0; i < 2 && t0 + i < t1; ++i) {
+      ok = af_wait(bar_k0 + 8 * i, 0u) && ok;
+      ph ^= 8u << i;
+      af_issue_s(tmem + kAfBN * i, sq, sk0 + i * kAfKBytes, bar_s0 + 8 * i);
     }
-  }
-  if (ok) {
-    red[cb][r] = m;
-    __syncthreads();
-    m = fmaxf(fmaxf(red[0][r], red[1][r]), fmaxf(red[2][r], red[3][r]));
-    __syncthreads();
   }
 
-  // ---- sweep 2: numerators, their quantization, O += P~ V^T ----
-  // software-pipelined: S(j + 1) is formed while tile j's numerators are quantized, O += P~(j) V(j) runs
-  // while the next tiles are stored, and the raw K and V blocks are fetched a tile ahead of their store
+  const int lim = af_row_limit(a, q);   // this row's last allowed key
   float l = 0.0f;
-  RawBlock kf = fetch_k(1), vf = fetch_v(1);
-  if (ok && live > 0) {
-    af_fence_before();
-    __syncthreads();          // every thread has read its last S of sweep 1
-    store_k(fetch_k(0), 0);
-    store_v(fetch_v(0), 0);
-    af_proxy_fence();
-    af_fence_before();
-    __syncthreads();
-    mma_s(0);
-  }
-  for (int64_t j = 0; j < live && ok; ++j) {
-    const int b = (int)(j & 1);
-    if (j + 1 < live) store_k(kf, b ^ 1);     // that buffer's last reader, S(j - 1), has completed
-    if (j > 0) {
-      ok = wait_all(bar_o, ph_o);              // O(j - 1) complete: its V and P~ buffers are free
-      if (!ok) break;
-    }
-    if (j + 1 < live) store_v(vf, b ^ 1);
-    kf = fetch_k(j + 2);
-    vf = fetch_v(j + 2);
-    af_proxy_fence();
-    af_fence_before();
-    ok = b ? wait_all(bar_s[1], ph_s[1]) : wait_all(bar_s[0], ph_s[0]);   // S(j) complete; K(j + 1), V(j + 1) visible
-    if (!ok) break;
-    if (j + 1 < live) mma_s(b ^ 1);
-    float s[16], x[16];
-    scores(b, s);
-    const int64_t k0 = j * kAfBN + 16 * cb;
+  for (int j = t0; j < t1; ++j) {
+    const int b = (j - t0) & 1;
+    ok = af_wait(bar_s0 + 8 * b, (ph >> b) & 1u) && ok;   // S(j) complete, K buffer b free
+    ph ^= 1u << b;
+    af_fence_after();
+    if (t == 0 && j + 2 < t1) af_fetch_tile(sk0 + b * kAfKBytes, kx + (int64_t)(j + 2) * kAfTileBytes, bar_k0 + 8 * b);
+    const uint32_t ts = tmem + t_lane + kAfBN * b + 16 * cb;
+    const int k0 = j * kAfBN + 16 * cb;
+    float x[16];
+    af_ld16(ts, x);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(x[i], sc_s);
     if (a.s_out) {
-      float* so = a.s_out + (h * a.Tq + q) * a.Tk + k0;
+      float* so = a.s_out + row * a.Tk + k0;
 #pragma unroll
-      for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(so + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
+      for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(so + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = s[i];
-    if (!exp_fast16(m, x)) {
+    if (!exp_fast16(m, x)) {   // rare: a numerator below the fast method's range; the scores again, by pairs
+      af_ld16(ts, x);
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
-        float ea = __fsub_rn(s[i], m), eb = __fsub_rn(s[i + 1], m);
+        float ea = __fsub_rn(__fmul_rn(x[i], sc_s), m), eb = __fsub_rn(__fmul_rn(x[i + 1], sc_s), m);
         exp_ss2(ea, eb);
         x[i] = ea;
         x[i + 1] = eb;
       }
     }
-    if (k0 + 15 > lim) {
+    af_fence_before();
+    const int rem = lim - k0;
+    if (rem < 15) {
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        if (k0 + i > lim) x[i] = 0.0f;
+        if (i > rem) x[i] = 0.0f;
     }
     u64 x2[8];
 #pragma unroll
@@ -477,68 +574,122 @@ __global__ void __launch_bounds__(kAfThreads, 1) attn_fused_kernel(const AttnFus
     uint32_t wlo, whi, scale;
     af_quantize_block<NC>(x2, tab, thr, inv6g, a.f_lo, a.f_hi, wlo, whi, scale);
     if (a.p_codes) {
-      *reinterpret_cast<uint2*>(a.p_codes + ((h * a.Tq + q) * bpr_v + k0 / 16) * 8) = make_uint2(wlo, whi);
+      *reinterpret_cast<uint2*>(a.p_codes + (row * bpr_v + k0 / 16) * 8) = make_uint2(wlo, whi);
       a.p_sf[af_sf_index(h, q, k0 / 16, a.Tq, bpr_v)] = (uint8_t)scale;
     }
-    uint4 lo, hi;
-    af_dequant_block(make_uint2(wlo, whi), scale, lo, hi);
-    af_store_block(sP(b), r, cb, kSboN, lo, hi);
+    if (j > t0) {   // O += P~(j-1) V(j-1) complete: the P~ buffer and V buffer b^1 are free
+      ok = af_wait(bar_o, (ph >> 2) & 1u) && ok;
+      ph ^= 4u;
+    }
+    if (t == 0 && j + 1 < t1)
+      af_fetch_tile(sv0 + (b ^ 1) * kAfVBytes, vx + (int64_t)(j + 1) * kAfTileBytes, bar_v0 + 8 * (b ^ 1));
+    {
+      uint4 lo, hi;
+      af_dequant_block(make_uint2(wlo, whi), scale, lo, hi);
+      af_store_block(sP, r, cb, kAfSboN, lo, hi);
+    }
     af_proxy_fence();
     af_fence_before();
-    __syncthreads();
+    if (af_half_sync_or(half, !ok)) {
+      ok = false;
+      break;
+    }
     if (t == 0) {
+      ok = af_wait(bar_v0 + 8 * b, (ph >> (5 + b)) & 1u) && ok;   // V(j) landed
+      ph ^= 32u << b;
       af_fence_after();
-      const uint32_t idesc = af_idesc(kAfD);
-#pragma unroll
-      for (int s2 = 0; s2 < kAfBN / 16; ++s2)
-        af_mma(tmem + 2 * kAfBN, af_desc(af_smem(sP(b)) + 256 * s2, kSboN), af_desc(af_smem(sV(b)) + 256 * s2, kSboN),
-               idesc, (j > 0 || s2 > 0) ? 1u : 0u);
-      af_commit(bar_o);
+      af_issue_o(tmem + 2 * kAfBN, sp, sv0 + b * kAfVBytes, j > t0, bar_o);
+      if (j + 2 < t1) {
+        ok = af_wait(bar_k0 + 8 * b, (ph >> (3 + b)) & 1u) && ok;   // K(j + 2) landed
+        ph ^= 8u << b;
+        af_issue_s(tmem + kAfBN * b, sq, sk0 + b * kAfKBytes, bar_s0 + 8 * b);
+      }
     }
   }
-  if (ok && live > 0) ok = wait_all(bar_o, ph_o);   // the last O += P~ V^T
+  ok = !af_half_sync_or(half, !ok);   // thread 0's waits after the last barrier included
+  if (ok && t1 > t0) {   // the last O += P~ V^T
+    ok = af_wait(bar_o, (ph >> 2) & 1u);
+    ok = !af_half_sync_or(half, !ok);
+    af_fence_after();
+  }
 
   // tiles past every row's last allowed key: P~ is a zero block there (scale 0, zero codes), which is what
   // the verification outputs receive; the products skip those tiles
-  if (ok && a.p_codes) {
-    for (int64_t j = live; j < ntiles; ++j) {
+  if (ok && a.p_codes && split == a.splits - 1) {
+    for (int64_t j = live; j < a.Tk / kAfBN; ++j) {
       const int64_t c = j * (kAfBN / 16) + cb;
-      *reinterpret_cast<uint2*>(a.p_codes + ((h * a.Tq + q) * bpr_v + c) * 8) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(a.p_codes + (row * bpr_v + c) * 8) = make_uint2(0u, 0u);
       a.p_sf[af_sf_index(h, q, c, a.Tq, bpr_v)] = 0;
     }
   }
 
-  // ---- epilogue ----
-  if (ok) {
-    red[cb][r] = l;
-    __syncthreads();
-    l = __fadd_rn(__fadd_rn(__fadd_rn(red[0][r], red[1][r]), red[2][r]), red[3][r]);
+  // ---- epilogue: the range's O accumulator and row sum, or with one range the result ----
+  if (ok && split < a.splits) {
+    red[half][cb][r] = l;
+    af_half_sync(half);
+    l = __fadd_rn(__fadd_rn(__fadd_rn(red[half][0][r], red[half][1][r]), red[half][2][r]), red[half][3][r]);
+    const float sc_o = __fmul_rn(gp, *a.v_g);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
+    for (int hh = 0; hh < 2; ++hh) {
       float o[16];
-      if (live > 0) {
-        af_ld16(tmem + t_lane + 2 * kAfBN + 32 * cb + 16 * half, o);
-      } else {   // no key allowed for any row: the product is 0 (and 0 / 0 is what the chain gives)
+      if (t1 > t0) {
+        af_ld16(tmem + t_lane + 2 * kAfBN + 32 * cb + 16 * hh, o);
+      } else {   // no tile in this range: the accumulator is 0
 #pragma unroll
         for (int i = 0; i < 16; ++i) o[i] = 0.0f;
       }
-      float* op = a.out + (h * a.Tq + q) * kAfD + 32 * cb + 16 * half;
+      if (a.splits == 1) {   // with every key in one range: O = fl(fl(acc g_p g_v) / l) (0 / 0 with no key)
+        float* op = a.out + row * kAfD + 32 * cb + 16 * hh;
 #pragma unroll
-      for (int i = 0; i < 16; i += 4)
-        *reinterpret_cast<float4*>(op + i) =
-            make_float4(__fdiv_rn(__fmul_rn(o[i], sc_o), l), __fdiv_rn(__fmul_rn(o[i + 1], sc_o), l),
-                        __fdiv_rn(__fmul_rn(o[i + 2], sc_o), l), __fdiv_rn(__fmul_rn(o[i + 3], sc_o), l));
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(op + i) =
+              make_float4(__fdiv_rn(__fmul_rn(o[i], sc_o), l), __fdiv_rn(__fmul_rn(o[i + 1], sc_o), l),
+                          __fdiv_rn(__fmul_rn(o[i + 2], sc_o), l), __fdiv_rn(__fmul_rn(o[i + 3], sc_o), l));
+      } else {
+        float* op = a.ws_o + ((int64_t)split * a.H * a.Tq + row) * kAfD + 32 * cb + 16 * hh;
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) *reinterpret_cast<float4*>(op + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+      }
     }
     if (cb == 0) {
-      a.row_max[h * a.Tq + q] = m;
-      a.row_sum[h * a.Tq + q] = l;
+      if (a.splits == 1) {
+        a.row_max[row] = m;
+        a.row_sum[row] = l;
+      } else {
+        a.ws_l[(int64_t)split * a.H * a.Tq + row] = l;
+      }
     }
-  } else if (t == 0 && a.status) {
-    atomicExch(a.status, 1);
   }
+  if (!ok && t == 0 && a.status) atomicExch(a.status, 1);
   af_fence_before();
   __syncthreads();
-  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAfTmemCols));
+  if (tid < 32) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "r"(kAfTmemCols));
+}
+
+// ---------------------------------------------------------------------------------------------------------
+// The ranges combined (splits > 1): a thread per 4 elements of O.
+// ---------------------------------------------------------------------------------------------------------
+__global__ void attn_combine_kernel(const AttnFusedParams a) {
+  const int64_t rows = a.H * a.Tq, i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * (kAfD / 4)) return;
+  const int64_t row = i / (kAfD / 4), c4 = i % (kAfD / 4);
+  float l = 0.0f, m = -INFINITY;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int s = 0; s < a.splits; ++s) {
+    const int64_t sr = (int64_t)s * rows + row;
+    l = __fadd_rn(l, a.ws_l[sr]);
+    m = fmaxf(m, a.ws_max[sr]);
+    const float4 o = *reinterpret_cast<const float4*>(a.ws_o + sr * kAfD + 4 * c4);
+    acc = make_float4(__fadd_rn(acc.x, o.x), __fadd_rn(acc.y, o.y), __fadd_rn(acc.z, o.z), __fadd_rn(acc.w, o.w));
+  }
+  const float sc_o = __fmul_rn(__fdiv_rn(1.0f, kTensorDiv), *a.v_g);
+  *reinterpret_cast<float4*>(a.out + row * kAfD + 4 * c4) =
+      make_float4(__fdiv_rn(__fmul_rn(acc.x, sc_o), l), __fdiv_rn(__fmul_rn(acc.y, sc_o), l),
+                  __fdiv_rn(__fmul_rn(acc.z, sc_o), l), __fdiv_rn(__fmul_rn(acc.w, sc_o), l));
+  if (c4 == 0) {
+    a.row_max[row] = m;
+    a.row_sum[row] = l;
+  }
 }
 
 }  // namespace nvfp4

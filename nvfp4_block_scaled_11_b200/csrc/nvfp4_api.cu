@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <initializer_list>
 #include <mutex>
@@ -693,48 +694,129 @@ int nvfp4_softmax_quantize_mma(const float* s, int64_t batch, int64_t Tq, int64_
 
 }  // extern "C"
 
-// One launch of the fused attention kernel for window width NC; its shared-memory limit is raised once per
-// instantiation (each kernel has its own attribute).
+// The fused attention's kernels raise their shared-memory limit once per device (the attribute belongs to
+// the kernel on the current device); one instantiation, so one record, per kernel.
+template <auto* kernel>
+int af_raise_smem(int bytes) {
+  static std::mutex mu;
+  static uint64_t done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> g(mu);
+  if ((done >> dev) & 1u) return NVFP4_OK;
+  // the largest shared-memory carveout, so that two CTAs of the numerator kernel fit on an SM
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  done |= 1ull << dev;
+  return NVFP4_OK;
+}
+
 template <int NC>
-int launch_attn_fused(const AttnFusedParams& a, dim3 grid, cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(attn_fused_kernel<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kAfSmemBytes);
-  });
-  if (attr != cudaSuccess) return NVFP4_ERR_CUDA;
-  attn_fused_kernel<NC><<<grid, kAfThreads, kAfSmemBytes, st>>>(a);
+int launch_attn_fused(const AttnFusedParams& a, cudaStream_t st) {
+  int rc = af_raise_smem<attn_rowmax_kernel>(kAfMaxSmemBytes);
+  if (rc == NVFP4_OK) rc = af_raise_smem<attn_fused_kernel<NC>>(kAfSmemBytes);
+  if (rc != NVFP4_OK) return rc;
+  attn_expand_kernel<<<dim3((unsigned)(a.Tk / kAfBN), (unsigned)a.H, 2), kAfThreads, 0, st>>>(a);
+  // a CTA runs two key ranges, one per half
+  const dim3 grid((unsigned)(a.Tq / kAfBM), (unsigned)((a.splits + 1) / 2), (unsigned)a.H);
+  attn_rowmax_kernel<<<grid, kAfCtaThreads, kAfMaxSmemBytes, st>>>(a);
+  attn_fused_kernel<NC><<<grid, kAfCtaThreads, kAfSmemBytes, st>>>(a);
+  if (a.splits > 1) {
+    const int64_t n = a.H * a.Tq * (kAfD / 4);
+    attn_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a);
+  }
   return last_error();
+}
+
+// Workspace: the ranges' O accumulators (splits > 1), row sums (splits > 1) and row maxima, then, from a
+// 256-byte boundary, the K and V^T tiles in FP16 (16 KB per 64 keys and head each).
+int64_t af_tiles_offset(int64_t H, int64_t Tq, int64_t splits) {
+  const int64_t rows = H * Tq;
+  return (splits * rows * 4 + (splits > 1 ? splits * rows * (kAfD + 1) * 4 : 0) + 255) / 256 * 256;
+}
+size_t af_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int64_t splits) {
+  return (size_t)(af_tiles_offset(H, Tq, splits) + 2 * H * (Tk / kAfBN) * (int64_t)kAfTileBytes);
 }
 
 extern "C" {
 
+size_t nvfp4_attention_fused_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int splits) {
+  if (H < 0 || Tq < 0 || Tk < 0 || Tk % kAfBN != 0 || splits < 1 || splits > kAfMaxSplits ||
+      checked_prod({H, Tq, kAfD + 2, splits, 4}) < 0 || checked_prod({H, Tk, 2 * kAfD * 2}) < 0)
+    return 0;
+  return af_workspace_bytes(H, Tq, Tk, splits);
+}
+
+int nvfp4_attention_fused_splits(int64_t H, int64_t Tq, int64_t Tk, int* splits) {
+  if (!splits) return NVFP4_ERR_ARG;
+  if (H < 0 || Tq < 0 || Tk < 0 || Tq % kAfBM != 0 || Tk % kAfBN != 0) return NVFP4_ERR_SIZE;
+  *splits = 1;
+  const int64_t qt = H * (Tq / kAfBM), tiles = Tk / kAfBN;
+  if (qt == 0 || tiles == 0) return NVFP4_OK;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      af_raise_smem<attn_fused_kernel<9>>(kAfSmemBytes) != NVFP4_OK ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_fused_kernel<9>, kAfCtaThreads, kAfSmemBytes) !=
+          cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  const int64_t slots = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+  // waves of equal CTAs, each running two ranges of 1/s of a query tile's keys side by side: s ranges cost
+  // ceil(qt ceil(s/2) / slots) / s; ranges of at least 8 tiles; the smallest s within 2 % of the best (fewer
+  // ranges to combine)
+  const int64_t smax = std::max<int64_t>(1, std::min<int64_t>(kAfMaxSplits, tiles / 8));
+  auto cost = [&](int64_t s) { return (double)((qt * ((s + 1) / 2) + slots - 1) / slots) / (double)s; };
+  double best = 1e30;
+  for (int64_t s = 1; s <= smax; ++s) best = std::min(best, cost(s));
+  for (int64_t s = 1; s <= smax; ++s)
+    if (cost(s) <= best * 1.02) {
+      *splits = (int)s;
+      break;
+    }
+  return NVFP4_OK;
+}
+
 int nvfp4_attention_fused(const uint8_t* q_codes, const uint8_t* q_sf, const float* q_gscale, const uint8_t* k_codes,
                           const uint8_t* k_sf, const float* k_gscale, const uint8_t* v_codes_t, const uint8_t* v_sf_t,
                           const float* v_gscale, int64_t H, int64_t Tq, int64_t Tk, int64_t D, float alpha, int causal,
-                          int64_t q_offset, int f_lo, int f_hi, float* out, float* row_max, float* row_sum,
-                          float* s_out, uint8_t* p_codes, uint8_t* p_sf, int* status, void* stream) {
+                          int64_t q_offset, int f_lo, int f_hi, int splits, void* workspace, size_t workspace_bytes,
+                          float* out, float* row_max, float* row_sum, float* s_out, uint8_t* p_codes, uint8_t* p_sf,
+                          int* status, void* stream) {
   const int nc = f_hi - f_lo + 1;
   if (!window_ok(f_lo, f_hi) || (nc != 1 && nc != 9 && nc != 17)) return NVFP4_ERR_ARG;
+  if (splits < 1 || splits > kAfMaxSplits) return NVFP4_ERR_ARG;
   if (H < 0 || Tq < 0 || Tk < 0 || D != kAfD || Tq % kAfBM != 0 || Tk % kAfBN != 0) return NVFP4_ERR_SIZE;
-  if (H > 65535 || checked_prod({H, Tq, Tk}) < 0 || checked_prod({H, Tq, D}) < 0) return NVFP4_ERR_SIZE;
+  if (H > 65535 || Tk >= ((int64_t)1 << 26) || checked_prod({H, Tq, Tk}) < 0 ||
+      checked_prod({H, Tq, D + 2, splits, 4}) < 0)
+    return NVFP4_ERR_SIZE;
   if (H == 0 || Tq == 0) return NVFP4_OK;
   if (Tk == 0) return NVFP4_ERR_SIZE;   // no keys: nothing to attend to
   if (!q_codes || !q_sf || !q_gscale || !k_codes || !k_sf || !k_gscale || !v_codes_t || !v_sf_t || !v_gscale ||
-      !out || !row_max || !row_sum || ((p_codes == nullptr) != (p_sf == nullptr)))
+      !out || !row_max || !row_sum || !workspace || ((p_codes == nullptr) != (p_sf == nullptr)))
     return NVFP4_ERR_ARG;
-  if (!aligned(q_codes, 8) || !aligned(k_codes, 8) || !aligned(v_codes_t, 8) || !aligned(out, 16) ||
+  if (checked_prod({H, Tk, 2 * D * 2}) < 0 || workspace_bytes < af_workspace_bytes(H, Tq, Tk, splits))
+    return NVFP4_ERR_SIZE;
+  if (!aligned(q_codes, 8) || !aligned(k_codes, 8) || !aligned(v_codes_t, 8) || !aligned(k_sf, 4) || !aligned(out, 16) ||
       !aligned(q_gscale, 4) || !aligned(k_gscale, 4) || !aligned(v_gscale, 4) || !aligned(row_max, 4) ||
-      !aligned(row_sum, 4) || (s_out && !aligned(s_out, 16)) || (p_codes && !aligned(p_codes, 8)) ||
-      (status && !aligned(status, 4)))
+      !aligned(row_sum, 4) || !aligned(workspace, 16) || (s_out && !aligned(s_out, 16)) ||
+      (p_codes && !aligned(p_codes, 8)) || (status && !aligned(status, 4)))
     return NVFP4_ERR_ALIGN;
+  // workspace: the O accumulators first (16-byte aligned rows), then the row sums and the row maxima
+  const int64_t rows = H * Tq;
+  float* ws = static_cast<float*>(workspace);
+  float* ws_o = splits > 1 ? ws : nullptr;
+  float* ws_l = splits > 1 ? ws + (int64_t)splits * rows * kAfD : nullptr;
+  float* ws_max = splits > 1 ? ws_l + (int64_t)splits * rows : ws;
+  uint8_t* kx = static_cast<uint8_t*>(workspace) + af_tiles_offset(H, Tq, splits);
+  uint8_t* vx = kx + H * (Tk / kAfBN) * (int64_t)kAfTileBytes;
   AttnFusedParams a{q_codes, q_sf, q_gscale, k_codes, k_sf, k_gscale, v_codes_t, v_sf_t, v_gscale, H, Tq, Tk,
-                    alpha, causal ? 1 : 0, q_offset, f_lo, f_hi, out, row_max, row_sum, s_out, p_codes, p_sf, status};
-  const dim3 grid((unsigned)(Tq / kAfBM), (unsigned)H);
+                    alpha, causal ? 1 : 0, q_offset, f_lo, f_hi, splits, ws_max, ws_l, ws_o, kx, vx, out, row_max,
+                    row_sum, s_out, p_codes, p_sf, status};
   cudaStream_t st = S(stream);
-  if (nc == 9) return launch_attn_fused<9>(a, grid, st);
-  if (nc == 1) return launch_attn_fused<1>(a, grid, st);
-  return launch_attn_fused<17>(a, grid, st);
+  if (nc == 9) return launch_attn_fused<9>(a, st);
+  if (nc == 1) return launch_attn_fused<1>(a, st);
+  return launch_attn_fused<17>(a, st);
 }
 
 int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void* stream) {

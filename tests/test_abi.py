@@ -180,7 +180,7 @@ def _ctype_of(decl: str):
         return ctypes.c_char_p if d.startswith("char") else ctypes.c_void_p
     base = d.rsplit(" ", 1)[0] if " " in d else d
     return {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "int32_t": ctypes.c_int, "uint32_t": ctypes.c_uint32,
-            "float": ctypes.c_float}[base]
+            "float": ctypes.c_float, "size_t": ctypes.c_size_t}[base]
 
 
 def test_binding_signatures_match_the_header():

@@ -29,7 +29,7 @@ def _inputs(H, Tq, Tk, seed, D=128):
     return q, k, v
 
 
-def _check(H, Tq, Tk, causal, q_offset, window, seed):
+def _check(H, Tq, Tk, causal, q_offset, window, seed, splits=None):
     D = 128
     q, k, v = _inputs(H, Tq, Tk, seed)
     f_lo, f_hi = window
@@ -39,7 +39,7 @@ def _check(H, Tq, Tk, causal, q_offset, window, seed):
     alpha = D ** -0.5
     out, m, l, s, pc, psf, status = nv.attention_fused(
         qc.view(H, Tq, D // 2), qsf, qg, kc.view(H, Tk, D // 2), ksf, kg, vc.view(H, D, Tk // 2), vsf, vg,
-        causal, q_offset, alpha, f_lo, f_hi, verify=True)
+        causal, q_offset, alpha, f_lo, f_hi, verify=True, splits=splits)
     torch.cuda.synchronize()
     assert status.item() == 0
     # operands from the oracle (linear scales), to form the exact products
@@ -80,15 +80,35 @@ def _check(H, Tq, Tk, causal, q_offset, window, seed):
     return out
 
 
-@pytest.mark.parametrize("H,Tq,Tk,causal,q_offset,window", [
-    (2, 128, 256, False, 0, (-2, 6)),
-    (1, 256, 512, True, 256, (-2, 6)),     # queries at the end of the keys
-    (1, 256, 256, True, 0, (-2, 6)),       # square causal: the first CTA skips the keys past its last row
-    (2, 128, 192, True, 64, (-8, 8)),
-    (1, 128, 64, False, 0, (0, 0)),        # one tile, max-scaling
+@pytest.mark.parametrize("H,Tq,Tk,causal,q_offset,window,splits", [
+    (2, 128, 256, False, 0, (-2, 6), None),
+    (2, 128, 256, False, 0, (-2, 6), 1),    # one range: the numerator kernel writes the result itself
+    (1, 256, 512, True, 256, (-2, 6), 3),   # queries at the end of the keys; ranges of 2 and 3 tiles
+    (1, 256, 256, True, 0, (-2, 6), 3),     # square causal: the first query tile has 2 live tiles, one range empty
+    (2, 128, 192, True, 64, (-8, 8), 2),
+    (1, 128, 64, False, 0, (0, 0), 2),      # one tile, max-scaling; the first range empty
+    (1, 128, 1024, True, 896, (-2, 6), 5),  # ragged ranges of 3 and 4 tiles
 ])
-def test_fused_attention_stages_match_oracle(H, Tq, Tk, causal, q_offset, window):
-    _check(H, Tq, Tk, causal, q_offset, window, seed=H * 1000 + Tk + Tq)
+def test_fused_attention_stages_match_oracle(H, Tq, Tk, causal, q_offset, window, splits):
+    _check(H, Tq, Tk, causal, q_offset, window, seed=H * 1000 + Tk + Tq, splits=splits)
+
+
+def test_fused_attention_split_counts_agree():
+    """Every split count gives the same scores, P~, row maxima and (within the summation bound) O."""
+    H, Tq, Tk, D = 1, 128, 512, 128
+    q, k, v = _inputs(H, Tq, Tk, 11)
+    qc, qsf, qg = nv._prologue_operand(q.cuda(), True, 0, -2, 6)
+    kc, ksf, kg = nv._prologue_operand(k.cuda(), True, 0, -2, 6)
+    vc, vsf, vg = nv.quantize_mma_t(v.cuda(), -2, 6)
+    res = [nv.attention_fused(qc.view(H, Tq, D // 2), qsf, qg, kc.view(H, Tk, D // 2), ksf, kg,
+                              vc.view(H, D, Tk // 2), vsf, vg, True, Tk - Tq, D ** -0.5, -2, 6, verify=True,
+                              splits=s) for s in (1, 2, 4, 8)]
+    o1 = res[0][0].cpu().double()
+    for r in res[1:]:
+        assert r[6].item() == 0
+        assert torch.equal(r[3], res[0][3]) and torch.equal(r[4], res[0][4]) and torch.equal(r[5], res[0][5])
+        assert torch.equal(r[1], res[0][1])
+        assert ((r[0].cpu().double() - o1).abs() <= 1e-5 * o1.abs().max()).all()
 
 
 def test_fused_attention_end_to_end_entry_point():
@@ -114,9 +134,16 @@ def test_fused_attention_argument_errors():
     import ctypes
     P = lambda t: ctypes.c_void_p(t.data_ptr())
     o = torch.zeros(128 * 128, dtype=torch.float32, device=dev)
-    args = lambda Tq, Tk, D, lo, hi: (P(z8), P(z8), P(g), P(z8), P(z8), P(g), P(z8), P(z8), P(g), 1, Tq, Tk, D,
-                                      ctypes.c_float(1.0), 0, 0, lo, hi, P(o), P(g), P(g), None, None, None, None, None)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=dev)
+    args = lambda Tq, Tk, D, lo, hi, splits=1, wsb=1 << 20: (
+        P(z8), P(z8), P(g), P(z8), P(z8), P(g), P(z8), P(z8), P(g), 1, Tq, Tk, D, ctypes.c_float(1.0), 0, 0, lo, hi,
+        splits, P(ws), wsb, P(o), P(g), P(g), None, None, None, None, None)
     assert L.nvfp4_attention_fused(*args(100, 64, 128, -2, 6)) == -2     # Tq % 128
     assert L.nvfp4_attention_fused(*args(128, 48, 128, -2, 6)) == -2     # Tk % 64
     assert L.nvfp4_attention_fused(*args(128, 64, 64, -2, 6)) == -2      # D != 128
     assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 5)) == -1     # 8 offsets
+    assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=0)) == -1
+    assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=65)) == -1
+    need = L.nvfp4_attention_fused_workspace_bytes(1, 128, 64, 2)
+    assert need == (2 * 128 * 4 + 2 * 128 * 129 * 4 + 255) // 256 * 256 + 2 * 64 * 128 * 2
+    assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=2, wsb=need - 1)) == -2   # workspace too small
