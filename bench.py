@@ -1220,17 +1220,26 @@ def run_attn(args, rank, world, dev):
     f_ws = nv.attention_fused_workspace(H, Tq, Tk, f_splits, dev) if fused_ok else None
 
     def step_fused(evs=None):
+        # V's quantization runs on a second stream beside Q's and K's and joins before the attention call
+        cur = torch.cuda.current_stream(dev)
         if evs:
-            evs[0].record(stream)
+            evs[0].record(cur)
+        fork = torch.cuda.Event()
+        fork.record(cur)
+        vside.wait_event(fork)
+        with torch.cuda.stream(vside):
+            nv.quantize_mma_t(v, args.f_lo, args.f_hi, codes=vc, sf=vsf, gscale=vg)
+        vdone = torch.cuda.Event()
+        vdone.record(vside)
         nv.kv_mixed_mma(q4, 0, 0, True, args.f_lo, args.f_hi, codes=qc4, sf=qsf, gscale=qg)
         nv.kv_mixed_mma(k4, 0, 0, True, args.f_lo, args.f_hi, codes=kc4, sf=ksf, gscale=kg)
-        nv.quantize_mma_t(v, args.f_lo, args.f_hi, codes=vc, sf=vsf, gscale=vg)
+        cur.wait_event(vdone)
         if evs:
-            evs[1].record(stream)
+            evs[1].record(cur)
         nv.attention_fused(qc, qsf, qg, kc, ksf, kg, vc, vsf, vg, True, Tk - Tq, scale, args.f_lo, args.f_hi,
                            out=fo, m=fm, l=fl, status=fst, splits=f_splits, workspace=f_ws)
         if evs:
-            evs[2].record(stream)
+            evs[2].record(cur)
         return fo
 
     fused = None

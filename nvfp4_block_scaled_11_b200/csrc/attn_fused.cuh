@@ -417,7 +417,10 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_rowmax_kernel(const Att
   }
 
   const int lim = af_row_limit(a, q);   // this row's last allowed key
-  float m = -INFINITY;
+  // rounding is monotone: for a positive finite scale c, the largest fl(c s) is fl(c max s), so whole
+  // blocks below the row's limit take the maximum of the raw sums (mr) and multiply once at the end
+  const bool pos_scale = sc_s > 0.0f && sc_s <= FLT_MAX;
+  float m = -INFINITY, mr = -INFINITY;
   for (int j = t0; j < t1; ++j) {
     const int b = (j - t0) % kAfMaxStages, b2 = (j + 2 - t0) % kAfMaxStages;
     ok = af_wait(bar_s0 + 8 * b, (ph_s >> b) & 1u) && ok;   // S(j) complete: K buffer b free
@@ -429,9 +432,17 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_rowmax_kernel(const Att
     af_ld16(tmem + t_lane + kAfBN * b + 16 * cb, s);
     af_fence_before();
     const int rem = lim - (j * kAfBN + 16 * cb);   // keys of the block at or below the row's limit
+    if (pos_scale && rem >= 15) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i <= rem) m = fmaxf(m, __fmul_rn(s[i], sc_s));
+      for (int i = 0; i < 8; ++i) s[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] = fmaxf(s[i], s[i + 4]);
+      mr = fmaxf(mr, fmaxf(fmaxf(s[0], s[2]), fmaxf(s[1], s[3])));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i <= rem) m = fmaxf(m, __fmul_rn(s[i], sc_s));
+    }
     if (af_half_sync_or(half, !ok)) {   // every thread has read S(j - 2)'s buffer, which S(j + 2) reuses
       ok = false;
       break;
@@ -444,6 +455,7 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_rowmax_kernel(const Att
     }
   }
   ok = !af_half_sync_or(half, !ok);   // thread 0's waits after the last barrier included
+  m = fmaxf(m, __fmul_rn(mr, sc_s));
   if (ok && split < a.splits) {
     red[half][cb][r] = m;
     af_half_sync(half);
@@ -530,7 +542,8 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   }
 
   const int lim = af_row_limit(a, q);   // this row's last allowed key
-  float l = 0.0f;
+  const u64 sc_s2 = pk2(sc_s, sc_s);
+  u64 l2 = pk2(0.0f, 0.0f);
   for (int j = t0; j < t1; ++j) {
     const int b = (j - t0) & 1;
     ok = af_wait(bar_s0 + 8 * b, (ph >> b) & 1u) && ok;   // S(j) complete, K buffer b free
@@ -542,7 +555,7 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
     float x[16];
     af_ld16(ts, x);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = __fmul_rn(x[i], sc_s);
+    for (int i = 0; i < 16; i += 2) upk2(mul2(pk2(x[i], x[i + 1]), sc_s2), x[i], x[i + 1]);
     if (a.s_out) {
       float* so = a.s_out + row * a.Tk + k0;
 #pragma unroll
@@ -568,8 +581,8 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
     u64 x2[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      l = __fadd_rn(__fadd_rn(l, x[2 * k]), x[2 * k + 1]);
       x2[k] = pk2(x[2 * k], x[2 * k + 1]);
+      l2 = add2(l2, x2[k]);   // two partial row sums (the sum's order is unspecified)
     }
     uint32_t wlo, whi, scale;
     af_quantize_block<NC>(x2, tab, thr, inv6g, a.f_lo, a.f_hi, wlo, whi, scale);
@@ -624,6 +637,9 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   }
 
   // ---- epilogue: the range's O accumulator and row sum, or with one range the result ----
+  float l, l_hi;
+  upk2(l2, l, l_hi);
+  l = __fadd_rn(l, l_hi);
   if (ok && split < a.splits) {
     red[half][cb][r] = l;
     af_half_sync(half);
