@@ -340,13 +340,14 @@ int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void
  *   S = nvfp4_gemm_nt(Q, K, alpha);  nvfp4_softmax_quantize_mma(S, causal, q_offset, f_lo, f_hi);
  *   O = nvfp4_gemm_nt(P~, V^T);  nvfp4_rows_divide(O, row_sum)
  * without the scores leaving the SMs.  Per head and 128 query rows, the 64-key tiles holding an allowed key
- * are cut into `splits` contiguous ranges.  Kernels run on `stream`: one forms S tile by tile on the
- * tensor cores (in tensor memory) and takes each range's row maxima; one forms S again, the numerators
- * exp(S - m) with m the maximum over all ranges, quantizes them (window [f_lo, f_hi] of 1, 9 or 17 offsets,
- * tensor scale fl(1/2688)) and accumulates P~ V^T per range; with splits > 1 a third adds the ranges'
- * accumulators and row sums and divides.  A first kernel writes K and V^T into the workspace as FP16 tiles.  Both products are FP32 sums of the exact products of the NVFP4
- * operands (the summation order differs from nvfp4_gemm_nt's and depends on splits); P~'s codes are those
- * of nvfp4_softmax_quantize_mma applied to this call's scores.
+ * are cut into `splits` contiguous ranges.  Kernels run on `stream`: the first writes Q, K and V^T into the
+ * workspace as FP16 tiles (exact); one forms S on the tensor cores (in tensor memory) and takes row maxima
+ * over (splits + 1) / 2 ranges; one forms S again per range, the numerators exp(S - m) with m the maximum
+ * over all keys, quantizes them (window [f_lo, f_hi] of 1, 9 or 17 offsets, tensor scale fl(1/2688)) and
+ * accumulates P~ V^T; with splits > 1 the last adds the ranges' accumulators and row sums and divides.
+ * Both products are FP32 sums of the exact products of the NVFP4 operands (the summation order differs from
+ * nvfp4_gemm_nt's and depends on splits); P~'s codes are those of nvfp4_softmax_quantize_mma applied to this
+ * call's scores.
  * Operands (device, from the library's quantizers): q_codes [H, Tq, D/2] with q_sf the tile layout of the
  * H [Tq, D] matrices (nvfp4_quantize_mma / nvfp4_kv_mixed_mma) and q_gscale; k_* likewise for [H, Tk, D];
  * v_codes_t [H, D, Tk/2] with v_sf_t the tile layout of the H [D, Tk] matrices (nvfp4_quantize_mma_t).
@@ -355,7 +356,7 @@ int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void
  * key k allowed for query q iff k <= q + q_offset.
  * splits: 1 .. 64 (nvfp4_attention_fused_splits gives the count that fills the current device; any count
  * gives a valid result).  workspace: caller-owned device memory, 16-byte aligned, at least
- * nvfp4_attention_fused_workspace_bytes(H, Tq, Tk, splits) bytes (NVFP4_ERR_SIZE otherwise); it holds K
+ * nvfp4_attention_fused_workspace_bytes(H, Tq, Tk, splits) bytes (NVFP4_ERR_SIZE otherwise); it holds Q, K
  * and V^T expanded to FP16 tiles (exact) and the ranges' row maxima, row sums and accumulators between the
  * kernels, so calls that share a workspace must be ordered on one stream.
  * Outputs: out [H, Tq, D] FP32 (16-byte aligned), row_max and row_sum [H * Tq].  Optional (NULL to skip;
@@ -378,8 +379,8 @@ int nvfp4_attention_fused_splits(int64_t H, int64_t Tq, int64_t Tk, int* splits)
 
 /* Bytes of workspace nvfp4_attention_fused needs for H heads, Tq query rows, Tk keys and `splits` ranges:
  * the ranges' row maxima (4 H Tq splits bytes) and, when splits > 1, row sums and O accumulators
- * (4 H Tq splits (D + 1)), rounded up to 256, plus K and V^T in FP16 (2 H Tk D 2 bytes); 0 for invalid
- * arguments.  Host only. */
+ * (4 H Tq splits (D + 1)), rounded up to 256, plus K, V^T and Q in FP16 ((2 Tk + Tq) H D 2 bytes); 0 for
+ * invalid arguments.  Host only. */
 size_t nvfp4_attention_fused_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int splits);
 
 /* Host only, for verification: the byte offsets at which nvfp4_gemm_nt reads the scale of (matrix l,

@@ -50,19 +50,17 @@ constexpr int kAfD = 128;          // head dimension (the first MMA's K, the sec
 constexpr int kAfThreads = 512;    // a half: 16 warps, 4 per TMEM lane quadrant, one 16-key block each per tile
 constexpr int kAfCtaThreads = 2 * kAfThreads;   // two halves, one key range each
 constexpr int kAfMaxSplits = 64;   // key ranges per query tile
-constexpr int kAfMaxStages = 4;       // row-max kernel: K tiles and S buffers per half
-constexpr int kAfTmemColsMax = 512;   // row-max kernel: per half four S buffers (4 x 64 columns)
+constexpr int kAfTmemColsMax = 512;   // row-max kernel: four S buffers of 128 columns
 constexpr int kAfTmemCols = 512;      // numerator kernel: per half an S double buffer and O (128 columns)
 
-// dynamic shared memory: Q (128 x 128 FP16), shared by the halves, then per half
-//   row maxima:  K tiles (64 x 128) x 4;
-//   numerators:  K tiles x 2, V^T tiles (128 x 64) x 2 and a P~ tile (128 x 64)
+// dynamic shared memory: Q (128 x 128 FP16), then
+//   row maxima:  four stages of two K tiles (64 x 128 each);
+//   numerators:  per half K tiles x 2, V^T tiles (128 x 64) x 2 and a P~ tile (128 x 64)
 constexpr int kAfQBytes = kAfBM * kAfD * 2;
 constexpr int kAfKBytes = kAfBN * kAfD * 2;
 constexpr int kAfVBytes = kAfD * kAfBN * 2;
 constexpr int kAfPBytes = kAfBM * kAfBN * 2;
 constexpr int kAfHalfBytes = 2 * kAfKBytes + 2 * kAfVBytes + kAfPBytes;
-constexpr int kAfMaxSmemBytes = kAfQBytes + 2 * kAfMaxStages * kAfKBytes;
 constexpr int kAfSmemBytes = kAfQBytes + 2 * kAfHalfBytes;
 
 struct AttnFusedParams {
@@ -82,11 +80,13 @@ struct AttnFusedParams {
   int64_t q_offset;
   int f_lo, f_hi;
   int splits;               // key ranges per query tile
-  float* ws_max;            // [splits, H * Tq] the ranges' row maxima
+  float* ws_max;            // [max_splits, H * Tq] the row-max kernel's ranges' row maxima
   float* ws_l;              // [splits, H * Tq] the ranges' row sums (splits > 1)
   float* ws_o;              // [splits, H * Tq, D] the ranges' O accumulators (splits > 1)
+  int max_splits;           // key ranges per query tile of the row-max kernel ((splits + 1) / 2)
   uint8_t* kx;              // [H, Tk / 64] K tiles in FP16, the MMA's shared-memory layout (16 KB each)
   uint8_t* vx;              // [H, Tk / 64] V^T tiles likewise
+  uint8_t* qx;              // [H, Tq / 64] Q tiles likewise (two make a CTA's 128 rows)
   float* out;               // [H, Tq, D]
   float* row_max;           // [H * Tq]
   float* row_sum;           // [H * Tq]
@@ -289,15 +289,26 @@ constexpr uint32_t kAfSboN = 128 * kAfBN / 8;   // tiles whose K is a key tile (
 constexpr uint32_t kAfTileBytes = 16384;        // a K tile (64 x 128) or a V^T tile (128 x 64) in FP16
 
 // ---------------------------------------------------------------------------------------------------------
-// K and V^T as FP16 tiles in the MMA's shared-memory layout (exact: v * E4M3(s), no tensor scale), once per
-// call: kx[h][j] the 64 x 128 K tile j, vx[h][j] the 128 x 64 V^T tile j, 16 KB each, so that the kernels
-// below fetch a tile with one bulk copy.  Grid (Tk / 64, H, 2), 512 threads: one 16-element block each, the
-// eight rows of a core matrix in consecutive threads (128 contiguous bytes per chunk column).
+// Q, K and V^T as FP16 tiles in the MMA's shared-memory layout (exact: v * E4M3(s), no tensor scale), once
+// per call: kx[h][j] the 64 x 128 K tile j, vx[h][j] the 128 x 64 V^T tile j, qx[h][j] the 64 x 128 Q tile j,
+// 16 KB each, so that the kernels below fetch a tile with one bulk copy (two consecutive K or Q tiles form
+// one 128-row tile of the same layout).  Grid (max(Tk, Tq) / 64, H, 3), 512 threads: one 16-element block
+// each, the eight rows of a core matrix in consecutive threads (128 contiguous bytes per chunk column).
 // ---------------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kAfThreads) attn_expand_kernel(const AttnFusedParams a) {
   const int t = threadIdx.x;
   const int64_t j = blockIdx.x, h = blockIdx.y, tiles = a.Tk / kAfBN;
   uint4 lo, hi;
+  if (blockIdx.z == 2) {   // Q: 64 rows x 8 blocks, as K
+    if (j >= a.Tq / kAfBN) return;
+    const int r = (t >> 6) * 8 + (t & 7), kb = (t >> 3) & 7;
+    const int64_t row = j * kAfBN + r;
+    const uint2 cw = *reinterpret_cast<const uint2*>(a.q_codes + ((h * a.Tq + row) * (kAfD / 16) + kb) * 8);
+    af_dequant_block(cw, a.q_sf[af_sf_index(h, row, kb, a.Tq, kAfD / 16)], lo, hi);
+    af_store_block(a.qx + (h * (a.Tq / kAfBN) + j) * kAfTileBytes, r, kb, kAfSboD, lo, hi);
+    return;
+  }
+  if (j >= tiles) return;
   if (blockIdx.z == 0) {   // K: 64 keys (8 row groups of 8) x 8 blocks
     const int r = (t >> 6) * 8 + (t & 7), kb = (t >> 3) & 7;
     const int64_t key = j * kAfBN + r;
@@ -321,14 +332,12 @@ __device__ __forceinline__ void af_fetch_tile(uint32_t dst, const uint8_t* src, 
                ::"r"(dst), "l"(src), "n"(kAfTileBytes), "r"(bar) : "memory");
 }
 
-// The CTA's 128 Q rows: 1024 blocks, one per thread of the CTA.
-__device__ __forceinline__ void af_load_q(const AttnFusedParams& a, uint8_t* sq, int64_t h, int64_t q0, int tid) {
-  const int row = tid >> 3, kb = tid & 7;
-  const int64_t qr = q0 + row;
-  uint4 lo, hi;
-  const uint2 cw = *reinterpret_cast<const uint2*>(a.q_codes + ((h * a.Tq + qr) * (kAfD / 16) + kb) * 8);
-  af_dequant_block(cw, a.q_sf[af_sf_index(h, qr, kb, a.Tq, kAfD / 16)], lo, hi);
-  af_store_block(sq, row, kb, kAfSboD, lo, hi);
+// The CTA's 128 Q rows (two FP16 tiles, 32 KB) by one bulk copy, its bytes counted on `bar`.  One thread.
+__device__ __forceinline__ void af_fetch_q(const AttnFusedParams& a, uint32_t dst, int64_t h, int64_t q0, uint32_t bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "n"(2 * kAfTileBytes) : "memory");
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(a.qx + (h * (a.Tq / kAfBN) + q0 / kAfBN) * kAfTileBytes), "n"(2 * kAfTileBytes),
+               "r"(bar) : "memory");
 }
 
 // Barrier of one half (named barrier 1 + half, 512 threads); the _or form also returns whether p was set
@@ -345,128 +354,170 @@ __device__ __forceinline__ void af_half_sync(int half) {
   asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(kAfThreads) : "memory");
 }
 
-// S = Q K^T (64 columns of TMEM from tmem_d), completion on bar; issued by one thread.
-__device__ __forceinline__ void af_issue_s(uint32_t tmem_d, uint32_t sq, uint32_t sk, uint32_t bar) {
+// S = Q K^T (64 columns of TMEM from tmem_d), completion on bar; issued by one thread.  dq, dk: the
+// descriptors of the Q and K tiles (the descriptor of the K step s is the tile's plus 256 s bytes, 16 s in
+// the start-address field, which cannot carry out of it below 256 KB of shared memory).
+__device__ __forceinline__ void af_issue_s(uint32_t tmem_d, uint64_t dq, uint64_t dk, uint32_t bar) {
   const uint32_t idesc = af_idesc(kAfBN);
 #pragma unroll
-  for (int s = 0; s < kAfD / 16; ++s)
-    af_mma(tmem_d, af_desc(sq + 256 * s, kAfSboD), af_desc(sk + 256 * s, kAfSboD), idesc, s > 0 ? 1u : 0u);
+  for (int s = 0; s < kAfD / 16; ++s) af_mma(tmem_d, dq + 16 * s, dk + 16 * s, idesc, s > 0 ? 1u : 0u);
   af_commit(bar);
 }
 // O (+)= P~ V^T (128 columns of TMEM from tmem_d), completion on bar; issued by one thread.
-__device__ __forceinline__ void af_issue_o(uint32_t tmem_d, uint32_t sp, uint32_t sv, bool acc, uint32_t bar) {
+__device__ __forceinline__ void af_issue_o(uint32_t tmem_d, uint64_t dp, uint64_t dv, bool acc, uint32_t bar) {
   const uint32_t idesc = af_idesc(kAfD);
 #pragma unroll
-  for (int s = 0; s < kAfBN / 16; ++s)
-    af_mma(tmem_d, af_desc(sp + 256 * s, kAfSboN), af_desc(sv + 256 * s, kAfSboN), idesc, (acc || s > 0) ? 1u : 0u);
+  for (int s = 0; s < kAfBN / 16; ++s) af_mma(tmem_d, dp + 16 * s, dv + 16 * s, idesc, (acc || s > 0) ? 1u : 0u);
   af_commit(bar);
 }
 
 // ---------------------------------------------------------------------------------------------------------
-// Row maxima of two key ranges per CTA (one per half): grid (Tq / 128, ceil(splits / 2), H), 1024 threads.
-// Per half: four K tiles in shared memory and four S buffers in TMEM; K(j + 4) is fetched once S(j) has
-// read its buffer, S(j + 2) is issued after the half's barrier of tile j (its K fetched two tiles earlier).
+// Row maxima of one key range per CTA: grid (Tq / 128, splits, H), 16 consumer warps and one producer warp.
+// The range is walked in pairs of 64-key tiles (two consecutive FP16 tiles form one 128-row tile of the
+// same layout): the producer fetches a pair with one bulk copy into one of four K stages and, once it has
+// landed and the consumers have released that stage's TMEM buffer, issues S = Q K^T for it (N = 128, or
+// 64 for a last single tile) -- the MMA issue blocks the issuing thread for about the MMA's duration, so it
+// runs in a warp of its own; the consumers read each S, take the row maxima and release the buffer.
 // ---------------------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kAfCtaThreads, 1) attn_rowmax_kernel(const AttnFusedParams a) {
-  extern __shared__ __align__(1024) uint8_t af_dyn[];
-  __shared__ float red[2][4][kAfBM];
-  __shared__ __align__(8) uint64_t bars[2][2][kAfMaxStages];   // per half: S complete, K landed
-  __shared__ uint32_t tmem_slot;
+constexpr int kAfMaxPairs = 4;                               // K stages and S buffers (128 columns each)
+constexpr int kAfMaxThreads = kAfThreads + 32;
+constexpr int kAfMaxSmemBytes = kAfQBytes + kAfMaxPairs * 2 * kAfKBytes;
 
-  const int tid = threadIdx.x, half = tid / kAfThreads, t = tid % kAfThreads, w = t >> 5, lane = t & 31;
-  const int qd = w & 3, cb = w >> 2;          // TMEM lane quadrant; 16-key block of the tile
-  const int r = 32 * qd + lane;               // this thread's query row within the CTA
-  const int split = 2 * blockIdx.y + half;
+__global__ void __launch_bounds__(kAfMaxThreads, 1) attn_rowmax_kernel(const AttnFusedParams a) {
+  extern __shared__ __align__(1024) uint8_t af_dyn[];
+  __shared__ float red[4][kAfBM];
+  __shared__ __align__(8) uint64_t bars[3][kAfMaxPairs];   // K landed, S complete, S released
+  __shared__ __align__(8) uint64_t bar_q_store;              // Q landed
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_fail;
+
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const bool producer = w == kAfThreads / 32;
+  const int qd = w & 3, cb = w >> 2;          // consumers: TMEM lane quadrant; 32-key quarter of a pair
+  const int r = 32 * qd + lane;               // consumers: this thread's query row within the CTA
+  const int split = blockIdx.y;
   const int64_t h = blockIdx.z, q0 = (int64_t)blockIdx.x * kAfBM, q = q0 + r;
   const int live = af_live_tiles(a, q0);
-  int t0 = 0, t1 = 0;
-  if (split < a.splits) af_range(live, split, a.splits, t0, t1);
+  int t0, t1;
+  af_range(live, split, a.max_splits, t0, t1);
+  const int pairs = (t1 - t0 + 1) / 2;
   uint8_t* const sQ = af_dyn;
-  uint8_t* const sK0 = af_dyn + kAfQBytes + half * kAfMaxStages * kAfKBytes;
+  uint8_t* const sK0 = af_dyn + kAfQBytes;
   const uint8_t* const kx = a.kx + h * (a.Tk / kAfBN) * kAfTileBytes;
+  const uint32_t bar_k0 = af_smem(&bars[0][0]), bar_s0 = af_smem(&bars[1][0]), bar_f0 = af_smem(&bars[2][0]);
+  const uint32_t bar_q = af_smem(&bar_q_store);
 
-  if (tid < 32) {
+  if (w == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(af_smem(&tmem_slot)),
                  "r"(kAfTmemColsMax));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  const uint32_t bar_s0 = af_smem(&bars[half][0][0]), bar_k0 = af_smem(&bars[half][1][0]);
-  const uint32_t sq = af_smem(sQ), sk0 = af_smem(sK0);
-  if (t == 0) {
-    for (int i = 0; i < 2 * kAfMaxStages; ++i)
+  // the tiles of pair u: t0 + 2u and, unless it is past the range, t0 + 2u + 1
+  auto pair_tiles = [&](int u) { return min(2, t1 - t0 - 2 * u); };
+  auto fetch_pair = [&](int u, int i) {
+    const uint32_t bytes = (uint32_t)pair_tiles(u) * kAfTileBytes;
+    const uint32_t bar = bar_k0 + 8 * i;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(af_smem(sK0) + (uint32_t)i * 2 * kAfKBytes), "l"(kx + (int64_t)(t0 + 2 * u) * kAfTileBytes),
+                 "r"(bytes), "r"(bar) : "memory");
+  };
+  if (producer && lane == 0) {
+    for (int i = 0; i < kAfMaxPairs; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_k0 + 8 * i));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_s0 + 8 * i));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar_f0 + 8 * i), "n"(kAfThreads / 32));
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_q));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int i = 0; i < kAfMaxStages && t0 + i < t1; ++i)
-      af_fetch_tile(sk0 + i * kAfKBytes, kx + (int64_t)(t0 + i) * kAfTileBytes, bar_k0 + 8 * i);
+    if (pairs > 0) af_fetch_q(a, af_smem(sQ), h, q0, bar_q);
+    for (int u = 0; u < kAfMaxPairs && u < pairs; ++u) fetch_pair(u, u);
+    s_fail = 0;
   }
-  if (live > 0) af_load_q(a, sQ, h, q0, tid);
   const float sc_s = __fmul_rn(__fmul_rn(a.alpha, *a.q_g), *a.k_g);
   af_proxy_fence();
   af_fence_before();
   __syncthreads();
   af_fence_after();
-  const uint32_t tmem = tmem_slot + (uint32_t)(half * kAfMaxStages * kAfBN), t_lane = (uint32_t)(32 * qd) << 16;
-  uint32_t ph_s = 0, ph_k = 0;   // parity bit per stage: S complete (all threads), K landed (thread 0)
+  const uint32_t tmem = tmem_slot;
   bool ok = true;
-  if (t == 0) {
-    for (int i = 0; i < 2 && t0 + i < t1; ++i) {
-      ok = af_wait(bar_k0 + 8 * i, 0u) && ok;
-      ph_k ^= 1u << i;
-      af_issue_s(tmem + kAfBN * i, sq, sk0 + i * kAfKBytes, bar_s0 + 8 * i);
-    }
-  }
 
-  const int lim = af_row_limit(a, q);   // this row's last allowed key
-  // rounding is monotone: for a positive finite scale c, the largest fl(c s) is fl(c max s), so whole
-  // blocks below the row's limit take the maximum of the raw sums (mr) and multiply once at the end
-  const bool pos_scale = sc_s > 0.0f && sc_s <= FLT_MAX;
-  float m = -INFINITY, mr = -INFINITY;
-  for (int j = t0; j < t1; ++j) {
-    const int b = (j - t0) % kAfMaxStages, b2 = (j + 2 - t0) % kAfMaxStages;
-    ok = af_wait(bar_s0 + 8 * b, (ph_s >> b) & 1u) && ok;   // S(j) complete: K buffer b free
-    ph_s ^= 1u << b;
-    af_fence_after();
-    if (t == 0 && j + kAfMaxStages < t1)
-      af_fetch_tile(sk0 + b * kAfKBytes, kx + (int64_t)(j + kAfMaxStages) * kAfTileBytes, bar_k0 + 8 * b);
-    float s[16];
-    af_ld16(tmem + t_lane + kAfBN * b + 16 * cb, s);
-    af_fence_before();
-    const int rem = lim - (j * kAfBN + 16 * cb);   // keys of the block at or below the row's limit
-    if (pos_scale && rem >= 15) {
+  if (producer) {
+    if (lane == 0) {
+      const uint64_t dq = af_desc(af_smem(sQ), kAfSboD), dk0 = af_desc(af_smem(sK0), kAfSboD);
+      if (pairs > 0) ok = af_wait(bar_q, 0u) && ok;   // Q landed
+      for (int u = 0; u < pairs; ++u) {
+        const int i = u % kAfMaxPairs;
+        const uint32_t par = (uint32_t)(u / kAfMaxPairs) & 1u;
+        ok = af_wait(bar_k0 + 8 * i, par) && ok;                               // K pair u landed
+        if (u >= kAfMaxPairs) ok = af_wait(bar_f0 + 8 * i, par ^ 1u) && ok;    // S(u - 4) released
+        af_fence_after();
+        const uint32_t n = (uint32_t)pair_tiles(u) * kAfBN, idesc = af_idesc(n);
+        const uint64_t dk = dk0 + (uint64_t)i * (2 * kAfKBytes >> 4);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s[i] = fmaxf(s[i], s[i + 8]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s[i] = fmaxf(s[i], s[i + 4]);
-      mr = fmaxf(mr, fmaxf(fmaxf(s[0], s[2]), fmaxf(s[1], s[3])));
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (i <= rem) m = fmaxf(m, __fmul_rn(s[i], sc_s));
+        for (int s = 0; s < kAfD / 16; ++s)
+          af_mma(tmem + (uint32_t)i * 2 * kAfBN, dq + 16 * s, dk + 16 * s, idesc, s > 0 ? 1u : 0u);
+        af_commit(bar_s0 + 8 * i);
+        // the stage of pair u - 1 is free once S(u - 1) has completed: fetch pair u + 3 into it
+        if (u >= 1 && u - 1 + kAfMaxPairs < pairs) {
+          const int ip = (u - 1) % kAfMaxPairs;
+          ok = af_wait(bar_s0 + 8 * ip, (uint32_t)((u - 1) / kAfMaxPairs) & 1u) && ok;
+          fetch_pair(u - 1 + kAfMaxPairs, ip);
+        }
+      }
+      if (!ok) s_fail = 1;
     }
-    if (af_half_sync_or(half, !ok)) {   // every thread has read S(j - 2)'s buffer, which S(j + 2) reuses
-      ok = false;
-      break;
-    }
-    if (t == 0 && j + 2 < t1) {
-      ok = af_wait(bar_k0 + 8 * b2, (ph_k >> b2) & 1u) && ok;   // K(j + 2) landed
-      ph_k ^= 1u << b2;
+  } else {
+    const int lim = af_row_limit(a, q);   // this row's last allowed key
+    // rounding is monotone: for a positive finite scale c, the largest fl(c s) is fl(c max s), so whole
+    // blocks below the row's limit take the maximum of the raw sums (mr) and multiply once at the end
+    const bool pos_scale = sc_s > 0.0f && sc_s <= FLT_MAX;
+    float m = -INFINITY, mr = -INFINITY;
+    for (int u = 0; u < pairs; ++u) {
+      const int i = u % kAfMaxPairs;
+      ok = af_wait(bar_s0 + 8 * i, (uint32_t)(u / kAfMaxPairs) & 1u) && ok;   // S(u) complete
       af_fence_after();
-      af_issue_s(tmem + kAfBN * b2, sq, sk0 + b2 * kAfKBytes, bar_s0 + 8 * b2);
+      const bool mine = 32 * cb < pair_tiles(u) * kAfBN;   // a single last tile has 64 keys
+      float s[16], s2[16];
+      if (mine) {
+        const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)i * 2 * kAfBN + 32 * cb;
+        af_ld16(ta, s);
+        af_ld16(ta + 16, s2);
+      }
+      af_fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_f0 + 8 * i) : "memory");
+      if (mine) {
+        const int rem = lim - ((t0 + 2 * u) * kAfBN + 32 * cb);   // keys at or below the row's limit
+        if (pos_scale && rem >= 31) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) s[k] = fmaxf(s[k], s2[k]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) s[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) s[k] = fmaxf(s[k], s[k + 4]);
+          mr = fmaxf(mr, fmaxf(fmaxf(s[0], s[2]), fmaxf(s[1], s[3])));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            if (k <= rem) m = fmaxf(m, __fmul_rn(s[k], sc_s));
+            if (k + 16 <= rem) m = fmaxf(m, __fmul_rn(s2[k], sc_s));
+          }
+        }
+      }
     }
+    m = fmaxf(m, __fmul_rn(mr, sc_s));
+    red[cb][r] = m;
+    if (!ok) s_fail = 1;
   }
-  ok = !af_half_sync_or(half, !ok);   // thread 0's waits after the last barrier included
-  m = fmaxf(m, __fmul_rn(mr, sc_s));
-  if (ok && split < a.splits) {
-    red[half][cb][r] = m;
-    af_half_sync(half);
-    if (cb == 0)
-      a.ws_max[((int64_t)split * a.H + h) * a.Tq + q] =
-          fmaxf(fmaxf(red[half][0][r], red[half][1][r]), fmaxf(red[half][2][r], red[half][3][r]));
-  }
-  if (!ok && t == 0 && a.status) atomicExch(a.status, 1);
+  __syncthreads();
+  const bool failed = s_fail != 0;
+  if (!failed && !producer && cb == 0)
+    a.ws_max[((int64_t)split * a.H + h) * a.Tq + q] = fmaxf(fmaxf(red[0][r], red[1][r]), fmaxf(red[2][r], red[3][r]));
+  if (failed && tid == 0 && a.status) atomicExch(a.status, 1);
   af_fence_before();
   __syncthreads();
-  if (tid < 32) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "r"(kAfTmemColsMax));
+  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAfTmemColsMax));
 }
 
 // ---------------------------------------------------------------------------------------------------------
@@ -482,6 +533,7 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   __shared__ float thr[128];
   __shared__ float red[2][4][kAfBM];
   __shared__ __align__(8) uint64_t bars[2][7];   // per half: S 0, S 1, O, K landed 0, 1, V landed 0, 1
+  __shared__ __align__(8) uint64_t bar_q_store;   // Q landed
   __shared__ uint32_t tmem_slot;
   CandEntry* tab = tab_store + kTabPad;
 
@@ -513,6 +565,19 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   const uint32_t bar_s0 = af_smem(&bars[half][0]), bar_o = af_smem(&bars[half][2]);
   const uint32_t bar_k0 = af_smem(&bars[half][3]), bar_v0 = af_smem(&bars[half][5]);
   const uint32_t sq = af_smem(sQ), sk0 = af_smem(sK0), sv0 = af_smem(sV0), sp = af_smem(sP);
+  const uint32_t bar_q = af_smem(&bar_q_store);
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_q));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // fetched when a half has tiles (that half's issuing thread waits for it, so no copy is left in flight)
+    bool work = false;
+    for (int s = 2 * (int)blockIdx.y; s < min(2 * (int)blockIdx.y + 2, a.splits); ++s) {
+      int r0, r1;
+      af_range(live, s, a.splits, r0, r1);
+      work = work || r0 < r1;
+    }
+    if (work) af_fetch_q(a, sq, h, q0, bar_q);
+  }
   if (t == 0) {
     for (int i = 0; i < 7; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_s0 + 8 * i));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -522,8 +587,7 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   }
   // the row maximum over all ranges (the row-max kernel's)
   float m = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) m = fmaxf(m, a.ws_max[(int64_t)s * a.H * a.Tq + row]);
-  if (live > 0) af_load_q(a, sQ, h, q0, tid);
+  for (int s = 0; s < a.max_splits; ++s) m = fmaxf(m, a.ws_max[(int64_t)s * a.H * a.Tq + row]);
   const float sc_s = __fmul_rn(__fmul_rn(a.alpha, *a.q_g), *a.k_g);
   af_proxy_fence();
   af_fence_before();
@@ -533,11 +597,14 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   // parity bits: bits 0, 1 S buffers and bit 2 O (all threads); bits 3, 4 K and 5, 6 V landed (thread 0)
   uint32_t ph = 0;
   bool ok = true;
+  const uint64_t dq = af_desc(sq, kAfSboD), dk0 = af_desc(sk0, kAfSboD);
+  const uint64_t dv0 = af_desc(sv0, kAfSboN), dp = af_desc(sp, kAfSboN);
   if (t == 0) {
+    if (t0 < t1) ok = af_wait(bar_q, 0u) && ok;   // Q landed
     for (int i = 0; i < 2 && t0 + i < t1; ++i) {
       ok = af_wait(bar_k0 + 8 * i, 0u) && ok;
       ph ^= 8u << i;
-      af_issue_s(tmem + kAfBN * i, sq, sk0 + i * kAfKBytes, bar_s0 + 8 * i);
+      af_issue_s(tmem + kAfBN * i, dq, dk0 + i * (kAfKBytes >> 4), bar_s0 + 8 * i);
     }
   }
 
@@ -611,11 +678,11 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
       ok = af_wait(bar_v0 + 8 * b, (ph >> (5 + b)) & 1u) && ok;   // V(j) landed
       ph ^= 32u << b;
       af_fence_after();
-      af_issue_o(tmem + 2 * kAfBN, sp, sv0 + b * kAfVBytes, j > t0, bar_o);
+      af_issue_o(tmem + 2 * kAfBN, dp, dv0 + b * (kAfVBytes >> 4), j > t0, bar_o);
       if (j + 2 < t1) {
         ok = af_wait(bar_k0 + 8 * b, (ph >> (3 + b)) & 1u) && ok;   // K(j + 2) landed
         ph ^= 8u << b;
-        af_issue_s(tmem + kAfBN * b, sq, sk0 + b * kAfKBytes, bar_s0 + 8 * b);
+        af_issue_s(tmem + kAfBN * b, dq, dk0 + b * (kAfKBytes >> 4), bar_s0 + 8 * b);
       }
     }
   }
@@ -694,7 +761,7 @@ __global__ void attn_combine_kernel(const AttnFusedParams a) {
   for (int s = 0; s < a.splits; ++s) {
     const int64_t sr = (int64_t)s * rows + row;
     l = __fadd_rn(l, a.ws_l[sr]);
-    m = fmaxf(m, a.ws_max[sr]);
+    if (s < a.max_splits) m = fmaxf(m, a.ws_max[sr]);
     const float4 o = *reinterpret_cast<const float4*>(a.ws_o + sr * kAfD + 4 * c4);
     acc = make_float4(__fadd_rn(acc.x, o.x), __fadd_rn(acc.y, o.y), __fadd_rn(acc.z, o.z), __fadd_rn(acc.w, o.w));
   }

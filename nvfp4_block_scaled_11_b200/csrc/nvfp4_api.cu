@@ -717,10 +717,11 @@ int launch_attn_fused(const AttnFusedParams& a, cudaStream_t st) {
   int rc = af_raise_smem<attn_rowmax_kernel>(kAfMaxSmemBytes);
   if (rc == NVFP4_OK) rc = af_raise_smem<attn_fused_kernel<NC>>(kAfSmemBytes);
   if (rc != NVFP4_OK) return rc;
-  attn_expand_kernel<<<dim3((unsigned)(a.Tk / kAfBN), (unsigned)a.H, 2), kAfThreads, 0, st>>>(a);
-  // a CTA runs two key ranges, one per half
+  attn_expand_kernel<<<dim3((unsigned)(std::max(a.Tk, a.Tq) / kAfBN), (unsigned)a.H, 3), kAfThreads, 0, st>>>(a);
+  attn_rowmax_kernel<<<dim3((unsigned)(a.Tq / kAfBM), (unsigned)a.max_splits, (unsigned)a.H), kAfMaxThreads,
+                       kAfMaxSmemBytes, st>>>(a);
+  // a numerator CTA runs two key ranges, one per half
   const dim3 grid((unsigned)(a.Tq / kAfBM), (unsigned)((a.splits + 1) / 2), (unsigned)a.H);
-  attn_rowmax_kernel<<<grid, kAfCtaThreads, kAfMaxSmemBytes, st>>>(a);
   attn_fused_kernel<NC><<<grid, kAfCtaThreads, kAfSmemBytes, st>>>(a);
   if (a.splits > 1) {
     const int64_t n = a.H * a.Tq * (kAfD / 4);
@@ -730,20 +731,20 @@ int launch_attn_fused(const AttnFusedParams& a, cudaStream_t st) {
 }
 
 // Workspace: the ranges' O accumulators (splits > 1), row sums (splits > 1) and row maxima, then, from a
-// 256-byte boundary, the K and V^T tiles in FP16 (16 KB per 64 keys and head each).
+// 256-byte boundary, the K, V^T and Q tiles in FP16 (16 KB per 64 keys or query rows and head each).
 int64_t af_tiles_offset(int64_t H, int64_t Tq, int64_t splits) {
   const int64_t rows = H * Tq;
   return (splits * rows * 4 + (splits > 1 ? splits * rows * (kAfD + 1) * 4 : 0) + 255) / 256 * 256;
 }
 size_t af_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int64_t splits) {
-  return (size_t)(af_tiles_offset(H, Tq, splits) + 2 * H * (Tk / kAfBN) * (int64_t)kAfTileBytes);
+  return (size_t)(af_tiles_offset(H, Tq, splits) + (2 * H * (Tk / kAfBN) + H * (Tq / kAfBN)) * (int64_t)kAfTileBytes);
 }
 
 extern "C" {
 
 size_t nvfp4_attention_fused_workspace_bytes(int64_t H, int64_t Tq, int64_t Tk, int splits) {
   if (H < 0 || Tq < 0 || Tk < 0 || Tk % kAfBN != 0 || splits < 1 || splits > kAfMaxSplits ||
-      checked_prod({H, Tq, kAfD + 2, splits, 4}) < 0 || checked_prod({H, Tk, 2 * kAfD * 2}) < 0)
+      checked_prod({H, Tq, kAfD + 2, splits, 4}) < 0 || checked_prod({H, Tk + Tq, 2 * kAfD * 2}) < 0)
     return 0;
   return af_workspace_bytes(H, Tq, Tk, splits);
 }
@@ -795,7 +796,7 @@ int nvfp4_attention_fused(const uint8_t* q_codes, const uint8_t* q_sf, const flo
   if (!q_codes || !q_sf || !q_gscale || !k_codes || !k_sf || !k_gscale || !v_codes_t || !v_sf_t || !v_gscale ||
       !out || !row_max || !row_sum || !workspace || ((p_codes == nullptr) != (p_sf == nullptr)))
     return NVFP4_ERR_ARG;
-  if (checked_prod({H, Tk, 2 * D * 2}) < 0 || workspace_bytes < af_workspace_bytes(H, Tq, Tk, splits))
+  if (checked_prod({H, Tk + Tq, 2 * D * 2}) < 0 || workspace_bytes < af_workspace_bytes(H, Tq, Tk, splits))
     return NVFP4_ERR_SIZE;
   if (!aligned(q_codes, 8) || !aligned(k_codes, 8) || !aligned(v_codes_t, 8) || !aligned(k_sf, 4) || !aligned(out, 16) ||
       !aligned(q_gscale, 4) || !aligned(k_gscale, 4) || !aligned(v_gscale, 4) || !aligned(row_max, 4) ||
@@ -810,9 +811,10 @@ int nvfp4_attention_fused(const uint8_t* q_codes, const uint8_t* q_sf, const flo
   float* ws_max = splits > 1 ? ws_l + (int64_t)splits * rows : ws;
   uint8_t* kx = static_cast<uint8_t*>(workspace) + af_tiles_offset(H, Tq, splits);
   uint8_t* vx = kx + H * (Tk / kAfBN) * (int64_t)kAfTileBytes;
+  uint8_t* qx = vx + H * (Tk / kAfBN) * (int64_t)kAfTileBytes;
   AttnFusedParams a{q_codes, q_sf, q_gscale, k_codes, k_sf, k_gscale, v_codes_t, v_sf_t, v_gscale, H, Tq, Tk,
-                    alpha, causal ? 1 : 0, q_offset, f_lo, f_hi, splits, ws_max, ws_l, ws_o, kx, vx, out, row_max,
-                    row_sum, s_out, p_codes, p_sf, status};
+                    alpha, causal ? 1 : 0, q_offset, f_lo, f_hi, splits, ws_max, ws_l, ws_o, (splits + 1) / 2,
+                    kx, vx, qx, out, row_max, row_sum, s_out, p_codes, p_sf, status};
   cudaStream_t st = S(stream);
   if (nc == 9) return launch_attn_fused<9>(a, st);
   if (nc == 1) return launch_attn_fused<1>(a, st);

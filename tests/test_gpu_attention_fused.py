@@ -145,5 +145,5 @@ def test_fused_attention_argument_errors():
     assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=0)) == -1
     assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=65)) == -1
     need = L.nvfp4_attention_fused_workspace_bytes(1, 128, 64, 2)
-    assert need == (2 * 128 * 4 + 2 * 128 * 129 * 4 + 255) // 256 * 256 + 2 * 64 * 128 * 2
+    assert need == (2 * 128 * 4 + 2 * 128 * 129 * 4 + 255) // 256 * 256 + (2 * 64 + 128) * 128 * 2
     assert L.nvfp4_attention_fused(*args(128, 64, 128, -2, 6, splits=2, wsb=need - 1)) == -2   # workspace too small
