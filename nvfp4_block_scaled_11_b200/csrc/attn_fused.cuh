@@ -240,6 +240,30 @@ __device__ __forceinline__ void af_resolve_deferred(unsigned mask, const u64 (&x
   }
 }
 
+// A block's codes and scale byte as write_block stores them: 0x7F for a poisoned block, the chosen code
+// c0 + fstar, or (no usable code) scale 0 with sign-only zeros.
+__device__ __forceinline__ void af_encode_block(const u64 (&x2)[8], bool poisoned, int c0, int fstar,
+                                                const CandEntry* tab, uint32_t& wlo, uint32_t& whi,
+                                                uint32_t& scale) {
+  wlo = whi = 0u;
+  if (poisoned) {
+    scale = 0x7Fu;
+  } else if (fstar != -128) {
+    scale = (uint32_t)(c0 + fstar);
+    encode_pairs(x2, tab[scale].r, wlo, whi);
+  } else {
+    scale = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float lo, hi;
+      upk2(x2[k], lo, hi);
+      const uint32_t nib = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
+      if (k < 4) wlo |= nib << (8 * k);
+      else whi |= nib << (8 * (k - 4));
+    }
+  }
+}
+
 // One P~ block per lane: ScaleSearch with the tensor scale of the table (each lane's codes, scale byte, as
 // write_block would store them), without writing anything.  Called by all 32 lanes of a warp.
 template <int NC>
@@ -264,23 +288,7 @@ __device__ __forceinline__ void af_quantize_block(const u64 (&x2)[8], const Cand
     const unsigned dm = __ballot_sync(0xFFFFFFFFu, deferred);
     if (dm) af_resolve_deferred<NC>(dm, x2, c0, f_lo, f_hi, tab, fstar);
   }
-  wlo = whi = 0u;
-  if (poisoned) {
-    scale = 0x7Fu;
-  } else if (fstar != -128) {
-    scale = (uint32_t)(c0 + fstar);
-    encode_pairs(x2, tab[scale].r, wlo, whi);
-  } else {
-    scale = 0u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float lo, hi;
-      upk2(x2[k], lo, hi);
-      const uint32_t nib = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
-      if (k < 4) wlo |= nib << (8 * k);
-      else whi |= nib << (8 * (k - 4));
-    }
-  }
+  af_encode_block(x2, poisoned, c0, fstar, tab, wlo, whi, scale);
 }
 
 
@@ -594,12 +602,13 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
   __syncthreads();
   af_fence_after();
   const uint32_t tmem = tmem_slot + (uint32_t)(half * 4 * kAfBN), t_lane = (uint32_t)(32 * qd) << 16;
-  // parity bits: bits 0, 1 S buffers and bit 2 O (all threads); bits 3, 4 K and 5, 6 V landed (thread 0)
+  // parity bits: bits 0, 1 S buffers and bit 2 O (all threads); bits 3, 4 K landed (thread 32) and 5, 6 V
+  // landed (thread 0)
   uint32_t ph = 0;
   bool ok = true;
   const uint64_t dq = af_desc(sq, kAfSboD), dk0 = af_desc(sk0, kAfSboD);
   const uint64_t dv0 = af_desc(sv0, kAfSboN), dp = af_desc(sp, kAfSboN);
-  if (t == 0) {
+  if (t == 32) {   // the S products' thread (the O products': thread 0)
     if (t0 < t1) ok = af_wait(bar_q, 0u) && ok;   // Q landed
     for (int i = 0; i < 2 && t0 + i < t1; ++i) {
       ok = af_wait(bar_k0 + 8 * i, 0u) && ok;
@@ -616,7 +625,7 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
     ok = af_wait(bar_s0 + 8 * b, (ph >> b) & 1u) && ok;   // S(j) complete, K buffer b free
     ph ^= 1u << b;
     af_fence_after();
-    if (t == 0 && j + 2 < t1) af_fetch_tile(sk0 + b * kAfKBytes, kx + (int64_t)(j + 2) * kAfTileBytes, bar_k0 + 8 * b);
+    if (t == 32 && j + 2 < t1) af_fetch_tile(sk0 + b * kAfKBytes, kx + (int64_t)(j + 2) * kAfTileBytes, bar_k0 + 8 * b);
     const uint32_t ts = tmem + t_lane + kAfBN * b + 16 * cb;
     const int k0 = j * kAfBN + 16 * cb;
     float x[16];
@@ -674,16 +683,19 @@ __global__ void __launch_bounds__(kAfCtaThreads, 1) attn_fused_kernel(const Attn
       ok = false;
       break;
     }
+    // the issue of a product holds its thread for about the product's duration: O and S are issued from
+    // two warps (thread 0 and thread 32 of the half), so that neither is held back by both
     if (t == 0) {
       ok = af_wait(bar_v0 + 8 * b, (ph >> (5 + b)) & 1u) && ok;   // V(j) landed
       ph ^= 32u << b;
       af_fence_after();
       af_issue_o(tmem + 2 * kAfBN, dp, dv0 + b * (kAfVBytes >> 4), j > t0, bar_o);
-      if (j + 2 < t1) {
-        ok = af_wait(bar_k0 + 8 * b, (ph >> (3 + b)) & 1u) && ok;   // K(j + 2) landed
-        ph ^= 8u << b;
-        af_issue_s(tmem + kAfBN * b, dq, dk0 + b * (kAfKBytes >> 4), bar_s0 + 8 * b);
-      }
+    }
+    if (t == 32 && j + 2 < t1) {
+      ok = af_wait(bar_k0 + 8 * b, (ph >> (3 + b)) & 1u) && ok;   // K(j + 2) landed
+      ph ^= 8u << b;
+      af_fence_after();
+      af_issue_s(tmem + kAfBN * b, dq, dk0 + b * (kAfKBytes >> 4), bar_s0 + 8 * b);
     }
   }
   ok = !af_half_sync_or(half, !ok);   // thread 0's waits after the last barrier included

@@ -721,8 +721,8 @@ int launch_attn_fused(const AttnFusedParams& a, cudaStream_t st) {
   attn_rowmax_kernel<<<dim3((unsigned)(a.Tq / kAfBM), (unsigned)a.max_splits, (unsigned)a.H), kAfMaxThreads,
                        kAfMaxSmemBytes, st>>>(a);
   // a numerator CTA runs two key ranges, one per half
-  const dim3 grid((unsigned)(a.Tq / kAfBM), (unsigned)((a.splits + 1) / 2), (unsigned)a.H);
-  attn_fused_kernel<NC><<<grid, kAfCtaThreads, kAfSmemBytes, st>>>(a);
+  attn_fused_kernel<NC><<<dim3((unsigned)(a.Tq / kAfBM), (unsigned)((a.splits + 1) / 2), (unsigned)a.H),
+                          kAfCtaThreads, kAfSmemBytes, st>>>(a);
   if (a.splits > 1) {
     const int64_t n = a.H * a.Tq * (kAfD / 4);
     attn_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a);
