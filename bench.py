@@ -1340,6 +1340,38 @@ def run_attn(args, rank, world, dev):
         "cuda_graph": {"used_for_value": graph_used, "eager_ms_per_step": eager_ms / steps,
                        "v_quantize_on_second_stream": v_overlap_used},
     }
+    if not args.no_e2e and args.e2e_steps > 0:
+        # the schedule that set `value`, with every step's q, k, v copied in from pinned host memory and O
+        # read back
+        hq, hk, hv = (torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True) for t_ in (q, k, v))
+        hq.copy_(q), hk.copy_(k), hv.copy_(v)
+        ho = torch.empty((H, Tq, D), dtype=torch.float32, pin_memory=True)
+        run_step = step_fused if fused and fused["used_for_value"] else step
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            ho.copy_(run_step(), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        line["e2e"] = {"value": world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": sum(t_.numel() * t_.element_size() for t_ in (hq, hk, hv)),
+                       "d2h_bytes_per_step": ho.numel() * ho.element_size(),
+                       "schedule": "fused" if run_step is step_fused else "chain"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = attn_oracle_baseline(args)
     if world > 1:
