@@ -193,6 +193,21 @@ __device__ __forceinline__ void af_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 consecutive columns of this warp's TMEM lanes in one load (one wait).
+__device__ __forceinline__ void af_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+               "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                 "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                 "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void af_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void af_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void af_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -486,12 +501,8 @@ __global__ void __launch_bounds__(kAfMaxThreads, 1) attn_rowmax_kernel(const Att
       ok = af_wait(bar_s0 + 8 * i, (uint32_t)(u / kAfMaxPairs) & 1u) && ok;   // S(u) complete
       af_fence_after();
       const bool mine = 32 * cb < pair_tiles(u) * kAfBN;   // a single last tile has 64 keys
-      float s[16], s2[16];
-      if (mine) {
-        const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)i * 2 * kAfBN + 32 * cb;
-        af_ld16(ta, s);
-        af_ld16(ta + 16, s2);
-      }
+      float s[32];
+      if (mine) af_ld32(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)i * 2 * kAfBN + 32 * cb, s);
       af_fence_before();
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_f0 + 8 * i) : "memory");
@@ -499,7 +510,7 @@ __global__ void __launch_bounds__(kAfMaxThreads, 1) attn_rowmax_kernel(const Att
         const int rem = lim - ((t0 + 2 * u) * kAfBN + 32 * cb);   // keys at or below the row's limit
         if (pos_scale && rem >= 31) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) s[k] = fmaxf(s[k], s2[k]);
+          for (int k = 0; k < 16; ++k) s[k] = fmaxf(s[k], s[k + 16]);
 #pragma unroll
           for (int k = 0; k < 8; ++k) s[k] = fmaxf(s[k], s[k + 8]);
 #pragma unroll
@@ -507,10 +518,8 @@ __global__ void __launch_bounds__(kAfMaxThreads, 1) attn_rowmax_kernel(const Att
           mr = fmaxf(mr, fmaxf(fmaxf(s[0], s[2]), fmaxf(s[1], s[3])));
         } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 32; ++k)
             if (k <= rem) m = fmaxf(m, __fmul_rn(s[k], sc_s));
-            if (k + 16 <= rem) m = fmaxf(m, __fmul_rn(s2[k], sc_s));
-          }
         }
       }
     }
