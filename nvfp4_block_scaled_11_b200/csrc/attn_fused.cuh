@@ -4,40 +4,44 @@
 // ScaleSearchAttention > native NVFP4 execution: Q K^T and P V^T run as NVFP4 products with FP32
 // accumulation and the softmax numerators P~ are ScaleSearch-quantized before the second product.  The
 // unfused chain writes the FP32 scores to HBM and reads them twice; here they never leave the SM.  The
-// 64-key tiles that hold an allowed key of a 128-row query tile are cut into `splits` contiguous ranges,
-// one CTA per (query tile, range, head), so that the grid fills every SM whatever the number of query
-// tiles, and three kernels run in turn:
-//   row maxima:  per range, S = alpha g_q g_k (Q K^T) tile by tile into tensor memory (TMEM) and the
-//                maximum over each row's allowed keys, written per range;
-//   numerators:  per range, S again, m = the maximum over the ranges, P~ = exp(S - m) (the same exp
-//                method as the oracle), ScaleSearch of every 16-key block with the tensor scale
-//                fl(1/2688) (the library's certified fast score, the definition where it cannot decide),
-//                the quantized block written to shared memory as the A operand of O += P~ V^T in TMEM;
-//                the range's O accumulator and row sum l are written out (or, with one range, the result);
+// 64-key tiles that hold an allowed key of a 128-row query tile are cut into `splits` contiguous ranges so
+// that the grid fills every SM whatever the number of query tiles, and four kernels run in turn:
+//   expand:      Q, K and V^T written once as FP16 tiles in the MMA's shared-memory layout, so that every
+//                later tile is one bulk copy;
+//   row maxima:  per range ((splits + 1) / 2 of them), S = alpha g_q g_k (Q K^T) into tensor memory (TMEM)
+//                over pairs of tiles and the maximum over each row's allowed keys, written per range;
+//   numerators:  per range (two per CTA, one per 512-thread half), S again tile by tile, m = the maximum
+//                over all keys, P~ = exp(S - m) (the same exp method as the oracle), ScaleSearch of every
+//                16-key block with the tensor scale fl(1/2688) (the library's certified fast score, the
+//                definition where it cannot decide), the quantized block written to shared memory as the A
+//                operand of O += P~ V^T in TMEM; the range's O accumulator and row sum l are written out
+//                (or, with one range, the result);
 //   combine:     O = fl(fl(sum of the ranges' accumulators * fl(g_p g_v)) / l), l the sum of the ranges'.
 // Every result is the unfused chain's formula: P~'s codes are those of the definition applied to this
-// kernel's own scores, and both products are sums of exact terms accumulated in FP32.
+// call's own scores, and both products are sums of exact terms accumulated in FP32.
 //
 // The operands are the library's NVFP4 tensors (codes plus E4M3 scales in the tile layout).  Each 16-element
-// block is dequantized into shared memory as FP16 values v * E4M3(s) without the tensor scale: a product of
-// a 2-significant-bit E2M1 value and a 4-bit E4M3 scale lies in [2^-10, 2688] with at most 6 significant
-// bits, so it is exact in FP16, and the FP16 tensor-core MMA (kind::f16, FP32 accumulation) forms exactly
-// the products the block-scaled FP4 MMA forms.  This keeps scale factors out of TMEM; the quantizer, not the
-// tensor pipe, bounds this kernel.
+// block enters the tensor cores as FP16 values v * E4M3(s) without the tensor scale: a product of a
+// 2-significant-bit E2M1 value and a 4-bit E4M3 scale lies in [2^-10, 2688] with at most 6 significant bits,
+// so it is exact in FP16, and the FP16 tensor-core MMA (kind::f16, FP32 accumulation) forms exactly the
+// products the block-scaled FP4 MMA forms.  This keeps scale factors out of TMEM; the quantizer, not the
+// tensor pipe, bounds this work.
 //
 // Layout in shared memory (no swizzle, the MMA's K-major canonical layout): a matrix of R rows and K
 // columns of FP16 is stored as 16-byte chunks, chunk c (elements 8c..8c+7) of row r at
 //   (r mod 8) * 16 + (r div 8) * SBO + c * 128,   SBO = 128 * K / 8,
 // so one MMA instruction (K = 16: chunks 2s and 2s+1) reads from start + 256 s with LBO = 128 and that SBO.
+// Two such 64-row tiles one after the other are one 128-row tile of the same layout.
 //
-// Schedule of the numerator kernel (one CTA barrier per tile): the products of tile j + 1 were issued a tile
-// earlier; a thread waits for S(j), reads its 16 scores, forms and quantizes its block of P~(j), waits for
-// O += P~(j-1) V(j-1) (long finished), stores its block of P~(j), of V(j) and of K(j+2); after the barrier
-// one thread issues O += P~(j) V(j) and S(j+2).  P~ and V have one buffer each, K and S two, so that the CTA
-// needs 96 KB of shared memory and 256 TMEM columns and two CTAs share an SM.
+// Schedule of the numerator kernel (one barrier per tile and half): S(j) was issued two tiles earlier; a
+// thread waits for it, reads its 16 scores, forms and quantizes its block of P~(j), waits for O += P~(j-1)
+// V(j-1) (long finished), stores its block of P~(j); after the half's barrier one thread issues O += P~(j)
+// V(j) and another S(j + 2).  K(j + 2) is fetched once S(j) has read its buffer, V(j + 1) once O(j - 1) has
+// read its buffer.  Kernels that allocate TMEM run one CTA per SM, so each CTA holds two independent halves
+// (1024 threads, 64 registers): 192 KB of shared memory and all 512 TMEM columns.
 //
-// Waits on the MMA completion barriers are bounded; a wait that runs out sets a status word, every thread
-// of the CTA leaves, the TMEM allocation is released and the outputs of that CTA are left unwritten.
+// Waits on the MMA and copy completion barriers are bounded; a wait that runs out sets a status word, the
+// threads of the CTA leave, the TMEM allocation is released and the outputs are not valid.
 #pragma once
 
 #include "attention.cuh"
