@@ -78,8 +78,10 @@ __device__ __forceinline__ bool exp_fast16(float m, float (&x)[16]) {
     upk2(p2, pa, pb);
     upk2(t2, ta, tb);
     ok = ok && ta >= t_min && tb >= t_min;
-    x[i] = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
-    x[i + 1] = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+    // unsigned: the shift discards bits(t)'s high bits and the add wraps, both defined (a signed shift
+    // that overflows is undefined behaviour)
+    x[i] = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+    x[i + 1] = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
   }
   return ok;
 }

@@ -3,7 +3,9 @@ kernel's own intermediate values (returned only when asked for, for verification
 * S: each score within the FP32-accumulation bound (D + 4) 2^-24 |alpha g_q g_k| sum_d |q_d k_d| of the
   exact product of the same NVFP4 operands;
 * P~: the oracle's softmax quantizer applied to the kernel's scores gives the kernel's codes, tile-layout
-  scales and row maxima bit for bit, and its row sums within the FP32 summation bound;
+  scales and row maxima bit for bit, and its row sums within the FP32 summation bound; the oracle's
+  numerators summed in the call's order (per range, column block, even/odd accumulators) give the
+  kernel's row sums bit for bit;
 * O: each element within (Tk + 4) 2^-24 g_p g_v sum_k |p_k v_k| / l of the exact product of the oracle's
   P~ and V divided by the kernel's row sum, plus the division's rounding."""
 import numpy as np
@@ -27,6 +29,41 @@ def _inputs(H, Tq, Tk, seed, D=128):
     k = (torch.randn((H, Tk, D), generator=g) * 1.3).to(torch.bfloat16)
     v = torch.randn((H, Tk, D), generator=g).to(torch.bfloat16)
     return q, k, v
+
+
+def _row_sums_in_call_order(s, m, causal, q_offset, splits):
+    """The row sums the fused call forms, from the oracle's numerators exp(S - m) of the call's scores: per
+    key range (the 64-key tiles with an allowed key of the query tile, cut into `splits` ranges), per 16-key
+    column block cb of each tile, the even and odd elements summed in two FP32 accumulators tile by tile
+    and added; the four column blocks added in order; the ranges added in order."""
+    f = np.float32
+    H, Tq, Tk = s.shape
+    exp_ss = np.vectorize(lambda d: O.exp_ss(d), otypes=[np.float32])
+    keys = np.arange(Tk)[None, :]
+    out = np.zeros((H, Tq), np.float32)
+    for h in range(H):
+        for q0 in range(0, Tq, 128):
+            rows = np.arange(q0, q0 + 128)
+            lim = (rows + q_offset)[:, None] if causal else np.full((128, 1), Tk - 1)
+            lim_cta = q0 + 127 + q_offset if causal else Tk - 1
+            live = 0 if lim_cta < 0 else min(Tk // 64, lim_cta // 64 + 1)
+            d = (s[h, q0:q0 + 128].astype(np.float32) - m[h, q0:q0 + 128, None].astype(np.float32)).astype(np.float32)
+            x = np.where(keys <= lim, exp_ss(d), f(0))
+            total = np.zeros(128, np.float32)
+            for sp in range(splits):
+                t0, t1 = live * sp // splits, live * (sp + 1) // splits
+                part = np.zeros(128, np.float32)
+                for cb in range(4):
+                    lo = np.zeros(128, np.float32)
+                    hi = np.zeros(128, np.float32)
+                    for j in range(t0, t1):
+                        for kk in range(8):
+                            lo = (lo + x[:, 64 * j + 16 * cb + 2 * kk]).astype(np.float32)
+                            hi = (hi + x[:, 64 * j + 16 * cb + 2 * kk + 1]).astype(np.float32)
+                    part = (part + (lo + hi).astype(np.float32)).astype(np.float32) if cb else (lo + hi).astype(np.float32)
+                total = (total + part).astype(np.float32)
+            out[h, q0:q0 + 128] = total
+    return out
 
 
 def _check(H, Tq, Tk, causal, q_offset, window, seed, splits=None):
@@ -69,6 +106,11 @@ def _check(H, Tq, Tk, causal, q_offset, window, seed, splits=None):
     assert np.array_equal(m.cpu().numpy(), rm.reshape(-1))
     l_g = l.cpu().numpy().astype(np.float64).reshape(H, Tq)
     assert (np.abs(l_g - rl) <= (Tk + 4) * U * rl).all()
+    # ... and bit for bit the oracle's numerators summed in the call's order
+    nsplit = splits if splits is not None else nv.attention_fused_splits(H, Tq, Tk)
+    assert np.array_equal(l.cpu().numpy().reshape(H, Tq),
+                          _row_sums_in_call_order(s.cpu().numpy(), m.cpu().numpy().reshape(H, Tq), causal, q_offset,
+                                                  nsplit))
     # O; a row with no allowed key has l = 0 and O = 0 / 0 (NaN), as in the unfused chain
     d_ref = O.gemm_nt(rc, rs, rg, rvc, rvs, rvg, Tq, D, Tk, 1.0, H)
     pmag = np.stack([np.abs(O.block_values(rc.reshape(H, -1)[h], rs.reshape(H, -1)[h], Tq, Tk)) @
