@@ -89,3 +89,19 @@ def test_decode_reference_arm_lines(workload, extra):
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"].startswith(workload)
+
+
+@pytest.mark.gpu
+def test_attention_workload_line():
+    """The FP4-attention line: the fused call and the chain timed, the faster one sets `value`, and the
+    end-to-end figure copies q, k and v in and O back every step."""
+    d = _run("--workload", "attn_nvfp4", "--scale", "0.125", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+             "--e2e-steps", "3")
+    for key in ("metric", "value", "unit", "ms_per_step", "dtype", "config", "roofline", "e2e", "clocks",
+                "gpu_launches", "fused"):
+        assert key in d, key
+    assert d["unit"] == "TFLOP/s" and d["value"] > 0 and d["gpu_launches"] > 0
+    assert d["fused"]["status"] == 0 and d["fused"]["max_abs_diff_vs_chain"] < 1e-5
+    H, Tq, Tk, D = (d["config"][k] for k in ("H", "Tq", "Tk", "D"))
+    assert d["e2e"]["h2d_bytes_per_step"] == 2 * H * D * (Tq + 2 * Tk) and d["e2e"]["value"] > 0
+    assert d["e2e"]["d2h_bytes_per_step"] == 4 * H * Tq * D
