@@ -81,6 +81,35 @@ def test_other_entry_point_errors(L):
     assert L.nvfp4_quantize_ex(fake, 32, 0, 16, -2, 6, None, fake, fake, None, None, None, None) == -1
 
 
+def test_attention_fused_host_checks(L):
+    """The fused attention's workspace size and its argument errors, all decided on the host before any
+    launch (fake device pointers; no GPU needed)."""
+    W = L.nvfp4_attention_fused_workspace_bytes
+    # maxima only (one range), plus sums and accumulators (several), rounded to 256, then Q, K, V^T tiles
+    assert W(2, 256, 512, 1) == (2 * 256 * 4 + 255) // 256 * 256 + (2 * 512 + 256) * 2 * 128 * 2
+    assert W(2, 256, 512, 3) == (3 * 512 * 4 + 3 * 512 * 129 * 4 + 255) // 256 * 256 + (2 * 512 + 256) * 2 * 128 * 2
+    for bad in ((-1, 128, 64, 1), (1, 128, 63, 1), (1, 128, 64, 0), (1, 128, 64, 65)):
+        assert W(*bad) == 0, bad
+    fake = V(0x10000)
+    ws_ok = W(1, 128, 64, 1)
+
+    def call(Tq=128, Tk=64, D=128, lo=-2, hi=6, splits=1, ws=fake, wsb=ws_ok, kc=fake, ksf=fake, out=fake, pc=None,
+             psf=None):
+        return L.nvfp4_attention_fused(fake, fake, fake, kc, ksf, fake, fake, fake, fake, 1, Tq, Tk, D,
+                                       ctypes.c_float(1.0), 1, 0, lo, hi, splits, ws, wsb, out, fake, fake, None, pc,
+                                       psf, None, None)
+    assert call(Tq=100) == -2 and call(Tk=48) == -2 and call(D=64) == -2 and call(Tk=1 << 26) == -2
+    assert call(lo=-2, hi=5) == -1 and call(lo=0, hi=-1) == -1          # 8 offsets; empty window
+    assert call(splits=0) == -1 and call(splits=65) == -1
+    assert call(ws=None) == -1 and call(wsb=ws_ok - 1) == -2             # no workspace; too small
+    assert call(pc=fake) == -1                                           # codes without scales
+    assert call(kc=V(0x10004)) == -3 and call(ksf=V(0x10002)) == -3 and call(out=V(0x10008)) == -3
+    assert call(ws=V(0x10008)) == -3
+    assert L.nvfp4_attention_fused(fake, fake, fake, fake, fake, fake, fake, fake, fake, 0, 128, 64, 128,
+                                   ctypes.c_float(1.0), 1, 0, -2, 6, 1, None, 0, None, None, None, None, None, None,
+                                   None, None) == 0                       # no heads: nothing to do
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(TypeError):
