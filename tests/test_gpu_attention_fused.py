@@ -47,8 +47,9 @@ def _row_sums_in_call_order(s, m, causal, q_offset, splits):
             lim = (rows + q_offset)[:, None] if causal else np.full((128, 1), Tk - 1)
             lim_cta = q0 + 127 + q_offset if causal else Tk - 1
             live = 0 if lim_cta < 0 else min(Tk // 64, lim_cta // 64 + 1)
-            d = (s[h, q0:q0 + 128].astype(np.float32) - m[h, q0:q0 + 128, None].astype(np.float32)).astype(np.float32)
-            x = np.where(keys <= lim, exp_ss(d), f(0))
+            with np.errstate(invalid="ignore"):   # rows with no allowed key: m = -inf, every key masked
+                d = (s[h, q0:q0 + 128].astype(np.float32) - m[h, q0:q0 + 128, None].astype(np.float32)).astype(np.float32)
+                x = np.where(keys <= lim, exp_ss(d), f(0))
             total = np.zeros(128, np.float32)
             for sp in range(splits):
                 t0, t1 = live * sp // splits, live * (sp + 1) // splits
@@ -134,6 +135,10 @@ def _check(H, Tq, Tk, causal, q_offset, window, seed, splits=None):
     (1, 128, 64, False, 0, (0, 0), 2),      # one tile, max-scaling; the first range empty
     (1, 128, 1024, True, 896, (-2, 6), 5),  # ragged ranges of 3 and 4 tiles
     (1, 256, 192, True, -200, (-2, 6), 2),  # rows 0..199 see no key: m = -inf, l = 0, O = 0 / 0
+    (2, 384, 1536, True, 1152, (-2, 6), None),   # three query tiles, the device's split count
+    (3, 256, 768, False, 0, (-8, 8), 7),    # odd head count, seven ranges (a CTA's second half idle)
+    (1, 512, 512, True, 0, (0, 0), 4),      # square causal over four query tiles, max-scaling
+    (2, 128, 1024, True, 300, (-2, 6), 3),  # the limit inside a tile
 ])
 def test_fused_attention_stages_match_oracle(H, Tq, Tk, causal, q_offset, window, splits):
     _check(H, Tq, Tk, causal, q_offset, window, seed=H * 1000 + Tk + Tq, splits=splits)
