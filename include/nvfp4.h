@@ -347,7 +347,9 @@ int nvfp4_rows_divide(float* x, const float* l, int64_t rows, int64_t cols, void
  * accumulates P~ V^T; with splits > 1 the last adds the ranges' accumulators and row sums and divides.
  * Both products are FP32 sums of the exact products of the NVFP4 operands (the summation order differs from
  * nvfp4_gemm_nt's and depends on splits); P~'s codes are those of nvfp4_softmax_quantize_mma applied to this
- * call's scores.
+ * call's scores, and row_sum adds its numerators in a fixed order: per key range and 16-key column block of
+ * the 64-key tiles, the even and the odd keys in two FP32 sums tile by tile, added; the four column blocks,
+ * then the ranges, added in order.
  * Operands (device, from the library's quantizers): q_codes [H, Tq, D/2] with q_sf the tile layout of the
  * H [Tq, D] matrices (nvfp4_quantize_mma / nvfp4_kv_mixed_mma) and q_gscale; k_* likewise for [H, Tk, D];
  * v_codes_t [H, D, Tk/2] with v_sf_t the tile layout of the H [D, Tk] matrices (nvfp4_quantize_mma_t).
